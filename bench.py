@@ -1,0 +1,451 @@
+"""Benchmark of the int4 blockwise-quantised Qwen2 decoder step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Default workload (N = 1): the full 28-layer decoder_step at 1.5B shapes (hidden 1536, 12/2 heads
+x 128, intermediate 8960, vocab 151936 tied), symmetric int4 block-32 weights from N(0, 0.02)
+masters, batch 1, past P = 1024, sequences of 64 consecutive steps that each append to the
+GPU-resident KV cache (the length is reset to 1024 after every 64 steps).  A bench step is one
+decoder_step.  Inputs are seeded synthetic data; weights (1.2 GB) and the lm_head (467 MB) are far
+larger than L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): replicas only -- every rank runs its own decoder on its own GPU, no
+collective on the data path; value = tokens of all ranks / max-over-ranks device time.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = ("decode step µs & tok/s at batch 1; achieved HBM GB/s vs B200 peak (1.5B, 7B)")
+
+CONFIGS = {
+    # name: (shape, mode, past P, steps per sequence, description)
+    "decode-1p5b": (synth.SHAPE_1P5B, "int4", 1024, 64,
+                    "28-layer decoder_step, 1.5B shapes, int4 sym block-32, P=1024, batch 1"),
+    "decode-7b": (synth.SHAPE_7B, "int4", 4096, 64,
+                  "28-layer decoder_step, 7B shapes, int4 sym block-32, P=4096, batch 1"),
+    "decode-asr-1p5b": (synth.SHAPE_1P5B, "ternary", 4530, 256,
+                        "ASR-shaped long decode, 1.5B ternary, P=4530 -> 4785, batch 1"),
+    "layer-1p5b": (synth.Shape("layer", 1536, 1, 12, 2, 128, 8960, 151936, tied=True), "ternary",
+                   128, 64, "one decoder layer + lm_head, 1.5B shapes, ternary, P=128"),
+}
+
+
+def std_for(shape):
+    return 0.015 if shape.hidden == 3584 else 0.02
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------- bytes
+def phase_bytes(shape, P):
+    """Algorithmic bytes per launch of each decode phase at past length P (per layer, except
+    the lm_head which is per step)."""
+    H, D, Hq, Hkv, I, V = shape.hidden, shape.head_dim, shape.n_q, shape.n_kv, shape.inter, shape.vocab
+
+    def packed(N, K):
+        return N * (K // 32) * 18
+
+    qkv_rows = (Hq + 2 * Hkv) * D
+    return {
+        "qkv": packed(qkv_rows, H) + 2 * qkv_rows + 2 * H + 4 * H + 4 * qkv_rows,
+        "attn": 2 * Hkv * (P + 1) * D * 2 + 4 * qkv_rows + 4 * Hq * D,
+        "o_proj": packed(H, Hq * D) + 4 * Hq * D + 8 * H,
+        "gate_up": 2 * packed(I, H) + 2 * H + 4 * H + 4 * I,
+        "down": packed(H, I) + 4 * I + 8 * H,
+        "lm_head": V * H * 2 + 2 * H + 4 * H + 4 * V,
+    }
+
+
+def step_bytes(shape, P):
+    b = phase_bytes(shape, P)
+    return shape.layers * sum(v for k, v in b.items() if k != "lm_head") + b["lm_head"]
+
+
+# ----------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ------------------------------------------------------------------------------ CPU baseline
+class OracleSample:
+    """The oracle (as it stands) on a bounded sample of one decode step: one decoder layer
+    (weights dequantised inside the call, as the oracle always does) plus 1/L of the lm_head
+    rows.  L such samples make one step, so step time ~= L x sample time."""
+
+    def __init__(self, shape, mode, P, layers=2):
+        from oracle import decoder as odec
+        from oracle import pack as opack
+
+        std = std_for(shape)
+        self.shape, self.P = shape, P
+        self.layers = []
+        for li in range(layers):
+            lw = dict(synth.layer_vectors(shape, li))
+            for m in synth.MATRICES:
+                W = synth.master(shape, m, li, std)
+                lw[m] = (opack.pack_ternary(W, opack.ternary_scale(W)) if mode == "ternary"
+                         else opack.pack_sym_int4(W))
+            self.layers.append(lw)
+        tables = synth.model_tables(shape)
+        rows = -(-shape.vocab // shape.layers)
+        self.lm_slice = np.ascontiguousarray(tables["lm_head"][:rows])
+        self.final_norm = tables["final_norm"]
+        sub = synth.Shape(shape.name, shape.hidden, layers, shape.n_q, shape.n_kv,
+                          shape.head_dim, shape.inter, shape.vocab, shape.tied)
+        self.kp, self.vp = synth.past_kv(sub, P)
+        self.emb = synth.input_embeds(shape)[0]
+        self.cfg1 = odec.Config(shape.hidden, 1, shape.n_q, shape.n_kv, shape.head_dim,
+                                shape.inter, shape.vocab, shape.eps, shape.theta)
+        self.i = 0
+
+    def run(self):
+        """One sample; returns the scaled step time in seconds."""
+        from oracle import decoder as odec
+
+        li = self.i % len(self.layers)
+        self.i += 1
+        W1 = {"layers": [self.layers[li]]}
+        t0 = time.perf_counter()
+        r = odec.decoder_step(self.cfg1, dict(W1, lm_head=self.lm_slice,
+                                              final_norm=self.final_norm, embed=None),
+                              self.emb, self.P, [self.kp[li]], [self.vp[li]])
+        dt = time.perf_counter() - t0
+        assert np.isfinite(r["logits"]).all()
+        return dt * self.shape.layers
+
+    def describe(self, n):
+        return (f"oracle: {n} samples of one decoder layer (dequantised in the call) + 1/"
+                f"{self.shape.layers} of the lm_head rows at P={self.P}; step time = "
+                f"{self.shape.layers} x median sample")
+
+
+def oracle_sample_time(shape, mode, P, samples=8):
+    o = OracleSample(shape, mode, P)
+    ts = [o.run() for _ in range(samples)]
+    return statistics.median(ts), o.describe(samples), blas_threads()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------ ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from int4_blockwise_quantised_b200 import _vv
+    from int4_blockwise_quantised_b200.model import Decoder, PackedModel
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        import datetime
+
+        dist = dist_mod
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    shape, mode, P, seq, desc = CONFIGS[args.config]
+    std = std_for(shape)
+    vmode = _vv.VV_TERNARY if mode == "ternary" else _vv.VV_SYM_INT4
+    t0 = time.time()
+    model = PackedModel(shape, vmode, lambda li, m: synth.master(shape, m, li, std),
+                        lambda li: synth.layer_vectors(shape, li), synth.model_tables(shape),
+                        "cuda")
+    setup_s = time.time() - t0
+    cap = P + max(seq, 64) + 8
+    dec = Decoder(model, cap)
+    kp, vp = synth.past_kv(shape, P)
+    dec.k_cache[:, 0, :, :P] = torch.from_numpy(kp).cuda()
+    dec.v_cache[:, 0, :, :P] = torch.from_numpy(vp).cuda()
+    del kp, vp
+    dec.set_length(P)
+    stream = torch.cuda.current_stream()
+
+    # Device-resident inputs for the device-timed value: token ids fed back greedily.
+    tok = torch.tensor([151643 % shape.vocab], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([P], dtype=torch.int32, device="cuda")
+    logits = torch.empty(shape.vocab, dtype=torch.float32, device="cuda")
+
+    def one_step(i):
+        # i = index within the sequence; position = P + i; greedy token fed back on device.
+        if i == 0:
+            dec.set_length(P)
+            pos.fill_(P)
+        dec.step(pos, token=tok, logits=logits, argmax=tok)
+        pos.add_(1)
+
+    n_launch = dec.step_launches
+    # warm-up (also captures the graph)
+    for i in range(args.warmup):
+        one_step(i % seq)
+    dec.sync_status()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    extra = 0
+    for i in range(args.steps):
+        if i % seq == 0:
+            extra += 3  # set_length kernel + pos fill + (pos add counted below)
+        one_step(i % seq)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    dec.sync_status()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    tok_s = world * args.steps / (ms / 1e3)
+    gpu_launches = args.steps * (n_launch + 1) + extra  # + the position increment per step
+
+    # ---------------------------------------------------------------- e2e (host buffers)
+    emb_host = torch.from_numpy(synth.input_embeds(shape, 1)[0]).pin_memory()
+    pos_host = torch.tensor([P], dtype=torch.int32).pin_memory()
+    out_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    emb_dev = torch.empty(shape.hidden, dtype=torch.float16, device="cuda")
+    pos_dev = torch.empty(1, dtype=torch.int32, device="cuda")
+    am_dev = torch.empty(1, dtype=torch.int32, device="cuda")
+    e2e_steps = min(args.steps, 256)
+    for i in range(3):  # capture the e2e graph (different pointers) outside the timed region
+        dec.set_length(P)
+        emb_dev.copy_(emb_host, non_blocking=True)
+        pos_dev.copy_(pos_host, non_blocking=True)
+        dec.step(pos_dev, input_embeds=emb_dev, argmax=am_dev)
+        out_host.copy_(am_dev, non_blocking=True)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        if i % seq == 0:
+            dec.set_length(P)
+        pos_host[0] = P + (i % seq)
+        emb_dev.copy_(emb_host, non_blocking=True)
+        pos_dev.copy_(pos_host, non_blocking=True)
+        dec.step(pos_dev, input_embeds=emb_dev, argmax=am_dev)
+        out_host.copy_(am_dev, non_blocking=True)
+        stream.synchronize()  # the host reads the greedy token every step
+        _ = int(out_host[0])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_tok_s = world * e2e_steps / (e2e_ms / 1e3)
+
+    # ------------------------------------------------------- live per-kernel durations (profile)
+    prof_steps = 8
+    acc = {}
+    dec.set_length(P)
+    pos.fill_(P)
+    for i in range(prof_steps):
+        ph = dec.profile_step(pos, token=tok, logits=logits, argmax=tok)
+        pos.add_(1)
+        for k, v in ph.items():
+            acc[k] = acc.get(k, 0.0) + v / prof_steps
+    per_launch_ms = {k: (v if k == "lm_head" else v / shape.layers) for k, v in acc.items()}
+    pb = phase_bytes(shape, P + prof_steps // 2)
+    total_ms = {k: v for k, v in acc.items()}
+    dominant = max(total_ms, key=total_ms.get)
+    peak, peak_kind = peaks()
+    achieved = pb[dominant] / (per_launch_ms[dominant] * 1e-3) / 1e9
+    traffic = traffic_for(dominant)
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": pb[dominant],
+                "avg_launch_us": round(per_launch_ms[dominant] * 1e3, 2),
+                "phase_share": {k: round(v / sum(total_ms.values()), 4) for k, v in total_ms.items()}}
+
+    sb = step_bytes(shape, P + seq // 2)
+    result = {
+        "metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.config, "description": desc, "batch": 1, "past_P": P,
+                   "steps_per_sequence": seq, "weights": f"{mode} block-32",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (weights %.0f MB, L2 126 MB); no flush" % (
+                       sb / 1e6)},
+        "step_us": round(ms_per_step * 1e3, 2),
+        "hbm_gbs": round(sb / (ms_per_step * 1e-3) / 1e9, 1),
+        "hbm_frac_of_measured": round(sb / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "hbm_frac_of_8tbs": round(sb / (ms_per_step * 1e-3) / 8e12, 4),
+        "algorithmic_bytes_per_step": sb,
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_tok_s, 2), "unit": "tok/s",
+                "h2d_bytes_per_step": shape.hidden * 2 + 4, "d2h_bytes_per_step": 4,
+                "steps": e2e_steps,
+                "note": "public API: pinned host input_embeds + position -> device copy, graph step, "
+                        "argmax device->host read and stream sync every step"},
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+        "setup_s": round(setup_s, 1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        st, sample, thr = oracle_sample_time(shape, mode, P)
+        result["cpu_baseline"] = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr,
+                                  "kind": "oracle", "sample": sample}
+    dec.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernel's source
+    changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
+    return d["dram_bytes_per_launch"] if h == d.get("source_sha") else None
+
+
+# ------------------------------------------------------------------------------ reference arm
+def run_reference(args, rank):
+    """The oracle as the reference arm: every step is one bounded oracle sample (one layer +
+    1/L of the lm_head, scaled by L), on this arm's config, metric and unit."""
+    if rank != 0:
+        return
+    shape, mode, P, seq, desc = CONFIGS[args.config]
+    o = OracleSample(shape, mode, P)
+    for _ in range(args.warmup):
+        o.run()
+    t0 = time.perf_counter()
+    est = [o.run() for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    st = statistics.median(est)
+    value = 1.0 / st
+    result = {
+        "metric": METRIC, "value": round(value, 4), "unit": "tok/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(st * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.config, "description": desc, "batch": 1, "past_P": P},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tok/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": o.describe(args.steps)},
+        "e2e": {"value": round(value, 4), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 2),
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--config", default="decode-1p5b", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

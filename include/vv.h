@@ -1,0 +1,259 @@
+/*
+ * libvv — int4 blockwise-quantised Qwen2 decoder step on NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only.  "device" pointers are CUDA global-memory addresses on
+ * the current device; "host" pointers are ordinary CPU memory.  Half-precision values are passed
+ * as uint16_t bit patterns (IEEE binary16).  A stream argument is a cudaStream_t passed as
+ * void* (NULL = the legacy default stream).  Calls are asynchronous on that stream unless
+ * stated otherwise.
+ *
+ * Ownership: the caller allocates and owns every input, output, weight and KV-cache buffer;
+ * libvv borrows them for the duration of a call (or, for vv_decoder_create, for the decoder's
+ * lifetime) and never frees them.  libvv owns only the workspace a decoder allocates in
+ * vv_decoder_create and frees in vv_decoder_destroy.
+ *
+ * Errors: every call returns vv_status (VV_OK = 0).  No exception crosses the ABI.
+ * vv_last_error() returns the text of the calling thread's most recent error.  Errors found on
+ * the device (a wait that timed out, a token id out of range) are recorded in a device error
+ * word and reported by vv_sync_status() / vv_decoder_sync_status().
+ *
+ * Sources of the operations (web pages on the VibeVoice ONNX exports):
+ *   [BITNET]  "vibevoice-asr-bitnet-onnx" model page (Masterx): ternarisation formula,
+ *             MatMulNBits packing paragraph, tier table, decoder_init / decoder_step I/O listing.
+ *   [STATUS]  "VibeVoice-1.5B — Current Status" (Prince-1/VibeVoice-1.5B-Onnx): sections
+ *             "Architecture", "Done" (140 MatMulNBits + 28 GroupQueryAttention, int4 ModelBuilder
+ *             build) and "Inference (ONNX)" (KV-incremental decode loop, tied lm_head).
+ *   [ASR]     "VibeVoice-ASR — ONNX export for Vernacula": section "Highlights" (GPU-resident KV
+ *             cache, 1950 launches per step of framework overhead).
+ */
+#ifndef VV_H_
+#define VV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t vv_status;
+
+#define VV_OK 0
+#define VV_ERR_INVALID_ARG 1 /* null / misaligned pointer, bad enum value */
+#define VV_ERR_SHAPE 2       /* inconsistent or unsupported sizes */
+#define VV_ERR_CAPACITY 3    /* KV cache or workspace too small */
+#define VV_ERR_RANGE 4       /* index out of range (audio splice, position, token id) */
+#define VV_ERR_CUDA 5        /* a CUDA runtime call failed; text in vv_last_error */
+#define VV_ERR_TIMEOUT 6     /* a bounded device-side wait expired */
+
+/* Quantisation modes of vv_pack_nbits. */
+#define VV_SYM_INT4 0 /* scale = max|w_block| / 7 */
+#define VV_TERNARY 1  /* BitNet ternary with a per-tensor scale s */
+
+typedef void* vv_stream; /* cudaStream_t */
+
+/* Library version string (static storage). */
+const char* vv_version(void);
+
+/* Copy the calling thread's last error text into buf (NUL-terminated, truncated to n).
+ * Returns the last error code. */
+vv_status vv_last_error(char* buf, size_t n);
+
+/* Synchronise `stream` and return (and clear) the device error word of the current device. */
+vv_status vv_sync_status(vv_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Packing ([BITNET] ternarisation and MatMulNBits paragraphs; [STATUS] "Done": int4 build).
+ *
+ * Layout produced (the public ONNX Runtime MatMulNBits layout, bits = 4, block = 32):
+ *   q_out      device uint8  [N, KB, 16], KB = ceil(K / 32).  Block b of row n holds columns
+ *              32b .. 32b+31; byte j holds column 32b+2j in its low nibble and 32b+2j+1 in its
+ *              high nibble.  Stored code = round(w / scale) + 8 (implicit zero point 8).
+ *   scales_out device fp16   [N, KB].
+ * Dequantised weight = (code - 8) * scale.  Columns past K are padded with code 8.
+ */
+
+/* Per-tensor ternary scale s = 1 / mean(|W|) ([BITNET] ternarisation formula).
+ * w: device fp32 [count].  s_out: HOST float.  mean is the correctly rounded float64 sum of
+ * |w| divided by count (float64), s = float32(1.0 / mean); a zero tensor gives s = +inf.
+ * Synchronous: returns after the value is on the host.  count in [1, 2^40). */
+vv_status vv_ternary_scale(const float* w, int64_t count, float* s_out, vv_stream stream);
+
+/* Quantise and pack W [N, K] (device fp32, row-major).
+ *   mode VV_TERNARY:  code = round(clamp(float32(w * s), -1, 1)) + 8 in {7, 8, 9};
+ *                     every block's scale = fp16(float32(1 / s)); s = ternary_s (from
+ *                     vv_ternary_scale); s not finite or <= 0 -> all codes 8, scale 0.
+ *   mode VV_SYM_INT4: scale = fp16(float32(max|w_block|) / 7);
+ *                     code = clamp(round(float32(w / scale)), -8, 7) + 8; zero scale -> codes 8.
+ * round() is half away from zero; all arithmetic is IEEE float32 without contraction, so the
+ * result is bit-reproducible.  block must be 32.  Inputs must be finite.
+ * Errors: VV_ERR_INVALID_ARG (null, mode), VV_ERR_SHAPE (N, K < 1, block != 32). */
+vv_status vv_pack_nbits(const float* w, int64_t N, int64_t K, int32_t block, int32_t mode,
+                        float ternary_s, uint8_t* q_out, uint16_t* scales_out,
+                        vv_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * MatMulNBits ([STATUS] "Done": com.microsoft::MatMulNBits, 5 per layer).
+ *   y[m, n] = sum_k x[m, k] * (code[n, k] - 8) * scale[n, k / 32]  (+ bias[n])
+ * x device fp16 [M, K]; q/scales as produced by vv_pack_nbits for [N, K]; bias device fp16 [N]
+ * or NULL; y device fp16 [M, N].  Products and sums in fp32, one rounding to fp16 at the end.
+ * 1 <= M <= 8 runs the dequant-fused GEMV (each weight byte read once for all M rows).
+ * Requirements: K % 32 == 0, block == 32, all pointers 16-byte aligned.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (K % 32, M outside [1, 8], N < 1). */
+vv_status vv_matmul_nbits(const uint16_t* x, const uint8_t* q, const uint16_t* scales,
+                          const uint16_t* bias, int64_t M, int64_t N, int64_t K, int32_t block,
+                          uint16_t* y, vv_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Grouped-query decode attention ([STATUS] "Done": com.microsoft::GroupQueryAttention, one per
+ * layer; [BITNET] decoder_step: past keys/values [L, 1, Hkv, P, D]).
+ *   out[h, :] = softmax(scale * q[h, :] . K[g, t, :] for t < len) . V[g, :, :],  g = h / (Hq/Hkv)
+ * q device fp16 [Hq, D] (already rotated); k_cache / v_cache device fp16 [Hkv, cap, D]
+ * (positions 0..len-1 valid, stride cap); out device fp16 [Hq, D].  All positions < len are
+ * visible (decoder_step has no mask input).  Softmax and accumulation in fp32.
+ * ws: device workspace of at least vv_gqa_decode_attn_workspace_size(Hq, Hkv, D, cap) bytes,
+ * zero-filled once before its first use; every call leaves its counters at zero again.  Calls
+ * sharing one ws must not overlap on the GPU.
+ * Requirements: D == 128, 1 <= Hkv <= 64, Hq % Hkv == 0, Hq / Hkv <= 8, 1 <= len <= cap.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CAPACITY (ws too small). */
+size_t vv_gqa_decode_attn_workspace_size(int32_t Hq, int32_t Hkv, int32_t D, int32_t cap);
+vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                             int32_t len, int32_t cap, int32_t Hq, int32_t Hkv, int32_t D,
+                             float scale, uint16_t* out, void* ws, size_t ws_bytes,
+                             vv_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Final RMSNorm + fp16 lm_head + greedy argmax ([BITNET]: lm_head stays fp16, greedy decode;
+ * [STATUS] "Inference (ONNX)": logits = hidden . embed^T with the tied table).
+ *   xn = x / sqrt(mean(x^2) + eps) * gamma;  logits[v] = sum_h w_lm[v, h] * xn[h]  (fp32)
+ *   idx = argmax_v logits[v], lowest index on ties.
+ * x device fp32 [H] (the residual before the final norm); gamma device fp16 [H]; w_lm device
+ * fp16 [V, H]; logits device fp32 [V] or NULL; idx device int32 [1].
+ * ws: device workspace of vv_lm_head_argmax_workspace_size(V) bytes, zero-filled once before
+ * its first use (left zeroed by every call).  Requirements: H % 256 == 0, H <= 16384.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CAPACITY. */
+size_t vv_lm_head_argmax_workspace_size(int64_t V);
+vv_status vv_lm_head_argmax(const float* x, const uint16_t* gamma, const uint16_t* w_lm,
+                            int64_t V, int64_t H, float eps, float* logits, int32_t* idx,
+                            void* ws, size_t ws_bytes, vv_stream stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Decoder ([BITNET] decoder_init / decoder_step contracts; [ASR] "Highlights": KV cache kept
+ * resident on the GPU, step replayed as one CUDA graph instead of ~1950 launches).
+ *
+ * The KV cache is the caller's: k_cache and v_cache are device fp16 [L, 1, Hkv, cap, D] each.
+ * "past K/V in, present K/V out" happens in place: after a call, positions 0..length-1 of the
+ * cache are the present keys/values (viewed [L, 1, Hkv, length, D] with stride cap).
+ * Keys are stored after RoPE.
+ */
+typedef struct vv_config {
+  int32_t hidden;      /* H  (1536 for the 1.5B backbone, 3584 for 7B) */
+  int32_t layers;      /* L  (28) */
+  int32_t n_q;         /* query heads  (12 / 28) */
+  int32_t n_kv;        /* key-value heads (2 / 4) */
+  int32_t head_dim;    /* D  (128; the only supported value) */
+  int32_t inter;       /* SwiGLU intermediate (8960 / 18944) */
+  int32_t vocab;       /* V  (151936 / 152064) */
+  float eps;           /* RMSNorm epsilon (1e-6) */
+  float rope_theta;    /* RoPE base (1e6) */
+  int32_t kv_capacity; /* cap: slots per layer and head in the caller's cache */
+  int32_t max_position;/* RoPE table length: position ids must lie in [0, max_position) */
+  int32_t max_prefill; /* largest S accepted by vv_decoder_init (0 = no prefill workspace) */
+} vv_config;
+
+typedef struct vv_packed_matrix {
+  const uint8_t* q;       /* device uint8 [N, K/32, 16] */
+  const uint16_t* scales; /* device fp16 [N, K/32] */
+} vv_packed_matrix;
+
+typedef struct vv_layer_weights {
+  const uint16_t* input_norm; /* fp16 [H]   RMSNorm before attention */
+  const uint16_t* post_norm;  /* fp16 [H]   RMSNorm before the MLP */
+  vv_packed_matrix wq;        /* [Hq*D, H] */
+  vv_packed_matrix wk;        /* [Hkv*D, H] */
+  vv_packed_matrix wv;        /* [Hkv*D, H] */
+  vv_packed_matrix wo;        /* [H, Hq*D] */
+  vv_packed_matrix wgate;     /* [I, H] */
+  vv_packed_matrix wup;       /* [I, H] */
+  vv_packed_matrix wdown;     /* [H, I] */
+  const uint16_t* bq;         /* fp16 [Hq*D]  (q/k/v carry biases in Qwen2) */
+  const uint16_t* bk;         /* fp16 [Hkv*D] */
+  const uint16_t* bv;         /* fp16 [Hkv*D] */
+} vv_layer_weights;
+
+typedef struct vv_model_weights {
+  const uint16_t* embed;          /* device fp16 [V, H] token embedding table */
+  const uint16_t* lm_head;        /* device fp16 [V, H]; equal to embed when tied */
+  const uint16_t* final_norm;     /* device fp16 [H] */
+  const vv_layer_weights* layers; /* HOST array of L entries, copied by vv_decoder_create */
+} vv_model_weights;
+
+typedef struct vv_decoder vv_decoder;
+
+/* Create a decoder on the current device.  All weight pointers are borrowed for the decoder's
+ * lifetime; k_cache/v_cache likewise.  Allocates the decoder's workspace.  Length starts at 0.
+ * Requirements: head_dim == 128, n_kv <= 64, n_q % n_kv == 0, n_q/n_kv <= 8, hidden and inter multiples of
+ * 256, 1 <= kv_capacity, 1 <= max_position.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CUDA (allocation). */
+vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* weights,
+                            uint16_t* k_cache, uint16_t* v_cache, vv_decoder** out);
+vv_status vv_decoder_destroy(vv_decoder* dec);
+
+/* Set the number of valid cache positions (rewind / reset / adopt a cache filled elsewhere).
+ * Enqueued on `stream`.  Errors: VV_ERR_CAPACITY if len > kv_capacity, VV_ERR_RANGE if < 0. */
+vv_status vv_decoder_set_length(vv_decoder* dec, int32_t len, vv_stream stream);
+int32_t vv_decoder_length(const vv_decoder* dec);
+
+/* One decode step at batch 1 (decoder_step).
+ *   input_embeds: device fp16 [H], or NULL to gather row *token_id of the embedding table
+ *   token_id:     device int32 [1] (used only when input_embeds is NULL)
+ *   position_id:  device int32 [1]; RoPE angle = position * theta^(-2i/D)
+ *   logits:       device fp32 [V] or NULL
+ *   argmax_out:   device int32 [1] or NULL (greedy token, lowest index on ties)
+ * Appends this position's K/V at slot `length` of every layer, then length += 1.  The first
+ * call with a given set of pointers captures the step as a CUDA graph; later calls replay it.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_CAPACITY (length == kv_capacity).  A position outside
+ * [0, max_position) or a token outside [0, V) is reported by vv_decoder_sync_status. */
+vv_status vv_decoder_step(vv_decoder* dec, const uint16_t* input_embeds, const int32_t* token_id,
+                          const int32_t* position_id, float* logits, int32_t* argmax_out,
+                          vv_stream stream);
+
+/* Prefill (decoder_init): embeds = embed[input_ids]; rows [audio_offset, audio_offset + N) are
+ * replaced by audio_features; causal attention over the S positions; writes present K/V at
+ * slots 0..S-1, sets length = S, and emits the last position's logits / argmax.
+ *   input_ids, position_ids: device int32 [S]; audio_features: device fp16 [N, H] or NULL (N=0)
+ * Errors: VV_ERR_RANGE (audio_offset + N > S, negative offset), VV_ERR_CAPACITY (S > cap or
+ * S > max_prefill), VV_ERR_INVALID_ARG. */
+vv_status vv_decoder_init(vv_decoder* dec, const int32_t* input_ids, const int32_t* position_ids,
+                          int64_t S, const uint16_t* audio_features, int64_t N,
+                          int64_t audio_offset, float* logits, int32_t* argmax_out,
+                          vv_stream stream);
+
+/* Debug tap: when layer_out (device fp32 [L, H]) is non-NULL, each later step writes the
+ * residual stream after every layer into it (init writes the last position's).  NULL turns it
+ * off.  Changing it re-captures the step graph. */
+vv_status vv_decoder_set_trace(vv_decoder* dec, float* layer_out);
+
+/* Turn CUDA-graph replay of the step on (default) or off (plain launches every call). */
+vv_status vv_decoder_set_graph(vv_decoder* dec, int32_t enable);
+
+/* Synchronise `stream` and return (and clear) the device error word. */
+vv_status vv_decoder_sync_status(vv_decoder* dec, vv_stream stream);
+
+/* Profiling tap: run one step with plain launches (no graph, no launch overlap) and CUDA events
+ * around every launch on `stream`; phase_ms (HOST float[6]) receives the device time summed over
+ * layers of [qkv, attention, o-proj, gate/up, down, lm_head].  Appends a position like
+ * vv_decoder_step.  Synchronous.  Errors as vv_decoder_step. */
+vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
+                                  const int32_t* token_id, const int32_t* position_id,
+                                  float* logits, int32_t* argmax_out, float* phase_ms,
+                                  vv_stream stream);
+
+/* Number of kernel launches one vv_decoder_step enqueues (for launch accounting). */
+int32_t vv_decoder_step_launches(const vv_decoder* dec);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VV_H_ */

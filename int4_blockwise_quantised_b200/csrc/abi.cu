@@ -1,0 +1,73 @@
+// Library-wide entry points: version, error text, device error word.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "vv_device.cuh"
+#include "vv_internal.h"
+
+namespace vv {
+
+__device__ int g_device_error = 0;
+
+namespace {
+thread_local vv_status t_last_code = VV_OK;
+thread_local char t_last_text[512] = "";
+}  // namespace
+
+vv_status set_error(vv_status code, const char* fmt, ...) {
+  t_last_code = code;
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_text, sizeof(t_last_text), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+vv_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return VV_OK;
+  return set_error(VV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+}  // namespace vv
+
+extern "C" {
+
+const char* vv_version(void) { return "libvv 0.1 (sm_100a)"; }
+
+vv_status vv_last_error(char* buf, size_t n) {
+  if (buf && n) {
+    strncpy(buf, vv::t_last_text, n - 1);
+    buf[n - 1] = '\0';
+  }
+  return vv::t_last_code;
+}
+
+vv_status vv_sync_status(vv_stream stream) {
+  VV_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int err = 0;
+  VV_CUDA(cudaMemcpyFromSymbol(&err, vv::g_device_error, sizeof(int)));
+  if (err != 0) {
+    const int zero = 0;
+    VV_CUDA(cudaMemcpyToSymbol(vv::g_device_error, &zero, sizeof(int)));
+    return vv::set_error(err, "device-side error %d recorded by a kernel", err);
+  }
+  return VV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,369 @@
+// Grouped-query decode attention over a GPU-resident fp16 KV cache
+// ("VibeVoice-1.5B — Current Status", section "Done": one GroupQueryAttention per layer;
+// "vibevoice-asr-bitnet-onnx": decoder_step past keys/values [L, 1, Hkv, P, D];
+// "VibeVoice-ASR — ONNX export for Vernacula", section "Highlights": the cache stays on the GPU).
+//
+//   out[h] = softmax(scale * q[h] . K[g, t]  for all t) . V[g],  g = h / (Hq / Hkv)
+//
+// Split-K ("flash decoding"): grid = (chunks, Hkv).  A CTA owns one KV head and a run of 64-
+// position tiles; one K/V tile load serves all G = Hq/Hkv query heads of the group.  Tiles move
+// global -> shared with cp.async.bulk (positions of one head are contiguous) into a double
+// buffer; softmax is online in fp32 in the log2 domain.  Each CTA writes (m, l, o) partials; the
+// last CTA of a head (arrival counter, no spinning) merges them and resets the counter.
+//
+// Fused decoder mode: the QKV GEMV left q/k/v pre-RoPE in fp32.  Every CTA rotates its group's
+// q (RoPE, table built on the host in float64); the CTA holding the last tile also rotates k,
+// rounds k and v to fp16, stores them at slot `length` of the cache and into its own tile.
+// Past tiles are prefetched before griddepcontrol.wait: they were written by kernels at least
+// one whole step (and a non-overlapped kernel boundary) earlier.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "vv_device.cuh"
+#include "vv_internal.h"
+
+namespace vv {
+namespace {
+
+constexpr int D = 128;
+constexpr int TT = 64;  // positions per tile
+constexpr int kThreads = 256;
+constexpr int kMaxG = 8;
+constexpr int kPartStride = 132;  // floats per (chunk, head) partial: m, l, pad, pad, o[128]
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnSmem {
+  __half k[2][TT * D];
+  __half v[2][TT * D];
+  float q[kMaxG][D];
+  float s[kMaxG][TT];
+  float m[kMaxG], l[kMaxG], corr[kMaxG];
+  float mw[kMaxG];  // merge weights scratch
+  uint64_t bar[2];
+  int is_last;
+};
+
+template <bool FUSED>
+__global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
+  const int c = blockIdx.x, g = blockIdx.y, nchunks = gridDim.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv;
+
+  // Past positions: standalone len, fused *length (stable: set a whole step earlier).
+  const int past = FUSED ? *a.length : a.len;
+  const int npos = FUSED ? past + 1 : past;
+  const int ntiles = (npos + TT - 1) / TT;
+  const int tpc = (ntiles + nchunks - 1) / nchunks;
+  const int t_begin = c * tpc;
+  const int t_end = min(t_begin + tpc, ntiles);
+  const int active = (ntiles + tpc - 1) / tpc;  // chunks that own at least one tile
+
+  pdl_launch_dependents();
+  if (t_begin >= t_end) {  // no work; not counted in `active`
+    pdl_wait();
+    return;
+  }
+
+  const __half* kc = reinterpret_cast<const __half*>(a.k_cache) + (size_t)g * a.cap * D;
+  const __half* vc = reinterpret_cast<const __half*>(a.v_cache) + (size_t)g * a.cap * D;
+
+  if (tid == 0) {
+    mbar_init(&sm.bar[0], 1);
+    mbar_init(&sm.bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // Issue the bulk load of tile t into buffer b: rows [t*TT, min(t*TT+TT, past)) from the cache.
+  auto issue = [&](int t, int b) {
+    const int p0 = t * TT;
+    const int p1 = min(p0 + TT, past);
+    const uint32_t bytes = p1 > p0 ? (uint32_t)(p1 - p0) * D * 2 : 0u;
+    mbar_arrive_expect_tx(&sm.bar[b], 2 * bytes);
+    if (bytes) {
+      bulk_g2s(sm.k[b], kc + (size_t)p0 * D, bytes, &sm.bar[b]);
+      bulk_g2s(sm.v[b], vc + (size_t)p0 * D, bytes, &sm.bar[b]);
+    }
+  };
+  if (tid == 0) {
+    issue(t_begin, 0);
+    if (t_begin + 1 < t_end) issue(t_begin + 1, 1);
+  }
+
+  pdl_wait();
+
+  // ---- q of the group (rotated, scaled into the log2 domain) and, fused, the new k/v.
+  int pos = 0;
+  if (FUSED) {
+    pos = *a.position;
+    if (pos < 0 || pos >= a.max_position) {
+      if (tid == 0) set_device_error(VV_ERR_RANGE);
+      pos = min(max(pos, 0), a.max_position - 1);
+    }
+  }
+  const float qscale = a.scale * kLog2e;
+  for (int i = tid; i < G * D; i += kThreads) {
+    const int h = i / D, d = i % D;
+    float qv;
+    if (FUSED) {
+      const float* qh = a.qkv + (size_t)(g * G + h) * D;
+      const int fi = d & (D / 2 - 1);
+      const float cs = a.rope_cos[(size_t)pos * (D / 2) + fi];
+      const float sn = a.rope_sin[(size_t)pos * (D / 2) + fi];
+      const float x1 = __ldcg(qh + fi), x2 = __ldcg(qh + fi + D / 2);
+      qv = d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+    } else {
+      qv = __half2float(reinterpret_cast<const __half*>(a.q_f16)[(size_t)(g * G + h) * D + d]);
+    }
+    sm.q[h][d] = qv * qscale;
+  }
+  // The CTA owning the last tile rotates the new key, rounds k/v to fp16 and stores them at
+  // slot `past`; the row enters shared memory when that tile is processed (the bulk copies of
+  // every tile cover only rows < past, and an earlier tile may still occupy the buffer).
+  const bool owns_new = FUSED && (t_end == ntiles);
+  __half my_kn = __float2half_rn(0.f), my_vn = __float2half_rn(0.f);
+  if (owns_new && tid < D) {
+    const int d = tid;
+    const float* kh = a.qkv + (size_t)(a.Hq + g) * D;
+    const float* vh = a.qkv + (size_t)(a.Hq + a.Hkv + g) * D;
+    const int fi = d & (D / 2 - 1);
+    const float cs = a.rope_cos[(size_t)pos * (D / 2) + fi];
+    const float sn = a.rope_sin[(size_t)pos * (D / 2) + fi];
+    const float x1 = __ldcg(kh + fi), x2 = __ldcg(kh + fi + D / 2);
+    my_kn = __float2half_rn(d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn);
+    my_vn = __float2half_rn(__ldcg(vh + d));
+    a.k_cache[((size_t)g * a.cap + past) * D + d] = __half_as_ushort(my_kn);
+    a.v_cache[((size_t)g * a.cap + past) * D + d] = __half_as_ushort(my_vn);
+  }
+  if (tid < kMaxG) {
+    sm.m[tid] = -INFINITY;
+    sm.l[tid] = 0.f;
+  }
+  __syncthreads();
+
+  // Output ownership: thread -> dim d = tid % 128, heads hh, hh+2, hh+4, hh+6 (hh = tid / 128).
+  const int od = tid & (D - 1), hh = tid >> 7;
+  float o[kMaxG / 2];
+#pragma unroll
+  for (int j = 0; j < kMaxG / 2; ++j) o[j] = 0.f;
+
+  // q fragment per lane for the score phase: dims 4*lane .. 4*lane+3 of every head.
+  float4 qf[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h)
+    qf[h] = h < G ? *reinterpret_cast<const float4*>(&sm.q[h][4 * lane]) : make_float4(0, 0, 0, 0);
+
+  for (int t = t_begin; t < t_end; ++t) {
+    const int b = (t - t_begin) & 1;
+    mbar_wait(&sm.bar[b], ((t - t_begin) >> 1) & 1);
+    const int p0 = t * TT;
+    const int n = min(TT, npos - p0);
+    if (owns_new && t == ntiles - 1) {
+      if (tid < D) {
+        sm.k[b][(past - p0) * D + tid] = my_kn;
+        sm.v[b][(past - p0) * D + tid] = my_vn;
+      }
+      __syncthreads();
+    }
+
+    // scores: warp w -> positions w, w+8, ...
+    for (int p = warp; p < n; p += kThreads / 32) {
+      const uint2 kr = *reinterpret_cast<const uint2*>(&sm.k[b][p * D + 4 * lane]);
+      const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kr.x));
+      const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kr.y));
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < G) {
+          float sdot = qf[h].x * k01.x + qf[h].y * k01.y + qf[h].z * k23.x + qf[h].w * k23.y;
+          sdot = warp_sum(sdot);
+          if (lane == 0) sm.s[h][p] = sdot;
+        }
+      }
+    }
+    __syncthreads();
+    // online softmax per head: warp h
+    if (warp < G) {
+      const int h = warp;
+      const float s0 = lane < n ? sm.s[h][lane] : -INFINITY;
+      const float s1 = lane + 32 < n ? sm.s[h][lane + 32] : -INFINITY;
+      const float mt = warp_max(fmaxf(s0, s1));
+      const float mo = sm.m[h];
+      const float mn = fmaxf(mo, mt);
+      const float e0 = lane < n ? exp2f(s0 - mn) : 0.f;
+      const float e1 = lane + 32 < n ? exp2f(s1 - mn) : 0.f;
+      sm.s[h][lane] = e0;
+      sm.s[h][lane + 32] = e1;
+      const float sum = warp_sum(e0 + e1);
+      if (lane == 0) {
+        const float cr = exp2f(mo - mn);  // mo = -inf on the first tile -> 0
+        sm.corr[h] = cr;
+        sm.l[h] = sm.l[h] * cr + sum;
+        sm.m[h] = mn;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kMaxG / 2; ++j) {
+      const int h = hh + 2 * j;
+      if (h < G) o[j] *= sm.corr[h];
+    }
+    for (int p = 0; p < n; ++p) {
+      const float vv = __half2float(sm.v[b][p * D + od]);
+#pragma unroll
+      for (int j = 0; j < kMaxG / 2; ++j) {
+        const int h = hh + 2 * j;
+        if (h < G) o[j] = fmaf(sm.s[h][p], vv, o[j]);
+      }
+    }
+    __syncthreads();  // buffer b and the score rows are free again
+    if (tid == 0 && t + 2 < t_end) issue(t + 2, b);
+  }
+
+  if (active == 1) {
+#pragma unroll
+    for (int j = 0; j < kMaxG / 2; ++j) {
+      const int h = hh + 2 * j;
+      if (h < G) {
+        const float r = o[j] / sm.l[h];
+        const size_t idx = (size_t)(g * G + h) * D + od;
+        if (FUSED) a.out_f32[idx] = r;
+        else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(r);
+      }
+    }
+    return;
+  }
+
+  // ---- partials, then the last CTA of this head merges.
+  float* part = a.ws_part + ((size_t)g * nchunks + c) * kMaxG * kPartStride;
+#pragma unroll
+  for (int j = 0; j < kMaxG / 2; ++j) {
+    const int h = hh + 2 * j;
+    if (h < G) part[h * kPartStride + 4 + od] = o[j];
+  }
+  if (tid < G) {
+    part[tid * kPartStride + 0] = sm.m[tid];
+    part[tid * kPartStride + 1] = sm.l[tid];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(&a.ws_count[g], 1);
+    sm.is_last = (prev == active - 1);
+  }
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+
+  const float* base = a.ws_part + (size_t)g * nchunks * kMaxG * kPartStride;
+  // per head: M = max m_c, L = sum l_c 2^(m_c - M)
+  if (warp < G) {
+    const int h = warp;
+    float mx = -INFINITY;
+    for (int cc = lane; cc < active; cc += 32) mx = fmaxf(mx, __ldcg(base + ((size_t)cc * kMaxG + h) * kPartStride));
+    mx = warp_max(mx);
+    float L = 0.f;
+    for (int cc = lane; cc < active; cc += 32) {
+      const float* pp = base + ((size_t)cc * kMaxG + h) * kPartStride;
+      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - mx);
+    }
+    L = warp_sum(L);
+    if (lane == 0) {
+      sm.m[h] = mx;
+      sm.l[h] = L;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kMaxG / 2; ++j) {
+    const int h = hh + 2 * j;
+    if (h < G) {
+      float acc = 0.f;
+      const float mx = sm.m[h];
+      for (int cc = 0; cc < active; ++cc) {
+        const float* pp = base + ((size_t)cc * kMaxG + h) * kPartStride;
+        acc = fmaf(__ldcg(pp + 4 + od), exp2f(__ldcg(pp) - mx), acc);
+      }
+      const float r = acc / sm.l[h];
+      const size_t idx = (size_t)(g * G + h) * D + od;
+      if (FUSED) a.out_f32[idx] = r;
+      else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(r);
+    }
+  }
+  if (tid == 0) a.ws_count[g] = 0;
+}
+
+}  // namespace
+
+int attn_default_chunks(int Hkv, int cap) {
+  const int tiles = (cap + TT - 1) / TT;
+  int per_head = sm_count() / (Hkv > 0 ? Hkv : 1);
+  if (per_head < 1) per_head = 1;
+  return tiles < per_head ? (tiles > 0 ? tiles : 1) : per_head;
+}
+
+size_t attn_workspace_bytes(int Hq, int Hkv, int nchunks) {
+  (void)Hq;
+  return (size_t)Hkv * nchunks * kMaxG * kPartStride * sizeof(float) + 256;
+}
+
+cudaError_t launch_attn(const AttnArgs& a, bool fused, cudaStream_t s, bool pdl) {
+  const size_t smem = sizeof(AttnSmem);
+  dim3 grid(a.nchunks, a.Hkv);
+  if (fused) {
+    auto k = attn_decode_kernel<true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch(k, grid, dim3(kThreads), smem, s, pdl, a);
+  }
+  auto k = attn_decode_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch(k, grid, dim3(kThreads), smem, s, pdl, a);
+}
+
+}  // namespace vv
+
+extern "C" size_t vv_gqa_decode_attn_workspace_size(int32_t Hq, int32_t Hkv, int32_t D_,
+                                                    int32_t cap) {
+  if (Hkv <= 0 || cap <= 0 || D_ != 128) return 0;
+  const int nch = vv::attn_default_chunks(Hkv, cap);
+  return vv::attn_workspace_bytes(Hq, Hkv, nch);
+}
+
+extern "C" vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cache,
+                                        const uint16_t* v_cache, int32_t len, int32_t cap,
+                                        int32_t Hq, int32_t Hkv, int32_t D_, float scale,
+                                        uint16_t* out, void* ws, size_t ws_bytes,
+                                        vv_stream stream) {
+  VV_CHECK_ARG(q && k_cache && v_cache && out && ws, "vv_gqa_decode_attn: null pointer");
+  VV_CHECK_ARG(vv::aligned16(q) && vv::aligned16(k_cache) && vv::aligned16(v_cache) &&
+                   vv::aligned16(out) && vv::aligned16(ws),
+               "vv_gqa_decode_attn: pointers must be 16-byte aligned");
+  VV_CHECK_SHAPE(D_ == 128, "vv_gqa_decode_attn: D=%d (only 128)", D_);
+  VV_CHECK_SHAPE(Hkv >= 1 && Hkv <= 64 && Hq >= Hkv && Hq % Hkv == 0 && Hq / Hkv <= 8,
+                 "vv_gqa_decode_attn: Hq=%d Hkv=%d", Hq, Hkv);
+  VV_CHECK_SHAPE(cap >= 1 && len >= 1 && len <= cap, "vv_gqa_decode_attn: len=%d cap=%d", len,
+                 cap);
+  const int nch = vv::attn_default_chunks(Hkv, cap);
+  const size_t need = vv::attn_workspace_bytes(Hq, Hkv, nch);
+  if (ws_bytes < need)
+    return vv::set_error(VV_ERR_CAPACITY, "vv_gqa_decode_attn: workspace %zu < %zu", ws_bytes,
+                         need);
+  vv::AttnArgs a = {};
+  a.q_f16 = q;
+  a.k_cache = const_cast<uint16_t*>(k_cache);
+  a.v_cache = const_cast<uint16_t*>(v_cache);
+  a.len = len;
+  a.cap = cap;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.scale = scale;
+  a.out_f16 = out;
+  a.ws_part = static_cast<float*>(ws);
+  a.ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + need - 256);
+  a.nchunks = nch;
+  return vv::cuda_check(vv::launch_attn(a, false, static_cast<cudaStream_t>(stream), false),
+                        "attention launch");
+}

@@ -1,0 +1,419 @@
+// The decoder object: decoder_step / decoder_init of the Qwen2 backbone
+// ("vibevoice-asr-bitnet-onnx": decoder_init / decoder_step I/O listing; "VibeVoice-1.5B —
+// Current Status", section "Architecture": pre-norm Qwen2 with q/k/v bias, GQA).
+//
+// Step = 5 kernels per layer + 1:
+//   qkv   : RMSNorm(x) -> [Wq;Wk;Wv] int4 GEMV + bias (layer 0 reads the embedding row)
+//   attn  : RoPE(q,k) at position, append k/v at slot `length`, split-K GQA attention
+//   o     : x += Wo . attn
+//   gateup: RMSNorm(x) -> gate/up int4 GEMV -> silu(g) * u
+//   down  : x += Wd . h
+//   head  : RMSNorm(x) -> fp16 lm_head GEMV -> logits, argmax; length += 1
+// The residual x stays fp32 in the workspace.  Position and length live in device memory, so the
+// whole step is captured once as a CUDA graph and replayed ("VibeVoice-ASR — ONNX export for
+// Vernacula", section "Highlights": ~1950 launches per step of framework overhead under ONNX
+// Runtime).  Every kernel after the first is launched with programmatic dependent launch so its
+// weight prefetch overlaps the previous kernel.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "vv_device.cuh"
+#include "vv_internal.h"
+#include "decoder_state.h"
+
+namespace vv {
+
+__global__ void set_int_kernel(int32_t* p, int32_t v) { *p = v; }
+__global__ void add_int_kernel(int32_t* p, int32_t v) { *p += v; }
+
+namespace {
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+}  // namespace
+
+cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
+                         const int32_t* position, float* logits, int32_t* argmax,
+                         cudaStream_t s, bool head, cudaEvent_t* ev) {
+  // ev (profiling): 2 events per launch, recorded around each kernel; PDL off so the events
+  // bracket exactly one kernel.
+  const bool pdl = ev == nullptr;
+  int evi = 0;
+  auto mark = [&]() {
+    if (ev) cudaEventRecord(ev[evi++], s);
+  };
+  const vv_config& c = d->cfg;
+  const int H = c.hidden, D = c.head_dim, Hq = c.n_q, Hkv = c.n_kv, I = c.inter;
+  const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
+  cudaError_t e;
+  for (int l = 0; l < c.layers; ++l) {
+    const vv_layer_weights& w = d->layers[l];
+    QkvArgs qa = {};
+    qa.w[0] = GemvWeights{w.wq.q, w.wq.scales};
+    qa.w[1] = GemvWeights{w.wk.q, w.wk.scales};
+    qa.w[2] = GemvWeights{w.wv.q, w.wv.scales};
+    qa.rows[0] = Hq * D;
+    qa.rows[1] = Hkv * D;
+    qa.rows[2] = Hkv * D;
+    qa.bias[0] = w.bq;
+    qa.bias[1] = w.bk;
+    qa.bias[2] = w.bv;
+    qa.K = H;
+    qa.x_resid_in = d->x_resid;
+    if (l == 0) {
+      qa.embeds = embeds;
+      qa.embed_table = embeds ? nullptr : d->embed;
+      qa.token = token;
+      qa.vocab = c.vocab;
+      qa.x_resid_out = d->x_resid;
+    }
+    qa.gamma = w.input_norm;
+    qa.eps = c.eps;
+    qa.out = d->qkv;
+    // The first kernel of a step is not overlapped with the previous step (it reads the
+    // caller's inputs and the length written by the previous step's last kernel).
+    mark();
+    if ((e = launch_qkv(qa, s, pdl && l > 0)) != cudaSuccess) return e;
+    mark();
+
+    AttnArgs aa = {};
+    aa.qkv = d->qkv;
+    aa.position = position;
+    aa.length = d->d_length;
+    aa.rope_cos = d->rope_cos;
+    aa.rope_sin = d->rope_sin;
+    aa.max_position = c.max_position;
+    aa.k_cache = d->k_cache + (size_t)l * layer_kv;
+    aa.v_cache = d->v_cache + (size_t)l * layer_kv;
+    aa.cap = c.kv_capacity;
+    aa.Hq = Hq;
+    aa.Hkv = Hkv;
+    aa.scale = 1.0f / sqrtf((float)D);
+    aa.out_f32 = d->o;
+    aa.ws_part = d->attn_part;
+    aa.ws_count = d->attn_count;
+    aa.nchunks = d->attn_chunks;
+    mark();
+    if ((e = launch_attn(aa, true, s, pdl)) != cudaSuccess) return e;
+    mark();
+
+    ResidArgs ro = {};
+    ro.w = GemvWeights{w.wo.q, w.wo.scales};
+    ro.N = H;
+    ro.K = Hq * D;
+    ro.x = d->o;
+    ro.x_resid = d->x_resid;
+    mark();
+    if ((e = launch_resid(ro, s, pdl)) != cudaSuccess) return e;
+    mark();
+
+    GateUpArgs ga = {};
+    ga.wg = GemvWeights{w.wgate.q, w.wgate.scales};
+    ga.wu = GemvWeights{w.wup.q, w.wup.scales};
+    ga.N = I;
+    ga.K = H;
+    ga.x_resid = d->x_resid;
+    ga.gamma = w.post_norm;
+    ga.eps = c.eps;
+    ga.h = d->h;
+    mark();
+    if ((e = launch_gateup(ga, s, pdl)) != cudaSuccess) return e;
+    mark();
+
+    ResidArgs rd = {};
+    rd.w = GemvWeights{w.wdown.q, w.wdown.scales};
+    rd.N = H;
+    rd.K = I;
+    rd.x = d->h;
+    rd.x_resid = d->x_resid;
+    rd.trace = d->trace ? d->trace + (size_t)l * H : nullptr;
+    mark();
+    if ((e = launch_resid(rd, s, pdl)) != cudaSuccess) return e;
+    mark();
+  }
+  if (!head) {
+    add_int_kernel<<<1, 1, 0, s>>>(d->d_length, 1);
+    return cudaGetLastError();
+  }
+  LmHeadArgs la = {};
+  la.x = d->x_resid;
+  la.gamma = d->final_norm;
+  la.w = d->lm_head;
+  la.V = c.vocab;
+  la.H = H;
+  la.eps = c.eps;
+  la.logits = logits;
+  la.idx = argmax ? argmax : d->d_argmax;
+  la.ws_val = d->lm_val;
+  la.ws_idx = d->lm_idx;
+  la.ws_count = d->lm_count;
+  la.length = d->d_length;
+  mark();
+  e = launch_lm_head(la, s, pdl);
+  mark();
+  return e;
+}
+
+}  // namespace vv
+
+using vv::set_error;
+
+extern "C" {
+
+vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uint16_t* k_cache,
+                            uint16_t* v_cache, vv_decoder** out) {
+  VV_CHECK_ARG(cfg && w && k_cache && v_cache && out && w->layers, "vv_decoder_create: null");
+  *out = nullptr;
+  const vv_config& c = *cfg;
+  VV_CHECK_SHAPE(c.head_dim == 128, "head_dim %d (only 128)", c.head_dim);
+  VV_CHECK_SHAPE(c.n_kv >= 1 && c.n_kv <= 64 && c.n_q % c.n_kv == 0 && c.n_q / c.n_kv <= 8,
+                 "n_q %d / n_kv %d", c.n_q, c.n_kv);
+  VV_CHECK_SHAPE(c.hidden >= 256 && c.hidden % 256 == 0 && c.hidden <= 16384, "hidden %d",
+                 c.hidden);
+  VV_CHECK_SHAPE(c.inter >= 256 && c.inter % 256 == 0 && c.inter <= 16384, "inter %d", c.inter);
+  VV_CHECK_SHAPE((c.n_q * c.head_dim) % 256 == 0 && c.n_q * c.head_dim <= 16384, "n_q*D %d",
+                 c.n_q * c.head_dim);
+  VV_CHECK_SHAPE(c.layers >= 1 && c.vocab >= 1 && c.kv_capacity >= 1 && c.max_position >= 1 &&
+                     c.max_prefill >= 0,
+                 "layers/vocab/capacity/max_position");
+  VV_CHECK_ARG(w->embed && w->lm_head && w->final_norm, "embed/lm_head/final_norm null");
+  VV_CHECK_ARG(vv::aligned16(k_cache) && vv::aligned16(v_cache) && vv::aligned16(w->lm_head) &&
+                   vv::aligned16(w->embed),
+               "cache / table pointers must be 16-byte aligned");
+  for (int l = 0; l < c.layers; ++l) {
+    const vv_layer_weights& L = w->layers[l];
+    const vv_packed_matrix* m[7] = {&L.wq, &L.wk, &L.wv, &L.wo, &L.wgate, &L.wup, &L.wdown};
+    for (auto* p : m)
+      VV_CHECK_ARG(p->q && p->scales && vv::aligned16(p->q) && vv::aligned16(p->scales),
+                   "layer %d: packed weight null or not 16-byte aligned", l);
+    VV_CHECK_ARG(L.input_norm && L.post_norm, "layer %d: norm gain null", l);
+  }
+
+  vv_decoder* d = new (std::nothrow) vv_decoder();
+  if (!d) return set_error(VV_ERR_CUDA, "out of host memory");
+  d->cfg = c;
+  d->layers.assign(w->layers, w->layers + c.layers);
+  d->embed = w->embed;
+  d->lm_head = w->lm_head;
+  d->final_norm = w->final_norm;
+  d->k_cache = k_cache;
+  d->v_cache = v_cache;
+  cudaGetDevice(&d->device);
+
+  const int H = c.hidden, D = c.head_dim;
+  d->attn_chunks = vv::attn_default_chunks(c.n_kv, c.kv_capacity);
+  const int lm_grid = vv::lm_head_grid(c.vocab);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = vv::align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_x = take((size_t)H * 4);
+  const size_t o_qkv = take((size_t)(c.n_q + 2 * c.n_kv) * D * 4);
+  const size_t o_o = take((size_t)c.n_q * D * 4);
+  const size_t o_h = take((size_t)c.inter * 4);
+  const size_t o_cos = take((size_t)c.max_position * (D / 2) * 4);
+  const size_t o_sin = take((size_t)c.max_position * (D / 2) * 4);
+  const size_t o_len = take(16);
+  const size_t o_arg = take(16);
+  const size_t attn_b = vv::attn_workspace_bytes(c.n_q, c.n_kv, d->attn_chunks);
+  const size_t o_part = take(attn_b);
+  const size_t o_lmv = take((size_t)lm_grid * 4);
+  const size_t o_lmi = take((size_t)lm_grid * 4);
+  const size_t o_lmc = take(16);
+  d->ws_bytes = off;
+  vv_status st = vv::cuda_check(cudaMalloc(&d->ws, d->ws_bytes), "cudaMalloc(decoder workspace)");
+  if (st) {
+    delete d;
+    return st;
+  }
+  st = vv::cuda_check(cudaMemset(d->ws, 0, d->ws_bytes), "cudaMemset");
+  unsigned char* b = d->ws;
+  d->x_resid = reinterpret_cast<float*>(b + o_x);
+  d->qkv = reinterpret_cast<float*>(b + o_qkv);
+  d->o = reinterpret_cast<float*>(b + o_o);
+  d->h = reinterpret_cast<float*>(b + o_h);
+  d->rope_cos = reinterpret_cast<float*>(b + o_cos);
+  d->rope_sin = reinterpret_cast<float*>(b + o_sin);
+  d->d_length = reinterpret_cast<int32_t*>(b + o_len);
+  d->d_argmax = reinterpret_cast<int32_t*>(b + o_arg);
+  d->attn_part = reinterpret_cast<float*>(b + o_part);
+  d->attn_count = reinterpret_cast<int*>(b + o_part + attn_b - 256);
+  d->lm_val = reinterpret_cast<float*>(b + o_lmv);
+  d->lm_idx = reinterpret_cast<int*>(b + o_lmi);
+  d->lm_count = reinterpret_cast<int*>(b + o_lmc);
+
+  // RoPE tables: angle = pos * theta^(-2i/D) in float64, cos/sin rounded once to fp32.
+  if (!st) {
+    std::vector<float> cs((size_t)c.max_position * (D / 2)), sn(cs.size());
+    for (int i = 0; i < D / 2; ++i) {
+      const double inv = std::pow((double)c.rope_theta, -2.0 * i / (double)D);
+      for (int p = 0; p < c.max_position; ++p) {
+        const double ang = (double)p * inv;
+        cs[(size_t)p * (D / 2) + i] = (float)std::cos(ang);
+        sn[(size_t)p * (D / 2) + i] = (float)std::sin(ang);
+      }
+    }
+    st = vv::cuda_check(cudaMemcpy(d->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice),
+                        "copy rope cos");
+    if (!st)
+      st = vv::cuda_check(
+          cudaMemcpy(d->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice),
+          "copy rope sin");
+  }
+  if (st) {
+    cudaFree(d->ws);
+    delete d;
+    return st;
+  }
+  *out = d;
+  return VV_OK;
+}
+
+vv_status vv_decoder_destroy(vv_decoder* d) {
+  if (!d) return VV_OK;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  cudaSetDevice(d->device);
+  if (d->gexec) cudaGraphExecDestroy(d->gexec);
+  if (d->ws) cudaFree(d->ws);
+  if (d->pws) cudaFree(d->pws);
+  cudaSetDevice(cur);
+  delete d;
+  return VV_OK;
+}
+
+vv_status vv_decoder_set_length(vv_decoder* d, int32_t len, vv_stream stream) {
+  VV_CHECK_ARG(d, "null decoder");
+  if (len < 0) return set_error(VV_ERR_RANGE, "length %d < 0", len);
+  if (len > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "length %d > capacity %d", len, d->cfg.kv_capacity);
+  vv::set_int_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(d->d_length, len);
+  VV_CUDA(cudaGetLastError());
+  d->len_host = len;
+  return VV_OK;
+}
+
+int32_t vv_decoder_length(const vv_decoder* d) { return d ? d->len_host : -1; }
+
+vv_status vv_decoder_set_trace(vv_decoder* d, float* layer_out) {
+  VV_CHECK_ARG(d, "null decoder");
+  d->trace = layer_out;
+  return VV_OK;
+}
+
+vv_status vv_decoder_set_graph(vv_decoder* d, int32_t enable) {
+  VV_CHECK_ARG(d, "null decoder");
+  d->use_graph = enable != 0;
+  return VV_OK;
+}
+
+int32_t vv_decoder_step_launches(const vv_decoder* d) { return d ? d->cfg.layers * 5 + 1 : 0; }
+
+vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int32_t* token_id,
+                          const int32_t* position_id, float* logits, int32_t* argmax_out,
+                          vv_stream stream) {
+  VV_CHECK_ARG(d && position_id, "vv_decoder_step: null decoder or position");
+  VV_CHECK_ARG(input_embeds || token_id, "vv_decoder_step: need input_embeds or token_id");
+  VV_CHECK_ARG(!input_embeds || vv::aligned16(input_embeds), "input_embeds not 16-byte aligned");
+  if (d->len_host + 1 > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "KV cache full (%d of %d)", d->len_host,
+                     d->cfg.kv_capacity);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!d->use_graph) {
+    VV_CUDA(vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s, true, nullptr));
+    d->len_host += 1;
+    return VV_OK;
+  }
+  const void* key[6] = {input_embeds, token_id, position_id, logits, argmax_out, d->trace};
+  bool same = d->gexec != nullptr;
+  for (int i = 0; i < 6 && same; ++i) same = key[i] == d->gkey[i];
+  if (!same) {
+    if (d->gexec) {
+      cudaGraphExecDestroy(d->gexec);
+      d->gexec = nullptr;
+    }
+    cudaGraph_t g = nullptr;
+    VV_CUDA(cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed));
+    cudaError_t le = vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s, true, nullptr);
+    cudaError_t ee = cudaStreamEndCapture(s, &g);
+    if (le != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      return vv::cuda_check(le, "step capture (launch)");
+    }
+    VV_CUDA(ee);
+    cudaError_t ie = cudaGraphInstantiate(&d->gexec, g, 0);
+    cudaGraphDestroy(g);
+    VV_CUDA(ie);
+    for (int i = 0; i < 6; ++i) d->gkey[i] = key[i];
+  }
+  VV_CUDA(cudaGraphLaunch(d->gexec, s));
+  d->len_host += 1;
+  return VV_OK;
+}
+
+vv_status vv_decoder_profile_step(vv_decoder* d, const uint16_t* input_embeds,
+                                  const int32_t* token_id, const int32_t* position_id,
+                                  float* logits, int32_t* argmax_out, float* phase_ms,
+                                  vv_stream stream) {
+  VV_CHECK_ARG(d && position_id && phase_ms, "vv_decoder_profile_step: null pointer");
+  VV_CHECK_ARG(input_embeds || token_id, "vv_decoder_profile_step: need input_embeds or token");
+  if (d->len_host + 1 > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "KV cache full (%d of %d)", d->len_host,
+                     d->cfg.kv_capacity);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = 2 * (d->cfg.layers * 5 + 1);
+  std::vector<cudaEvent_t> ev(n, nullptr);
+  vv_status st = VV_OK;
+  for (int i = 0; i < n && !st; ++i) st = vv::cuda_check(cudaEventCreate(&ev[i]), "event");
+  if (!st)
+    st = vv::cuda_check(vv::enqueue_step(d, input_embeds, token_id, position_id, logits,
+                                         argmax_out, s, true, ev.data()),
+                        "profile step");
+  if (!st) st = vv::cuda_check(cudaStreamSynchronize(s), "sync");
+  if (!st) {
+    for (int i = 0; i < 6; ++i) phase_ms[i] = 0.f;
+    for (int k = 0; k < n / 2; ++k) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, ev[2 * k], ev[2 * k + 1]);
+      const int phase = (k == n / 2 - 1) ? 5 : (k % 5);
+      phase_ms[phase] += ms;
+    }
+    d->len_host += 1;
+  }
+  for (auto e : ev)
+    if (e) cudaEventDestroy(e);
+  return st;
+}
+
+vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t* position_ids,
+                          int64_t S, const uint16_t* audio_features, int64_t N,
+                          int64_t audio_offset, float* logits, int32_t* argmax_out,
+                          vv_stream stream) {
+  VV_CHECK_ARG(d && input_ids && position_ids, "vv_decoder_init: null pointer");
+  VV_CHECK_ARG(N == 0 || audio_features, "vv_decoder_init: audio_features null with N > 0");
+  VV_CHECK_ARG(!audio_features || vv::aligned16(audio_features), "audio_features misaligned");
+  if (S < 1) return set_error(VV_ERR_SHAPE, "S=%lld", (long long)S);
+  if (N < 0 || audio_offset < 0 || audio_offset + N > S)
+    return set_error(VV_ERR_RANGE, "audio_offset %lld + N %lld > S %lld", (long long)audio_offset,
+                     (long long)N, (long long)S);
+  if (S > d->cfg.kv_capacity || S > d->cfg.max_prefill)
+    return set_error(VV_ERR_CAPACITY, "S=%lld > capacity %d or max_prefill %d", (long long)S,
+                     d->cfg.kv_capacity, d->cfg.max_prefill);
+  VV_CUDA(vv::prefill_run(d, input_ids, position_ids, (int)S, audio_features, (int)N,
+                          (int)audio_offset, logits, argmax_out,
+                          static_cast<cudaStream_t>(stream)));
+  d->len_host = (int32_t)S;
+  return VV_OK;
+}
+
+vv_status vv_decoder_sync_status(vv_decoder* d, vv_stream stream) {
+  VV_CHECK_ARG(d, "null decoder");
+  return vv_sync_status(stream);
+}
+
+}  // extern "C"

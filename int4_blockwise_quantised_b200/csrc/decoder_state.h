@@ -1,0 +1,59 @@
+// Decoder state shared by decoder.cu and prefill.cu (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <vector>
+
+#include "../../include/vv.h"
+
+struct vv_decoder {
+  vv_config cfg;
+  std::vector<vv_layer_weights> layers;
+  const uint16_t* embed = nullptr;
+  const uint16_t* lm_head = nullptr;
+  const uint16_t* final_norm = nullptr;
+  uint16_t* k_cache = nullptr;
+  uint16_t* v_cache = nullptr;
+  int device = 0;
+
+  unsigned char* ws = nullptr;
+  size_t ws_bytes = 0;
+  float* x_resid = nullptr;
+  float* qkv = nullptr;
+  float* o = nullptr;
+  float* h = nullptr;
+  float* rope_cos = nullptr;
+  float* rope_sin = nullptr;
+  int32_t* d_length = nullptr;
+  int32_t* d_argmax = nullptr;
+  float* attn_part = nullptr;
+  int* attn_count = nullptr;
+  int attn_chunks = 1;
+  float* lm_val = nullptr;
+  int* lm_idx = nullptr;
+  int* lm_count = nullptr;
+  // prefill workspace (allocated lazily by the prefill path)
+  unsigned char* pws = nullptr;
+  size_t pws_bytes = 0;
+
+  int32_t len_host = 0;
+  float* trace = nullptr;
+  bool use_graph = true;
+  cudaGraphExec_t gexec = nullptr;
+  const void* gkey[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+};
+
+
+namespace vv {
+__global__ void set_int_kernel(int32_t* p, int32_t v);
+__global__ void add_int_kernel(int32_t* p, int32_t v);
+// Enqueue one decode step (plain launches).  head=false skips the lm_head and only advances the
+// device length (used by the token-by-token prefill).
+cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
+                         const int32_t* position, float* logits, int32_t* argmax, cudaStream_t s,
+                         bool head, cudaEvent_t* events = nullptr);
+cudaError_t prefill_run(vv_decoder* dec, const int32_t* ids, const int32_t* pos, int S,
+                        const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
+                        cudaStream_t s);
+}  // namespace vv

@@ -1,0 +1,247 @@
+"""GPU parity of the decoder (decoder_step / decoder_init through the C ABI) against the oracle.
+
+Contract: every layer output (the residual after the MLP) and the logits within 2e-3 normwise;
+the appended K/V at slot P equal to the oracle's fp16 values to 1 ulp and every other cache slot
+untouched; greedy argmax equal wherever the oracle's top-2 margin exceeds 1e-2.  Multi-step runs
+are teacher-forced with the oracle's tokens (trajectories never fork at near-ties).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import TOL, gpu_model, normwise, ocfg, oracle_model
+from oracle import decoder as odec
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def need_gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def fill_cache(dec, kp, vp):
+    P = kp.shape[2]
+    dec.k_cache[:, 0, :, :P] = dev(kp)
+    dec.v_cache[:, 0, :, :P] = dev(vp)
+    dec.set_length(P)
+
+
+def ulp_close(a16, b16):
+    a = a16.astype(np.float64)
+    b = b16.astype(np.float64)
+    return np.all(np.abs(a - b) <= np.spacing(np.abs(b16)).astype(np.float64) * 1.0001)
+
+
+def run_steps(shape, mode, P, steps, cap=None, graph=True, check_kv=True, layers_oracle=None):
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    cfg = ocfg(shape)
+    W = oracle_model(shape, mode)
+    model = gpu_model(shape, mode)
+    cap = cap or P + steps + 5
+    dec = Decoder(model, cap)
+    dec.set_graph(graph)
+    kp, vp = synth.past_kv(shape, P)
+    fill_cache(dec, kp, vp)
+    kc = [kp[l].copy() for l in range(shape.layers)]
+    vc = [vp[l].copy() for l in range(shape.layers)]
+    trace = torch.zeros((shape.layers, shape.hidden), dtype=torch.float32, device="cuda")
+    dec.set_trace(trace)
+    emb = synth.input_embeds(shape, steps)
+    pos_t = torch.zeros(1, dtype=torch.int32, device="cuda")
+    emb_t = torch.zeros(shape.hidden, dtype=torch.float16, device="cuda")
+    logits = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+    amax = torch.zeros(1, dtype=torch.int32, device="cuda")
+    worst = 0.0
+    for s in range(steps):
+        pos = P + s + (128 - P if P == 128 and s == 0 else 0)
+        pos_t.fill_(pos)
+        emb_t.copy_(dev(emb[s]))
+        dec.step(pos_t, input_embeds=emb_t, logits=logits, argmax=amax)
+        dec.sync_status()
+        ora = odec.decoder_step(cfg, W, emb[s], pos, kc, vc)
+        lo = trace.cpu().numpy()
+        for l in range(shape.layers):
+            e = normwise(lo[l], ora["layer_out"][l])
+            worst = max(worst, e)
+            assert e <= TOL, f"step {s} layer {l}: {e}"
+        e = normwise(logits.cpu().numpy(), ora["logits"])
+        assert e <= TOL, f"step {s} logits: {e}"
+        ref = ora["logits"]
+        top2 = np.sort(ref)[-2:]
+        if top2[1] - top2[0] > 1e-2:
+            assert int(amax.item()) == ora["argmax"]
+        if check_kv:
+            slot = P + s
+            kg = dec.k_cache[:, 0, :, slot].cpu().numpy()
+            vg = dec.v_cache[:, 0, :, slot].cpu().numpy()
+            assert ulp_close(kg, ora["k_new"]) and ulp_close(vg, ora["v_new"])
+        for l in range(shape.layers):
+            kc[l] = np.concatenate([kc[l], ora["k_new"][l][:, None, :]], axis=1)
+            vc[l] = np.concatenate([vc[l], ora["v_new"][l][:, None, :]], axis=1)
+    # untouched slots: past positions bit-identical, beyond length still zero
+    n = P + steps
+    assert np.array_equal(dec.k_cache[:, 0, :, :P].cpu().numpy(), kp)
+    assert torch.count_nonzero(dec.k_cache[:, 0, :, n:]).item() == 0
+    assert dec.length == n
+    return worst
+
+
+def test_single_layer_ternary_config():
+    """One decoder layer, ternary weights, P = 128 at position 128 (one-layer workload)."""
+    shape = synth.Shape("layer1", 1536, 1, 12, 2, 128, 8960, 151936, tied=True)
+    run_steps(shape, "ternary", 128, 1)
+
+
+def test_tiny_int4_multistep_graph():
+    run_steps(synth.SHAPE_TINY, "int4", 5, 6)
+
+
+def test_tiny_int4_multistep_no_graph():
+    run_steps(synth.SHAPE_TINY, "int4", 70, 3, graph=False)
+
+
+def test_small_real_dims_multistep():
+    run_steps(synth.SHAPE_SMALL, "int4", 1024, 4)
+
+
+def test_small_ternary_long_context():
+    run_steps(synth.SHAPE_SMALL, "ternary", 4530, 2)
+
+
+def test_graph_and_plain_launches_bit_identical():
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.SHAPE_TINY
+    model = gpu_model(shape, "int4")
+    outs = []
+    for graph in (True, False):
+        dec = Decoder(model, 64)
+        dec.set_graph(graph)
+        kp, vp = synth.past_kv(shape, 9)
+        fill_cache(dec, kp, vp)
+        lg = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+        pos = torch.tensor([9], dtype=torch.int32, device="cuda")
+        tok = torch.tensor([17], dtype=torch.int32, device="cuda")
+        for _ in range(3):
+            dec.step(pos, token=tok, logits=lg)
+            pos += 1
+        torch.cuda.synchronize()
+        outs.append((lg.cpu().numpy().copy(), dec.k_cache.cpu().numpy().copy()))
+        dec.close()
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+def test_token_id_input_gathers_embedding():
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.SHAPE_TINY
+    model = gpu_model(shape, "int4")
+    W = oracle_model(shape, "int4")
+    dec = Decoder(model, 16)
+    kp, vp = synth.past_kv(shape, 3)
+    fill_cache(dec, kp, vp)
+    lg = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+    dec.step(torch.tensor([3], dtype=torch.int32, device="cuda"),
+             token=torch.tensor([421], dtype=torch.int32, device="cuda"), logits=lg)
+    dec.sync_status()
+    ora = odec.decoder_step(ocfg(shape), W, W["embed"][421], 3, list(kp), list(vp))
+    assert normwise(lg.cpu().numpy(), ora["logits"]) <= TOL
+
+
+def test_capacity_and_range_errors():
+    from int4_blockwise_quantised_b200 import _vv
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.SHAPE_TINY
+    model = gpu_model(shape, "int4")
+    dec = Decoder(model, 4, max_position=8)
+    pos = torch.tensor([0], dtype=torch.int32, device="cuda")
+    tok = torch.tensor([1], dtype=torch.int32, device="cuda")
+    for i in range(4):
+        pos.fill_(i)
+        dec.step(pos, token=tok)
+    dec.sync_status()
+    with pytest.raises(_vv.VVError) as e:
+        dec.step(pos, token=tok)
+    assert e.value.code == _vv.VV_ERR_CAPACITY
+    with pytest.raises(_vv.VVError):
+        dec.set_length(5)
+    dec.set_length(0)
+    pos.fill_(100)  # outside the RoPE table -> device-side range error, reported at sync
+    dec.step(pos, token=tok)
+    with pytest.raises(_vv.VVError) as e:
+        dec.sync_status()
+    assert e.value.code == _vv.VV_ERR_RANGE
+    tok.fill_(shape.vocab + 5)
+    pos.fill_(1)
+    dec.step(pos, token=tok)
+    with pytest.raises(_vv.VVError) as e:
+        dec.sync_status()
+    assert e.value.code == _vv.VV_ERR_RANGE
+    dec.sync_status()  # cleared
+
+
+# ------------------------------------------------------------------------------------ prefill
+@pytest.mark.parametrize("shape,mode,S,N", [(synth.SHAPE_TINY, "int4", 37, 20),
+                                            (synth.SHAPE_SMALL, "ternary", 70, 40)])
+def test_prefill_then_steps_match_oracle(shape, mode, S, N):
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    cfg = ocfg(shape)
+    W = oracle_model(shape, mode)
+    model = gpu_model(shape, mode)
+    ids, pos, feats, off = synth.asr_prompt(shape, N, prefix=7, suffix=S - N - 7)
+    dec = Decoder(model, S + 8, max_prefill=S)
+    trace = torch.zeros((shape.layers, shape.hidden), dtype=torch.float32, device="cuda")
+    dec.set_trace(trace)
+    lg = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+    am = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dec.init(dev(ids), dev(pos), dev(feats), off, logits=lg, argmax=am)
+    dec.sync_status()
+    ora = odec.decoder_init(cfg, W, ids, pos, feats, off)
+    assert dec.length == S
+    assert normwise(lg.cpu().numpy(), ora["logits"]) <= TOL
+    lo = trace.cpu().numpy()
+    for l in range(shape.layers):
+        assert normwise(lo[l], ora["layer_out"][l]) <= TOL
+    kg = dec.k_cache[:, 0, :, :S].cpu().numpy()
+    assert normwise(kg, ora["k"]) <= TOL
+    assert normwise(dec.v_cache[:, 0, :, :S].cpu().numpy(), ora["v"]) <= TOL
+    # continue decoding from the prefilled cache (teacher-forced with the oracle's argmax)
+    kc = [ora["k"][l] for l in range(shape.layers)]
+    vc = [ora["v"][l] for l in range(shape.layers)]
+    tok = ora["argmax"]
+    for s in range(2):
+        p = S + s
+        dec.step(torch.tensor([p], dtype=torch.int32, device="cuda"),
+                 token=torch.tensor([tok], dtype=torch.int32, device="cuda"), logits=lg)
+        st = odec.decoder_step(cfg, W, W["embed"][tok], p, kc, vc)
+        assert normwise(lg.cpu().numpy(), st["logits"]) <= TOL
+        kc = [np.concatenate([kc[l], st["k_new"][l][:, None]], 1) for l in range(shape.layers)]
+        vc = [np.concatenate([vc[l], st["v_new"][l][:, None]], 1) for l in range(shape.layers)]
+        tok = st["argmax"]
+
+
+def test_prefill_rejects_bad_splice():
+    from int4_blockwise_quantised_b200 import _vv
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.SHAPE_TINY
+    dec = Decoder(gpu_model(shape, "int4"), 32, max_prefill=16)
+    ids = torch.zeros(10, dtype=torch.int32, device="cuda")
+    feats = torch.zeros((5, shape.hidden), dtype=torch.float16, device="cuda")
+    with pytest.raises(_vv.VVError) as e:
+        dec.init(ids, ids, feats, audio_offset=6)
+    assert e.value.code == _vv.VV_ERR_RANGE
+    with pytest.raises(_vv.VVError) as e:
+        dec.init(torch.zeros(20, dtype=torch.int32, device="cuda"),
+                 torch.zeros(20, dtype=torch.int32, device="cuda"))
+    assert e.value.code == _vv.VV_ERR_CAPACITY
