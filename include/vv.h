@@ -249,7 +249,21 @@ vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
                                   float* logits, int32_t* argmax_out, float* phase_ms,
                                   vv_stream stream);
 
-/* Number of kernel launches one vv_decoder_step enqueues (for launch accounting). */
+/* Timeline tap of the persistent step kernel: runs one step (appending a position like
+ * vv_decoder_step, without graph capture) with every CTA recording the device clock
+ * (%globaltimer, ns) at fixed points of its schedule: kernel start, then for each layer
+ * [x staged (QKV)], barrier arrive/exit before attention, barrier arrive/exit before o-proj,
+ * x staged, arrive/exit, x staged (gate/up), arrive/exit, x staged (down); layers > 0 start
+ * with arrive/exit before QKV; then arrive/exit, x staged (lm_head), end.  stamps: HOST
+ * uint64 [grid * max_per_cta]; *grid_out and *per_cta_out receive the CTA count and the number
+ * of stamps each CTA wrote.  Synchronous.  VV_ERR_CAPACITY when max_per_cta is too small. */
+vv_status vv_decoder_step_timeline(vv_decoder* dec, const uint16_t* input_embeds,
+                                   const int32_t* token_id, const int32_t* position_id,
+                                   uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,
+                                   int32_t* per_cta_out, vv_stream stream);
+
+/* Number of kernel launches one vv_decoder_step enqueues (for launch accounting): 1 for the
+ * persistent step kernel (default), 5 per layer + 1 with VV_STEP=kernels in the environment. */
 int32_t vv_decoder_step_launches(const vv_decoder* dec);
 
 #ifdef __cplusplus

@@ -89,6 +89,8 @@ def _load():
         "vv_decoder_sync_status": (S, [P, P]),
         "vv_decoder_step_launches": (c_int32, [P]),
         "vv_decoder_profile_step": (S, [P, P, P, P, P, P, POINTER(c_float), P]),
+        "vv_decoder_step_timeline": (S, [P, P, P, P, P, c_int32, POINTER(c_int32),
+                                         POINTER(c_int32), P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

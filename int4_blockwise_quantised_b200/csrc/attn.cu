@@ -31,6 +31,7 @@ constexpr int kThreads = 256;
 constexpr int kMaxG = 8;
 constexpr int kPartStride = 132;  // floats per (chunk, head) partial: m, l, pad, pad, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxChunks = 256;  // upper bound of grid.x (chunks per KV head)
 
 struct AttnSmem {
   __half k[2][TT * D];
@@ -38,7 +39,7 @@ struct AttnSmem {
   float q[kMaxG][D];
   float s[kMaxG][TT];
   float m[kMaxG], l[kMaxG], corr[kMaxG];
-  float mw[kMaxG];  // merge weights scratch
+  float mw[kMaxChunks][kMaxG];  // merge weights 2^(m_c - M) / L per (chunk, head)
   uint64_t bar[2];
   int is_last;
 };
@@ -169,16 +170,34 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
     }
 
     // scores: warp w -> positions w, w+8, ...
-    for (int p = warp; p < n; p += kThreads / 32) {
+    for (int p = warp; p < n; p += 2 * (kThreads / 32)) {
+      const int p2 = p + kThreads / 32;
+      const bool has2 = p2 < n;
       const uint2 kr = *reinterpret_cast<const uint2*>(&sm.k[b][p * D + 4 * lane]);
+      const uint2 kr2 = has2 ? *reinterpret_cast<const uint2*>(&sm.k[b][p2 * D + 4 * lane])
+                             : make_uint2(0u, 0u);
       const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kr.x));
       const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kr.y));
+      const float2 j01 = __half22float2(*reinterpret_cast<const __half2*>(&kr2.x));
+      const float2 j23 = __half22float2(*reinterpret_cast<const __half2*>(&kr2.y));
+      float sd[2 * kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) {
-        if (h < G) {
-          float sdot = qf[h].x * k01.x + qf[h].y * k01.y + qf[h].z * k23.x + qf[h].w * k23.y;
-          sdot = warp_sum(sdot);
-          if (lane == 0) sm.s[h][p] = sdot;
+        sd[h] = qf[h].x * k01.x + qf[h].y * k01.y + qf[h].z * k23.x + qf[h].w * k23.y;
+        sd[kMaxG + h] = qf[h].x * j01.x + qf[h].y * j01.y + qf[h].z * j23.x + qf[h].w * j23.y;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 2 * kMaxG; ++i) sd[i] += __shfl_xor_sync(0xffffffffu, sd[i], o);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          if (h < G) {
+            sm.s[h][p] = sd[h];
+            if (has2) sm.s[h][p2] = sd[kMaxG + h];
+          }
         }
       }
     }
@@ -257,38 +276,46 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
   __threadfence();
 
   const float* base = a.ws_part + (size_t)g * nchunks * kMaxG * kPartStride;
-  // per head: M = max m_c, L = sum l_c 2^(m_c - M)
+  // per head: M = max m_c, L = sum l_c 2^(m_c - M); weights w_c = 2^(m_c - M) / L to smem
   if (warp < G) {
     const int h = warp;
     float mx = -INFINITY;
-    for (int cc = lane; cc < active; cc += 32) mx = fmaxf(mx, __ldcg(base + ((size_t)cc * kMaxG + h) * kPartStride));
+    for (int cc = lane; cc < active; cc += 32)
+      mx = fmaxf(mx, __ldcg(base + ((size_t)cc * kMaxG + h) * kPartStride));
     mx = warp_max(mx);
     float L = 0.f;
     for (int cc = lane; cc < active; cc += 32) {
       const float* pp = base + ((size_t)cc * kMaxG + h) * kPartStride;
-      L += __ldcg(pp + 1) * exp2f(__ldcg(pp) - mx);
+      const float e = exp2f(__ldcg(pp) - mx);
+      sm.mw[cc][h] = e;
+      L += __ldcg(pp + 1) * e;
     }
     L = warp_sum(L);
-    if (lane == 0) {
-      sm.m[h] = mx;
-      sm.l[h] = L;
-    }
+    const float invL = 1.f / L;
+    for (int cc = lane; cc < active; cc += 32) sm.mw[cc][h] *= invL;
   }
   __syncthreads();
+  // out[h][d] = sum_c w_c o_c[h][d]: independent loads, 8 chunks in flight per thread
 #pragma unroll
   for (int j = 0; j < kMaxG / 2; ++j) {
     const int h = hh + 2 * j;
     if (h < G) {
       float acc = 0.f;
-      const float mx = sm.m[h];
-      for (int cc = 0; cc < active; ++cc) {
-        const float* pp = base + ((size_t)cc * kMaxG + h) * kPartStride;
-        acc = fmaf(__ldcg(pp + 4 + od), exp2f(__ldcg(pp) - mx), acc);
+      int cc = 0;
+      for (; cc + 8 <= active; cc += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          v[u] = __ldcg(base + ((size_t)(cc + u) * kMaxG + h) * kPartStride + 4 + od);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc = fmaf(sm.mw[cc + u][h], v[u], acc);
       }
-      const float r = acc / sm.l[h];
+      for (; cc < active; ++cc)
+        acc = fmaf(sm.mw[cc][h], __ldcg(base + ((size_t)cc * kMaxG + h) * kPartStride + 4 + od),
+                   acc);
       const size_t idx = (size_t)(g * G + h) * D + od;
-      if (FUSED) a.out_f32[idx] = r;
-      else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(r);
+      if (FUSED) a.out_f32[idx] = acc;
+      else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(acc);
     }
   }
   if (tid == 0) a.ws_count[g] = 0;
@@ -300,7 +327,8 @@ int attn_default_chunks(int Hkv, int cap) {
   const int tiles = (cap + TT - 1) / TT;
   int per_head = sm_count() / (Hkv > 0 ? Hkv : 1);
   if (per_head < 1) per_head = 1;
-  return tiles < per_head ? (tiles > 0 ? tiles : 1) : per_head;
+  int n = tiles < per_head ? (tiles > 0 ? tiles : 1) : per_head;
+  return n > kMaxChunks ? kMaxChunks : n;
 }
 
 size_t attn_workspace_bytes(int Hq, int Hkv, int nchunks) {

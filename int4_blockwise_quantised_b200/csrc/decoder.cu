@@ -18,6 +18,8 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -38,9 +40,19 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
                          const int32_t* position, float* logits, int32_t* argmax,
                          cudaStream_t s, bool head, cudaEvent_t* ev) {
+  if (d->persistent && ev == nullptr && head) {
+    StepParams p = d->step;
+    p.input_embeds = reinterpret_cast<const __half*>(embeds);
+    p.token = token;
+    p.position = position;
+    p.logits = logits;
+    p.argmax = argmax ? argmax : d->d_argmax;
+    p.trace = d->trace;
+    return launch_step(p, s);
+  }
   // ev (profiling): 2 events per launch, recorded around each kernel; PDL off so the events
   // bracket exactly one kernel.
-  const bool pdl = ev == nullptr;
+  const bool pdl = ev == nullptr && d->use_pdl;
   int evi = 0;
   auto mark = [&]() {
     if (ev) cudaEventRecord(ev[evi++], s);
@@ -202,6 +214,8 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   d->k_cache = k_cache;
   d->v_cache = v_cache;
   cudaGetDevice(&d->device);
+  // VV_PDL=0 launches the step without programmatic dependent launch (diagnostics).
+  if (const char* e = getenv("VV_PDL")) d->use_pdl = atoi(e) != 0;
 
   const int H = c.hidden, D = c.head_dim;
   d->attn_chunks = vv::attn_default_chunks(c.n_kv, c.kv_capacity);
@@ -225,6 +239,16 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   const size_t o_lmv = take((size_t)lm_grid * 4);
   const size_t o_lmi = take((size_t)lm_grid * 4);
   const size_t o_lmc = take(16);
+  // persistent step kernel
+  const int grid = vv::sm_count();
+  const int max_tiles = vv::step_max_tiles(c.kv_capacity);
+  const size_t o_spart = take(vv::step_attn_part_floats(c.n_kv, max_tiles) * 4);
+  const size_t o_scnt = take((size_t)c.n_kv * 4);
+  const size_t o_hval = take((size_t)grid * 4);
+  const size_t o_hidx = take((size_t)grid * 4);
+  const size_t o_hcnt = take(16);
+  const size_t o_bar = take(16);
+  const size_t o_layers = take(sizeof(vv::StepLayer) * c.layers);
   d->ws_bytes = off;
   vv_status st = vv::cuda_check(cudaMalloc(&d->ws, d->ws_bytes), "cudaMalloc(decoder workspace)");
   if (st) {
@@ -246,6 +270,84 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   d->lm_val = reinterpret_cast<float*>(b + o_lmv);
   d->lm_idx = reinterpret_cast<int*>(b + o_lmi);
   d->lm_count = reinterpret_cast<int*>(b + o_lmc);
+
+  {
+    vv::StepParams& p = d->step;
+    p.H = H;
+    p.L = c.layers;
+    p.Hq = c.n_q;
+    p.Hkv = c.n_kv;
+    p.I = c.inter;
+    p.V = c.vocab;
+    p.eps = c.eps;
+    p.scale = 1.0f / sqrtf((float)D);
+    d->d_layers = reinterpret_cast<vv::StepLayer*>(b + o_layers);
+    p.layers = d->d_layers;
+    p.embed = reinterpret_cast<const __half*>(w->embed);
+    p.lm_head = reinterpret_cast<const __half*>(w->lm_head);
+    p.final_norm = reinterpret_cast<const __half*>(w->final_norm);
+    p.k_cache = reinterpret_cast<__half*>(k_cache);
+    p.v_cache = reinterpret_cast<__half*>(v_cache);
+    p.cap = c.kv_capacity;
+    p.rope_cos = d->rope_cos;
+    p.rope_sin = d->rope_sin;
+    p.max_position = c.max_position;
+    p.x_resid = d->x_resid;
+    p.qkv = d->qkv;
+    p.attn_out = d->o;
+    p.h = d->h;
+    p.attn_part = reinterpret_cast<float*>(b + o_spart);
+    p.attn_count = reinterpret_cast<int*>(b + o_scnt);
+    p.max_tiles = max_tiles;
+    p.head_val = reinterpret_cast<float*>(b + o_hval);
+    p.head_idx = reinterpret_cast<int*>(b + o_hidx);
+    p.head_count = reinterpret_cast<int*>(b + o_hcnt);
+    p.length = d->d_length;
+    p.bar_count = reinterpret_cast<unsigned*>(b + o_bar);
+    p.bar_gen = reinterpret_cast<unsigned*>(b + o_bar + 4);
+    p.grid = grid;
+    p.nstages = 4;
+    p.x_floats = std::max(std::max(H, c.n_q * D), c.inter);
+    const size_t fixed = vv::step_smem_bytes(0, p.nstages, p.x_floats);
+    int smem_max = 0;
+    cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, d->device);
+    if (smem_max <= 0) smem_max = 232448;
+    const long avail = (long)smem_max - (long)fixed;
+    p.stage_bytes = (int)((avail / p.nstages) / 1024 * 1024);
+    std::vector<vv::StepLayer> hl(c.layers);
+    for (int l = 0; l < c.layers; ++l) {
+      const vv_layer_weights& L = w->layers[l];
+      const vv_packed_matrix* m[7] = {&L.wq, &L.wk, &L.wv, &L.wo, &L.wgate, &L.wup, &L.wdown};
+      hl[l].in_norm = reinterpret_cast<const __half*>(L.input_norm);
+      hl[l].post_norm = reinterpret_cast<const __half*>(L.post_norm);
+      for (int k = 0; k < 7; ++k) {
+        hl[l].q[k] = m[k]->q;
+        hl[l].s[k] = reinterpret_cast<const __half*>(m[k]->scales);
+      }
+      hl[l].bias[0] = reinterpret_cast<const __half*>(L.bq);
+      hl[l].bias[1] = reinterpret_cast<const __half*>(L.bk);
+      hl[l].bias[2] = reinterpret_cast<const __half*>(L.bv);
+    }
+    if (!st)
+      st = vv::cuda_check(cudaMemcpy(d->d_layers, hl.data(), sizeof(vv::StepLayer) * c.layers,
+                                     cudaMemcpyHostToDevice),
+                          "copy layer table");
+    int nb = 0;
+    if (!st && H > 32 * grid)
+      st = set_error(VV_ERR_SHAPE, "hidden %d > 32 x SM count (persistent step)", H);
+    if (!st) st = vv::cuda_check(vv::step_configure(p, &nb), "step kernel configuration");
+    if (!st && nb < 1) {
+      int regs = 0, mt = 0, ss = 0, lb = 0;
+      vv::step_func_info(&regs, &mt, &ss, &lb);
+      st = set_error(VV_ERR_SHAPE,
+                     "persistent step: no stage size >= 32 KB fits one CTA per SM (regs %d, "
+                     "max threads %d, static smem %d, local %d, threads %d, smem optin %d)",
+                     regs, mt, ss, lb, vv::step_threads(), smem_max);
+    }
+    if (!st && max_tiles > 256)
+      st = set_error(VV_ERR_SHAPE, "kv_capacity %d > 16384 (persistent step)", c.kv_capacity);
+  }
+  if (const char* e = getenv("VV_STEP")) d->persistent = strcmp(e, "kernels") != 0;
 
   // RoPE tables: angle = pos * theta^(-2i/D) in float64, cos/sin rounded once to fp32.
   if (!st) {
@@ -280,6 +382,7 @@ vv_status vv_decoder_destroy(vv_decoder* d) {
   cudaGetDevice(&cur);
   cudaSetDevice(d->device);
   if (d->gexec) cudaGraphExecDestroy(d->gexec);
+  if (d->capture_stream) cudaStreamDestroy(d->capture_stream);
   if (d->ws) cudaFree(d->ws);
   if (d->pws) cudaFree(d->pws);
   cudaSetDevice(cur);
@@ -312,7 +415,10 @@ vv_status vv_decoder_set_graph(vv_decoder* d, int32_t enable) {
   return VV_OK;
 }
 
-int32_t vv_decoder_step_launches(const vv_decoder* d) { return d ? d->cfg.layers * 5 + 1 : 0; }
+int32_t vv_decoder_step_launches(const vv_decoder* d) {
+  if (!d) return 0;
+  return d->persistent ? 1 : d->cfg.layers * 5 + 1;
+}
 
 vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int32_t* token_id,
                           const int32_t* position_id, float* logits, int32_t* argmax_out,
@@ -337,10 +443,16 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
       cudaGraphExecDestroy(d->gexec);
       d->gexec = nullptr;
     }
+    // Capture on the decoder's own stream (capture executes nothing, and the caller's stream
+    // may be the legacy default stream, which cannot be captured); replay on the caller's.
+    if (!d->capture_stream)
+      VV_CUDA(cudaStreamCreateWithFlags(&d->capture_stream, cudaStreamNonBlocking));
+    cudaStream_t cs = d->capture_stream;
     cudaGraph_t g = nullptr;
-    VV_CUDA(cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed));
-    cudaError_t le = vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s, true, nullptr);
-    cudaError_t ee = cudaStreamEndCapture(s, &g);
+    VV_CUDA(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+    cudaError_t le =
+        vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, cs, true, nullptr);
+    cudaError_t ee = cudaStreamEndCapture(cs, &g);
     if (le != cudaSuccess) {
       if (g) cudaGraphDestroy(g);
       return vv::cuda_check(le, "step capture (launch)");
@@ -388,6 +500,48 @@ vv_status vv_decoder_profile_step(vv_decoder* d, const uint16_t* input_embeds,
   for (auto e : ev)
     if (e) cudaEventDestroy(e);
   return st;
+}
+
+vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
+                                   const int32_t* token_id, const int32_t* position_id,
+                                   uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,
+                                   int32_t* per_cta_out, vv_stream stream) {
+  VV_CHECK_ARG(d && position_id && stamps && grid_out && per_cta_out, "null pointer");
+  VV_CHECK_ARG(input_embeds || token_id, "need input_embeds or token_id");
+  const int need = 14 * d->cfg.layers + 8;
+  if (max_per_cta < need)
+    return set_error(VV_ERR_CAPACITY, "max_per_cta %d < %d", max_per_cta, need);
+  if (d->len_host + 1 > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "KV cache full");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = d->step.grid;
+  uint64_t* dst = nullptr;
+  VV_CUDA(cudaMalloc(&dst, sizeof(uint64_t) * grid * max_per_cta));
+  vv_status st = vv::cuda_check(cudaMemsetAsync(dst, 0, sizeof(uint64_t) * grid * max_per_cta, s),
+                                "memset");
+  vv::StepParams p = d->step;
+  p.input_embeds = reinterpret_cast<const __half*>(input_embeds);
+  p.token = token_id;
+  p.position = position_id;
+  p.logits = nullptr;
+  p.argmax = d->d_argmax;
+  p.trace = d->trace;
+  p.stamps = dst;
+  p.max_stamps = max_per_cta;
+  if (!st) st = vv::cuda_check(vv::launch_step(p, s), "timeline step");
+  if (!st)
+    st = vv::cuda_check(cudaMemcpyAsync(stamps, dst, sizeof(uint64_t) * grid * max_per_cta,
+                                        cudaMemcpyDeviceToHost, s),
+                        "copy stamps");
+  if (!st) st = vv::cuda_check(cudaStreamSynchronize(s), "sync");
+  cudaFree(dst);
+  if (st) return st;
+  int n = 0;
+  while (n < max_per_cta - 3 && stamps[n] != 0) ++n;
+  *grid_out = grid;
+  *per_cta_out = n;
+  d->len_host += 1;
+  return VV_OK;
 }
 
 vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t* position_ids,

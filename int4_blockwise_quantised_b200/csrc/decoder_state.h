@@ -6,6 +6,7 @@
 #include <vector>
 
 #include "../../include/vv.h"
+#include "step.h"
 
 struct vv_decoder {
   vv_config cfg;
@@ -40,7 +41,12 @@ struct vv_decoder {
   int32_t len_host = 0;
   float* trace = nullptr;
   bool use_graph = true;
+  bool use_pdl = true;
+  bool persistent = true;          // one cooperative kernel per step (default)
+  vv::StepParams step = {};        // persistent-kernel parameters (per-call pointers patched)
+  vv::StepLayer* d_layers = nullptr;
   cudaGraphExec_t gexec = nullptr;
+  cudaStream_t capture_stream = nullptr;  // graphs are captured here, launched on the caller's
   const void* gkey[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
 };
 

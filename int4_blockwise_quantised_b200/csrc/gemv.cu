@@ -51,20 +51,35 @@ __device__ void stage_x(float* xs, const float* __restrict__ src32, const __half
                         const __half* __restrict__ gamma, float eps, int K, int tid, int nthreads,
                         float* red_tmp) {
   const int nhb = K >> 4;
+  constexpr int kReg = 4;  // float4 chunks held in registers per thread (K <= 16 * nthreads)
+  auto load4 = [&](int k) -> float4 {
+    if (src32) return __ldcg(reinterpret_cast<const float4*>(src32 + k));
+    const uint2 h = __ldcg(reinterpret_cast<const uint2*>(src16 + k));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  };
+  const bool in_regs = K <= kReg * 4 * nthreads;
+  float4 v[kReg];
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kReg; ++i) {
+      const int k = (tid + i * nthreads) * 4;
+      v[i] = k < K ? load4(k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   float inv = 1.f;
   if (NORM) {
     float ss = 0.f;
-    for (int k = tid * 4; k < K; k += nthreads * 4) {
-      float4 v;
-      if (src32) {
-        v = __ldcg(reinterpret_cast<const float4*>(src32 + k));
-      } else {
-        const uint2 h = __ldcg(reinterpret_cast<const uint2*>(src16 + k));
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
-        v = make_float4(a.x, a.y, b.x, b.y);
+    if (in_regs) {
+#pragma unroll
+      for (int i = 0; i < kReg; ++i)
+        ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    } else {
+      for (int k = tid * 4; k < K; k += nthreads * 4) {
+        const float4 t = load4(k);
+        ss += t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
       }
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     }
     ss = warp_sum(ss);
     if ((tid & 31) == 0) red_tmp[tid >> 5] = ss;
@@ -73,23 +88,23 @@ __device__ void stage_x(float* xs, const float* __restrict__ src32, const __half
     for (int i = 0; i < nthreads / 32; ++i) tot += red_tmp[i];
     inv = rsqrtf(tot / (float)K + eps);
   }
-  for (int k = tid * 4; k < K; k += nthreads * 4) {
-    float v[4];
-    if (src32) {
-      const float4 t = __ldcg(reinterpret_cast<const float4*>(src32 + k));
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else {
-      const uint2 h = __ldcg(reinterpret_cast<const uint2*>(src16 + k));
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
-      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
-      v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-    }
+  auto put = [&](int k, float4 t) {
+    float y[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float y = v[i];
-      if (NORM) y = y * inv * __half2float(gamma[k + i]);
-      xs[x_slot(k + i, nhb)] = y;
+      float yy = y[i];
+      if (NORM) yy = yy * inv * __half2float(gamma[k + i]);
+      xs[x_slot(k + i, nhb)] = yy;
     }
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int i = 0; i < kReg; ++i) {
+      const int k = (tid + i * nthreads) * 4;
+      if (k < K) put(k, v[i]);
+    }
+  } else {
+    for (int k = tid * 4; k < K; k += nthreads * 4) put(k, load4(k));
   }
   compute_bar(nthreads);
 }

@@ -1,0 +1,952 @@
+// Persistent decode-step kernel: the whole decoder_step (all layers + lm_head) in one
+// cooperative launch ("vibevoice-asr-bitnet-onnx": decoder_step contract; "VibeVoice-ASR — ONNX
+// export for Vernacula", section "Highlights": the step's ~1950 launches are the overhead to
+// remove).
+//
+// One CTA per SM.  Warp 0..NW-1 compute, warp NW is the producer.
+//
+// The producer walks a static per-CTA schedule of everything the step streams from HBM -- for each
+// layer: its rows of [Wq;Wk;Wv], its K/V tiles, its rows of Wo, of Wgate+Wup, of Wdown; then its
+// rows of the lm_head -- and moves it with cp.async.bulk into a ring of shared-memory stages.
+// Weights and past K/V do not depend on the step's activations, so the producer never waits for
+// them: HBM keeps streaming across phase boundaries, limited only by the ring's depth.
+//
+// Compute warps walk the same schedule.  Before each phase they pass a grid-wide barrier (the
+// phase's input is an activation vector produced by every CTA), stage that vector in shared
+// memory / registers (with the fused RMSNorm where the layer has one), then consume the phase's
+// stages.  Phases per layer:
+//   QKV  : y = [Wq;Wk;Wv] . RMSNorm(x) + b              -> qkv (fp32)
+//   ATTN : per (kv head, 64-position tile): RoPE(q), RoPE(k_new) + append at slot `length`,
+//          online-softmax partial; the last CTA of a head merges the partials -> attn (fp32)
+//   O    : x += Wo . attn
+//   GU   : h = silu(Wg . RMSNorm(x)) * (Wu . RMSNorm(x))
+//   DOWN : x += Wd . h
+// then HEAD: logits = W_lm . RMSNorm(x), argmax (last CTA reduces), length += 1.
+//
+// The grid barrier is an arrival counter plus a generation word in global memory; every wait is
+// bounded (VV_ERR_TIMEOUT in the device error word after 2 s, then the kernel carries on).  The
+// cooperative launch guarantees that all CTAs are resident.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "vv_device.cuh"
+#include "vv_internal.h"
+#include "step.h"
+
+namespace vv {
+namespace {
+
+constexpr int NW = 15;                 // compute warps (+1 producer: 512 threads, 4-warp register granules)
+constexpr int kThreads = (NW + 1) * 32;
+constexpr int D = 128;
+constexpr int TT = 64;                 // attention tile (positions)
+constexpr int kMaxG = 8;
+constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kRegHB = 3;              // half-blocks per lane held in registers (K <= 1536)
+
+enum Phase { PH_QKV = 0, PH_ATTN, PH_O, PH_GU, PH_DOWN, PH_HEAD };
+
+__device__ __forceinline__ void cbar() {  // compute warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+}
+
+__device__ __forceinline__ void cta_range(int n, int cta, int ncta, int& r0, int& r1) {
+  r0 = (int)((int64_t)n * cta / ncta);
+  r1 = (int)((int64_t)n * (cta + 1) / ncta);
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u32(unsigned* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Timeline tap: thread 0 of each CTA records %globaltimer at fixed points of the schedule
+// (barrier arrival, barrier exit, x staged, end) when p.stamps is set.
+__device__ __forceinline__ void stamp(const StepParams& p, int& k) {
+  if (p.stamps && threadIdx.x == 0) {
+    if (k < p.max_stamps) p.stamps[(size_t)blockIdx.x * p.max_stamps + k] = globaltimer_ns();
+    ++k;
+  }
+}
+
+// Grid-wide barrier among the compute warps of all CTAs.  The arrival counter only grows during
+// a launch (barrier k completes when it reaches (k + 1) * gridDim.x) and the last CTA of the
+// lm_head phase resets it, so an arrival is one fire-and-forget release-add and the wait one
+// acquire poll.  Bounded wait.
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ void grid_barrier(const StepParams& p, unsigned& nbar, int& sk) {
+  cbar();
+  stamp(p, sk);
+  if (threadIdx.x == 0) {
+    const unsigned target = (nbar + 1) * gridDim.x;
+    red_release_add(p.bar_count, 1u);
+    if (ld_acquire_u32(p.bar_count) < target) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_u32(p.bar_count) < target) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          set_device_error(VV_ERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
+  ++nbar;
+  stamp(p, sk);
+  cbar();
+}
+
+// --------------------------------------------------------------------------------- schedule
+// Rows per stage of a packed matrix with K columns (codes + scales per row), nseg matrices per
+// stage (gate/up share a stage).
+__device__ __forceinline__ int packed_row_bytes(int K) { return (K >> 5) * 18; }
+__device__ __forceinline__ int rows_per_stage(int row_bytes, int nseg, int stage_bytes) {
+  int r = stage_bytes / (row_bytes * nseg);
+  return r > 64 ? 64 : r;
+}
+
+// Rows per stage of a phase: bounded by the stage size, and for the split-K (large K) path by
+// kSplitRows so that kSplitRows x kSplitW = NW warps share a stage.
+constexpr int kSplitW = 3;                // warps per row when K is large
+constexpr int kSplitRows = NW / kSplitW;  // 5 rows per stage
+__device__ __forceinline__ int phase_rps(int K, int nseg, int stage_bytes) {
+  const int r = rows_per_stage((K >> 5) * 18, nseg, stage_bytes);
+  return K > 32 * kRegHB * 16 ? min(r, kSplitRows) : r;
+}
+
+struct Ring {
+  uint64_t wait_ns;  // time this thread spent blocked in ring waits (timeline tap)
+  unsigned char* base;
+  uint64_t* full;
+  uint64_t* empty;
+  int stage_bytes;
+  int nstages;
+  int idx;  // running stage counter
+  __device__ unsigned char* slot_ptr(int i) const { return base + (size_t)(i % nstages) * stage_bytes; }
+};
+
+// Producer side of one stage: wait for the slot, post the byte count, issue the copies.
+struct Copy {
+  const void* src;
+  uint32_t bytes;
+  uint32_t dst_off;
+};
+
+// Ring wait with wait-time accounting.
+__device__ __forceinline__ void ring_wait(Ring& r, uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  mbar_wait(bar, parity);
+  r.wait_ns += globaltimer_ns() - t0;
+}
+
+__device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t pol) {
+  const int s = r.idx++;
+  const int slot = s % r.nstages;
+  if (s >= r.nstages) ring_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
+  uint32_t tot = 0;
+  for (int i = 0; i < n; ++i) tot += c[i].bytes;
+  mbar_arrive_expect_tx(&r.full[slot], tot);
+  unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
+  for (int i = 0; i < n; ++i)
+    if (c[i].bytes) bulk_g2s_stream(dst + c[i].dst_off, c[i].src, c[i].bytes, &r.full[slot], pol);
+}
+
+// Stream rows [r0, r1) of a packed matrix (and optionally the same rows of a second one).
+__device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, const uint8_t* q1,
+                               const __half* s1, int K, int r0, int r1, uint64_t pol) {
+  const int nseg = q1 ? 2 : 1;
+  const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
+  const int rps = phase_rps(K, nseg, r.stage_bytes);
+  for (int a = r0; a < r1; a += rps) {
+    const int n = min(rps, r1 - a);
+    Copy c[4];
+    int k = 0;
+    // layout: [seg0 codes (rps rows)][seg1 codes][seg0 scales][seg1 scales]
+    c[k++] = Copy{q0 + (size_t)a * rq, (uint32_t)(n * rq), 0u};
+    if (q1) c[k++] = Copy{q1 + (size_t)a * rq, (uint32_t)(n * rq), (uint32_t)(rps * rq)};
+    c[k++] = Copy{reinterpret_cast<const unsigned char*>(s0) + (size_t)a * rs, (uint32_t)(n * rs),
+                  (uint32_t)(nseg * rps * rq)};
+    if (q1)
+      c[k++] = Copy{reinterpret_cast<const unsigned char*>(s1) + (size_t)a * rs,
+                    (uint32_t)(n * rs), (uint32_t)(nseg * rps * rq + rps * rs)};
+    produce(r, c, k, pol);
+  }
+}
+
+// Tiles (kv head g, tile t) owned by this CTA: items i = cta + k * ncta < Hkv * ntiles.
+__device__ __forceinline__ int ntiles_for(int past) { return (past + 1 + TT - 1) / TT; }
+
+__device__ void producer(const StepParams& p, Ring& r, int past) {
+  const uint64_t pol = policy_evict_first();
+  const int cta = blockIdx.x, ncta = gridDim.x;
+  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv, I = p.I;
+  const int nqkv = (Hq + 2 * Hkv) * D;
+  const int nt = ntiles_for(past);
+  for (int l = 0; l < p.L; ++l) {
+    const StepLayer& w = p.layers[l];
+    // QKV: logical rows [0, nqkv) over the three matrices
+    int r0, r1;
+    cta_range(nqkv, cta, ncta, r0, r1);
+    const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
+    for (int m = 0; m < 3; ++m) {
+      const int a = max(r0, bounds[m]), b = min(r1, bounds[m + 1]);
+      if (a < b) produce_packed(r, w.q[m], w.s[m], nullptr, nullptr, H, a - bounds[m], b - bounds[m], pol);
+    }
+    // ATTN: past K/V rows of the tiles
+    for (int it = cta; it < Hkv * nt; it += ncta) {
+      const int g = it / nt, t = it % nt;
+      const int p0 = t * TT, p1 = min(p0 + TT, past);
+      const uint32_t bytes = p1 > p0 ? (uint32_t)(p1 - p0) * D * 2 : 0u;
+      const size_t off = ((size_t)(l * Hkv + g) * p.cap + p0) * D;
+      Copy c[2] = {Copy{p.k_cache + off, bytes, 0u}, Copy{p.v_cache + off, bytes, TT * D * 2}};
+      produce(r, c, 2, pol);
+    }
+    cta_range(H, cta, ncta, r0, r1);
+    produce_packed(r, w.q[3], w.s[3], nullptr, nullptr, Hq * D, r0, r1, pol);
+    cta_range(I, cta, ncta, r0, r1);
+    produce_packed(r, w.q[4], w.s[4], w.q[5], w.s[5], H, r0, r1, pol);
+    cta_range(H, cta, ncta, r0, r1);
+    produce_packed(r, w.q[6], w.s[6], nullptr, nullptr, I, r0, r1, pol);
+  }
+  // HEAD: fp16 rows of the lm_head
+  int r0, r1;
+  cta_range(p.V, cta, ncta, r0, r1);
+  const int rb = H * 2;
+  const int rps = min(64, r.stage_bytes / rb);
+  for (int a = r0; a < r1; a += rps) {
+    const int n = min(rps, r1 - a);
+    Copy c[1] = {Copy{p.lm_head + (size_t)a * H, (uint32_t)(n * rb), 0u}};
+    produce(r, c, 1, pol);
+  }
+}
+
+// ------------------------------------------------------------------------ compute helpers
+// x staging.  Source fp32 (or fp16 embedding row), optional RMSNorm with fp16 gamma; the result
+// is rounded once to fp16 (the GEMV's activation type) and stored in the half2-pair layout of the
+// dequant-dot: element k (hb = k/16, word = (k/8)%2, j = k%8) goes to uint4 (word * NHB + hb),
+// component j%4, half j/4, i.e. the pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7) of each word.  A warp
+// reading half-blocks hb = lane + 32i touches consecutive 16-byte chunks (no bank conflicts).
+// All compute threads; ends with a compute barrier.
+__device__ __forceinline__ int xh_slot(int k, int nhb) {
+  const int hb = k >> 4, word = (k >> 3) & 1, j = k & 7;
+  return ((word * nhb + hb) * 4 + (j & 3)) * 2 + (j >> 2);
+}
+
+__device__ void stage_x(__half* xs, float* red, const float* src32, const __half* src16,
+                        const __half* gamma, float eps, int K, float* copy_out) {
+  const int tid = threadIdx.x;
+  constexpr int NT = NW * 32;
+  constexpr int kReg = 5;  // float4 chunks per thread kept in registers (K <= 4 * 5 * NT = 9600)
+  const int nhb = K >> 4;
+  auto load4 = [&](int k) -> float4 {
+    if (src32) return __ldcg(reinterpret_cast<const float4*>(src32 + k));
+    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(src16 + k));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  };
+  auto put = [&](int k, float4 t, float inv) {
+    float y[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float u = y[e];
+      if (gamma) u = u * inv * __half2float(gamma[k + e]);
+      xs[xh_slot(k + e, nhb)] = __float2half_rn(u);
+    }
+  };
+  auto norm_inv = [&](float ss) {
+    ss = warp_sum(ss);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    cbar();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) tot += red[i];
+    return rsqrtf(tot / (float)K + eps);
+  };
+  if (K > kReg * 4 * NT) {  // large K (7B down projection): two passes over the source
+    float ss = 0.f;
+    for (int k = tid * 4; k < K; k += NT * 4) {
+      const float4 t = load4(k);
+      if (copy_out) *reinterpret_cast<float4*>(copy_out + k) = t;
+      ss += t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
+    }
+    const float inv = gamma ? norm_inv(ss) : 1.f;
+    for (int k = tid * 4; k < K; k += NT * 4) put(k, load4(k), inv);
+    cbar();
+    return;
+  }
+  float4 v[kReg];
+  uint2 gv[kReg];  // gamma halves, loaded with x so their latency overlaps
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kReg; ++i) {
+    const int k = (tid + i * NT) * 4;
+    if (k < K) {
+      if (gamma) gv[i] = *reinterpret_cast<const uint2*>(gamma + k);
+      v[i] = load4(k);
+      if (copy_out) *reinterpret_cast<float4*>(copy_out + k) = v[i];
+      ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    } else {
+      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  const float inv = gamma ? norm_inv(ss) : 1.f;
+#pragma unroll
+  for (int i = 0; i < kReg; ++i) {
+    const int k = (tid + i * NT) * 4;
+    if (k < K) {
+      float y[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      if (gamma) {
+        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].x));
+        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].y));
+        y[0] *= inv * g01.x;
+        y[1] *= inv * g01.y;
+        y[2] *= inv * g23.x;
+        y[3] *= inv * g23.y;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xs[xh_slot(k + e, nhb)] = __float2half_rn(y[e]);
+    }
+  }
+  cbar();
+}
+
+// Dot of one half-block (8 bytes of codes = 16 columns) with its two x words (half2 pairs).
+__device__ __forceinline__ float hb_doth(uint2 wv, uint4 xa, uint4 xb) {
+  return dot8_h(wv.x, xa) + dot8_h(wv.y, xb);
+}
+
+// Consume the stages of a packed-matrix phase.  fin(row, y0, y1) is called once per output row
+// (y1: the up value of a gate/up pair, nseg = 2).
+//  * K <= 1536 (x in registers xr): each warp takes 4 rows per pass (or 2 gate/up pairs) for
+//    instruction-level parallelism; lanes stride the half-blocks; shuffle reduction.
+//  * larger K (x in shared memory, interleaved): each row is split over kSplitW warps, partial
+//    sums meet in shared memory (red2) and the first warp of the row finishes it.
+template <class Fin>
+__device__ __forceinline__ void consume_packed(Ring& r, const __half* xs, const uint4 (&xr)[kRegHB][2],
+                                               bool regx, int K, int r0, int r1, int nseg,
+                                               float* red2, Fin fin) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KB = K >> 5, NHB = K >> 4;
+  const int rq = KB * 16, rs = KB * 2;
+  const int rps = phase_rps(K, nseg, r.stage_bytes);
+  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+  for (int a = r0; a < r1; a += rps) {
+    const int n = min(rps, r1 - a);
+    const int s = r.idx++;
+    const int slot = s % r.nstages;
+    ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
+    const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
+    const unsigned char* scb = st + (size_t)nseg * rps * rq;
+    auto rowq = [&](int sg, int lr) { return st + (size_t)(sg * rps + lr) * rq; };
+    auto rows = [&](int sg, int lr) {
+      return reinterpret_cast<const __half*>(scb + (size_t)(sg * rps + lr) * rs);
+    };
+    if (regx) {
+      // R = 4 row slots per warp pass: (seg, row) pairs
+      const int units = n * nseg;
+      for (int u0 = warp * 4; u0 < units; u0 += NW * 4) {
+        int sg[4], lr[4];
+        bool ok[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int u = u0 + k;
+          ok[k] = u < units;
+          const int uu = ok[k] ? u : u0;
+          // nseg == 2: units (2i, 2i+1) are (gate i, up i)
+          sg[k] = nseg == 2 ? (uu & 1) : 0;
+          lr[k] = nseg == 2 ? (uu >> 1) : uu;
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kRegHB; ++j) {
+          const int hb = lane + 32 * j;
+          if (hb < NHB) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint2 wv = *reinterpret_cast<const uint2*>(rowq(sg[k], lr[k]) + hb * 8);
+              const float sc = __half2float(rows(sg[k], lr[k])[hb >> 1]);
+              acc[k] = fmaf(sc, hb_doth(wv, xr[j][0], xr[j][1]), acc[k]);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = warp_sum(acc[k]);
+        if (lane == 0) {
+          if (nseg == 2) {
+            if (ok[0]) fin(a + lr[0], acc[0], acc[1]);
+            if (ok[2]) fin(a + lr[2], acc[2], acc[3]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (ok[k]) fin(a + lr[k], acc[k], 0.f);
+          }
+        }
+      }
+    } else {
+      // split-K: warp w -> row w / kSplitW, slice w % kSplitW
+      const int lrow = warp / kSplitW, slice = warp % kSplitW;
+      float acc0 = 0.f, acc1 = 0.f;
+      if (lrow < n) {
+        const unsigned char* q0 = rowq(0, lrow);
+        const __half* sc0 = rows(0, lrow);
+        const unsigned char* q1 = rowq(nseg - 1, lrow);
+        const __half* sc1 = rows(nseg - 1, lrow);
+        for (int hb = lane + 32 * slice; hb < NHB; hb += 32 * kSplitW) {
+          const uint4 xa = xs4[hb], xb = xs4[NHB + hb];
+          const uint2 w0 = *reinterpret_cast<const uint2*>(q0 + hb * 8);
+          acc0 = fmaf(__half2float(sc0[hb >> 1]), hb_doth(w0, xa, xb), acc0);
+          if (nseg == 2) {
+            const uint2 w1 = *reinterpret_cast<const uint2*>(q1 + hb * 8);
+            acc1 = fmaf(__half2float(sc1[hb >> 1]), hb_doth(w1, xa, xb), acc1);
+          }
+        }
+      }
+      acc0 = warp_sum(acc0);
+      acc1 = warp_sum(acc1);
+      if (lane == 0) {
+        red2[warp * 2 + 0] = acc0;
+        red2[warp * 2 + 1] = acc1;
+      }
+      cbar();
+      if (lane == 0 && slice == 0 && lrow < n) {
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < kSplitW; ++k) {
+          y0 += red2[(warp + k) * 2 + 0];
+          y1 += red2[(warp + k) * 2 + 1];
+        }
+        fin(a + lrow, y0, y1);
+      }
+      cbar();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.empty[slot]);
+  }
+}
+
+// Preload the lane's half-blocks of x (fp16 pair layout in xs) into registers.
+__device__ __forceinline__ void load_xr(const __half* xs, uint4 (&xr)[kRegHB][2], int K) {
+  const int lane = threadIdx.x & 31;
+  const int NHB = K >> 4;
+  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+#pragma unroll
+  for (int j = 0; j < kRegHB; ++j) {
+    const int hb = lane + 32 * j;
+    xr[j][0] = hb < NHB ? xs4[hb] : make_uint4(0u, 0u, 0u, 0u);
+    xr[j][1] = hb < NHB ? xs4[NHB + hb] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+struct AttnScratch {
+  float cs[D / 2], sn[D / 2];  // RoPE cos/sin at this step's position
+  float q[kMaxG][D];
+  float s[kMaxG][TT];
+  float m[kMaxG], l[kMaxG];
+  float mw[256][kMaxG];
+  int is_last;
+};
+
+// One attention tile item: scores, softmax, P.V for the G heads of kv head g.
+__device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
+                          int past, int pos) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.Hq / p.Hkv;
+  const int nt = ntiles_for(past);
+  const int npos = past + 1;
+  const int p0 = t * TT;
+  const int n = min(TT, npos - p0);
+  const float* qkv = p.qkv;
+  // q of the group, rotated and scaled into the log2 domain
+  const float qscale = p.scale * kLog2e;
+  for (int i = tid; i < G * D; i += NW * 32) {
+    const int h = i / D, d = i % D;
+    const float* qh = qkv + (size_t)(g * G + h) * D;
+    const int fi = d & (D / 2 - 1);
+    const float cs = as.cs[fi], sn = as.sn[fi];
+    const float x1 = __ldcg(qh + fi), x2 = __ldcg(qh + fi + D / 2);
+    as.q[h][d] = (d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn) * qscale;
+  }
+  const int s = r.idx++;
+  const int slot = s % r.nstages;
+  ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
+  __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
+  __half* vt = kt + TT * D;
+  if (t == nt - 1 && tid < D) {  // this tile holds the new position: rotate k, append k/v
+    const int d = tid;
+    const float* kh = qkv + (size_t)(p.Hq + g) * D;
+    const float* vh = qkv + (size_t)(p.Hq + p.Hkv + g) * D;
+    const int fi = d & (D / 2 - 1);
+    const float cs = as.cs[fi], sn = as.sn[fi];
+    const float x1 = __ldcg(kh + fi), x2 = __ldcg(kh + fi + D / 2);
+    const __half kn = __float2half_rn(d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn);
+    const __half vn = __float2half_rn(__ldcg(vh + d));
+    const size_t off = ((size_t)(l * p.Hkv + g) * p.cap + past) * D + d;
+    p.k_cache[off] = kn;
+    p.v_cache[off] = vn;
+    kt[(past - p0) * D + d] = kn;
+    vt[(past - p0) * D + d] = vn;
+  }
+  cbar();
+  // scores: warp w -> head w/2, positions (w%2)*32 + lane; chunk order rotated by lane so the
+  // 16-byte k loads of a warp hit distinct banks.
+  for (int item = warp; item < 2 * G; item += NW) {
+    const int h = item >> 1, pp = (item & 1) * 32 + lane;
+    {
+      float sc = -INFINITY;
+      if (pp < n) {
+        const __half* kr = kt + pp * D;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          const int cc = (c + lane) & 15;
+          const uint4 kv = *reinterpret_cast<const uint4*>(kr + cc * 8);
+          const float4 qa = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
+          const float4 qb = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
+          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa.x, qa.y), acc);
+          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa.z, qa.w), acc);
+          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb.x, qb.y), acc);
+          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb.z, qb.w), acc);
+        }
+        sc = acc.x + acc.y;
+      }
+      as.s[h][pp] = sc;
+    }
+  }
+  cbar();
+  if (warp < G) {  // softmax statistics of this tile, per head
+    const int h = warp;
+    const float s0 = as.s[h][lane], s1 = as.s[h][lane + 32];
+    const float mt = warp_max(fmaxf(s0, s1));
+    const float e0 = lane < n ? exp2f(s0 - mt) : 0.f;
+    const float e1 = lane + 32 < n ? exp2f(s1 - mt) : 0.f;
+    as.s[h][lane] = e0;
+    as.s[h][lane + 32] = e1;
+    const float sum = warp_sum(e0 + e1);
+    if (lane == 0) {
+      as.m[h] = mt;
+      as.l[h] = sum;
+    }
+  }
+  cbar();
+  // P.V: (head, dim) pairs over all compute threads
+  {
+    float* part = p.attn_part + ((size_t)(g * p.max_tiles + t) * kMaxG) * kPart;
+    for (int idx = tid; idx < G * D; idx += NW * 32) {
+      const int h = idx >> 7, d = idx & (D - 1);
+      float o = 0.f;
+      const float* ph = as.s[h];
+      for (int pp = 0; pp < n; ++pp) o = fmaf(ph[pp], __half2float(vt[pp * D + d]), o);
+      part[h * kPart + 4 + d] = o;
+    }
+    if (tid < G) {
+      part[tid * kPart + 0] = as.m[tid];
+      part[tid * kPart + 1] = as.l[tid];
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&r.empty[slot]);
+  // publish; the last tile of head g to finish merges all of g's partials
+  __threadfence();
+  cbar();
+  if (tid == 0) {
+    const int prev = atomicAdd(&p.attn_count[g], 1);
+    as.is_last = prev == nt - 1;
+  }
+  cbar();
+  if (!as.is_last) return;
+  __threadfence();
+  const float* base = p.attn_part + (size_t)g * p.max_tiles * kMaxG * kPart;
+  if (warp < G) {
+    const int h = warp;
+    float mx = -INFINITY;
+    for (int c = lane; c < nt; c += 32) mx = fmaxf(mx, __ldcg(base + ((size_t)c * kMaxG + h) * kPart));
+    mx = warp_max(mx);
+    float L = 0.f;
+    for (int c = lane; c < nt; c += 32) {
+      const float* pp = base + ((size_t)c * kMaxG + h) * kPart;
+      const float e = exp2f(__ldcg(pp) - mx);
+      as.mw[c][h] = e;
+      L += __ldcg(pp + 1) * e;
+    }
+    L = warp_sum(L);
+    const float inv = 1.f / L;
+    for (int c = lane; c < nt; c += 32) as.mw[c][h] *= inv;
+  }
+  cbar();
+  for (int idx = tid; idx < G * D; idx += NW * 32) {
+    const int h = idx >> 7, d = idx & (D - 1);
+    float acc = 0.f;
+    for (int c0 = 0; c0 < nt; c0 += 16) {
+      const int m = min(16, nt - c0);
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        v[u] = u < m ? __ldcg(base + ((size_t)(c0 + u) * kMaxG + h) * kPart + 4 + d) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (u < m) acc = fmaf(as.mw[c0 + u][h], v[u], acc);
+    }
+    p.attn_out[(size_t)(g * G + h) * D + d] = acc;
+  }
+  if (tid == 0) p.attn_count[g] = 0;
+}
+
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  Ring r;
+  r.wait_ns = 0;
+  r.base = smem;
+  r.stage_bytes = p.stage_bytes;
+  r.nstages = p.nstages;
+  r.idx = 0;
+  __half* xs = reinterpret_cast<__half*>(smem + (size_t)p.nstages * p.stage_bytes);
+  AttnScratch& as = *reinterpret_cast<AttnScratch*>(smem + (size_t)p.nstages * p.stage_bytes +
+                                                     (size_t)p.x_floats * 4);
+  float* red = reinterpret_cast<float*>(&as + 1);  // [64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 64) + 15) &
+                                               ~uintptr_t(15));
+  r.full = bars;
+  r.empty = bars + p.nstages;
+  __shared__ float s_val[NW];
+  __shared__ int s_idx[NW];
+  __shared__ int s_last;
+
+  const int past = *p.length;
+  if (tid == 0) {
+    for (int i = 0; i < p.nstages; ++i) {
+      mbar_init(&r.full[i], 1);
+      mbar_init(&r.empty[i], NW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == NW) {
+    if (lane == 0) {
+      producer(p, r, past);
+      if (p.stamps) {
+        uint64_t* row = p.stamps + (size_t)blockIdx.x * p.max_stamps;
+        row[p.max_stamps - 1] = r.wait_ns;          // producer blocked on free slots
+        row[p.max_stamps - 2] = globaltimer_ns();   // producer done issuing
+      }
+    }
+    return;
+  }
+
+  // ----------------------------------------------------------------------------- compute
+  unsigned gen = 0;  // barriers passed in this launch
+  int sk = 0;        // timeline stamp index
+  stamp(p, sk);
+  const int cta = blockIdx.x, ncta = gridDim.x;
+  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv, I = p.I;
+  const int nqkv = (Hq + 2 * Hkv) * D;
+  const int nt = ntiles_for(past);
+  int pos = *p.position;
+  if (pos < 0 || pos >= p.max_position) {
+    if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
+    pos = min(max(pos, 0), p.max_position - 1);
+  }
+  uint4 xr[kRegHB][2];
+  for (int i = tid; i < D / 2; i += NW * 32) {
+    as.cs[i] = p.rope_cos[(size_t)pos * (D / 2) + i];
+    as.sn[i] = p.rope_sin[(size_t)pos * (D / 2) + i];
+  }
+  // This CTA's rows of the residual (the o-proj and down phases update exactly these rows).
+  int hr0, hr1;
+  cta_range(H, cta, ncta, hr0, hr1);
+  float* xown = red + 32;  // up to 32 rows (H <= 32 * gridDim.x)
+
+  for (int l = 0; l < p.L; ++l) {
+    const StepLayer& w = p.layers[l];
+    // ---------------------------------------------------------------- QKV
+    if (l == 0) {
+      const __half* e16 = p.input_embeds;
+      if (!e16) {
+        int tok = __ldcg(p.token);
+        if (tok < 0 || tok >= p.V) {
+          if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
+          tok = min(max(tok, 0), p.V - 1);
+        }
+        e16 = p.embed + (size_t)tok * H;
+      }
+      for (int i = tid; i < hr1 - hr0; i += NW * 32) xown[i] = __half2float(e16[hr0 + i]);
+      stage_x(xs, red, nullptr, e16, w.in_norm, p.eps, H, cta == 0 ? p.x_resid : nullptr);
+      stamp(p, sk);
+    } else {
+      grid_barrier(p, gen, sk);
+      stage_x(xs, red, p.x_resid, nullptr, w.in_norm, p.eps, H, nullptr);
+      stamp(p, sk);
+    }
+    const bool regH = H <= 32 * kRegHB * 16;
+    {
+      int r0, r1;
+      cta_range(nqkv, cta, ncta, r0, r1);
+      const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
+      // this CTA's q/k/v biases -> shared memory (as.q is free until the attention phase)
+      float* bias_s = &as.q[0][0];
+      for (int i = tid; i < r1 - r0; i += NW * 32) {
+        const int row = r0 + i;
+        const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
+        const __half* b = w.bias[m];
+        bias_s[i] = b ? __half2float(b[row - bounds[m]]) : 0.f;
+      }
+      if (regH) load_xr(xs, xr, H);
+      cbar();
+      for (int m = 0; m < 3; ++m) {
+        const int a = max(r0, bounds[m]), b = min(r1, bounds[m + 1]);
+        if (a < b) {
+          float* out = p.qkv + bounds[m];
+          const float* bs = bias_s + (bounds[m] - r0);
+          consume_packed(r, xs, xr, regH, H, a - bounds[m], b - bounds[m], 1, &as.s[0][0],
+                         [&](int row, float y, float) { out[row] = y + bs[row]; });
+        }
+      }
+    }
+    // ---------------------------------------------------------------- ATTN
+    grid_barrier(p, gen, sk);
+    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, pos);
+    // ---------------------------------------------------------------- O
+    grid_barrier(p, gen, sk);
+    stage_x(xs, red, p.attn_out, nullptr, nullptr, 0.f, Hq * D, nullptr);
+    stamp(p, sk);
+    const bool regO = Hq * D <= 32 * kRegHB * 16;
+    if (regO) load_xr(xs, xr, Hq * D);
+    {
+      int r0, r1;
+      cta_range(H, cta, ncta, r0, r1);
+      consume_packed(r, xs, xr, regO, Hq * D, r0, r1, 1, &as.s[0][0], [&](int row, float y, float) {
+        const float v = xown[row - hr0] + y;
+        xown[row - hr0] = v;
+        p.x_resid[row] = v;
+      });
+    }
+    // ---------------------------------------------------------------- GU
+    grid_barrier(p, gen, sk);
+    stage_x(xs, red, p.x_resid, nullptr, w.post_norm, p.eps, H, nullptr);
+    stamp(p, sk);
+    if (regH) load_xr(xs, xr, H);
+    {
+      int r0, r1;
+      cta_range(I, cta, ncta, r0, r1);
+      consume_packed(r, xs, xr, regH, H, r0, r1, 2, &as.s[0][0], [&](int row, float g, float u) {
+        p.h[row] = g / (1.f + __expf(-g)) * u;
+      });
+    }
+    // ---------------------------------------------------------------- DOWN
+    grid_barrier(p, gen, sk);
+    stage_x(xs, red, p.h, nullptr, nullptr, 0.f, I, nullptr);
+    stamp(p, sk);
+    {
+      int r0, r1;
+      cta_range(H, cta, ncta, r0, r1);
+      float* tr = p.trace ? p.trace + (size_t)l * H : nullptr;
+      consume_packed(r, xs, xr, false, I, r0, r1, 1, &as.s[0][0], [&](int row, float y, float) {
+        const float v = xown[row - hr0] + y;
+        xown[row - hr0] = v;
+        p.x_resid[row] = v;
+        if (tr) tr[row] = v;
+      });
+    }
+  }
+  // ------------------------------------------------------------------------------ HEAD
+  grid_barrier(p, gen, sk);
+  stage_x(xs, red, p.x_resid, nullptr, p.final_norm, p.eps, H, nullptr);
+  stamp(p, sk);
+  float best = -INFINITY;
+  int best_i = 0x7fffffff;
+  {
+    int r0, r1;
+    cta_range(p.V, cta, ncta, r0, r1);
+    const int rb = H * 2;
+    const int rps = min(64, r.stage_bytes / rb);
+    const int nch = H >> 3;  // 16-byte chunks per row
+    // x of 16-byte weight chunk c (8 columns: half-block c/2, word c%2) = pair word (c%2, c/2);
+    // held in registers for c = lane + 32 j when the row fits (H <= 1536)
+    const int nhb = H >> 4;
+    const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+    const bool regHead = nch <= 32 * 2 * kRegHB;
+    if (regHead) {
+#pragma unroll
+      for (int j = 0; j < 2 * kRegHB; ++j) {
+        const int c = lane + 32 * j;
+        xr[j >> 1][j & 1] = c < nch ? xs4[(c & 1) * nhb + (c >> 1)] : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    for (int a = r0; a < r1; a += rps) {
+      const int n = min(rps, r1 - a);
+      const int s = r.idx++;
+      const int slot = s % r.nstages;
+      ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
+      const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
+      for (int i = warp; i < n; i += NW) {
+        const unsigned char* row = st + (size_t)i * rb;
+        float acc = 0.f;
+        // weights (w0,w1)(w2,w3)(w4,w5)(w6,w7) against x pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7)
+        auto chunk = [&](const uint4 wv, const uint4 xv) {
+          uint32_t p04, p15, p26, p37;
+          asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(p04) : "r"(wv.x), "r"(wv.z));
+          asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(p15) : "r"(wv.x), "r"(wv.z));
+          asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(p26) : "r"(wv.y), "r"(wv.w));
+          asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(p37) : "r"(wv.y), "r"(wv.w));
+          acc = fma2_f16_f32(p04, xv.x, acc);
+          acc = fma2_f16_f32(p15, xv.y, acc);
+          acc = fma2_f16_f32(p26, xv.z, acc);
+          acc = fma2_f16_f32(p37, xv.w, acc);
+        };
+        if (regHead) {
+#pragma unroll
+          for (int j = 0; j < 2 * kRegHB; ++j) {
+            const int c = lane + 32 * j;
+            if (c < nch) chunk(*reinterpret_cast<const uint4*>(row + c * 16), xr[j >> 1][j & 1]);
+          }
+        } else {
+          for (int c = lane; c < nch; c += 32)
+            chunk(*reinterpret_cast<const uint4*>(row + c * 16), xs4[(c & 1) * nhb + (c >> 1)]);
+        }
+        const float v = warp_sum(acc);
+        if (lane == 0) {
+          const int vr = a + i;
+          if (p.logits) p.logits[vr] = v;
+          if (better(v, vr, best, best_i)) {
+            best = v;
+            best_i = vr;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&r.empty[slot]);
+    }
+  }
+  if (lane == 0) {
+    s_val[warp] = best;
+    s_idx[warp] = best_i;
+  }
+  cbar();
+  stamp(p, sk);
+  if (tid == 0) {
+    float bv = s_val[0];
+    int bi = s_idx[0];
+    for (int w2 = 1; w2 < NW; ++w2)
+      if (better(s_val[w2], s_idx[w2], bv, bi)) {
+        bv = s_val[w2];
+        bi = s_idx[w2];
+      }
+    p.head_val[cta] = bv;
+    p.head_idx[cta] = bi;
+    __threadfence();
+    s_last = atomicAdd(p.head_count, 1) == ncta - 1;
+  }
+  cbar();
+  if (!s_last) return;
+  __threadfence();
+  if (warp == 0) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = lane; i < ncta; i += 32) {
+      const float v = __ldcg(p.head_val + i);
+      const int ix = __ldcg(p.head_idx + i);
+      if (better(v, ix, bv, bi)) {
+        bv = v;
+        bi = ix;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      *p.argmax = bi == 0x7fffffff ? 0 : bi;
+      *p.head_count = 0;
+      *p.bar_count = 0u;  // every CTA has passed every barrier of this launch
+      *p.length = past + 1;
+    }
+  }
+}
+
+}  // namespace
+
+size_t step_smem_bytes(int stage_bytes, int nstages, int x_floats) {
+  return (size_t)nstages * stage_bytes + (size_t)x_floats * 4 + sizeof(AttnScratch) + 64 * 4 +
+         2 * nstages * 8 + 64;
+}
+
+int step_threads() { return kThreads; }
+
+size_t step_attn_part_floats(int Hkv, int max_tiles) {
+  return (size_t)Hkv * max_tiles * kMaxG * kPart;
+}
+
+int step_max_tiles(int cap) { return (cap + TT - 1) / TT; }
+
+// Pick the largest stage size (>= 32 KB, 1 KB steps) for which one CTA per SM is resident.
+cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
+  cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  *blocks_per_sm = 0;
+  for (; p.stage_bytes >= 32 * 1024; p.stage_bytes -= 1024) {
+    const size_t smem = step_smem_bytes(p.stage_bytes, p.nstages, p.x_floats);
+    e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    int nb = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, step_kernel, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (nb >= 1) {
+      *blocks_per_sm = nb;
+      return cudaSuccess;
+    }
+  }
+  return cudaSuccess;
+}
+
+void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_bytes) {
+  cudaFuncAttributes fa = {};
+  cudaFuncGetAttributes(&fa, step_kernel);
+  *regs = fa.numRegs;
+  *max_threads = fa.maxThreadsPerBlock;
+  *static_smem = (int)fa.sharedSizeBytes;
+  *local_bytes = (int)fa.localSizeBytes;
+}
+
+cudaError_t launch_step(const StepParams& p, cudaStream_t s) {
+  const size_t smem = step_smem_bytes(p.stage_bytes, p.nstages, p.x_floats);
+  cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, step_kernel, p);
+}
+
+}  // namespace vv

@@ -1,0 +1,69 @@
+// Parameters of the persistent decode-step kernel (internal).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vv {
+
+struct StepLayer {
+  const __half* in_norm;
+  const __half* post_norm;
+  const uint8_t* q[7];   // wq, wk, wv, wo, wgate, wup, wdown codes
+  const __half* s[7];    // their scales
+  const __half* bias[3]; // bq, bk, bv
+};
+
+struct StepParams {
+  int H, L, Hq, Hkv, I, V;
+  float eps, scale;
+  const StepLayer* layers;  // device array [L]
+  const __half* embed;
+  const __half* lm_head;
+  const __half* final_norm;
+  __half* k_cache;
+  __half* v_cache;
+  int cap;
+  const float* rope_cos;
+  const float* rope_sin;
+  int max_position;
+  // per-step inputs / outputs
+  const __half* input_embeds;  // or nullptr -> embed[*token]
+  const int32_t* token;
+  const int32_t* position;
+  float* logits;     // may be nullptr
+  int32_t* argmax;
+  float* trace;      // [L, H] or nullptr
+  // workspace
+  float* x_resid;
+  float* qkv;
+  float* attn_out;
+  float* h;
+  float* attn_part;
+  int* attn_count;
+  int max_tiles;
+  float* head_val;
+  int* head_idx;
+  int* head_count;
+  int32_t* length;
+  unsigned* bar_count;
+  unsigned* bar_gen;
+  uint64_t* stamps;   // timeline tap [grid][max_stamps] (globaltimer ns) or nullptr
+  int max_stamps;
+  // launch shape
+  int grid;
+  int stage_bytes;
+  int nstages;
+  int x_floats;
+};
+
+size_t step_smem_bytes(int stage_bytes, int nstages, int x_floats);
+int step_threads();
+size_t step_attn_part_floats(int Hkv, int max_tiles);
+int step_max_tiles(int cap);
+cudaError_t step_configure(StepParams& p, int* blocks_per_sm);
+void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_bytes);
+cudaError_t launch_step(const StepParams& p, cudaStream_t s);
+
+}  // namespace vv

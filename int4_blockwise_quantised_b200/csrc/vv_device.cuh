@@ -170,6 +170,51 @@ __device__ __forceinline__ float2 dot8_nbits(uint32_t w, float4 x8e, float4 x8o,
   return acc;
 }
 
+// ----------------------------------------------------------------------------------------------
+// int4 dequant-dot, half2 form.  One 32-bit word of codes (elements 0..7) is unpacked with the
+// 0x6400 (= 1024.0 in fp16) magic: lop3 places nibble pairs (0,4), (1,5), (2,6), (3,7) into the
+// mantissas of two fp16 lanes, then one packed add/fma removes the bias, which yields the exact
+// values (code - 8) in fp16.  Products with fp16 activations are formed by the mixed-precision
+// fma.rn.f32.f16 (both factors fp16, exact product, fp32 accumulate), so nothing is rounded but
+// the fp32 sums.  x8 holds the activations as half2 pairs (x0,x4), (x1,x5), (x2,x6), (x3,x7).
+__device__ __forceinline__ void unpack8_h2(uint32_t w, uint32_t (&d)[4]) {
+  const uint32_t w8 = w >> 8;
+  uint32_t h0, h1, h2, h3;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h0) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h1) : "r"(w), "r"(0x00F000F0u), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h2) : "r"(w8), "r"(0x000F000Fu), "r"(0x64006400u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h3) : "r"(w8), "r"(0x00F000F0u), "r"(0x64006400u));
+  // (1024 + c) - 1032 = c - 8;  (1024 + 16c) / 16 - 72 = c - 8   (all exact in fp16)
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d[0]) : "r"(h0), "r"(0x64086408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d[1]) : "r"(h1), "r"(0x2C002C00u), "r"(0xD480D480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d[2]) : "r"(h2), "r"(0x64086408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d[3]) : "r"(h3), "r"(0x2C002C00u), "r"(0xD480D480u));
+}
+
+// acc += a.lo * b.lo + a.hi * b.hi with fp16 factors and an fp32 accumulator.
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float acc) {
+  asm("{\n\t.reg .f16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a), "r"(b));
+  return acc;
+}
+
+// Exact sum over one word: sum_i (code_i - 8) * x_i in fp32.
+__device__ __forceinline__ float dot8_h(uint32_t w, uint4 x8) {
+  uint32_t d[4];
+  unpack8_h2(w, d);
+  float acc = 0.f;
+  acc = fma2_f16_f32(d[0], x8.x, acc);
+  acc = fma2_f16_f32(d[1], x8.y, acc);
+  acc = fma2_f16_f32(d[2], x8.z, acc);
+  acc = fma2_f16_f32(d[3], x8.w, acc);
+  return acc;
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint16_t b) {
   return __half2float(__ushort_as_half(b));
 }

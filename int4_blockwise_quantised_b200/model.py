@@ -147,6 +147,20 @@ class Decoder:
                                               stream_handle(stream)))
         return dict(zip(self.PHASES, list(out)))
 
+    def step_timeline(self, position, input_embeds=None, token=None, stream=None):
+        """One persistent step with the timeline tap; returns uint64 ns array [grid, stamps]."""
+        maxn = 14 * self.model.shape.layers + 16
+        grid_max = 1024
+        buf = np.zeros(grid_max * maxn, dtype=np.uint64)
+        g = ctypes.c_int32()
+        n = ctypes.c_int32()
+        check(_vv.lib.vv_decoder_step_timeline(self.handle, ptr(input_embeds), ptr(token),
+                                               ptr(position), buf.ctypes.data, maxn,
+                                               ctypes.byref(g), ctypes.byref(n),
+                                               stream_handle(stream)))
+        full = buf[: g.value * maxn].reshape(g.value, maxn)
+        return full[:, : n.value], full
+
     def init(self, input_ids, position_ids, audio_features=None, audio_offset=0, logits=None,
              argmax=None, stream=None):
         S = input_ids.numel()

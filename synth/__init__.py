@@ -50,7 +50,7 @@ class Shape:
 SHAPE_1P5B = Shape("qwen2-1.5b", 1536, 28, 12, 2, 128, 8960, 151936, tied=True)
 SHAPE_7B = Shape("qwen2-7b", 3584, 28, 28, 4, 128, 18944, 152064, tied=False)
 # Small shapes for fast parity runs; several tiles and a ragged tail on every axis that has one.
-SHAPE_TINY = Shape("tiny", 256, 2, 4, 2, 128, 640, 1000, tied=True)
+SHAPE_TINY = Shape("tiny", 256, 2, 4, 2, 128, 768, 1000, tied=True)
 SHAPE_SMALL = Shape("small", 1536, 2, 12, 2, 128, 8960, 4099, tied=True)
 
 

@@ -125,8 +125,11 @@ def test_gemv_multirow(vv, M):
 def _attn_case(vv, Hq, Hkv, length, cap, seed, kscale=1.0):
     D = 128
     q = synth.normal_f16((Hq, D), 1.0, seed)
-    K = synth.normal_f16((Hkv, cap, D), kscale, seed + 1)
-    V = synth.normal_f16((Hkv, cap, D), 1.0, seed + 2)
+    # the valid positions are drawn independently of `cap`; slots past `length` stay zero
+    K = np.zeros((Hkv, cap, D), np.float16)
+    V = np.zeros((Hkv, cap, D), np.float16)
+    K[:, :length] = synth.normal_f16((Hkv, length, D), kscale, seed + 1)
+    V[:, :length] = synth.normal_f16((Hkv, length, D), 1.0, seed + 2)
     ref = oops.gqa_decode_attention(q.astype(np.float64), K[:, :length].astype(np.float64),
                                     V[:, :length].astype(np.float64), 1 / math.sqrt(D))
     ws = torch.zeros(vv.vv_gqa_decode_attn_workspace_size(Hq, Hkv, D, cap), dtype=torch.uint8,
