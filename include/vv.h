@@ -122,6 +122,28 @@ vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cache, const u
                              float scale, uint16_t* out, void* ws, size_t ws_bytes,
                              vv_stream stream);
 
+/* Same operation, arguments and requirements as vv_gqa_decode_attn, for callers that cannot
+ * allocate device memory when they run attention (an application that has given its whole GPU
+ * memory budget to its own pool, a real-time audio thread that may not call cudaMalloc because it
+ * can block and synchronise the device, a plugin that may not own allocations).  No workspace
+ * argument: the scratch (split-K partials and arrival counters) is a file-scope device array of
+ * 256 KiB that every GPU loading this library holds until the process exits.  No counterpart in
+ * the pages: this is a property of this library, not of the method.
+ *  - The first call on a device looks up the array's device address with that device current;
+ *    make that first call before any stream capture.
+ *  - The call allocates nothing (no cudaMalloc/cudaFree); it clears the arrival counters with
+ *    cudaMemsetAsync on `stream` and then launches the kernel.
+ *  - All calls share the one array, which keeps the previous call's partials: calls that overlap
+ *    on the GPU (different streams without ordering) race and corrupt each other's results.
+ *  - Errors: as vv_gqa_decode_attn, plus VV_ERR_CAPACITY when the shape needs more scratch than
+ *    the array holds: Hkv x chunks x 8 x 132 floats + 256 bytes must fit in 256 KiB, i.e.
+ *    Hkv x chunks <= 62 (chunks = min(ceil(cap/64), SMs/Hkv)); with 2 KV heads that is a cache of
+ *    up to 1984 positions, with 4 KV heads up to 960. */
+vv_status vv_gqa_decode_attn_noalloc(const uint16_t* q, const uint16_t* k_cache,
+                                     const uint16_t* v_cache, int32_t len, int32_t cap, int32_t Hq,
+                                     int32_t Hkv, int32_t D, float scale, uint16_t* out,
+                                     vv_stream stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Final RMSNorm + fp16 lm_head + greedy argmax ([BITNET]: lm_head stays fp16, greedy decode;
  * [STATUS] "Inference (ONNX)": logits = hidden . embed^T with the tied table).

@@ -75,6 +75,8 @@ def _load():
         "vv_gqa_decode_attn_workspace_size": (c_size_t, [c_int32, c_int32, c_int32, c_int32]),
         "vv_gqa_decode_attn": (S, [P, P, P, c_int32, c_int32, c_int32, c_int32, c_int32, c_float,
                                    P, P, c_size_t, P]),
+        "vv_gqa_decode_attn_noalloc": (S, [P, P, P, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                           c_float, P, P]),
         "vv_lm_head_argmax_workspace_size": (c_size_t, [c_int64]),
         "vv_lm_head_argmax": (S, [P, P, P, c_int64, c_int64, c_float, P, P, P, c_size_t, P]),
         "vv_decoder_create": (S, [POINTER(vv_config), POINTER(vv_model_weights), P, P,
@@ -192,6 +194,16 @@ def vv_gqa_decode_attn(q, k_cache, v_cache, length, scale, ws, stream=None, out=
     check(lib.vv_gqa_decode_attn(ptr(q), ptr(k_cache), ptr(v_cache), length, cap, Hq, Hkv, D,
                                  scale, ptr(o), ptr(ws), ws.numel() * ws.element_size(),
                                  stream_handle(stream)))
+    return o
+
+
+def vv_gqa_decode_attn_noalloc(q, k_cache, v_cache, length, scale, stream=None, out=None):
+    """Like vv_gqa_decode_attn, with the library's static scratch instead of a workspace."""
+    Hq, D = q.shape
+    Hkv, cap, _ = k_cache.shape
+    o = out if out is not None else torch.empty_like(q)
+    check(lib.vv_gqa_decode_attn_noalloc(ptr(q), ptr(k_cache), ptr(v_cache), length, cap, Hq, Hkv,
+                                         D, scale, ptr(o), stream_handle(stream)))
     return o
 
 

@@ -19,6 +19,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "vv_device.cuh"
 #include "vv_internal.h"
 
@@ -394,4 +396,78 @@ extern "C" vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cac
   a.nchunks = nch;
   return vv::cuda_check(vv::launch_attn(a, false, static_cast<cudaStream_t>(stream), false),
                         "attention launch");
+}
+
+// ------------------------------------------------------------------------------------------------
+// Scratch-free variant of vv_gqa_decode_attn.
+//
+// Some callers cannot allocate device memory at the point where they run attention: a host
+// application that has handed the whole GPU memory budget to its own pool (a serving engine that
+// pre-reserves the KV cache, a real-time audio pipeline that forbids allocation on its processing
+// thread because cudaMalloc can block and synchronise the device), or a plugin that is not
+// allowed to create allocations of its own.  For them the split-K partials and arrival counters
+// live in one file-scope device array instead of a caller workspace.  Every GPU that loads this
+// library holds the array (kNoAllocScratchBytes) until the process exits.
+namespace vv {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(256) << 10;  // 256 KiB
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};  // device address of the array, per device ordinal
+}  // namespace
+}  // namespace vv
+
+static __device__ __align__(256) unsigned char g_attn_scratch[vv::kNoAllocScratchBytes];
+
+extern "C" vv_status vv_gqa_decode_attn_noalloc(const uint16_t* q, const uint16_t* k_cache,
+                                                const uint16_t* v_cache, int32_t len, int32_t cap,
+                                                int32_t Hq, int32_t Hkv, int32_t D_, float scale,
+                                                uint16_t* out, vv_stream stream) {
+  VV_CHECK_ARG(q && k_cache && v_cache && out, "vv_gqa_decode_attn_noalloc: null pointer");
+  VV_CHECK_ARG(vv::aligned16(q) && vv::aligned16(k_cache) && vv::aligned16(v_cache) &&
+                   vv::aligned16(out),
+               "vv_gqa_decode_attn_noalloc: pointers must be 16-byte aligned");
+  VV_CHECK_SHAPE(D_ == 128, "vv_gqa_decode_attn_noalloc: D=%d (only 128)", D_);
+  VV_CHECK_SHAPE(Hkv >= 1 && Hkv <= 64 && Hq >= Hkv && Hq % Hkv == 0 && Hq / Hkv <= 8,
+                 "vv_gqa_decode_attn_noalloc: Hq=%d Hkv=%d", Hq, Hkv);
+  VV_CHECK_SHAPE(cap >= 1 && len >= 1 && len <= cap, "vv_gqa_decode_attn_noalloc: len=%d cap=%d",
+                 len, cap);
+  const int nch = vv::attn_default_chunks(Hkv, cap);
+  const size_t need = vv::attn_workspace_bytes(Hq, Hkv, nch);
+  if (need > vv::kNoAllocScratchBytes)
+    return vv::set_error(VV_ERR_CAPACITY,
+                         "vv_gqa_decode_attn_noalloc: needs %zu bytes of scratch, the static array "
+                         "holds %zu (use vv_gqa_decode_attn with a caller workspace)",
+                         need, vv::kNoAllocScratchBytes);
+  int dev = 0;
+  VV_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return vv::set_error(VV_ERR_INVALID_ARG, "device ordinal %d", dev);
+  void* base = nullptr;
+  {
+    // First call on a device: look up the array's device address with that device current.
+    std::lock_guard<std::mutex> lock(vv::g_noalloc_mu);
+    if (!vv::g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      VV_CUDA(cudaGetSymbolAddress(&p, g_attn_scratch));
+      vv::g_noalloc_ptr[dev] = p;
+    }
+    base = vv::g_noalloc_ptr[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(base);
+  // The arrival counters must start at zero (the partials are fully rewritten by every call).
+  VV_CUDA(cudaMemsetAsync(ws + need - 256, 0, 256, s));
+  vv::AttnArgs a = {};
+  a.q_f16 = q;
+  a.k_cache = const_cast<uint16_t*>(k_cache);
+  a.v_cache = const_cast<uint16_t*>(v_cache);
+  a.len = len;
+  a.cap = cap;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.scale = scale;
+  a.out_f16 = out;
+  a.ws_part = reinterpret_cast<float*>(ws);
+  a.ws_count = reinterpret_cast<int*>(ws + need - 256);
+  a.nchunks = nch;
+  return vv::cuda_check(vv::launch_attn(a, false, s, false), "attention (no-alloc) launch");
 }
