@@ -215,7 +215,7 @@ typedef struct vv_decoder vv_decoder;
 /* Create a decoder on the current device.  All weight pointers are borrowed for the decoder's
  * lifetime; k_cache/v_cache likewise.  Allocates the decoder's workspace.  Length starts at 0.
  * Requirements: head_dim == 128, n_kv <= 64, n_q % n_kv == 0, n_q/n_kv <= 8, hidden and inter multiples of
- * 256, 1 <= kv_capacity, 1 <= max_position.
+ * 256 (inter <= 32768), 1 <= kv_capacity, 1 <= max_position.
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CUDA (allocation). */
 vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* weights,
                             uint16_t* k_cache, uint16_t* v_cache, vv_decoder** out);

@@ -185,7 +185,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
                  "n_q %d / n_kv %d", c.n_q, c.n_kv);
   VV_CHECK_SHAPE(c.hidden >= 256 && c.hidden % 256 == 0 && c.hidden <= 16384, "hidden %d",
                  c.hidden);
-  VV_CHECK_SHAPE(c.inter >= 256 && c.inter % 256 == 0 && c.inter <= 16384, "inter %d", c.inter);
+  VV_CHECK_SHAPE(c.inter >= 256 && c.inter % 256 == 0 && c.inter <= 32768, "inter %d", c.inter);
   VV_CHECK_SHAPE((c.n_q * c.head_dim) % 256 == 0 && c.n_q * c.head_dim <= 16384, "n_q*D %d",
                  c.n_q * c.head_dim);
   VV_CHECK_SHAPE(c.layers >= 1 && c.vocab >= 1 && c.kv_capacity >= 1 && c.max_position >= 1 &&

@@ -44,6 +44,8 @@ constexpr int kMaxG = 8;
 constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRegHB = 3;              // half-blocks per lane held in registers (K <= 1536)
+constexpr int kMergeInO = 32;          // up to this many tiles per head, every CTA merges the
+                                       // attention partials while staging the o-projection input
 
 enum Phase { PH_QKV = 0, PH_ATTN, PH_O, PH_GU, PH_DOWN, PH_HEAD };
 
@@ -453,8 +455,66 @@ struct AttnScratch {
   float s[kMaxG][TT];
   float m[kMaxG], l[kMaxG];
   float mw[256][kMaxG];
+  float pv[4][kMaxG][D];  // P.V partial sums per position quarter
   int is_last;
 };
+
+__device__ __forceinline__ bool merge_in_o(const StepParams& p, int nt) {
+  return nt <= kMergeInO && p.Hkv * nt * (p.Hq / p.Hkv) <= 256 * kMaxG;
+}
+
+// Stage the o-projection input straight from the attention partials (merge_in_o case): per head
+// M = max_t m_t, L = sum_t l_t 2^(m_t - M), o[h][d] = sum_t 2^(m_t - M) o_t[h][d] / L; rounded to
+// fp16 into the GEMV layout.  w[(g*nt + t)*G + h] in shared memory.  Ends with a compute barrier.
+__device__ void stage_attn_merged(const StepParams& p, __half* xs, float* w, int nt) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.Hq / p.Hkv, K = p.Hq * D, nhb = K >> 4;
+  for (int hh = warp; hh < p.Hq; hh += NW) {
+    const int g = hh / G, h = hh % G;
+    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart;
+    float mt = -INFINITY, lt = 0.f;
+    if (lane < nt) {
+      mt = __ldcg(base + (size_t)lane * kMaxG * kPart);
+      lt = __ldcg(base + (size_t)lane * kMaxG * kPart + 1);
+    }
+    const float M = warp_max(mt);
+    const float e = lane < nt ? exp2f(mt - M) : 0.f;
+    const float L = warp_sum(lt * e);
+    if (lane < nt) w[(g * nt + lane) * G + h] = e / L;
+  }
+  cbar();
+  for (int k4 = tid; k4 < K / 4; k4 += NW * 32) {
+    const int k = k4 * 4;
+    const int hh = k >> 7, d = k & (D - 1);
+    const int g = hh / G, h = hh % G;
+    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart + 4 + d;
+    const float* wg = w + (size_t)g * nt * G + h;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < nt; t0 += 8) {
+      const int m = min(8, nt - t0);
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = u < m ? __ldcg(reinterpret_cast<const float4*>(base + (size_t)(t0 + u) * kMaxG * kPart))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (u < m) {
+          const float ww = wg[(t0 + u) * G];
+          acc.x = fmaf(ww, v[u].x, acc.x);
+          acc.y = fmaf(ww, v[u].y, acc.y);
+          acc.z = fmaf(ww, v[u].z, acc.z);
+          acc.w = fmaf(ww, v[u].w, acc.w);
+        }
+      }
+    }
+    xs[xh_slot(k + 0, nhb)] = __float2half_rn(acc.x);
+    xs[xh_slot(k + 1, nhb)] = __float2half_rn(acc.y);
+    xs[xh_slot(k + 2, nhb)] = __float2half_rn(acc.z);
+    xs[xh_slot(k + 3, nhb)] = __float2half_rn(acc.w);
+  }
+  cbar();
+}
 
 // One attention tile item: scores, softmax, P.V for the G heads of kv head g.
 __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
@@ -505,7 +565,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
       float sc = -INFINITY;
       if (pp < n) {
         const __half* kr = kt + pp * D;
-        float2 acc = make_float2(0.f, 0.f);
+        float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
           const int cc = (c + lane) & 15;
@@ -513,11 +573,11 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
           const float4 qa = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
           const float4 qb = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
           acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa.x, qa.y), acc);
-          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa.z, qa.w), acc);
+          acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa.z, qa.w), acc2);
           acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb.x, qb.y), acc);
-          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb.z, qb.w), acc);
+          acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb.z, qb.w), acc2);
         }
-        sc = acc.x + acc.y;
+        sc = (acc.x + acc.y) + (acc2.x + acc2.y);
       }
       as.s[h][pp] = sc;
     }
@@ -538,15 +598,33 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     }
   }
   cbar();
-  // P.V: (head, dim) pairs over all compute threads
+  // P.V: unit = (head h, 8-dim octet o, position quarter q); V rows read as 16-byte vectors,
+  // quarters combined through shared memory (as.pv), then written as the tile's partial.
   {
+    const int units = G * 16 * 4;
+    for (int u = tid; u < units; u += NW * 32) {
+      const int q = u & 3, o = (u >> 2) & 15, h = u >> 6;
+      float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+      const float* ph = as.s[h];
+      const int p_end = min(n, q * 16 + 16);
+      for (int pp = q * 16; pp < p_end; ++pp) {
+        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * D + o * 8);
+        const float w = ph[pp];
+        const float2 ww = make_float2(w, w);
+        a0 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.x)), ww, a0);
+        a1 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.y)), ww, a1);
+        a2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.z)), ww, a2);
+        a3 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.w)), ww, a3);
+      }
+      float4* dst = reinterpret_cast<float4*>(&as.pv[q][h][o * 8]);
+      dst[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
+      dst[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
+    }
+    cbar();
     float* part = p.attn_part + ((size_t)(g * p.max_tiles + t) * kMaxG) * kPart;
     for (int idx = tid; idx < G * D; idx += NW * 32) {
       const int h = idx >> 7, d = idx & (D - 1);
-      float o = 0.f;
-      const float* ph = as.s[h];
-      for (int pp = 0; pp < n; ++pp) o = fmaf(ph[pp], __half2float(vt[pp * D + d]), o);
-      part[h * kPart + 4 + d] = o;
+      part[h * kPart + 4 + d] = (as.pv[0][h][d] + as.pv[1][h][d]) + (as.pv[2][h][d] + as.pv[3][h][d]);
     }
     if (tid < G) {
       part[tid * kPart + 0] = as.m[tid];
@@ -555,7 +633,10 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   }
   __syncwarp();
   if (lane == 0) mbar_arrive(&r.empty[slot]);
-  // publish; the last tile of head g to finish merges all of g's partials
+  // Short caches: the partials are merged by every CTA when it stages the o-projection input
+  // (after the grid barrier, which orders these stores).  Long caches: the last tile of head g to
+  // finish merges g's partials here.
+  if (merge_in_o(p, nt)) return;
   __threadfence();
   cbar();
   if (tid == 0) {
@@ -583,20 +664,28 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     for (int c = lane; c < nt; c += 32) as.mw[c][h] *= inv;
   }
   cbar();
-  for (int idx = tid; idx < G * D; idx += NW * 32) {
-    const int h = idx >> 7, d = idx & (D - 1);
-    float acc = 0.f;
-    for (int c0 = 0; c0 < nt; c0 += 16) {
-      const int m = min(16, nt - c0);
-      float v[16];
+  for (int idx = tid; idx < G * (D / 4); idx += NW * 32) {
+    const int h = idx / (D / 4), d4 = idx % (D / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < nt; c0 += 8) {
+      const int m = min(8, nt - c0);
+      float4 v[8];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        v[u] = u < m ? __ldcg(base + ((size_t)(c0 + u) * kMaxG + h) * kPart + 4 + d) : 0.f;
+      for (int u = 0; u < 8; ++u)
+        v[u] = u < m ? __ldcg(reinterpret_cast<const float4*>(base + ((size_t)(c0 + u) * kMaxG + h) * kPart + 4) + d4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        if (u < m) acc = fmaf(as.mw[c0 + u][h], v[u], acc);
+      for (int u = 0; u < 8; ++u) {
+        if (u < m) {
+          const float w = as.mw[c0 + u][h];
+          acc.x = fmaf(w, v[u].x, acc.x);
+          acc.y = fmaf(w, v[u].y, acc.y);
+          acc.z = fmaf(w, v[u].z, acc.z);
+          acc.w = fmaf(w, v[u].w, acc.w);
+        }
+      }
     }
-    p.attn_out[(size_t)(g * G + h) * D + d] = acc;
+    *reinterpret_cast<float4*>(p.attn_out + (size_t)(g * G + h) * D + 4 * d4) = acc;
   }
   if (tid == 0) p.attn_count[g] = 0;
 }
@@ -616,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   r.idx = 0;
   __half* xs = reinterpret_cast<__half*>(smem + (size_t)p.nstages * p.stage_bytes);
   AttnScratch& as = *reinterpret_cast<AttnScratch*>(smem + (size_t)p.nstages * p.stage_bytes +
-                                                     (size_t)p.x_floats * 4);
+                                                     (size_t)p.x_floats * 2);
   float* red = reinterpret_cast<float*>(&as + 1);  // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 64) + 15) &
                                                ~uintptr_t(15));
@@ -722,7 +811,11 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, pos);
     // ---------------------------------------------------------------- O
     grid_barrier(p, gen, sk);
-    stage_x(xs, red, p.attn_out, nullptr, nullptr, 0.f, Hq * D, nullptr);
+    if (merge_in_o(p, nt)) {
+      stage_attn_merged(p, xs, &as.mw[0][0], nt);
+    } else {
+      stage_x(xs, red, p.attn_out, nullptr, nullptr, 0.f, Hq * D, nullptr);
+    }
     stamp(p, sk);
     const bool regO = Hq * D <= 32 * kRegHB * 16;
     if (regO) load_xr(xs, xr, Hq * D);
@@ -886,7 +979,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
 }  // namespace
 
 size_t step_smem_bytes(int stage_bytes, int nstages, int x_floats) {
-  return (size_t)nstages * stage_bytes + (size_t)x_floats * 4 + sizeof(AttnScratch) + 64 * 4 +
+  // x is staged in fp16: x_floats halves
+  return (size_t)nstages * stage_bytes + (size_t)x_floats * 2 + sizeof(AttnScratch) + 64 * 4 +
          2 * nstages * 8 + 64;
 }
 
