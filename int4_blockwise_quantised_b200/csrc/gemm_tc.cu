@@ -1,0 +1,364 @@
+// tcgen05 tensor-core GEMM for the prefill: C[M, N] = A[M, K] . B[N, K]^T, fp16 in, fp32 out.
+// (Prefill of decoder_init, "vibevoice-asr-bitnet-onnx": decoder_init contract; all projections
+// of the S prompt positions are real dense contractions.)
+//
+// One 128 x 256 output tile per CTA, K in blocks of 64:
+//   warp 0      : TMA producer (cp.async.bulk.tensor 2D, 128-byte swizzle, no multicast) into a
+//                 4-stage ring of (A 128x64, B 256x64) fp16 tiles, mbarrier complete_tx;
+//   warp 1      : allocates 256 TMEM columns, one thread issues tcgen05.mma kind::f16
+//                 (M=128, N=256, K=16, fp32 accumulate in TMEM), tcgen05.commit releases stages;
+//   warps 2..5  : epilogue -- tcgen05.ld 32 lanes x 32 columns per step, fused operation, store.
+// Epilogues: BIAS (fp32 out + fp16 bias), RESID (fp32 x += acc), SWIGLU (columns interleaved
+// gate/up -> fp16 silu(g) * u), F16 (fp16 out + fp16 bias).  Rows >= M are masked (TMA zero-fills the A tail).
+// Every mbarrier wait is bounded; TMEM is always released before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "vv_device.cuh"
+#include "vv_internal.h"
+#include "gemm_tc.h"
+
+namespace vv {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kStageA = BM * BK * 2;  // 16 KB
+constexpr uint32_t kStageB = BN * BK * 2;  // 32 KB
+constexpr uint32_t kTmemCols = 256;
+// instruction descriptor: D f32, A/B f16, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  // start address >> 4 | LBO 16 B (unused for swizzled K-major) | SBO 1024 B (8 rows x 128 B)
+  // | version 1 (bit 46) | layout SWIZZLE_128B (2 << 61)
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmEpilogue e, const int M, const int N, const int K) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + STAGES * kStageA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * kStageB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = N / BN;
+  const int m_blk = blockIdx.x / n_tiles, n_blk = blockIdx.x % n_tiles;
+  const int kblocks = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(tmem_full, 1);
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % STAGES;
+        if (kb >= STAGES) mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1);
+        mbar_arrive_expect_tx(&full[s], kStageA + kStageB);
+        tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m_blk * BM, &full[s]);
+        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, n_blk * BN, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % STAGES;
+        mbar_wait(&full[s], (kb / STAGES) & 1);
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * kStageB);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)  // 32 bytes per K=16 slice inside the swizzled row
+          umma_f16(tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), kIdesc,
+                   (kb > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);  // stage free once these MMAs have read it
+      }
+      umma_commit(tmem_full);  // accumulator complete
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31
+    const int q = warp & 3;
+    const int row = m_blk * BM + q * 32 + lane;
+    mbar_wait(tmem_full, 0);
+    tc_fence_after();
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+      if (row < M) {
+        const int col = n_blk * BN + c;
+        if (EPI == kEpiBias) {
+          float* out = e.out_f32 + (size_t)row * e.ldo + col;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 o;
+            o.x = v[j + 0] + (e.bias ? __half2float(e.bias[col + j + 0]) : 0.f);
+            o.y = v[j + 1] + (e.bias ? __half2float(e.bias[col + j + 1]) : 0.f);
+            o.z = v[j + 2] + (e.bias ? __half2float(e.bias[col + j + 2]) : 0.f);
+            o.w = v[j + 3] + (e.bias ? __half2float(e.bias[col + j + 3]) : 0.f);
+            *reinterpret_cast<float4*>(out + j) = o;
+          }
+        } else if (EPI == kEpiResid) {
+          float* out = e.out_f32 + (size_t)row * e.ldo + col;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 o = *reinterpret_cast<float4*>(out + j);
+            o.x += v[j + 0];
+            o.y += v[j + 1];
+            o.z += v[j + 2];
+            o.w += v[j + 3];
+            *reinterpret_cast<float4*>(out + j) = o;
+          }
+        } else if (EPI == kEpiF16) {
+          __half* out = e.out_f16 + (size_t)row * e.ldo + col;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            __half h8[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              h8[t] = __float2half_rn(v[j + t] + (e.bias ? __half2float(e.bias[col + j + t]) : 0.f));
+            *reinterpret_cast<uint4*>(out + j) = *reinterpret_cast<uint4*>(h8);
+          }
+        } else {  // SwiGLU over interleaved (gate, up) columns -> fp16
+          __half* out = e.out_f16 + (size_t)row * e.ldo + col / 2;
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            __half h4[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float g = v[2 * (j + t)], u = v[2 * (j + t) + 1];
+              h4[t] = __float2half_rn(g / (1.f + __expf(-g)) * u);
+            }
+            *reinterpret_cast<uint2*>(out + j) = *reinterpret_cast<uint2*>(h4);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// fp16 row-major [rows, cols] (cols contiguous), box {64 cols, box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* tm, const void* base, int rows, int cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmEpilogue& e, int M,
+                     int N, int K, int tiles, size_t smem, cudaStream_t s) {
+  cudaError_t err =
+      cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  gemm_tc_kernel<EPI><<<tiles, kThreads, smem, s>>>(ta, tb, e, M, N, K);
+  return cudaGetLastError();
+}
+
+// One thread per 32-weight block: 16 code bytes + one fp16 scale in, 32 fp16 out (64 bytes).
+__global__ void __launch_bounds__(256) dequant_f16_kernel(const DequantSrc src, int total_rows,
+                                                          int K, __half* __restrict__ out) {
+  const int KB = K >> 5;
+  const int64_t nblk = (int64_t)total_rows * KB;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    const int orow = (int)(b / KB), kb = (int)(b % KB);
+    int m, r;
+    if (src.interleave) {
+      m = orow & 1;
+      r = orow >> 1;
+    } else {
+      m = 0;
+      r = orow;
+      while (m < src.nseg - 1 && r >= src.rows[m]) r -= src.rows[m++];
+    }
+    const uint4 codes = *reinterpret_cast<const uint4*>(src.q[m] + ((size_t)r * KB + kb) * 16);
+    const float sc = __half2float(__ushort_as_half(src.s[m][(size_t)r * KB + kb]));
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)orow * K + (size_t)kb * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half h[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t byte = (w[i] >> (8 * j)) & 0xFFu;
+        h[2 * j] = __float2half_rn((float)((int)(byte & 0xF) - 8) * sc);
+        h[2 * j + 1] = __float2half_rn((float)((int)(byte >> 4) - 8) * sc);
+      }
+      dst[i] = *reinterpret_cast<const uint4*>(h);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
+                               cudaStream_t s) {
+  const int64_t nblk = (int64_t)total_rows * (K >> 5);
+  int64_t grid = (nblk + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  dequant_f16_kernel<<<(int)grid, 256, 0, s>>>(src, total_rows, K, out);
+  return cudaGetLastError();
+}
+
+size_t gemm_tc_smem() { return STAGES * (kStageA + kStageB) + 2 * STAGES * 8 + 64 + 1024; }
+
+cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s) {
+  if (M < 1 || N % BN != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
+  if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
+  const int tiles = ((M + BM - 1) / BM) * (N / BN);
+  const size_t smem = gemm_tc_smem();
+  switch (epi) {
+    case kEpiBias: return run_gemm<kEpiBias>(ta, tb, e, M, N, K, tiles, smem, s);
+    case kEpiResid: return run_gemm<kEpiResid>(ta, tb, e, M, N, K, tiles, smem, s);
+    case kEpiSwiglu: return run_gemm<kEpiSwiglu>(ta, tb, e, M, N, K, tiles, smem, s);
+    case kEpiF16: return run_gemm<kEpiF16>(ta, tb, e, M, N, K, tiles, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace vv
+
+extern "C" vv_status vv_matmul_nbits_tc(const uint16_t* x, const uint8_t* q,
+                                        const uint16_t* scales, const uint16_t* bias, int64_t M,
+                                        int64_t N, int64_t K, int32_t block, uint16_t* w_f16,
+                                        uint16_t* y, vv_stream stream) {
+  VV_CHECK_ARG(x && q && scales && w_f16 && y, "vv_matmul_nbits_tc: null pointer");
+  VV_CHECK_ARG(vv::aligned16(x) && vv::aligned16(q) && vv::aligned16(scales) &&
+                   vv::aligned16(w_f16) && vv::aligned16(y) && (!bias || vv::aligned16(bias)),
+               "vv_matmul_nbits_tc: pointers must be 16-byte aligned");
+  VV_CHECK_SHAPE(block == 32, "vv_matmul_nbits_tc: block %d (only 32)", block);
+  VV_CHECK_SHAPE(K >= 64 && K % 64 == 0 && K < (1 << 24), "vv_matmul_nbits_tc: K=%lld",
+                 (long long)K);
+  VV_CHECK_SHAPE(N >= 256 && N % 256 == 0 && N < (1 << 24), "vv_matmul_nbits_tc: N=%lld",
+                 (long long)N);
+  VV_CHECK_SHAPE(M >= 1 && M < (1 << 24), "vv_matmul_nbits_tc: M=%lld", (long long)M);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  vv::DequantSrc src = {};
+  src.q[0] = q;
+  src.s[0] = scales;
+  src.rows[0] = (int)N;
+  src.nseg = 1;
+  __half* w = reinterpret_cast<__half*>(w_f16);
+  VV_CUDA(vv::launch_dequant_f16(src, (int)N, (int)K, w, s));
+  vv::GemmEpilogue e = {};
+  e.out_f16 = reinterpret_cast<__half*>(y);
+  e.bias = reinterpret_cast<const __half*>(bias);
+  e.ldo = (int)N;
+  VV_CUDA(vv::launch_gemm_tc(x, w_f16, (int)M, (int)N, (int)K, vv::kEpiF16, e, s));
+  return VV_OK;
+}

@@ -1,0 +1,40 @@
+// tcgen05 GEMM for the prefill (internal).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vv {
+
+constexpr int kEpiBias = 0;    // out_f32[m, n] = acc + bias[n]
+constexpr int kEpiResid = 1;   // out_f32[m, n] += acc
+constexpr int kEpiSwiglu = 2;  // out_f16[m, n/2] = silu(acc[m, n]) * acc[m, n+1], n even
+constexpr int kEpiF16 = 3;     // out_f16[m, n] = fp16(acc + bias[n])
+
+struct GemmEpilogue {
+  float* out_f32;
+  __half* out_f16;
+  const __half* bias;
+  int ldo;  // row stride of the output in elements
+};
+
+size_t gemm_tc_smem();
+// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 256 == 0, K % 64 == 0.
+cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s);
+
+// Up to three packed MatMulNBits matrices (row segments, same K) dequantised into one fp16
+// [rows, K] matrix, element (code - 8) * scale rounded once to fp16.  interleave = 1 (two
+// segments of equal rows): output row 2n is row n of segment 0, row 2n + 1 row n of segment 1.
+struct DequantSrc {
+  const uint8_t* q[3];
+  const uint16_t* s[3];
+  int rows[3];
+  int nseg;
+  int interleave;
+};
+cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
+                               cudaStream_t s);
+
+}  // namespace vv

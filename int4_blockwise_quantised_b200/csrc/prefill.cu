@@ -2,18 +2,286 @@
 // writes audio_features over the <|speech_pad|> rows starting at audio_offset; present K/V of all
 // S positions; logits of the last position).
 //
-// This translation unit holds the embedding gather + audio splice and the prefill driver.
+// Tensor-core path, per layer (S prompt positions, fp32 residual X [S, H]):
+//   Xn  = RMSNorm(X)                                  (fp16, the GEMM operand)
+//   QKV = Xn . [Wq;Wk;Wv]^T + b                       tcgen05 GEMM, bias epilogue
+//   Q, K, V <- RoPE(QKV); K, V -> cache slots 0..S-1  (fp16)
+//   O   = causal GQA attention                       mma.sync flash attention
+//   X  += O . Wo^T                                    tcgen05 GEMM, residual epilogue
+//   Hm  = silu(Xn Wg^T) * (Xn Wu^T), Xn = RMSNorm(X)  tcgen05 GEMM over interleaved gate/up rows
+//   X  += Hm . Wd^T                                   tcgen05 GEMM, residual epilogue
+// Each packed int4 matrix is first dequantised to an fp16 copy ((code - 8) * scale, rounded once)
+// in a reused workspace buffer.  The last row then goes through the final RMSNorm + lm_head.
+// VV_PREFILL=steps in the environment selects the token-by-token path (one decode step per
+// position), kept as a cross-check of the tensor-core path.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
 
 #include "vv_device.cuh"
 #include "vv_internal.h"
 #include "decoder_state.h"
+#include "gemm_tc.h"
+#include "attn_prefill.h"
 
 namespace vv {
 namespace {
 
-// out[i] = audio[i - off] for off <= i < off + N, else embed[ids[i]] (fp16 rows of H).
+constexpr int D = 128;
+
+// X[s] = audio[s - off] for off <= s < off + N, else embed[ids[s]]  (fp32 rows of H).
+__global__ void __launch_bounds__(256) splice_x_kernel(const int32_t* __restrict__ ids, int S,
+                                                       const __half* __restrict__ embed, int V,
+                                                       int H, const __half* __restrict__ audio,
+                                                       int N, int off, float* __restrict__ x) {
+  const int row = blockIdx.x;
+  if (row >= S) return;
+  const __half* src;
+  if (row >= off && row < off + N) {
+    src = audio + (size_t)(row - off) * H;
+  } else {
+    int id = ids[row];
+    if (id < 0 || id >= V) {
+      if (threadIdx.x == 0) set_device_error(VV_ERR_RANGE);
+      id = min(max(id, 0), V - 1);
+    }
+    src = embed + (size_t)id * H;
+  }
+  for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)row * H + i] = __half2float(src[i]);
+}
+
+// Xn[s] = X[s] / sqrt(mean(X[s]^2) + eps) * gamma  -> fp16.  One CTA of 128 threads per row.
+__global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const float* __restrict__ x, int H,
+                                                           const __half* __restrict__ gamma,
+                                                           float eps, __half* __restrict__ out) {
+  const int row = blockIdx.x;
+  const float* xr = x + (size_t)row * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < H; i += 512) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  __shared__ float red[4];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  const float inv = rsqrtf((red[0] + red[1] + red[2] + red[3]) / (float)H + eps);
+  for (int i = threadIdx.x * 4; i < H; i += 512) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + i);
+    __half2 a = __floats2half2_rn(v.x * inv * __half2float(gamma[i]), v.y * inv * __half2float(gamma[i + 1]));
+    __half2 b = __floats2half2_rn(v.z * inv * __half2float(gamma[i + 2]), v.w * inv * __half2float(gamma[i + 3]));
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&a);
+    pk.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(out + (size_t)row * H + i) = pk;
+  }
+}
+
+// RoPE of q and k at position_ids[s], then Q -> fp16 [S, Hq*D]; K, V -> cache slot s (fp16).
+// grid (S, Hq + 2*Hkv), block 128 (one thread per dim).
+__global__ void __launch_bounds__(128) rope_kv_kernel(const float* __restrict__ qkv, int S,
+                                                      int Hq, int Hkv, const int32_t* __restrict__ pos_ids,
+                                                      const float* __restrict__ cos_t,
+                                                      const float* __restrict__ sin_t, int max_pos,
+                                                      __half* __restrict__ q_out,
+                                                      __half* __restrict__ kc, __half* __restrict__ vc,
+                                                      int cap) {
+  const int s = blockIdx.x, hh = blockIdx.y, d = threadIdx.x;
+  const int nqkv = (Hq + 2 * Hkv) * D;
+  const float* row = qkv + (size_t)s * nqkv;
+  if (hh >= Hq + Hkv) {  // value head
+    const int g = hh - Hq - Hkv;
+    vc[((size_t)g * cap + s) * D + d] = __float2half_rn(row[hh * D + d]);
+    return;
+  }
+  int pos = pos_ids[s];
+  if (pos < 0 || pos >= max_pos) {
+    if (d == 0) set_device_error(VV_ERR_RANGE);
+    pos = min(max(pos, 0), max_pos - 1);
+  }
+  const int fi = d & (D / 2 - 1);
+  const float cs = cos_t[(size_t)pos * (D / 2) + fi], sn = sin_t[(size_t)pos * (D / 2) + fi];
+  const float x1 = row[hh * D + fi], x2 = row[hh * D + fi + D / 2];
+  const float y = d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+  if (hh < Hq) {
+    q_out[(size_t)s * Hq * D + hh * D + d] = __float2half_rn(y);
+  } else {
+    const int g = hh - Hq;
+    kc[((size_t)g * cap + s) * D + d] = __float2half_rn(y);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+cudaError_t prefill_steps(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
+                          const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
+                          cudaStream_t s);
+
+}  // namespace
+
+cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
+                        const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
+                        cudaStream_t s) {
+  const char* mode = getenv("VV_PREFILL");
+  if (mode && strcmp(mode, "steps") == 0)
+    return prefill_steps(d, ids, pos, S, audio, N, off, logits, argmax, s);
+  const vv_config& c = d->cfg;
+  const int H = c.hidden, Hq = c.n_q, Hkv = c.n_kv, I = c.inter, HQD = Hq * D;
+  const int NQKV = (Hq + 2 * Hkv) * D;
+  const int SM = c.max_prefill;
+  // workspace layout (allocated once, sized for max_prefill)
+  size_t off_b = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off_b;
+    off_b = align256(off_b + bytes);
+    return o;
+  };
+  const size_t o_x = take((size_t)SM * H * 4);
+  const size_t o_xn = take((size_t)SM * (H > HQD ? H : HQD) * 2);
+  const size_t o_qkv = take((size_t)SM * NQKV * 4);
+  const size_t o_q = take((size_t)SM * HQD * 2);
+  const size_t o_h = take((size_t)SM * I * 2);
+  size_t wmax = (size_t)NQKV * H;
+  if ((size_t)2 * I * H > wmax) wmax = (size_t)2 * I * H;
+  if ((size_t)H * I > wmax) wmax = (size_t)H * I;
+  if ((size_t)H * HQD > wmax) wmax = (size_t)H * HQD;
+  const size_t o_w = take(wmax * 2);
+  const size_t o_bias = take((size_t)NQKV * 2);
+  const size_t need = off_b;
+  if (d->pws_bytes < need) {
+    if (d->pws) cudaFree(d->pws);
+    d->pws = nullptr;
+    d->pws_bytes = 0;
+    cudaError_t e = cudaMalloc(&d->pws, need);
+    if (e != cudaSuccess) return e;
+    d->pws_bytes = need;
+  }
+  unsigned char* b = d->pws;
+  float* X = reinterpret_cast<float*>(b + o_x);
+  __half* Xn = reinterpret_cast<__half*>(b + o_xn);  // also the attention output O
+  float* QKV = reinterpret_cast<float*>(b + o_qkv);
+  __half* Q = reinterpret_cast<__half*>(b + o_q);
+  __half* Hm = reinterpret_cast<__half*>(b + o_h);
+  __half* W = reinterpret_cast<__half*>(b + o_w);
+  __half* Bqkv = reinterpret_cast<__half*>(b + o_bias);
+  const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
+  cudaError_t e;
+
+  splice_x_kernel<<<S, 256, 0, s>>>(ids, S, reinterpret_cast<const __half*>(d->embed), c.vocab, H,
+                                    reinterpret_cast<const __half*>(audio), N, off, X);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int l = 0; l < c.layers; ++l) {
+    const vv_layer_weights& w = d->layers[l];
+    __half* kc = reinterpret_cast<__half*>(d->k_cache) + (size_t)l * layer_kv;
+    __half* vc = reinterpret_cast<__half*>(d->v_cache) + (size_t)l * layer_kv;
+    // ---- QKV
+    rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.input_norm), c.eps, Xn);
+    DequantSrc dq = {};
+    dq.q[0] = w.wq.q; dq.s[0] = w.wq.scales; dq.rows[0] = HQD;
+    dq.q[1] = w.wk.q; dq.s[1] = w.wk.scales; dq.rows[1] = Hkv * D;
+    dq.q[2] = w.wv.q; dq.s[2] = w.wv.scales; dq.rows[2] = Hkv * D;
+    dq.nseg = 3;
+    if ((e = launch_dequant_f16(dq, NQKV, H, W, s)) != cudaSuccess) return e;
+    const uint16_t* bsrc[3] = {w.bq, w.bk, w.bv};
+    const int brows[3] = {HQD, Hkv * D, Hkv * D};
+    int boff = 0;
+    for (int m = 0; m < 3; ++m) {
+      if (bsrc[m])
+        e = cudaMemcpyAsync(Bqkv + boff, bsrc[m], (size_t)brows[m] * 2, cudaMemcpyDeviceToDevice, s);
+      else
+        e = cudaMemsetAsync(Bqkv + boff, 0, (size_t)brows[m] * 2, s);
+      if (e != cudaSuccess) return e;
+      boff += brows[m];
+    }
+    GemmEpilogue ep = {};
+    ep.out_f32 = QKV;
+    ep.bias = Bqkv;
+    ep.ldo = NQKV;
+    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
+                            S, NQKV, H, kEpiBias, ep, s)) != cudaSuccess)
+      return e;
+    rope_kv_kernel<<<dim3(S, Hq + 2 * Hkv), D, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
+                                                      c.max_position, Q, kc, vc, c.kv_capacity);
+    // ---- attention -> O (in the Xn buffer)
+    AttnPrefillArgs aa = {};
+    aa.q = reinterpret_cast<const uint16_t*>(Q);
+    aa.k_cache = reinterpret_cast<const uint16_t*>(kc);
+    aa.v_cache = reinterpret_cast<const uint16_t*>(vc);
+    aa.out = reinterpret_cast<uint16_t*>(Xn);
+    aa.S = S;
+    aa.cap = c.kv_capacity;
+    aa.Hq = Hq;
+    aa.Hkv = Hkv;
+    aa.scale = 1.0f / sqrtf((float)D);
+    if ((e = launch_attn_prefill(aa, s)) != cudaSuccess) return e;
+    // ---- O projection + residual
+    dq = {};
+    dq.q[0] = w.wo.q; dq.s[0] = w.wo.scales; dq.rows[0] = H;
+    dq.nseg = 1;
+    if ((e = launch_dequant_f16(dq, H, HQD, W, s)) != cudaSuccess) return e;
+    ep = {};
+    ep.out_f32 = X;
+    ep.ldo = H;
+    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
+                            S, H, HQD, kEpiResid, ep, s)) != cudaSuccess)
+      return e;
+    // ---- gate/up + SwiGLU
+    rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.post_norm), c.eps, Xn);
+    dq = {};
+    dq.q[0] = w.wgate.q; dq.s[0] = w.wgate.scales; dq.rows[0] = I;
+    dq.q[1] = w.wup.q; dq.s[1] = w.wup.scales; dq.rows[1] = I;
+    dq.nseg = 2;
+    dq.interleave = 1;
+    if ((e = launch_dequant_f16(dq, 2 * I, H, W, s)) != cudaSuccess) return e;
+    ep = {};
+    ep.out_f16 = Hm;
+    ep.ldo = I;
+    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
+                            S, 2 * I, H, kEpiSwiglu, ep, s)) != cudaSuccess)
+      return e;
+    // ---- down + residual
+    dq = {};
+    dq.q[0] = w.wdown.q; dq.s[0] = w.wdown.scales; dq.rows[0] = H;
+    dq.nseg = 1;
+    if ((e = launch_dequant_f16(dq, H, I, W, s)) != cudaSuccess) return e;
+    ep = {};
+    ep.out_f32 = X;
+    ep.ldo = H;
+    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Hm), reinterpret_cast<const uint16_t*>(W),
+                            S, H, I, kEpiResid, ep, s)) != cudaSuccess)
+      return e;
+    if (d->trace) {
+      e = cudaMemcpyAsync(d->trace + (size_t)l * H, X + (size_t)(S - 1) * H, (size_t)H * 4,
+                          cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  // ---- last position: final norm + lm_head + argmax; the residual row feeds later steps
+  if ((e = cudaMemcpyAsync(d->x_resid, X + (size_t)(S - 1) * H, (size_t)H * 4,
+                           cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+    return e;
+  LmHeadArgs la = {};
+  la.x = d->x_resid;
+  la.gamma = d->final_norm;
+  la.w = d->lm_head;
+  la.V = c.vocab;
+  la.H = H;
+  la.eps = c.eps;
+  la.logits = logits;
+  la.idx = argmax ? argmax : d->d_argmax;
+  la.ws_val = d->lm_val;
+  la.ws_idx = d->lm_idx;
+  la.ws_count = d->lm_count;
+  la.length = nullptr;
+  if ((e = launch_lm_head(la, s, false)) != cudaSuccess) return e;
+  set_int_kernel<<<1, 1, 0, s>>>(d->d_length, S);
+  return cudaGetLastError();
+}
+
+namespace {
+// Token-by-token prefill: one decode step per prompt position (cross-check path).
 __global__ void __launch_bounds__(256) splice_kernel(const int32_t* __restrict__ ids, int S,
                                                      const uint16_t* __restrict__ embed, int V,
                                                      int H, const uint16_t* __restrict__ audio,
@@ -35,11 +303,9 @@ __global__ void __launch_bounds__(256) splice_kernel(const int32_t* __restrict__
   for (int i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = src[i];
 }
 
-}  // namespace
-
-cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
-                        const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
-                        cudaStream_t s) {
+cudaError_t prefill_steps(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
+                          const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
+                          cudaStream_t s) {
   const vv_config& c = d->cfg;
   const size_t need = (size_t)c.max_prefill * c.hidden * 2;
   if (d->pws_bytes < need) {
@@ -64,5 +330,6 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   }
   return cudaSuccess;
 }
+}  // namespace
 
 }  // namespace vv

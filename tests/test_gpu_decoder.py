@@ -186,7 +186,8 @@ def test_capacity_and_range_errors():
 
 # ------------------------------------------------------------------------------------ prefill
 @pytest.mark.parametrize("shape,mode,S,N", [(synth.SHAPE_TINY, "int4", 37, 20),
-                                            (synth.SHAPE_SMALL, "ternary", 70, 40)])
+                                            (synth.SHAPE_SMALL, "ternary", 70, 40),
+                                            (synth.SHAPE_SMALL, "int4", 300, 200)])
 def test_prefill_then_steps_match_oracle(shape, mode, S, N):
     from int4_blockwise_quantised_b200.model import Decoder
 
@@ -240,3 +241,29 @@ def test_prefill_rejects_bad_splice():
         dec.init(torch.zeros(20, dtype=torch.int32, device="cuda"),
                  torch.zeros(20, dtype=torch.int32, device="cuda"))
     assert e.value.code == _vv.VV_ERR_CAPACITY
+
+
+def test_prefill_full_length_one_layer():
+    """One 1.5B-sized layer over a full ASR prompt (S = 4530 positions: 36 row tiles with a
+    ragged tail, 71 causal key blocks), int4 weights, checked against the oracle."""
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.Shape("layer1", 1536, 1, 12, 2, 128, 8960, 151936, tied=True)
+    cfg = ocfg(shape)
+    W = oracle_model(shape, "int4")
+    model = gpu_model(shape, "int4")
+    S = 4530
+    N = synth.frames_for_audio(600.0)  # 10 minutes of 24 kHz audio -> 4500 frames
+    ids, pos, feats, off = synth.asr_prompt(shape, N, prefix=7, suffix=S - N - 7)
+    dec = Decoder(model, S + 8, max_prefill=S)
+    trace = torch.zeros((1, shape.hidden), dtype=torch.float32, device="cuda")
+    dec.set_trace(trace)
+    lg = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+    dec.init(dev(ids), dev(pos), dev(feats), off, logits=lg)
+    dec.sync_status()
+    ora = odec.decoder_init(cfg, W, ids, pos, feats, off)
+    assert normwise(lg.cpu().numpy(), ora["logits"]) <= TOL
+    assert normwise(trace.cpu().numpy()[0], ora["layer_out"][0]) <= TOL
+    assert normwise(dec.k_cache[:, 0, :, :S].cpu().numpy(), ora["k"]) <= TOL
+    assert normwise(dec.v_cache[:, 0, :, :S].cpu().numpy(), ora["v"]) <= TOL
+    assert torch.count_nonzero(dec.k_cache[:, 0, :, S:]).item() == 0

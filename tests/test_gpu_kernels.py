@@ -121,6 +121,61 @@ def test_gemv_multirow(vv, M):
     assert normwise(Y.cpu().numpy().astype(np.float64), ref) <= 1e-3
 
 
+# ------------------------------------------------------------- tensor-core MatMulNBits (many rows)
+def test_gemm_tc_one_hot_layout_exact(vv):
+    """Row m of x is one-hot at column k_m: y[m] must be the fp16 dequantised column k_m exactly
+    (single product, fp32 accumulate, one rounding).  Columns span swizzle chunks and K blocks."""
+    N, K = 512, 1536
+    W = synth.normal_f32((N, K), 0.02, 19)
+    q, sc = opack.pack_sym_int4(W)
+    deq = opack.dequant(q, sc, K)
+    cols = [0, 1, 7, 8, 15, 16, 31, 32, 63, 64, 100, 777, 1000, 1535]
+    X = np.zeros((len(cols), K), np.float16)
+    for i, k in enumerate(cols):
+        X[i, k] = 1.0
+    Y = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc)).cpu().numpy()
+    for i, k in enumerate(cols):
+        assert np.array_equal(Y[i], deq[:, k].astype(np.float16)), (i, k)
+
+
+GEMM_TC_SHAPES = [(1, 256, 64), (37, 1024, 1536), (128, 2048, 1536), (129, 512, 8960),
+                  (300, 1536, 8960), (513, 256, 3584)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_TC_SHAPES)
+def test_gemm_tc_random(vv, M, N, K):
+    """Random x, bias: within 1e-3 normwise (fp16 weight rounding 2^-12 relative, fp32
+    accumulation, fp16 output rounding)."""
+    W = synth.normal_f32((N, K), 0.02, M + N + K)
+    q, sc = opack.pack_sym_int4(W)
+    X = synth.normal_f16((M, K), 1.0, 21)
+    b = synth.normal_f16((N,), 0.02, 22)
+    ref = oops.matmul_nbits(X.astype(np.float64), q, sc, K, b)
+    Y = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc), dev(b))
+    assert normwise(Y.cpu().numpy().astype(np.float64), ref) <= 1e-3
+
+
+def test_gemm_tc_ternary_matches_gemv(vv):
+    """Ternary weights: the tensor-core path and the GEMV path agree row by row (M = 8)."""
+    N, K = 1536, 1536
+    W = synth.normal_f32((N, K), 0.02, 23)
+    s = opack.ternary_scale(W)
+    q, sc = opack.pack_ternary(W, s)
+    X = synth.normal_f16((8, K), 1.0, 24)
+    a = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc)).cpu().numpy().astype(np.float64)
+    g = vv.vv_matmul_nbits(dev(X), dev(q), dev(sc)).cpu().numpy().astype(np.float64)
+    assert normwise(a, g) <= 1e-3
+
+
+def test_gemm_tc_rejects_bad_shapes(vv):
+    q = torch.zeros((100, 2, 16), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((100, 2), dtype=torch.float16, device="cuda")
+    x = torch.zeros((4, 64), dtype=torch.float16, device="cuda")
+    with pytest.raises(vv.VVError) as e:
+        vv.vv_matmul_nbits_tc(x, q, sc)
+    assert e.value.code == vv.VV_ERR_SHAPE
+
+
 # ---------------------------------------------------------------------------------- attention
 def _attn_case(vv, Hq, Hkv, length, cap, seed, kscale=1.0):
     D = 128
