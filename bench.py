@@ -45,6 +45,14 @@ CONFIGS = {
 }
 
 
+PREFILL_CONFIGS = {
+    # name: (shape, mode, S, audio frames N, description)
+    "prefill-asr-1p5b": (synth.SHAPE_1P5B, "int4", 4530, 4500,
+                         "28-layer decoder_init, 1.5B shapes, int4 sym block-32, S=4530 (20 text "
+                         "ids + 4500 spliced audio_features + 10 text ids), batch 1"),
+}
+
+
 def std_for(shape):
     return 0.015 if shape.hidden == 3584 else 0.02
 
@@ -75,6 +83,16 @@ def phase_bytes(shape, P):
         "down": packed(H, I) + 4 * I + 8 * H,
         "lm_head": V * H * 2 + 2 * H + 4 * H + 4 * V,
     }
+
+
+def prefill_flops(shape, S):
+    """Algorithmic FLOPs of one decoder_init over S positions: the GEMM part (q/k/v, o, gate/up,
+    down over all S rows) and the causal attention part (QK^T and PV over the S(S+1)/2 visible
+    pairs), plus the last row's lm_head."""
+    H, D, Hq, Hkv, I, V = shape.hidden, shape.head_dim, shape.n_q, shape.n_kv, shape.inter, shape.vocab
+    gemm = 2 * S * (H * (Hq + 2 * Hkv) * D + Hq * D * H + H * 2 * I + I * H) * shape.layers
+    attn = 2 * 2 * Hq * D * (S * (S + 1) // 2) * shape.layers
+    return {"gemm": gemm, "attention": attn, "lm_head": 2 * V * H}
 
 
 def step_bytes(shape, P):
@@ -367,11 +385,220 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "setup_s": round(setup_s, 1),
     }
+    if args.config == "decode-1p5b" and not args.no_prefill:
+        # decoder_init at S = 4530 on the same int4 1.5B weights (the ASR prefill workload)
+        pshape, _, pS, pN, _ = PREFILL_CONFIGS["prefill-asr-1p5b"]
+        dec.close()
+        pr = measure_prefill(model, pshape, pS, pN, 10, 3, dist, world)
+        result["prefill"] = {"workload": "prefill-asr-1p5b", "value": round(pr["tok_s"], 1),
+                             "unit": "tok/s", "ms": round(pr["ms"], 3),
+                             "tflops_whole_prefill": round(pr["tflops_whole"], 1),
+                             "e2e_tok_s": round(pr["e2e_tok_s"], 1), "roofline": pr["roofline"]}
+        result["gpu_launches_prefill"] = pr["launches"] * 10
+        dec = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         st, sample, thr = oracle_sample_time(shape, mode, P)
         result["cpu_baseline"] = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr,
                                   "kind": "oracle", "sample": sample}
+    if dec is not None:
+        dec.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------------- prefill
+def prefill_inputs(shape, S, N):
+    prefix = 20
+    ids, pos, feats, off = synth.asr_prompt(shape, N, prefix=prefix, suffix=S - N - prefix)
+    assert ids.size == S
+    return ids, pos, feats, off
+
+
+def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
+    """Device-timed decoder_init over S positions (inputs resident), the end-to-end variant
+    (pinned host ids / positions / audio_features copied in, argmax read back, every step), and
+    the per-kind breakdown from one profiled prefill."""
+    import torch
+
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    dec = Decoder(model, S + 8, max_prefill=S)
+    ids, pos, feats, off = prefill_inputs(shape, S, N)
+    ids_d, pos_d, feats_d = (torch.from_numpy(a).cuda() for a in (ids, pos, feats))
+    logits = torch.empty(shape.vocab, dtype=torch.float32, device="cuda")
+    am = torch.empty(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        dec.init(ids_d, pos_d, feats_d, off, logits=logits, argmax=am)
+    dec.sync_status()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        dec.init(ids_d, pos_d, feats_d, off, logits=logits, argmax=am)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    dec.sync_status()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per = ms / steps
+    # end to end: host buffers in, greedy token out
+    ids_h, pos_h, feats_h = (torch.from_numpy(a).pin_memory() for a in (ids, pos, feats))
+    out_h = torch.empty(1, dtype=torch.int32).pin_memory()
+    e2e_steps = max(3, min(steps, 20))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        ids_d.copy_(ids_h, non_blocking=True)
+        pos_d.copy_(pos_h, non_blocking=True)
+        feats_d.copy_(feats_h, non_blocking=True)
+        dec.init(ids_d, pos_d, feats_d, off, argmax=am)
+        out_h.copy_(am, non_blocking=True)
+        stream.synchronize()
+        _ = int(out_h[0])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    kind_ms, kind_n = dec.profile_init(ids_d, pos_d, feats_d, off, logits=logits, argmax=am)
+    dec.sync_status()
     dec.close()
+    fl = prefill_flops(shape, S)
+    mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = mp.get("bf16_tflops", 1590.0)
+    peak_sus = mp.get("bf16_tflops_sustained", 1400.0)
+    kind = "measured" if mp else "fallback"
+    gemm_ms = kind_ms["gemm"]
+    ach = fl["gemm"] / (gemm_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 kind::f16, 128x256 tiles)",
+            "achieved": round(ach, 1), "peak": peak, "peak_kind": f"{kind} bf16 burst (fp16 dense "
+            "rate = bf16 on B200, nominal ratio 1)", "unit": "TFLOP/s",
+            "frac": round(ach / peak, 4), "frac_of_sustained": round(ach / peak_sus, 4),
+            "traffic": traffic_for("gemm_tc"),
+            "algorithmic_flops_per_launch": fl["gemm"] // max(kind_n["gemm"], 1),
+            "avg_launch_us": round(gemm_ms * 1e3 / max(kind_n["gemm"], 1), 2),
+            "launches_per_prefill": kind_n["gemm"],
+            "breakdown_ms": {k: round(v, 3) for k, v in kind_ms.items()},
+            "breakdown_launches": kind_n,
+            "attention_tflops": round(fl["attention"] / (kind_ms["attention"] * 1e-3) / 1e12, 1)
+            if kind_ms["attention"] > 0 else None}
+    total_fl = fl["gemm"] + fl["attention"] + fl["lm_head"]
+    return {
+        "tok_s": world * S / (ms_per * 1e-3), "ms": ms_per, "steps": steps,
+        "e2e_tok_s": world * S / (e2e_ms * 1e-3), "e2e_ms": e2e_ms,
+        "h2d_bytes": ids.nbytes + pos.nbytes + feats.nbytes, "d2h_bytes": 4,
+        "tflops_whole": total_fl / (ms_per * 1e-3) / 1e12, "roofline": roof, "clocks": clk,
+        "launches": sum(kind_n.values()),
+    }
+
+
+class OraclePrefillSample:
+    """The oracle on a bounded sample of one decoder_init: one decoder layer over all S
+    positions (weights dequantised inside the call) plus the lm_head row; prefill time =
+    L x that sample."""
+
+    def __init__(self, shape, mode, S, N):
+        from oracle import decoder as odec
+        from oracle import pack as opack
+
+        std = std_for(shape)
+        self.shape = shape
+        lw = dict(synth.layer_vectors(shape, 0))
+        for m in synth.MATRICES:
+            W = synth.master(shape, m, 0, std)
+            lw[m] = (opack.pack_ternary(W, opack.ternary_scale(W)) if mode == "ternary"
+                     else opack.pack_sym_int4(W))
+        tables = synth.model_tables(shape)
+        self.W = {"layers": [lw], "embed": tables["embed"], "lm_head": tables["lm_head"],
+                  "final_norm": tables["final_norm"]}
+        self.cfg1 = odec.Config(shape.hidden, 1, shape.n_q, shape.n_kv, shape.head_dim,
+                                shape.inter, shape.vocab, shape.eps, shape.theta)
+        self.inputs = prefill_inputs(shape, S, N)
+        self.S = S
+
+    def run(self):
+        from oracle import decoder as odec
+
+        ids, pos, feats, off = self.inputs
+        t0 = time.perf_counter()
+        r = odec.decoder_init(self.cfg1, self.W, ids, pos, feats, off)
+        dt = time.perf_counter() - t0
+        assert np.isfinite(r["logits"]).all()
+        return dt * self.shape.layers
+
+    def describe(self, n):
+        return (f"oracle: {n} sample(s) of decoder_init with one decoder layer over all "
+                f"S={self.S} positions (+ the last row's lm_head); prefill time = "
+                f"{self.shape.layers} x sample")
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+
+    from int4_blockwise_quantised_b200 import _vv
+    from int4_blockwise_quantised_b200.model import PackedModel
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        import datetime
+
+        dist = dist_mod
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    shape, mode, S, N, desc = PREFILL_CONFIGS[args.config]
+    vmode = _vv.VV_TERNARY if mode == "ternary" else _vv.VV_SYM_INT4
+    t0 = time.time()
+    model = PackedModel(shape, vmode, lambda li, m: synth.master(shape, m, li, std_for(shape)),
+                        lambda li: synth.layer_vectors(shape, li), synth.model_tables(shape),
+                        "cuda")
+    setup_s = time.time() - t0
+    r = measure_prefill(model, shape, S, N, args.steps, args.warmup, dist, world)
+    result = {
+        "metric": "prefill tok/s (decoder_init, batch 1); tensor-core GEMM TFLOP/s vs B200 peak",
+        "value": round(r["tok_s"], 1), "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(r["ms"], 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": args.config, "description": desc, "S": S, "audio_frames": N,
+                   "weights": f"{mode} block-32",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (weights 1.2 GB read and 120 MB activations "
+                         "per layer); no flush"},
+        "tflops_whole_prefill": round(r["tflops_whole"], 1),
+        "roofline": r["roofline"],
+        "e2e": {"value": round(r["e2e_tok_s"], 1), "unit": "tok/s",
+                "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"],
+                "note": "public API: pinned host input_ids + position_ids + audio_features -> "
+                        "device, decoder_init, argmax device->host read + sync every step"},
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": r["clocks"], "setup_s": round(setup_s, 1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        o = OraclePrefillSample(shape, mode, S, N)
+        st = o.run()
+        result["cpu_baseline"] = {"value": round(S / st, 3), "unit": "tok/s",
+                                  "cores": blas_threads(), "kind": "oracle",
+                                  "sample": o.describe(1)}
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -431,6 +658,9 @@ def run_reference(args, rank):
     1/L of the lm_head, scaled by L), on this arm's config, metric and unit."""
     if rank != 0:
         return
+    if args.config in PREFILL_CONFIGS:
+        run_reference_prefill(args)
+        return
     shape, mode, P, seq, desc = CONFIGS[args.config]
     o = OracleSample(shape, mode, P)
     for _ in range(args.warmup):
@@ -455,12 +685,43 @@ def run_reference(args, rank):
     print(json.dumps(result), flush=True)
 
 
+def run_reference_prefill(args):
+    """Reference arm for a prefill config: the oracle's decoder_init on one layer over all S
+    positions per step (scaled by L); at most 1 warm-up and 3 timed samples (each is tens of
+    seconds of CPU work)."""
+    shape, mode, S, N, desc = PREFILL_CONFIGS[args.config]
+    o = OraclePrefillSample(shape, mode, S, N)
+    warm, steps = min(args.warmup, 1), min(args.steps, 3)
+    for _ in range(warm):
+        o.run()
+    t0 = time.perf_counter()
+    est = [o.run() for _ in range(steps)]
+    wall = time.perf_counter() - t0
+    st = statistics.median(est)
+    value = S / st
+    print(json.dumps({
+        "metric": "prefill tok/s (decoder_init, batch 1); tensor-core GEMM TFLOP/s vs B200 peak",
+        "value": round(value, 3), "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": warm,
+        "ms_per_step": round(st * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.config, "description": desc, "S": S, "audio_frames": N},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": o.describe(steps)},
+        "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 2),
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=16)
-    ap.add_argument("--config", default="decode-1p5b", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="decode-1p5b",
+                    choices=sorted(CONFIGS) + sorted(PREFILL_CONFIGS))
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill measurement added to the default decode line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -470,6 +731,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.config in PREFILL_CONFIGS:
+        run_prefill(args, rank, world, local_rank)
         return
     run_ours(args, rank, world, local_rank)
 

@@ -284,6 +284,18 @@ vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
                                   float* logits, int32_t* argmax_out, float* phase_ms,
                                   vv_stream stream);
 
+/* Profiling variant of vv_decoder_init: the same prefill (same arguments, same results and
+ * cache contents), with a CUDA event recorded after every launch.  Synchronous.  phase_ms: HOST
+ * float [5] and launches: HOST int32 [5] receive the device time and the number of launches (or
+ * copies) of each kind: [0] embedding splice, RMSNorm, RoPE/KV write, bias and trace copies;
+ * [1] weight dequantisation to fp16; [2] tensor-core GEMMs; [3] causal attention; [4] final
+ * norm + lm_head + argmax.  Errors as vv_decoder_init. */
+vv_status vv_decoder_profile_init(vv_decoder* dec, const int32_t* input_ids,
+                                  const int32_t* position_ids, int64_t S,
+                                  const uint16_t* audio_features, int64_t N, int64_t audio_offset,
+                                  float* logits, int32_t* argmax_out, float* phase_ms,
+                                  int32_t* launches, vv_stream stream);
+
 /* Timeline tap of the persistent step kernel: runs one step (appending a position like
  * vv_decoder_step, without graph capture) with every CTA recording the device clock
  * (%globaltimer, ns) at fixed points of its schedule: kernel start, then for each layer
@@ -291,7 +303,10 @@ vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
  * x staged, arrive/exit, x staged (gate/up), arrive/exit, x staged (down); layers > 0 start
  * with arrive/exit before QKV; then arrive/exit, x staged (lm_head), end.  stamps: HOST
  * uint64 [grid * max_per_cta]; *grid_out and *per_cta_out receive the CTA count and the number
- * of stamps each CTA wrote.  Synchronous.  VV_ERR_CAPACITY when max_per_cta is too small. */
+ * of stamps each CTA wrote.  The last 8 entries of each CTA's row are not stamps: compute
+ * thread 0's time blocked on the stage ring per phase kind (QKV, attention, o-proj, gate/up,
+ * down, lm_head; ns), then the producer's finishing time and its time blocked on free slots.
+ * Synchronous.  VV_ERR_CAPACITY when max_per_cta < 14 L + 11. */
 vv_status vv_decoder_step_timeline(vv_decoder* dec, const uint16_t* input_embeds,
                                    const int32_t* token_id, const int32_t* position_id,
                                    uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,

@@ -508,7 +508,7 @@ vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
                                    int32_t* per_cta_out, vv_stream stream) {
   VV_CHECK_ARG(d && position_id && stamps && grid_out && per_cta_out, "null pointer");
   VV_CHECK_ARG(input_embeds || token_id, "need input_embeds or token_id");
-  const int need = 14 * d->cfg.layers + 8;
+  const int need = 14 * d->cfg.layers + 11;
   if (max_per_cta < need)
     return set_error(VV_ERR_CAPACITY, "max_per_cta %d < %d", max_per_cta, need);
   if (d->len_host + 1 > d->cfg.kv_capacity)
@@ -563,6 +563,46 @@ vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t
                           static_cast<cudaStream_t>(stream)));
   d->len_host = (int32_t)S;
   return VV_OK;
+}
+
+vv_status vv_decoder_profile_init(vv_decoder* d, const int32_t* input_ids,
+                                  const int32_t* position_ids, int64_t S,
+                                  const uint16_t* audio_features, int64_t N, int64_t audio_offset,
+                                  float* logits, int32_t* argmax_out, float* phase_ms,
+                                  int32_t* launches, vv_stream stream) {
+  VV_CHECK_ARG(d && input_ids && position_ids && phase_ms && launches,
+               "vv_decoder_profile_init: null pointer");
+  VV_CHECK_ARG(N == 0 || audio_features, "vv_decoder_profile_init: audio_features null");
+  VV_CHECK_ARG(!audio_features || vv::aligned16(audio_features), "audio_features misaligned");
+  if (S < 1) return set_error(VV_ERR_SHAPE, "S=%lld", (long long)S);
+  if (N < 0 || audio_offset < 0 || audio_offset + N > S)
+    return set_error(VV_ERR_RANGE, "audio_offset %lld + N %lld > S %lld", (long long)audio_offset,
+                     (long long)N, (long long)S);
+  if (S > d->cfg.kv_capacity || S > d->cfg.max_prefill)
+    return set_error(VV_ERR_CAPACITY, "S=%lld > capacity %d or max_prefill %d", (long long)S,
+                     d->cfg.kv_capacity, d->cfg.max_prefill);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  vv::PrefillTimer t;
+  vv_status st = vv::cuda_check(vv::prefill_run(d, input_ids, position_ids, (int)S, audio_features,
+                                                (int)N, (int)audio_offset, logits, argmax_out, s,
+                                                &t),
+                                "profile prefill");
+  if (!st) st = vv::cuda_check(cudaStreamSynchronize(s), "sync");
+  if (!st) {
+    for (int k = 0; k < vv::kPfKinds; ++k) {
+      phase_ms[k] = 0.f;
+      launches[k] = 0;
+    }
+    for (size_t i = 1; i < t.ev.size(); ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, t.ev[i - 1], t.ev[i]);
+      phase_ms[t.kind[i]] += ms;
+      launches[t.kind[i]] += 1;
+    }
+    d->len_host = (int32_t)S;
+  }
+  for (auto e : t.ev) cudaEventDestroy(e);
+  return st;
 }
 
 vv_status vv_decoder_sync_status(vv_decoder* d, vv_stream stream) {

@@ -52,6 +52,13 @@ struct vv_decoder {
 
 
 namespace vv {
+// Optional event trail of one prefill: an event after every launch, tagged with the launch's
+// kind (kPfMisc: splice / norm / RoPE / copies, kPfDequant, kPfGemm, kPfAttn, kPfHead).
+enum { kPfMisc = 0, kPfDequant = 1, kPfGemm = 2, kPfAttn = 3, kPfHead = 4, kPfKinds = 5 };
+struct PrefillTimer {
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> kind;
+};
 __global__ void set_int_kernel(int32_t* p, int32_t v);
 __global__ void add_int_kernel(int32_t* p, int32_t v);
 // Enqueue one decode step (plain launches).  head=false skips the lm_head and only advances the
@@ -61,5 +68,5 @@ cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* t
                          bool head, cudaEvent_t* events = nullptr);
 cudaError_t prefill_run(vv_decoder* dec, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
-                        cudaStream_t s);
+                        cudaStream_t s, PrefillTimer* timer = nullptr);
 }  // namespace vv

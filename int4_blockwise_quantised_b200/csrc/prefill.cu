@@ -123,7 +123,21 @@ cudaError_t prefill_steps(vv_decoder* d, const int32_t* ids, const int32_t* pos,
 
 cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
-                        cudaStream_t s) {
+                        cudaStream_t s, PrefillTimer* timer) {
+  // mark(k): the work enqueued since the previous mark is of kind k
+  auto mark = [&](int k) -> cudaError_t {
+    if (!timer) return cudaSuccess;
+    cudaEvent_t ev;
+    cudaError_t err = cudaEventCreate(&ev);
+    if (err != cudaSuccess) return err;
+    timer->ev.push_back(ev);
+    timer->kind.push_back(k);
+    return cudaEventRecord(ev, s);
+  };
+#define VV_MARK(k)                                   \
+  do {                                               \
+    if ((e = mark(k)) != cudaSuccess) return e;      \
+  } while (0)
   const char* mode = getenv("VV_PREFILL");
   if (mode && strcmp(mode, "steps") == 0)
     return prefill_steps(d, ids, pos, S, audio, N, off, logits, argmax, s);
@@ -169,21 +183,25 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
   cudaError_t e;
 
+  VV_MARK(kPfMisc);
   splice_x_kernel<<<S, 256, 0, s>>>(ids, S, reinterpret_cast<const __half*>(d->embed), c.vocab, H,
                                     reinterpret_cast<const __half*>(audio), N, off, X);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  VV_MARK(kPfMisc);
   for (int l = 0; l < c.layers; ++l) {
     const vv_layer_weights& w = d->layers[l];
     __half* kc = reinterpret_cast<__half*>(d->k_cache) + (size_t)l * layer_kv;
     __half* vc = reinterpret_cast<__half*>(d->v_cache) + (size_t)l * layer_kv;
     // ---- QKV
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.input_norm), c.eps, Xn);
+    VV_MARK(kPfMisc);
     DequantSrc dq = {};
     dq.q[0] = w.wq.q; dq.s[0] = w.wq.scales; dq.rows[0] = HQD;
     dq.q[1] = w.wk.q; dq.s[1] = w.wk.scales; dq.rows[1] = Hkv * D;
     dq.q[2] = w.wv.q; dq.s[2] = w.wv.scales; dq.rows[2] = Hkv * D;
     dq.nseg = 3;
     if ((e = launch_dequant_f16(dq, NQKV, H, W, s)) != cudaSuccess) return e;
+    VV_MARK(kPfDequant);
     const uint16_t* bsrc[3] = {w.bq, w.bk, w.bv};
     const int brows[3] = {HQD, Hkv * D, Hkv * D};
     int boff = 0;
@@ -195,6 +213,7 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
       if (e != cudaSuccess) return e;
       boff += brows[m];
     }
+    VV_MARK(kPfMisc);
     GemmEpilogue ep = {};
     ep.out_f32 = QKV;
     ep.bias = Bqkv;
@@ -202,8 +221,10 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
                             S, NQKV, H, kEpiBias, ep, s)) != cudaSuccess)
       return e;
+    VV_MARK(kPfGemm);
     rope_kv_kernel<<<dim3(S, Hq + 2 * Hkv), D, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
                                                       c.max_position, Q, kc, vc, c.kv_capacity);
+    VV_MARK(kPfMisc);
     // ---- attention -> O (in the Xn buffer)
     AttnPrefillArgs aa = {};
     aa.q = reinterpret_cast<const uint16_t*>(Q);
@@ -216,46 +237,55 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     aa.Hkv = Hkv;
     aa.scale = 1.0f / sqrtf((float)D);
     if ((e = launch_attn_prefill(aa, s)) != cudaSuccess) return e;
+    VV_MARK(kPfAttn);
     // ---- O projection + residual
     dq = {};
     dq.q[0] = w.wo.q; dq.s[0] = w.wo.scales; dq.rows[0] = H;
     dq.nseg = 1;
     if ((e = launch_dequant_f16(dq, H, HQD, W, s)) != cudaSuccess) return e;
+    VV_MARK(kPfDequant);
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;
     if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
                             S, H, HQD, kEpiResid, ep, s)) != cudaSuccess)
       return e;
+    VV_MARK(kPfGemm);
     // ---- gate/up + SwiGLU
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.post_norm), c.eps, Xn);
+    VV_MARK(kPfMisc);
     dq = {};
     dq.q[0] = w.wgate.q; dq.s[0] = w.wgate.scales; dq.rows[0] = I;
     dq.q[1] = w.wup.q; dq.s[1] = w.wup.scales; dq.rows[1] = I;
     dq.nseg = 2;
     dq.interleave = 1;
     if ((e = launch_dequant_f16(dq, 2 * I, H, W, s)) != cudaSuccess) return e;
+    VV_MARK(kPfDequant);
     ep = {};
     ep.out_f16 = Hm;
     ep.ldo = I;
     if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
                             S, 2 * I, H, kEpiSwiglu, ep, s)) != cudaSuccess)
       return e;
+    VV_MARK(kPfGemm);
     // ---- down + residual
     dq = {};
     dq.q[0] = w.wdown.q; dq.s[0] = w.wdown.scales; dq.rows[0] = H;
     dq.nseg = 1;
     if ((e = launch_dequant_f16(dq, H, I, W, s)) != cudaSuccess) return e;
+    VV_MARK(kPfDequant);
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;
     if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Hm), reinterpret_cast<const uint16_t*>(W),
                             S, H, I, kEpiResid, ep, s)) != cudaSuccess)
       return e;
+    VV_MARK(kPfGemm);
     if (d->trace) {
       e = cudaMemcpyAsync(d->trace + (size_t)l * H, X + (size_t)(S - 1) * H, (size_t)H * 4,
                           cudaMemcpyDeviceToDevice, s);
       if (e != cudaSuccess) return e;
+      VV_MARK(kPfMisc);
     }
   }
   // ---- last position: final norm + lm_head + argmax; the residual row feeds later steps
@@ -276,8 +306,12 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   la.ws_count = d->lm_count;
   la.length = nullptr;
   if ((e = launch_lm_head(la, s, false)) != cudaSuccess) return e;
+  VV_MARK(kPfHead);
   set_int_kernel<<<1, 1, 0, s>>>(d->d_length, S);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  VV_MARK(kPfMisc);
+  return cudaSuccess;
+#undef VV_MARK
 }
 
 namespace {

@@ -132,6 +132,8 @@ struct Ring {
   int stage_bytes;
   int nstages;
   int idx;  // running stage counter
+  int ph;          // phase kind of the stages being consumed (timeline tap)
+  uint64_t* tapw;  // timeline tap: per-phase-kind ring wait of compute thread 0 (else null)
   __device__ unsigned char* slot_ptr(int i) const { return base + (size_t)(i % nstages) * stage_bytes; }
 };
 
@@ -147,7 +149,9 @@ __device__ __forceinline__ void ring_wait(Ring& r, uint64_t* bar, uint32_t parit
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
   mbar_wait(bar, parity);
-  r.wait_ns += globaltimer_ns() - t0;
+  const uint64_t dt = globaltimer_ns() - t0;
+  r.wait_ns += dt;
+  if (r.tapw) r.tapw[r.ph] += dt;
 }
 
 __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t pol) {
@@ -327,6 +331,56 @@ __device__ __forceinline__ float hb_doth(uint2 wv, uint4 xa, uint4 xb) {
   return dot8_h(wv.x, xa) + dot8_h(wv.y, xb);
 }
 
+// One stage of the register-x path: warp w takes units [w R, w R + R), then [w R + NW R, ...);
+// unit u is (segment, row) = (u & 1, u >> 1) for gate/up pairs, else (0, u).  Lanes stride the
+// half-blocks; one shuffle reduction per unit; lane 0 finishes the rows.
+template <int R, class RowQ, class RowS, class Fin>
+__device__ __forceinline__ void regx_pass(RowQ rowq, RowS rows, const uint4 (&xr)[kRegHB][2], int K,
+                                          int units, int nseg, int a, Fin fin) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NHB = K >> 4;
+  for (int u0 = warp * R; u0 < units; u0 += NW * R) {
+    int sg[R], lr[R];
+    bool ok[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int u = u0 + k;
+      ok[k] = u < units;
+      const int uu = ok[k] ? u : u0;
+      sg[k] = nseg == 2 ? (uu & 1) : 0;
+      lr[k] = nseg == 2 ? (uu >> 1) : uu;
+    }
+    float acc[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) acc[k] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kRegHB; ++j) {
+      const int hb = lane + 32 * j;
+      if (hb < NHB) {
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+          const uint2 wv = *reinterpret_cast<const uint2*>(rowq(sg[k], lr[k]) + hb * 8);
+          const float sc = __half2float(rows(sg[k], lr[k])[hb >> 1]);
+          acc[k] = fmaf(sc, hb_doth(wv, xr[j][0], xr[j][1]), acc[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) acc[k] = warp_sum(acc[k]);
+    if (lane == 0) {
+      if (nseg == 2) {
+#pragma unroll
+        for (int k = 0; k + 1 < R; k += 2)
+          if (ok[k]) fin(a + lr[k], acc[k], acc[k + 1]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < R; ++k)
+          if (ok[k]) fin(a + lr[k], acc[k], 0.f);
+      }
+    }
+  }
+}
+
 // Consume the stages of a packed-matrix phase.  fin(row, y0, y1) is called once per output row
 // (y1: the up value of a gate/up pair, nseg = 2).
 //  * K <= 1536 (x in registers xr): each warp takes 4 rows per pass (or 2 gate/up pairs) for
@@ -354,46 +408,16 @@ __device__ __forceinline__ void consume_packed(Ring& r, const __half* xs, const 
       return reinterpret_cast<const __half*>(scb + (size_t)(sg * rps + lr) * rs);
     };
     if (regx) {
-      // R = 4 row slots per warp pass: (seg, row) pairs
+      // R row slots per warp pass: as many as keep every warp busy (R = 1 for the small
+      // phases, up to 4 for instruction-level parallelism when rows are plentiful); gate/up
+      // pairs stay inside one warp (R >= 2).
       const int units = n * nseg;
-      for (int u0 = warp * 4; u0 < units; u0 += NW * 4) {
-        int sg[4], lr[4];
-        bool ok[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int u = u0 + k;
-          ok[k] = u < units;
-          const int uu = ok[k] ? u : u0;
-          // nseg == 2: units (2i, 2i+1) are (gate i, up i)
-          sg[k] = nseg == 2 ? (uu & 1) : 0;
-          lr[k] = nseg == 2 ? (uu >> 1) : uu;
-        }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < kRegHB; ++j) {
-          const int hb = lane + 32 * j;
-          if (hb < NHB) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint2 wv = *reinterpret_cast<const uint2*>(rowq(sg[k], lr[k]) + hb * 8);
-              const float sc = __half2float(rows(sg[k], lr[k])[hb >> 1]);
-              acc[k] = fmaf(sc, hb_doth(wv, xr[j][0], xr[j][1]), acc[k]);
-            }
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = warp_sum(acc[k]);
-        if (lane == 0) {
-          if (nseg == 2) {
-            if (ok[0]) fin(a + lr[0], acc[0], acc[1]);
-            if (ok[2]) fin(a + lr[2], acc[2], acc[3]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (ok[k]) fin(a + lr[k], acc[k], 0.f);
-          }
-        }
-      }
+      if (nseg == 1 && units <= NW)
+        regx_pass<1>(rowq, rows, xr, K, units, nseg, a, fin);
+      else if (units <= 2 * NW)
+        regx_pass<2>(rowq, rows, xr, K, units, nseg, a, fin);
+      else
+        regx_pass<4>(rowq, rows, xr, K, units, nseg, a, fin);
     } else {
       // split-K: warp w -> row w / kSplitW, slice w % kSplitW
       const int lrow = warp / kSplitW, slice = warp % kSplitW;
@@ -465,58 +489,64 @@ __device__ __forceinline__ bool merge_in_o(const StepParams& p, int nt) {
 
 // Stage the o-projection input straight from the attention partials (merge_in_o case): per head
 // M = max_t m_t, L = sum_t l_t 2^(m_t - M), o[h][d] = sum_t 2^(m_t - M) o_t[h][d] / L; rounded to
-// fp16 into the GEMV layout.  w[(g*nt + t)*G + h] in shared memory.  Ends with a compute barrier.
-__device__ void stage_attn_merged(const StepParams& p, __half* xs, float* w, int nt) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// fp16 into the GEMV layout.  Each thread merges its 4 dims online over batches of 6 tiles, the
+// batch's m, l and o loads all in flight together.  Ends with a compute barrier.
+__device__ void stage_attn_merged(const StepParams& p, __half* xs, int nt) {
+  const int tid = threadIdx.x;
   const int G = p.Hq / p.Hkv, K = p.Hq * D, nhb = K >> 4;
-  for (int hh = warp; hh < p.Hq; hh += NW) {
-    const int g = hh / G, h = hh % G;
-    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart;
-    float mt = -INFINITY, lt = 0.f;
-    if (lane < nt) {
-      mt = __ldcg(base + (size_t)lane * kMaxG * kPart);
-      lt = __ldcg(base + (size_t)lane * kMaxG * kPart + 1);
-    }
-    const float M = warp_max(mt);
-    const float e = lane < nt ? exp2f(mt - M) : 0.f;
-    const float L = warp_sum(lt * e);
-    if (lane < nt) w[(g * nt + lane) * G + h] = e / L;
-  }
-  cbar();
+  constexpr int kB = 6;
   for (int k4 = tid; k4 < K / 4; k4 += NW * 32) {
     const int k = k4 * 4;
     const int hh = k >> 7, d = k & (D - 1);
     const int g = hh / G, h = hh % G;
-    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart + 4 + d;
-    const float* wg = w + (size_t)g * nt * G + h;
+    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart;
+    float M = -INFINITY, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t0 = 0; t0 < nt; t0 += 8) {
-      const int m = min(8, nt - t0);
-      float4 v[8];
+    for (int t0 = 0; t0 < nt; t0 += kB) {
+      float4 v[kB];
+      float mt[kB], lt[kB];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = u < m ? __ldcg(reinterpret_cast<const float4*>(base + (size_t)(t0 + u) * kMaxG * kPart))
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (u < m) {
-          const float ww = wg[(t0 + u) * G];
-          acc.x = fmaf(ww, v[u].x, acc.x);
-          acc.y = fmaf(ww, v[u].y, acc.y);
-          acc.z = fmaf(ww, v[u].z, acc.z);
-          acc.w = fmaf(ww, v[u].w, acc.w);
+      for (int u = 0; u < kB; ++u) {
+        if (t0 + u < nt) {
+          const float* pt = base + (size_t)(t0 + u) * kMaxG * kPart;
+          mt[u] = __ldcg(pt);
+          lt[u] = __ldcg(pt + 1);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(pt + 4 + d));
+        } else {
+          mt[u] = -INFINITY;
+          lt[u] = 0.f;
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+      float bm = M;
+#pragma unroll
+      for (int u = 0; u < kB; ++u) bm = fmaxf(bm, mt[u]);
+      const float c = exp2f(M - bm);  // 0 on the first batch (M = -inf)
+      L *= c;
+      acc.x *= c;
+      acc.y *= c;
+      acc.z *= c;
+      acc.w *= c;
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const float e = exp2f(mt[u] - bm);
+        L = fmaf(lt[u], e, L);
+        acc.x = fmaf(e, v[u].x, acc.x);
+        acc.y = fmaf(e, v[u].y, acc.y);
+        acc.z = fmaf(e, v[u].z, acc.z);
+        acc.w = fmaf(e, v[u].w, acc.w);
+      }
+      M = bm;
     }
-    xs[xh_slot(k + 0, nhb)] = __float2half_rn(acc.x);
-    xs[xh_slot(k + 1, nhb)] = __float2half_rn(acc.y);
-    xs[xh_slot(k + 2, nhb)] = __float2half_rn(acc.z);
-    xs[xh_slot(k + 3, nhb)] = __float2half_rn(acc.w);
+    const float inv = 1.f / L;
+    xs[xh_slot(k + 0, nhb)] = __float2half_rn(acc.x * inv);
+    xs[xh_slot(k + 1, nhb)] = __float2half_rn(acc.y * inv);
+    xs[xh_slot(k + 2, nhb)] = __float2half_rn(acc.z * inv);
+    xs[xh_slot(k + 3, nhb)] = __float2half_rn(acc.w * inv);
   }
   cbar();
 }
 
-// One attention tile item: scores, softmax, P.V for the G heads of kv head g.
 __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
                           int past, int pos) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -526,30 +556,52 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   const int p0 = t * TT;
   const int n = min(TT, npos - p0);
   const float* qkv = p.qkv;
-  // q of the group, rotated and scaled into the log2 domain
+  // q of the group (rotated, scaled into the log2 domain) and, on the tile holding the new
+  // position, the new k/v: every global load is issued before any is used (one L2 round trip).
   const float qscale = p.scale * kLog2e;
-  for (int i = tid; i < G * D; i += NW * 32) {
-    const int h = i / D, d = i % D;
-    const float* qh = qkv + (size_t)(g * G + h) * D;
-    const int fi = d & (D / 2 - 1);
-    const float cs = as.cs[fi], sn = as.sn[fi];
-    const float x1 = __ldcg(qh + fi), x2 = __ldcg(qh + fi + D / 2);
-    as.q[h][d] = (d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn) * qscale;
+  const bool newpos = t == nt - 1;
+  constexpr int kQPer = (kMaxG * D + NW * 32 - 1) / (NW * 32);  // q element pairs per thread
+  float qa[kQPer], qb[kQPer];
+#pragma unroll
+  for (int j = 0; j < kQPer; ++j) {
+    const int i = tid + j * NW * 32;
+    qa[j] = qb[j] = 0.f;
+    if (i < G * D) {
+      const int h = i / D, d = i % D;
+      const float* qh = qkv + (size_t)(g * G + h) * D;
+      const int fi = d & (D / 2 - 1);
+      qa[j] = __ldcg(qh + fi);
+      qb[j] = __ldcg(qh + fi + D / 2);
+    }
+  }
+  float ka = 0.f, kb = 0.f, vv = 0.f;
+  if (newpos && tid < D) {
+    const int d = tid, fi = d & (D / 2 - 1);
+    const float* kh = qkv + (size_t)(p.Hq + g) * D;
+    ka = __ldcg(kh + fi);
+    kb = __ldcg(kh + fi + D / 2);
+    vv = __ldcg(qkv + (size_t)(p.Hq + p.Hkv + g) * D + d);
+  }
+#pragma unroll
+  for (int j = 0; j < kQPer; ++j) {
+    const int i = tid + j * NW * 32;
+    if (i < G * D) {
+      const int h = i / D, d = i % D;
+      const int fi = d & (D / 2 - 1);
+      const float cs = as.cs[fi], sn = as.sn[fi];
+      as.q[h][d] = (d < D / 2 ? qa[j] * cs - qb[j] * sn : qb[j] * cs + qa[j] * sn) * qscale;
+    }
   }
   const int s = r.idx++;
   const int slot = s % r.nstages;
   ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
   __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
   __half* vt = kt + TT * D;
-  if (t == nt - 1 && tid < D) {  // this tile holds the new position: rotate k, append k/v
-    const int d = tid;
-    const float* kh = qkv + (size_t)(p.Hq + g) * D;
-    const float* vh = qkv + (size_t)(p.Hq + p.Hkv + g) * D;
-    const int fi = d & (D / 2 - 1);
+  if (newpos && tid < D) {  // this tile holds the new position: rotate k, append k/v
+    const int d = tid, fi = d & (D / 2 - 1);
     const float cs = as.cs[fi], sn = as.sn[fi];
-    const float x1 = __ldcg(kh + fi), x2 = __ldcg(kh + fi + D / 2);
-    const __half kn = __float2half_rn(d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn);
-    const __half vn = __float2half_rn(__ldcg(vh + d));
+    const __half kn = __float2half_rn(d < D / 2 ? ka * cs - kb * sn : kb * cs + ka * sn);
+    const __half vn = __float2half_rn(vv);
     const size_t off = ((size_t)(l * p.Hkv + g) * p.cap + past) * D + d;
     p.k_cache[off] = kn;
     p.v_cache[off] = vn;
@@ -699,6 +751,12 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   Ring r;
   r.wait_ns = 0;
+  r.ph = 0;
+  // timeline tap: the last 8 stamps of a CTA's row hold thread 0's ring wait per phase kind
+  // (QKV, ATTN, O, GU, DOWN, HEAD at max-8 .. max-3), then the producer's done time and its
+  // blocked time.
+  r.tapw = (p.stamps && threadIdx.x == 0) ? p.stamps + (size_t)blockIdx.x * p.max_stamps + p.max_stamps - 8
+                                          : nullptr;
   r.base = smem;
   r.stage_bytes = p.stage_bytes;
   r.nstages = p.nstages;
@@ -763,6 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   for (int l = 0; l < p.L; ++l) {
     const StepLayer& w = p.layers[l];
     // ---------------------------------------------------------------- QKV
+    r.ph = 0;
     if (l == 0) {
       const __half* e16 = p.input_embeds;
       if (!e16) {
@@ -807,12 +866,14 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       }
     }
     // ---------------------------------------------------------------- ATTN
+    r.ph = 1;
     grid_barrier(p, gen, sk);
     for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, pos);
     // ---------------------------------------------------------------- O
+    r.ph = 2;
     grid_barrier(p, gen, sk);
     if (merge_in_o(p, nt)) {
-      stage_attn_merged(p, xs, &as.mw[0][0], nt);
+      stage_attn_merged(p, xs, nt);
     } else {
       stage_x(xs, red, p.attn_out, nullptr, nullptr, 0.f, Hq * D, nullptr);
     }
@@ -829,6 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       });
     }
     // ---------------------------------------------------------------- GU
+    r.ph = 3;
     grid_barrier(p, gen, sk);
     stage_x(xs, red, p.x_resid, nullptr, w.post_norm, p.eps, H, nullptr);
     stamp(p, sk);
@@ -841,6 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       });
     }
     // ---------------------------------------------------------------- DOWN
+    r.ph = 4;
     grid_barrier(p, gen, sk);
     stage_x(xs, red, p.h, nullptr, nullptr, 0.f, I, nullptr);
     stamp(p, sk);
@@ -857,6 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     }
   }
   // ------------------------------------------------------------------------------ HEAD
+  r.ph = 5;
   grid_barrier(p, gen, sk);
   stage_x(xs, red, p.x_resid, nullptr, p.final_norm, p.eps, H, nullptr);
   stamp(p, sk);

@@ -168,3 +168,17 @@ class Decoder:
         check(_vv.lib.vv_decoder_init(self.handle, ptr(input_ids), ptr(position_ids), S,
                                       ptr(audio_features), N, audio_offset, ptr(logits),
                                       ptr(argmax), stream_handle(stream)))
+
+    PREFILL_KINDS = ("misc", "dequant", "gemm", "attention", "lm_head")
+
+    def profile_init(self, input_ids, position_ids, audio_features=None, audio_offset=0,
+                     logits=None, argmax=None, stream=None):
+        """decoder_init with an event after every launch; returns ({kind: ms}, {kind: launches})."""
+        S = input_ids.numel()
+        N = 0 if audio_features is None else audio_features.shape[0]
+        ms = (ctypes.c_float * 5)()
+        n = (ctypes.c_int32 * 5)()
+        check(_vv.lib.vv_decoder_profile_init(self.handle, ptr(input_ids), ptr(position_ids), S,
+                                              ptr(audio_features), N, audio_offset, ptr(logits),
+                                              ptr(argmax), ms, n, stream_handle(stream)))
+        return dict(zip(self.PREFILL_KINDS, list(ms))), dict(zip(self.PREFILL_KINDS, list(n)))
