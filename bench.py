@@ -488,7 +488,7 @@ def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
     kind = "measured" if mp else "fallback"
     gemm_ms = kind_ms["gemm"]
     ach = fl["gemm"] / (gemm_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 kind::f16, 128x256 tiles)",
+    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 kind::f16, persistent, 128x256 or 128x128 tiles, 2 TMEM accumulators)",
             "achieved": round(ach, 1), "peak": peak, "peak_kind": f"{kind} bf16 burst (fp16 dense "
             "rate = bf16 on B200, nominal ratio 1)", "unit": "TFLOP/s",
             "frac": round(ach / peak, 4), "frac_of_sustained": round(ach / peak_sus, 4),

@@ -2,15 +2,20 @@
 // (Prefill of decoder_init, "vibevoice-asr-bitnet-onnx": decoder_init contract; all projections
 // of the S prompt positions are real dense contractions.)
 //
-// One 128 x 256 output tile per CTA, K in blocks of 64:
+// Persistent: one CTA per SM walks the 128 x BN output tiles (BN = 256, or 128 when that fills
+// the last wave of SMs better), K in blocks of 64.
 //   warp 0      : TMA producer (cp.async.bulk.tensor 2D, 128-byte swizzle, no multicast) into a
-//                 4-stage ring of (A 128x64, B 256x64) fp16 tiles, mbarrier complete_tx;
-//   warp 1      : allocates 256 TMEM columns, one thread issues tcgen05.mma kind::f16
-//                 (M=128, N=256, K=16, fp32 accumulate in TMEM), tcgen05.commit releases stages;
-//   warps 2..5  : epilogue -- tcgen05.ld 32 lanes x 32 columns per step, fused operation, store.
+//                 ring of (A 128x64, B BNx64) fp16 stages, mbarrier complete_tx; the ring runs on
+//                 across tile boundaries;
+//   warp 1      : allocates 2 x BN TMEM columns (two accumulators), one thread issues
+//                 tcgen05.mma kind::f16 (M = 128, N = BN, K = 16, fp32 accumulate in TMEM);
+//                 tcgen05.commit releases stages and hands a finished accumulator over;
+//   warps 2..5  : epilogue -- tcgen05.ld 32 lanes x 32 columns per step, fused operation, store;
+//                 the accumulator is released back to the MMA warp, so the epilogue of tile i
+//                 overlaps the main loop of tile i + 1.
 // Epilogues: BIAS (fp32 out + fp16 bias), RESID (fp32 x += acc), SWIGLU (columns interleaved
-// gate/up -> fp16 silu(g) * u), F16 (fp16 out + fp16 bias).  Rows >= M are masked (TMA zero-fills the A tail).
-// Every mbarrier wait is bounded; TMEM is always released before the CTA exits.
+// gate/up -> fp16 silu(g) * u), F16 (fp16 out + fp16 bias).  Rows >= M are masked (TMA
+// zero-fills the A tail).  Every mbarrier wait is bounded; TMEM is released before the CTA exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -25,13 +30,19 @@
 namespace vv {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64;
 constexpr int kThreads = 192;
 constexpr uint32_t kStageA = BM * BK * 2;  // 16 KB
-constexpr uint32_t kStageB = BN * BK * 2;  // 32 KB
-constexpr uint32_t kTmemCols = 256;
-// instruction descriptor: D f32, A/B f16, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t kRingBytes = 192 * 1024;
+template <int BN>
+struct Cfg {
+  static constexpr uint32_t kStageB = BN * BK * 2;
+  static constexpr int kStages = kRingBytes / (kStageA + kStageB);  // 4 (BN 256) or 6 (BN 128)
+  static constexpr uint32_t kTmemCols = 2 * BN;                     // two accumulators
+  // instruction descriptor: D f32, A/B f16, both K-major, N = BN, M = 128
+  static constexpr uint32_t kIdesc =
+      (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   // start address >> 4 | LBO 16 B (unused for swizzled K-major) | SBO 1024 B (8 rows x 128 B)
@@ -89,24 +100,77 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <int EPI>
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, const float (&v)[32], int row,
+                                               int col) {
+  if (EPI == kEpiBias) {
+    float* out = e.out_f32 + (size_t)row * e.ldo + col;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float4 o;
+      o.x = v[j + 0] + (e.bias ? __half2float(e.bias[col + j + 0]) : 0.f);
+      o.y = v[j + 1] + (e.bias ? __half2float(e.bias[col + j + 1]) : 0.f);
+      o.z = v[j + 2] + (e.bias ? __half2float(e.bias[col + j + 2]) : 0.f);
+      o.w = v[j + 3] + (e.bias ? __half2float(e.bias[col + j + 3]) : 0.f);
+      *reinterpret_cast<float4*>(out + j) = o;
+    }
+  } else if (EPI == kEpiResid) {
+    float* out = e.out_f32 + (size_t)row * e.ldo + col;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float4 o = *reinterpret_cast<float4*>(out + j);
+      o.x += v[j + 0];
+      o.y += v[j + 1];
+      o.z += v[j + 2];
+      o.w += v[j + 3];
+      *reinterpret_cast<float4*>(out + j) = o;
+    }
+  } else if (EPI == kEpiF16) {
+    __half* out = e.out_f16 + (size_t)row * e.ldo + col;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      __half h8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        h8[t] = __float2half_rn(v[j + t] + (e.bias ? __half2float(e.bias[col + j + t]) : 0.f));
+      *reinterpret_cast<uint4*>(out + j) = *reinterpret_cast<uint4*>(h8);
+    }
+  } else {  // SwiGLU over interleaved (gate, up) columns -> fp16
+    __half* out = e.out_f16 + (size_t)row * e.ldo + col / 2;
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+      __half h4[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float g = v[2 * (j + t)], u = v[2 * (j + t) + 1];
+        h4[t] = __float2half_rn(g / (1.f + __expf(-g)) * u);
+      }
+      *reinterpret_cast<uint2*>(out + j) = *reinterpret_cast<uint2*>(h4);
+    }
+  }
+}
+
+template <int EPI, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmEpilogue e, const int M, const int N, const int K) {
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sA = smem;
   unsigned char* sB = smem + STAGES * kStageA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * kStageB);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::kStageB);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;    // [2] epilogue -> MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = N / BN;
-  const int m_blk = blockIdx.x / n_tiles, n_blk = blockIdx.x % n_tiles;
+  const int tiles = ((M + BM - 1) / BM) * n_tiles;
   const int kblocks = K / BK;
 
   if (threadIdx.x == 0) {
@@ -114,7 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(tmem_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+    }
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
@@ -122,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
+                 "r"(C::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -133,87 +200,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % STAGES;
-        if (kb >= STAGES) mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1);
-        mbar_arrive_expect_tx(&full[s], kStageA + kStageB);
-        tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m_blk * BM, &full[s]);
-        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, n_blk * BN, &full[s]);
+      int g = 0;  // running k-block counter across tiles
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (g >= STAGES) mbar_wait(&empty[s], ((g / STAGES) - 1) & 1);
+          mbar_arrive_expect_tx(&full[s], kStageA + C::kStageB);
+          tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m_blk * BM, &full[s]);
+          tma_load_2d(sB + s * C::kStageB, &tmB, kb * BK, n_blk * BN, &full[s]);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % STAGES;
-        mbar_wait(&full[s], (kb / STAGES) & 1);
+      int g = 0, i = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2) mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1);  // epilogue done with it
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * kStageB);
+        const uint32_t d = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % STAGES;
+          mbar_wait(&full[s], (g / STAGES) & 1);
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * C::kStageB);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)  // 32 bytes per K=16 slice inside the swizzled row
-          umma_f16(tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), kIdesc,
-                   (kb > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&empty[s]);  // stage free once these MMAs have read it
+          for (int k = 0; k < BK / 16; ++k)  // 32 bytes per K=16 slice inside the swizzled row
+            umma_f16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), C::kIdesc,
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);  // stage free once these MMAs have read it
+        }
+        umma_commit(&acc_full[buf]);  // accumulator complete
       }
-      umma_commit(tmem_full);  // accumulator complete
     }
     __syncwarp();
   } else {
     // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31
     const int q = warp & 3;
-    const int row = m_blk * BM + q * 32 + lane;
-    mbar_wait(tmem_full, 0);
-    tc_fence_after();
-    for (int c = 0; c < BN; c += 32) {
-      float v[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-      if (row < M) {
-        const int col = n_blk * BN + c;
-        if (EPI == kEpiBias) {
-          float* out = e.out_f32 + (size_t)row * e.ldo + col;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 o;
-            o.x = v[j + 0] + (e.bias ? __half2float(e.bias[col + j + 0]) : 0.f);
-            o.y = v[j + 1] + (e.bias ? __half2float(e.bias[col + j + 1]) : 0.f);
-            o.z = v[j + 2] + (e.bias ? __half2float(e.bias[col + j + 2]) : 0.f);
-            o.w = v[j + 3] + (e.bias ? __half2float(e.bias[col + j + 3]) : 0.f);
-            *reinterpret_cast<float4*>(out + j) = o;
-          }
-        } else if (EPI == kEpiResid) {
-          float* out = e.out_f32 + (size_t)row * e.ldo + col;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 o = *reinterpret_cast<float4*>(out + j);
-            o.x += v[j + 0];
-            o.y += v[j + 1];
-            o.z += v[j + 2];
-            o.w += v[j + 3];
-            *reinterpret_cast<float4*>(out + j) = o;
-          }
-        } else if (EPI == kEpiF16) {
-          __half* out = e.out_f16 + (size_t)row * e.ldo + col;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            __half h8[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              h8[t] = __float2half_rn(v[j + t] + (e.bias ? __half2float(e.bias[col + j + t]) : 0.f));
-            *reinterpret_cast<uint4*>(out + j) = *reinterpret_cast<uint4*>(h8);
-          }
-        } else {  // SwiGLU over interleaved (gate, up) columns -> fp16
-          __half* out = e.out_f16 + (size_t)row * e.ldo + col / 2;
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            __half h4[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float g = v[2 * (j + t)], u = v[2 * (j + t) + 1];
-              h4[t] = __float2half_rn(g / (1.f + __expf(-g)) * u);
-            }
-            *reinterpret_cast<uint2*>(out + j) = *reinterpret_cast<uint2*>(h4);
-          }
-        }
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+      const int buf = i & 1;
+      const int row = m_blk * BM + q * 32 + lane;
+      mbar_wait(&acc_full[buf], (i >> 1) & 1);
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(base + (uint32_t)c, v);
+        if (row < M) epilogue_chunk<EPI, BN>(e, v, row, n_blk * BN + c);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
@@ -221,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
+                 "r"(C::kTmemCols)
                  : "memory");
   }
 }
@@ -252,16 +292,6 @@ bool make_map(CUtensorMap* tm, const void* base, int rows, int cols, int box_row
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <int EPI>
-cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmEpilogue& e, int M,
-                     int N, int K, int tiles, size_t smem, cudaStream_t s) {
-  cudaError_t err =
-      cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  gemm_tc_kernel<EPI><<<tiles, kThreads, smem, s>>>(ta, tb, e, M, N, K);
-  return cudaGetLastError();
 }
 
 // One thread per 32-weight block: 16 code bytes + one fp16 scale in, 32 fp16 out (64 bytes).
@@ -312,23 +342,60 @@ cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __h
   return cudaGetLastError();
 }
 
-size_t gemm_tc_smem() { return STAGES * (kStageA + kStageB) + 2 * STAGES * 8 + 64 + 1024; }
+namespace {
 
-cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
-                           const GemmEpilogue& e, cudaStream_t s) {
-  if (M < 1 || N % BN != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
-  if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
+template <int BN>
+size_t smem_bytes() {
+  return Cfg<BN>::kStages * (kStageA + Cfg<BN>::kStageB) + 2 * Cfg<BN>::kStages * 8 + 4 * 8 + 16 +
+         1024;
+}
+
+template <int EPI, int BN>
+cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmEpilogue& e, int M,
+                     int N, int K, int grid, cudaStream_t s) {
+  const size_t smem = smem_bytes<BN>();
+  cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  gemm_tc_kernel<EPI, BN><<<grid, kThreads, smem, s>>>(ta, tb, e, M, N, K);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_bn(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                      const GemmEpilogue& e, cudaStream_t s) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
   const int tiles = ((M + BM - 1) / BM) * (N / BN);
-  const size_t smem = gemm_tc_smem();
+  const int grid = tiles < sm_count() ? tiles : sm_count();
   switch (epi) {
-    case kEpiBias: return run_gemm<kEpiBias>(ta, tb, e, M, N, K, tiles, smem, s);
-    case kEpiResid: return run_gemm<kEpiResid>(ta, tb, e, M, N, K, tiles, smem, s);
-    case kEpiSwiglu: return run_gemm<kEpiSwiglu>(ta, tb, e, M, N, K, tiles, smem, s);
-    case kEpiF16: return run_gemm<kEpiF16>(ta, tb, e, M, N, K, tiles, smem, s);
+    case kEpiBias: return run_gemm<kEpiBias, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiResid: return run_gemm<kEpiResid, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiSwiglu: return run_gemm<kEpiSwiglu, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiF16: return run_gemm<kEpiF16, BN>(ta, tb, e, M, N, K, grid, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+}  // namespace
+
+size_t gemm_tc_smem() { return smem_bytes<256>(); }
+
+// Wave efficiency of a tile count on the SMs: tiles / (waves * SMs).
+static double wave_eff(long tiles, int sms) {
+  const long waves = (tiles + sms - 1) / sms;
+  return (double)tiles / (double)(waves * sms);
+}
+
+cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s) {
+  if (M < 1 || N % 128 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
+  if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
+  const int sms = sm_count();
+  const long mt = (M + BM - 1) / BM;
+  // 256-wide tiles unless 128-wide ones fill the last wave clearly better (or N needs them)
+  const bool wide = N % 256 == 0 && wave_eff(mt * (N / 256), sms) >= wave_eff(mt * (N / 128), sms) - 0.1;
+  return wide ? launch_bn<256>(A, B, M, N, K, epi, e, s) : launch_bn<128>(A, B, M, N, K, epi, e, s);
 }
 
 }  // namespace vv
@@ -344,7 +411,7 @@ extern "C" vv_status vv_matmul_nbits_tc(const uint16_t* x, const uint8_t* q,
   VV_CHECK_SHAPE(block == 32, "vv_matmul_nbits_tc: block %d (only 32)", block);
   VV_CHECK_SHAPE(K >= 64 && K % 64 == 0 && K < (1 << 24), "vv_matmul_nbits_tc: K=%lld",
                  (long long)K);
-  VV_CHECK_SHAPE(N >= 256 && N % 256 == 0 && N < (1 << 24), "vv_matmul_nbits_tc: N=%lld",
+  VV_CHECK_SHAPE(N >= 128 && N % 128 == 0 && N < (1 << 24), "vv_matmul_nbits_tc: N=%lld",
                  (long long)N);
   VV_CHECK_SHAPE(M >= 1 && M < (1 << 24), "vv_matmul_nbits_tc: M=%lld", (long long)M);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
