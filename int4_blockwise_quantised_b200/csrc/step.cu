@@ -40,6 +40,8 @@ constexpr int NW = 15;                 // compute warps (+1 producer: 512 thread
 constexpr int kThreads = (NW + 1) * 32;
 constexpr int D = 128;
 constexpr int TT = 64;                 // attention tile (positions)
+constexpr int kRowH = D + 8;           // halves per K/V row in a stage: 272 bytes, so consecutive
+                                       // rows start 4 banks apart (conflict-free 16-byte reads)
 constexpr int kMaxG = 8;
 constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
@@ -166,6 +168,20 @@ __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t 
     if (c[i].bytes) bulk_g2s_stream(dst + c[i].dst_off, c[i].src, c[i].bytes, &r.full[slot], pol);
 }
 
+// One attention tile: `rows` past K rows and V rows (256 bytes each) into the padded row layout
+// (kRowH halves per row; V after TT K rows).
+__device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int rows, uint64_t pol) {
+  const int s = r.idx++;
+  const int slot = s % r.nstages;
+  if (s >= r.nstages) ring_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
+  mbar_arrive_expect_tx(&r.full[slot], (uint32_t)rows * D * 2 * 2);
+  unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
+  for (int i = 0; i < rows; ++i) {
+    bulk_g2s_stream(dst + (size_t)i * kRowH * 2, k + (size_t)i * D, D * 2, &r.full[slot], pol);
+    bulk_g2s_stream(dst + (size_t)(TT + i) * kRowH * 2, v + (size_t)i * D, D * 2, &r.full[slot], pol);
+  }
+}
+
 // Stream rows [r0, r1) of a packed matrix (and optionally the same rows of a second one).
 __device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, const uint8_t* q1,
                                const __half* s1, int K, int r0, int r1, uint64_t pol) {
@@ -211,10 +227,8 @@ __device__ void producer(const StepParams& p, Ring& r, int past) {
     for (int it = cta; it < Hkv * nt; it += ncta) {
       const int g = it / nt, t = it % nt;
       const int p0 = t * TT, p1 = min(p0 + TT, past);
-      const uint32_t bytes = p1 > p0 ? (uint32_t)(p1 - p0) * D * 2 : 0u;
       const size_t off = ((size_t)(l * Hkv + g) * p.cap + p0) * D;
-      Copy c[2] = {Copy{p.k_cache + off, bytes, 0u}, Copy{p.v_cache + off, bytes, TT * D * 2}};
-      produce(r, c, 2, pol);
+      produce_kv_rows(r, p.k_cache + off, p.v_cache + off, max(p1 - p0, 0), pol);
     }
     cta_range(H, cta, ncta, r0, r1);
     produce_packed(r, w.q[3], w.s[3], nullptr, nullptr, Hq * D, r0, r1, pol);
@@ -596,7 +610,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   const int slot = s % r.nstages;
   ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
   __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
-  __half* vt = kt + TT * D;
+  __half* vt = kt + TT * kRowH;
   if (newpos && tid < D) {  // this tile holds the new position: rotate k, append k/v
     const int d = tid, fi = d & (D / 2 - 1);
     const float cs = as.cs[fi], sn = as.sn[fi];
@@ -605,22 +619,22 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     const size_t off = ((size_t)(l * p.Hkv + g) * p.cap + past) * D + d;
     p.k_cache[off] = kn;
     p.v_cache[off] = vn;
-    kt[(past - p0) * D + d] = kn;
-    vt[(past - p0) * D + d] = vn;
+    kt[(past - p0) * kRowH + d] = kn;
+    vt[(past - p0) * kRowH + d] = vn;
   }
   cbar();
-  // scores: warp w -> head w/2, positions (w%2)*32 + lane; chunk order rotated by lane so the
-  // 16-byte k loads of a warp hit distinct banks.
+  // scores: warp w -> head w/2, positions (w%2)*32 + lane.  All lanes walk the chunks in the same
+  // order, so the q reads are broadcasts; the padded K rows keep the k reads conflict-free.
   for (int item = warp; item < 2 * G; item += NW) {
     const int h = item >> 1, pp = (item & 1) * 32 + lane;
     {
       float sc = -INFINITY;
       if (pp < n) {
-        const __half* kr = kt + pp * D;
+        const __half* kr = kt + pp * kRowH;
         float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-          const int cc = (c + lane) & 15;
+          const int cc = c;
           const uint4 kv = *reinterpret_cast<const uint4*>(kr + cc * 8);
           const float4 qa = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
           const float4 qb = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
@@ -650,17 +664,18 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     }
   }
   cbar();
-  // P.V: unit = (head h, 8-dim octet o, position quarter q); V rows read as 16-byte vectors,
-  // quarters combined through shared memory (as.pv), then written as the tile's partial.
+  // P.V: unit = (head h, 8-dim octet o, position quarter q); V rows read as 16-byte vectors (the
+  // 16 octets of a row on consecutive lanes: conflict-free), quarters combined through shared
+  // memory (as.pv), then written as the tile's partial.
   {
     const int units = G * 16 * 4;
     for (int u = tid; u < units; u += NW * 32) {
-      const int q = u & 3, o = (u >> 2) & 15, h = u >> 6;
+      const int o = u & 15, q = (u >> 4) & 3, h = u >> 6;
       float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
       const float* ph = as.s[h];
       const int p_end = min(n, q * 16 + 16);
       for (int pp = q * 16; pp < p_end; ++pp) {
-        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * D + o * 8);
+        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * kRowH + o * 8);
         const float w = ph[pp];
         const float2 ww = make_float2(w, w);
         a0 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.x)), ww, a0);
@@ -1062,7 +1077,8 @@ cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
                                        (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   *blocks_per_sm = 0;
-  for (; p.stage_bytes >= 32 * 1024; p.stage_bytes -= 1024) {
+  // a stage must hold one attention tile: 2 x TT padded rows of kRowH halves (34 KB)
+  for (; p.stage_bytes >= 2 * TT * kRowH * 2; p.stage_bytes -= 1024) {
     const size_t smem = step_smem_bytes(p.stage_bytes, p.nstages, p.x_floats);
     e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
