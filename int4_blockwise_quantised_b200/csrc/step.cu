@@ -156,10 +156,27 @@ __device__ __forceinline__ void ring_wait(Ring& r, uint64_t* bar, uint32_t parit
   if (r.tapw) r.tapw[r.ph] += dt;
 }
 
+// The producer's wait for a free slot: it runs stages ahead of the consumers, so it sleeps
+// between polls instead of spinning through the issue slots its SM sub-partition shares with
+// compute warps.  Bounded like every wait (kWaitLimitNs).
+__device__ __forceinline__ void producer_wait(Ring& r, uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  for (unsigned it = 1;; ++it) {
+    __nanosleep(256);
+    if (mbar_try_wait(bar, parity)) break;
+    if ((it & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_device_error(VV_ERR_TIMEOUT);
+      break;
+    }
+  }
+  r.wait_ns += globaltimer_ns() - t0;
+}
+
 __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t pol) {
   const int s = r.idx++;
   const int slot = s % r.nstages;
-  if (s >= r.nstages) ring_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
+  if (s >= r.nstages) producer_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
   uint32_t tot = 0;
   for (int i = 0; i < n; ++i) tot += c[i].bytes;
   mbar_arrive_expect_tx(&r.full[slot], tot);
@@ -173,7 +190,7 @@ __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t 
 __device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int rows, uint64_t pol) {
   const int s = r.idx++;
   const int slot = s % r.nstages;
-  if (s >= r.nstages) ring_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
+  if (s >= r.nstages) producer_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
   mbar_arrive_expect_tx(&r.full[slot], (uint32_t)rows * D * 2 * 2);
   unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
   for (int i = 0; i < rows; ++i) {
@@ -204,6 +221,28 @@ __device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, con
   }
 }
 
+// Stream logical rows [r0, r1) of [Wq; Wk; Wv] (bounds: first row of each matrix); a stage may
+// hold rows of two matrices, laid out as one matrix of consecutive rows.
+__device__ void produce_qkv(Ring& r, const StepLayer& w, int K, int r0, int r1,
+                            const int (&bounds)[4], uint64_t pol) {
+  const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
+  const int rps = phase_rps(K, 1, r.stage_bytes);
+  for (int a = r0; a < r1; a += rps) {
+    const int n = min(rps, r1 - a);
+    Copy c[6];
+    int k = 0;
+    for (int m = 0; m < 3; ++m) {
+      const int lo = max(a, bounds[m]), hi = min(a + n, bounds[m + 1]);
+      if (lo >= hi) continue;
+      c[k++] = Copy{w.q[m] + (size_t)(lo - bounds[m]) * rq, (uint32_t)((hi - lo) * rq),
+                    (uint32_t)((lo - a) * rq)};
+      c[k++] = Copy{reinterpret_cast<const unsigned char*>(w.s[m]) + (size_t)(lo - bounds[m]) * rs,
+                    (uint32_t)((hi - lo) * rs), (uint32_t)(rps * rq + (lo - a) * rs)};
+    }
+    produce(r, c, k, pol);
+  }
+}
+
 // Tiles (kv head g, tile t) owned by this CTA: items i = cta + k * ncta < Hkv * ntiles.
 __device__ __forceinline__ int ntiles_for(int past) { return (past + 1 + TT - 1) / TT; }
 
@@ -219,10 +258,7 @@ __device__ void producer(const StepParams& p, Ring& r, int past) {
     int r0, r1;
     cta_range(nqkv, cta, ncta, r0, r1);
     const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
-    for (int m = 0; m < 3; ++m) {
-      const int a = max(r0, bounds[m]), b = min(r1, bounds[m + 1]);
-      if (a < b) produce_packed(r, w.q[m], w.s[m], nullptr, nullptr, H, a - bounds[m], b - bounds[m], pol);
-    }
+    produce_qkv(r, w, H, r0, r1, bounds, pol);
     // ATTN: past K/V rows of the tiles
     for (int it = cta; it < Hkv * nt; it += ncta) {
       const int g = it / nt, t = it % nt;
@@ -870,15 +906,10 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       }
       if (regH) load_xr(xs, xr, H);
       cbar();
-      for (int m = 0; m < 3; ++m) {
-        const int a = max(r0, bounds[m]), b = min(r1, bounds[m + 1]);
-        if (a < b) {
-          float* out = p.qkv + bounds[m];
-          const float* bs = bias_s + (bounds[m] - r0);
-          consume_packed(r, xs, xr, regH, H, a - bounds[m], b - bounds[m], 1, &as.s[0][0],
-                         [&](int row, float y, float) { out[row] = y + bs[row]; });
-        }
-      }
+      // [Wq; Wk; Wv] as one matrix of nqkv rows (the producer joins the segments)
+      const float* bs = bias_s - r0;
+      consume_packed(r, xs, xr, regH, H, r0, r1, 1, &as.s[0][0],
+                     [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
     }
     // ---------------------------------------------------------------- ATTN
     r.ph = 1;
