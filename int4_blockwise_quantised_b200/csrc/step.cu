@@ -117,13 +117,18 @@ __device__ __forceinline__ int rows_per_stage(int row_bytes, int nseg, int stage
   return r > 64 ? 64 : r;
 }
 
-// Rows per stage of a phase: bounded by the stage size, and for the split-K (large K) path by
-// kSplitRows so that kSplitRows x kSplitW = NW warps share a stage.
+// Rows per stage of a phase: bounded by the stage size, and for the split-K (large K, few rows)
+// path by kSplitRows so that kSplitRows x kSplitW = NW warps share a stage.  `rows` is the
+// CTA's row count for the phase: with x in shared memory and at least 2 NW units, warps take
+// whole rows instead (row mode) and stages are filled.  Producer and consumers compute the same.
 constexpr int kSplitW = 3;                // warps per row when K is large
 constexpr int kSplitRows = NW / kSplitW;  // 5 rows per stage
-__device__ __forceinline__ int phase_rps(int K, int nseg, int stage_bytes) {
+__device__ __forceinline__ bool row_mode(int K, int nseg, int rows) {
+  return K > 32 * kRegHB * 16 && rows * nseg >= 2 * NW;
+}
+__device__ __forceinline__ int phase_rps(int K, int nseg, int stage_bytes, int rows) {
   const int r = rows_per_stage((K >> 5) * 18, nseg, stage_bytes);
-  return K > 32 * kRegHB * 16 ? min(r, kSplitRows) : r;
+  return (K > 32 * kRegHB * 16 && !row_mode(K, nseg, rows)) ? min(r, kSplitRows) : r;
 }
 
 struct Ring {
@@ -204,7 +209,7 @@ __device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, con
                                const __half* s1, int K, int r0, int r1, uint64_t pol) {
   const int nseg = q1 ? 2 : 1;
   const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
-  const int rps = phase_rps(K, nseg, r.stage_bytes);
+  const int rps = phase_rps(K, nseg, r.stage_bytes, r1 - r0);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     Copy c[4];
@@ -226,7 +231,7 @@ __device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, con
 __device__ void produce_qkv(Ring& r, const StepLayer& w, int K, int r0, int r1,
                             const int (&bounds)[4], uint64_t pol) {
   const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
-  const int rps = phase_rps(K, 1, r.stage_bytes);
+  const int rps = phase_rps(K, 1, r.stage_bytes, r1 - r0);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     Copy c[6];
@@ -381,6 +386,57 @@ __device__ __forceinline__ float hb_doth(uint2 wv, uint4 xa, uint4 xb) {
   return dot8_h(wv.x, xa) + dot8_h(wv.y, xb);
 }
 
+// One stage with x in shared memory and whole rows per warp (large K, rows plentiful): warp w
+// takes units [w R, w R + R), lanes stride the half-blocks, one shuffle reduction per unit; no
+// cross-warp reduction, so no barrier inside the stage.
+template <int R, class RowQ, class RowS, class Fin>
+__device__ __forceinline__ void smemx_pass(RowQ rowq, RowS rows, const uint4* xs4, int K, int units,
+                                           int nseg, int a, Fin fin) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NHB = K >> 4;
+  for (int u0 = warp * R; u0 < units; u0 += NW * R) {
+    const unsigned char* wq[R];
+    const __half* ws[R];
+    int lr[R];
+    bool ok[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int u = u0 + k;
+      ok[k] = u < units;
+      const int uu = ok[k] ? u : u0;
+      const int sg = nseg == 2 ? (uu & 1) : 0;
+      lr[k] = nseg == 2 ? (uu >> 1) : uu;
+      wq[k] = rowq(sg, lr[k]);
+      ws[k] = rows(sg, lr[k]);
+    }
+    float acc[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) acc[k] = 0.f;
+#pragma unroll 2
+    for (int hb = lane; hb < NHB; hb += 32) {
+      const uint4 xa = xs4[hb], xb = xs4[NHB + hb];
+#pragma unroll
+      for (int k = 0; k < R; ++k) {
+        const uint2 wv = *reinterpret_cast<const uint2*>(wq[k] + hb * 8);
+        acc[k] = fmaf(__half2float(ws[k][hb >> 1]), hb_doth(wv, xa, xb), acc[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) acc[k] = warp_sum(acc[k]);
+    if (lane == 0) {
+      if (nseg == 2) {
+#pragma unroll
+        for (int k = 0; k + 1 < R; k += 2)
+          if (ok[k]) fin(a + lr[k], acc[k], acc[k + 1]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < R; ++k)
+          if (ok[k]) fin(a + lr[k], acc[k], 0.f);
+      }
+    }
+  }
+}
+
 // One stage of the register-x path: warp w takes units [w R, w R + R), then [w R + NW R, ...);
 // unit u is (segment, row) = (u & 1, u >> 1) for gate/up pairs, else (0, u).  Lanes stride the
 // half-blocks; one shuffle reduction per unit; lane 0 finishes the rows.
@@ -444,7 +500,8 @@ __device__ __forceinline__ void consume_packed(Ring& r, const __half* xs, const 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = K >> 5, NHB = K >> 4;
   const int rq = KB * 16, rs = KB * 2;
-  const int rps = phase_rps(K, nseg, r.stage_bytes);
+  const int rps = phase_rps(K, nseg, r.stage_bytes, r1 - r0);
+  const bool rowmode = row_mode(K, nseg, r1 - r0);
   const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
@@ -468,6 +525,8 @@ __device__ __forceinline__ void consume_packed(Ring& r, const __half* xs, const 
         regx_pass<2>(rowq, rows, xr, K, units, nseg, a, fin);
       else
         regx_pass<4>(rowq, rows, xr, K, units, nseg, a, fin);
+    } else if (rowmode) {
+      smemx_pass<2>(rowq, rows, xs4, K, n * nseg, nseg, a, fin);
     } else {
       // split-K: warp w -> row w / kSplitW, slice w % kSplitW
       const int lrow = warp / kSplitW, slice = warp % kSplitW;

@@ -111,6 +111,20 @@ def test_small_ternary_long_context():
     run_steps(synth.SHAPE_SMALL, "ternary", 4530, 2)
 
 
+def test_wide_hidden_row_mode():
+    """hidden 2048 > 1536: x no longer fits in registers; gate/up (38 pairs per CTA) runs whole
+    rows per warp with x in shared memory, the other phases split K over warps."""
+    shape = synth.Shape("wide", 2048, 2, 16, 2, 128, 5632, 4099, tied=True)
+    run_steps(shape, "int4", 300, 2)
+
+
+def test_single_layer_7b_shapes():
+    """One decoder layer at 7B shapes (hidden 3584, 28/4 heads, intermediate 18944, untied
+    152064-row head): q/k/v (31 rows per CTA) and gate/up in row mode, o-proj and down split-K."""
+    shape = synth.Shape("layer7b", 3584, 1, 28, 4, 128, 18944, 152064, tied=False)
+    run_steps(shape, "int4", 128, 1)
+
+
 def test_graph_and_plain_launches_bit_identical():
     from int4_blockwise_quantised_b200.model import Decoder
 
