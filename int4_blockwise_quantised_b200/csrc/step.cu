@@ -809,28 +809,49 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   if (!as.is_last) return;
   __threadfence();
   const float* base = p.attn_part + (size_t)g * p.max_tiles * kMaxG * kPart;
-  if (warp < G) {
+  if (warp < G) {  // merge weights of head h: every m, l load in flight at once
     const int h = warp;
+    constexpr int kPer = 256 / 32;  // nt <= max_tiles <= 256
+    float mv[kPer], lv[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int c = lane + 32 * j;
+      mv[j] = -INFINITY;
+      lv[j] = 0.f;
+      if (c < nt) {
+        const float* pp = base + ((size_t)c * kMaxG + h) * kPart;
+        mv[j] = __ldcg(pp);
+        lv[j] = __ldcg(pp + 1);
+      }
+    }
     float mx = -INFINITY;
-    for (int c = lane; c < nt; c += 32) mx = fmaxf(mx, __ldcg(base + ((size_t)c * kMaxG + h) * kPart));
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) mx = fmaxf(mx, mv[j]);
     mx = warp_max(mx);
     float L = 0.f;
-    for (int c = lane; c < nt; c += 32) {
-      const float* pp = base + ((size_t)c * kMaxG + h) * kPart;
-      const float e = exp2f(__ldcg(pp) - mx);
-      as.mw[c][h] = e;
-      L += __ldcg(pp + 1) * e;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      mv[j] = exp2f(mv[j] - mx);  // 0 for absent tiles
+      L = fmaf(lv[j], mv[j], L);
     }
     L = warp_sum(L);
     const float inv = 1.f / L;
-    for (int c = lane; c < nt; c += 32) as.mw[c][h] *= inv;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+      if (lane + 32 * j < nt) as.mw[lane + 32 * j][h] = mv[j] * inv;
   }
   cbar();
-  for (int idx = tid; idx < G * (D / 4); idx += NW * 32) {
-    const int h = idx / (D / 4), d4 = idx % (D / 4);
+  // o merge: (head, 4-dim column) x tile half -> partial sums in as.pv, then the halves add up
+  const int cols = G * (D / 4);
+  const int halves = (NW * 32) / cols >= 2 ? 2 : 1;
+  const int tsplit = (nt + halves - 1) / halves;
+  for (int idx = tid; idx < cols * halves; idx += NW * 32) {
+    const int col = idx % cols, part = idx / cols;
+    const int h = col / (D / 4), d4 = col % (D / 4);
+    const int t0 = part * tsplit, t1 = min(nt, t0 + tsplit);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < nt; c0 += 8) {
-      const int m = min(8, nt - c0);
+    for (int c0 = t0; c0 < t1; c0 += 8) {
+      const int m = min(8, t1 - c0);
       float4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -846,6 +867,19 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
           acc.w = fmaf(w, v[u].w, acc.w);
         }
       }
+    }
+    *reinterpret_cast<float4*>(&as.pv[part][h][4 * d4]) = acc;
+  }
+  cbar();
+  for (int idx = tid; idx < cols; idx += NW * 32) {
+    const int h = idx / (D / 4), d4 = idx % (D / 4);
+    float4 acc = *reinterpret_cast<const float4*>(&as.pv[0][h][4 * d4]);
+    if (halves == 2) {
+      const float4 b2 = *reinterpret_cast<const float4*>(&as.pv[1][h][4 * d4]);
+      acc.x += b2.x;
+      acc.y += b2.y;
+      acc.z += b2.z;
+      acc.w += b2.w;
     }
     *reinterpret_cast<float4*>(p.attn_out + (size_t)(g * G + h) * D + 4 * d4) = acc;
   }
