@@ -100,6 +100,23 @@ def step_bytes(shape, P):
     return shape.layers * sum(v for k, v in b.items() if k != "lm_head") + b["lm_head"]
 
 
+# ----------------------------------------------------------------------------------- ranks
+def max_over_ranks(value, dist, device):
+    """The slowest rank's value (every rank gets it); the identity without a process group."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units of all ranks per second over the max-over-ranks time `ms` (weak scaling)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ----------------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -209,6 +226,16 @@ def oracle_sample_time(shape, mode, P, samples=8):
     return statistics.median(ts), o.describe(samples), blas_threads()
 
 
+def oracle_sample_time_1thread(shape, mode, P, samples=3):
+    """The same oracle sample with BLAS limited to one thread."""
+    from threadpoolctl import threadpool_limits
+
+    o = OracleSample(shape, mode, P)
+    with threadpool_limits(limits=1):
+        ts = [o.run() for _ in range(samples)]
+    return statistics.median(ts), o.describe(samples)
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -293,13 +320,24 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     dec.sync_status()
     ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     ms_per_step = ms / args.steps
-    tok_s = world * args.steps / (ms / 1e3)
+    tok_s = whole_job_rate(args.steps, world, ms)
     gpu_launches = args.steps * (n_launch + 1) + extra  # + the position increment per step
+
+    # -------------------------------------- per-step distribution (one sequence, not timed above)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(seq + 1)]
+    torch.cuda.synchronize()
+    step_ev[0].record(stream)
+    for i in range(seq):
+        one_step(i)
+        step_ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per_step = sorted(step_ev[i].elapsed_time(step_ev[i + 1]) * 1e3 for i in range(seq))
+    pct = {"p50": round(per_step[len(per_step) // 2], 2),
+           "p90": round(per_step[min(len(per_step) - 1, (9 * len(per_step)) // 10)], 2),
+           "steps": seq, "note": "per-step CUDA events over one sequence of steps from P "
+                                 "(includes the position increment), outside the timed region"}
 
     # ---------------------------------------------------------------- e2e (host buffers)
     emb_host = torch.from_numpy(synth.input_embeds(shape, 1)[0]).pin_memory()
@@ -334,11 +372,8 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_tok_s = world * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+    e2e_tok_s = whole_job_rate(e2e_steps, world, e2e_ms)
 
     # -------------------------------------------------- roofline of the dominant kernel
     # One persistent cooperative kernel per step: its average launch duration is the timed
@@ -371,6 +406,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (weights %.0f MB, L2 126 MB); no flush" % (
                        sb / 1e6)},
         "step_us": round(ms_per_step * 1e3, 2),
+        "step_us_percentiles": pct,
         "hbm_gbs": round(sb / (ms_per_step * 1e-3) / 1e9, 1),
         "hbm_frac_of_measured": round(sb / (ms_per_step * 1e-3) / 1e9 / peak, 4),
         "hbm_frac_of_8tbs": round(sb / (ms_per_step * 1e-3) / 8e12, 4),
@@ -399,7 +435,14 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         st, sample, thr = oracle_sample_time(shape, mode, P)
         result["cpu_baseline"] = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr,
-                                  "kind": "oracle", "sample": sample}
+                                  "kind": "oracle", "sample": sample,
+                                  "host_cpus": os.cpu_count()}
+        try:
+            st1, sample1 = oracle_sample_time_1thread(shape, mode, P)
+            result["cpu_baseline"]["one_thread"] = {"value": round(1.0 / st1, 4), "unit": "tok/s",
+                                                    "cores": 1, "sample": sample1}
+        except Exception as e:  # threadpoolctl missing: report the all-cores figure only
+            result["cpu_baseline"]["one_thread"] = {"error": str(e)[:200]}
     if dec is not None:
         dec.close()
     if dist:
@@ -450,10 +493,7 @@ def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
     clk = clocks.stop()
     dec.sync_status()
     ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     ms_per = ms / steps
     # end to end: host buffers in, greedy token out
     ids_h, pos_h, feats_h = (torch.from_numpy(a).pin_memory() for a in (ids, pos, feats))
@@ -473,10 +513,7 @@ def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
     kind_ms, kind_n = dec.profile_init(ids_d, pos_d, feats_d, off, logits=logits, argmax=am)
     dec.sync_status()
     dec.close()
@@ -488,7 +525,7 @@ def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
     kind = "measured" if mp else "fallback"
     gemm_ms = kind_ms["gemm"]
     ach = fl["gemm"] / (gemm_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 kind::f16, persistent, 128x256 or 128x128 tiles, 2 TMEM accumulators)",
+    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 kind::f16, persistent, 128 x 256, 192 or 128 tiles, 2 TMEM accumulators)",
             "achieved": round(ach, 1), "peak": peak, "peak_kind": f"{kind} bf16 burst (fp16 dense "
             "rate = bf16 on B200, nominal ratio 1)", "unit": "TFLOP/s",
             "frac": round(ach / peak, 4), "frac_of_sustained": round(ach / peak_sus, 4),
