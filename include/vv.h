@@ -109,7 +109,7 @@ vv_status vv_matmul_nbits(const uint16_t* x, const uint8_t* q, const uint16_t* s
  *   y[m, n] = fp16( sum_k x[m, k] * w16[n, k]  (+ bias[n]) ),  w16 = fp16((code - 8) * scale)
  * Two launches: W is dequantised into w_f16 (caller's device scratch, fp16 [N, K], overwritten),
  * then a tcgen05 tensor-core GEMM (fp16 operands, fp32 accumulation in tensor memory) writes y.
- * Same operands as vv_matmul_nbits; any M >= 1.  Requirements: N % 256 == 0, K % 64 == 0,
+ * Same operands as vv_matmul_nbits; any M >= 1.  Requirements: N % 128 == 0 or N % 192 == 0, K % 64 == 0,
  * block == 32, all pointers 16-byte aligned, M < 2^24.  The fp16 rounding of each dequantised
  * weight is the only difference from vv_matmul_nbits' arithmetic.
  * Errors: VV_ERR_INVALID_ARG (null, misaligned), VV_ERR_SHAPE (N, K, M out of range). */

@@ -2,8 +2,8 @@
 // (Prefill of decoder_init, "vibevoice-asr-bitnet-onnx": decoder_init contract; all projections
 // of the S prompt positions are real dense contractions.)
 //
-// Persistent: one CTA per SM walks the 128 x BN output tiles (BN = 256, or 128 when that fills
-// the last wave of SMs better), K in blocks of 64.
+// Persistent: one CTA per SM walks the 128 x BN output tiles (BN = 256, 192 or 128: the widest
+// that fills the last wave of SMs about as well as any), K in blocks of 64.
 //   warp 0      : TMA producer (cp.async.bulk.tensor 2D, 128-byte swizzle, no multicast) into a
 //                 ring of (A 128x64, B BNx64) fp16 stages, mbarrier complete_tx; the ring runs on
 //                 across tile boundaries;
@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "vv_device.cuh"
@@ -37,8 +38,9 @@ constexpr uint32_t kRingBytes = 192 * 1024;
 template <int BN>
 struct Cfg {
   static constexpr uint32_t kStageB = BN * BK * 2;
-  static constexpr int kStages = kRingBytes / (kStageA + kStageB);  // 4 (BN 256) or 6 (BN 128)
-  static constexpr uint32_t kTmemCols = 2 * BN;                     // two accumulators
+  static constexpr int kStages = kRingBytes / (kStageA + kStageB);  // 4 (BN 256, 192), 6 (BN 128)
+  // two accumulators of BN columns; the allocation is a power of two
+  static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;
   // instruction descriptor: D f32, A/B f16, both K-major, N = BN, M = 128
   static constexpr uint32_t kIdesc =
       (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
@@ -389,13 +391,22 @@ static double wave_eff(long tiles, int sms) {
 
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
-  if (M < 1 || N % 128 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
+  if (M < 1 || N % 64 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
   if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
   const int sms = sm_count();
   const long mt = (M + BM - 1) / BM;
-  // 256-wide tiles unless 128-wide ones fill the last wave clearly better (or N needs them)
-  const bool wide = N % 256 == 0 && wave_eff(mt * (N / 256), sms) >= wave_eff(mt * (N / 128), sms) - 0.1;
-  return wide ? launch_bn<256>(A, B, M, N, K, epi, e, s) : launch_bn<128>(A, B, M, N, K, epi, e, s);
+  // the widest tile whose wave efficiency is within 0.1 of the best available width
+  const int widths[3] = {256, 192, 128};
+  double best = 0.0;
+  for (int w : widths)
+    if (N % w == 0) best = std::max(best, wave_eff(mt * (N / w), sms));
+  for (int w : widths) {
+    if (N % w != 0 || wave_eff(mt * (N / w), sms) < best - 0.1) continue;
+    if (w == 256) return launch_bn<256>(A, B, M, N, K, epi, e, s);
+    if (w == 192) return launch_bn<192>(A, B, M, N, K, epi, e, s);
+    return launch_bn<128>(A, B, M, N, K, epi, e, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace vv
@@ -411,7 +422,8 @@ extern "C" vv_status vv_matmul_nbits_tc(const uint16_t* x, const uint8_t* q,
   VV_CHECK_SHAPE(block == 32, "vv_matmul_nbits_tc: block %d (only 32)", block);
   VV_CHECK_SHAPE(K >= 64 && K % 64 == 0 && K < (1 << 24), "vv_matmul_nbits_tc: K=%lld",
                  (long long)K);
-  VV_CHECK_SHAPE(N >= 128 && N % 128 == 0 && N < (1 << 24), "vv_matmul_nbits_tc: N=%lld",
+  VV_CHECK_SHAPE(N >= 128 && (N % 128 == 0 || N % 192 == 0) && N < (1 << 24),
+                 "vv_matmul_nbits_tc: N=%lld",
                  (long long)N);
   VV_CHECK_SHAPE(M >= 1 && M < (1 << 24), "vv_matmul_nbits_tc: M=%lld", (long long)M);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -20,7 +20,7 @@ struct GemmEpilogue {
 };
 
 size_t gemm_tc_smem();
-// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 256 == 0, K % 64 == 0.
+// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 128 == 0 or N % 192 == 0, K % 64 == 0.
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s);
 

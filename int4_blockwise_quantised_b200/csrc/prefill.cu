@@ -80,36 +80,60 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const float* __restri
 }
 
 // RoPE of q and k at position_ids[s], then Q -> fp16 [S, Hq*D]; K, V -> cache slot s (fp16).
-// grid (S, Hq + 2*Hkv), block 128 (one thread per dim).
-__global__ void __launch_bounds__(128) rope_kv_kernel(const float* __restrict__ qkv, int S,
+// One CTA per position; each thread takes 8 consecutive dims of one head (vector loads of x and
+// of its rotate-half partner, one 16-byte store).
+__global__ void __launch_bounds__(256) rope_kv_kernel(const float* __restrict__ qkv, int S,
                                                       int Hq, int Hkv, const int32_t* __restrict__ pos_ids,
                                                       const float* __restrict__ cos_t,
                                                       const float* __restrict__ sin_t, int max_pos,
                                                       __half* __restrict__ q_out,
                                                       __half* __restrict__ kc, __half* __restrict__ vc,
                                                       int cap) {
-  const int s = blockIdx.x, hh = blockIdx.y, d = threadIdx.x;
-  const int nqkv = (Hq + 2 * Hkv) * D;
-  const float* row = qkv + (size_t)s * nqkv;
-  if (hh >= Hq + Hkv) {  // value head
-    const int g = hh - Hq - Hkv;
-    vc[((size_t)g * cap + s) * D + d] = __float2half_rn(row[hh * D + d]);
-    return;
-  }
+  const int s = blockIdx.x;
+  const int nh = Hq + 2 * Hkv;
   int pos = pos_ids[s];
   if (pos < 0 || pos >= max_pos) {
-    if (d == 0) set_device_error(VV_ERR_RANGE);
+    if (threadIdx.x == 0) set_device_error(VV_ERR_RANGE);
     pos = min(max(pos, 0), max_pos - 1);
   }
-  const int fi = d & (D / 2 - 1);
-  const float cs = cos_t[(size_t)pos * (D / 2) + fi], sn = sin_t[(size_t)pos * (D / 2) + fi];
-  const float x1 = row[hh * D + fi], x2 = row[hh * D + fi + D / 2];
-  const float y = d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
-  if (hh < Hq) {
-    q_out[(size_t)s * Hq * D + hh * D + d] = __float2half_rn(y);
-  } else {
-    const int g = hh - Hq;
-    kc[((size_t)g * cap + s) * D + d] = __float2half_rn(y);
+  const float* row = qkv + (size_t)s * nh * D;
+  for (int c = threadIdx.x; c < nh * (D / 8); c += blockDim.x) {
+    const int hh = c / (D / 8), d0 = (c % (D / 8)) * 8;
+    const float* hr = row + hh * D;
+    float y[8];
+    if (hh >= Hq + Hkv) {  // value head: no rotation
+      const float4 a = *reinterpret_cast<const float4*>(hr + d0);
+      const float4 b = *reinterpret_cast<const float4*>(hr + d0 + 4);
+      y[0] = a.x; y[1] = a.y; y[2] = a.z; y[3] = a.w;
+      y[4] = b.x; y[5] = b.y; y[6] = b.z; y[7] = b.w;
+    } else {
+      const int f0 = d0 & (D / 2 - 1);
+      float x1[8], x2[8], cs[8], sn[8];
+      *reinterpret_cast<float4*>(x1) = *reinterpret_cast<const float4*>(hr + f0);
+      *reinterpret_cast<float4*>(x1 + 4) = *reinterpret_cast<const float4*>(hr + f0 + 4);
+      *reinterpret_cast<float4*>(x2) = *reinterpret_cast<const float4*>(hr + f0 + D / 2);
+      *reinterpret_cast<float4*>(x2 + 4) = *reinterpret_cast<const float4*>(hr + f0 + D / 2 + 4);
+      const float* ct = cos_t + (size_t)pos * (D / 2) + f0;
+      const float* st = sin_t + (size_t)pos * (D / 2) + f0;
+      *reinterpret_cast<float4*>(cs) = *reinterpret_cast<const float4*>(ct);
+      *reinterpret_cast<float4*>(cs + 4) = *reinterpret_cast<const float4*>(ct + 4);
+      *reinterpret_cast<float4*>(sn) = *reinterpret_cast<const float4*>(st);
+      *reinterpret_cast<float4*>(sn + 4) = *reinterpret_cast<const float4*>(st + 4);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        y[j] = d0 < D / 2 ? x1[j] * cs[j] - x2[j] * sn[j] : x2[j] * cs[j] + x1[j] * sn[j];
+    }
+    __align__(16) __half h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = __float2half_rn(y[j]);
+    __half* dst;
+    if (hh < Hq)
+      dst = q_out + (size_t)s * Hq * D + (size_t)hh * D + d0;
+    else if (hh < Hq + Hkv)
+      dst = kc + ((size_t)(hh - Hq) * cap + s) * D + d0;
+    else
+      dst = vc + ((size_t)(hh - Hq - Hkv) * cap + s) * D + d0;
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
   }
 }
 
@@ -222,7 +246,7 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
                             S, NQKV, H, kEpiBias, ep, s)) != cudaSuccess)
       return e;
     VV_MARK(kPfGemm);
-    rope_kv_kernel<<<dim3(S, Hq + 2 * Hkv), D, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
+    rope_kv_kernel<<<S, 256, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
                                                       c.max_position, Q, kc, vc, c.kv_capacity);
     VV_MARK(kPfMisc);
     // ---- attention -> O (in the Xn buffer)

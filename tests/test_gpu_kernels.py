@@ -138,11 +138,11 @@ def test_gemm_tc_one_hot_layout_exact(vv):
         assert np.array_equal(Y[i], deq[:, k].astype(np.float16)), (i, k)
 
 
-# 256- and 128-wide tiles, a single tile, ragged M tails, and enough tiles (4530 x 2048) that
+# 256-, 192- and 128-wide tiles, a single tile, ragged M tails, and enough tiles (4530 rows) that
 # every CTA of the persistent grid cycles through both accumulators
 GEMM_TC_SHAPES = [(1, 256, 64), (37, 1024, 1536), (128, 2048, 1536), (129, 512, 8960),
                   (300, 1536, 8960), (513, 256, 3584), (600, 128, 64), (1000, 1536, 512),
-                  (4530, 2048, 1536)]
+                  (4530, 2048, 1536), (4530, 1536, 1536)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_TC_SHAPES)
