@@ -284,6 +284,21 @@ vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
                                   float* logits, int32_t* argmax_out, float* phase_ms,
                                   vv_stream stream);
 
+/* Greedy generation on the device ("vibevoice-asr-bitnet-onnx": the driver's greedy decode
+ * with stop tokens): up to n_steps decode steps, the token of step i being the argmax of step
+ * i - 1 (step 0: *first_token), positions *position, *position + 1, ...; each step appends to
+ * the KV cache like vv_decoder_step.  A step whose argmax is one of stop_ids (HOST array of
+ * n_stop <= 8 ids, e.g. 151645 and 151643) ends the generation: the remaining launches return
+ * at once.  first_token, position: device int32 [1]; tokens_out: device int32 [n_steps], entry i
+ * = argmax of step i (entries past the stop are untouched); n_out: HOST int32, the number of
+ * steps run (the stop token included).  Needs the persistent step kernel.  Synchronous: one host
+ * synchronisation for the whole generation.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (n_steps < 1), VV_ERR_CAPACITY (length + n_steps >
+ * capacity); device-side range errors as vv_decoder_step. */
+vv_status vv_decoder_generate(vv_decoder* dec, const int32_t* first_token, const int32_t* position,
+                              int32_t n_steps, const int32_t* stop_ids, int32_t n_stop,
+                              int32_t* tokens_out, int32_t* n_out, vv_stream stream);
+
 /* Profiling variant of vv_decoder_init: the same prefill (same arguments, same results and
  * cache contents), with a CUDA event recorded after every launch.  Synchronous.  phase_ms: HOST
  * float [5] and launches: HOST int32 [5] receive the device time and the number of launches (or

@@ -92,6 +92,8 @@ def _load():
         "vv_decoder_sync_status": (S, [P, P]),
         "vv_decoder_step_launches": (c_int32, [P]),
         "vv_decoder_profile_step": (S, [P, P, P, P, P, P, POINTER(c_float), P]),
+        "vv_decoder_generate": (S, [P, P, P, c_int32, POINTER(c_int32), c_int32, P,
+                                    POINTER(c_int32), P]),
         "vv_decoder_profile_init": (S, [P, P, P, c_int64, P, c_int64, c_int64, P, P,
                                         POINTER(c_float), POINTER(c_int32), P]),
         "vv_decoder_step_timeline": (S, [P, P, P, P, P, c_int32, POINTER(c_int32),

@@ -234,6 +234,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   const size_t o_sin = take((size_t)c.max_position * (D / 2) * 4);
   const size_t o_len = take(16);
   const size_t o_arg = take(16);
+  const size_t o_gen = take(16);  // generation: done flag, token count, position
   const size_t attn_b = vv::attn_workspace_bytes(c.n_q, c.n_kv, d->attn_chunks);
   const size_t o_part = take(attn_b);
   const size_t o_lmv = take((size_t)lm_grid * 4);
@@ -265,6 +266,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   d->rope_sin = reinterpret_cast<float*>(b + o_sin);
   d->d_length = reinterpret_cast<int32_t*>(b + o_len);
   d->d_argmax = reinterpret_cast<int32_t*>(b + o_arg);
+  d->d_gen = reinterpret_cast<int32_t*>(b + o_gen);
   d->attn_part = reinterpret_cast<float*>(b + o_part);
   d->attn_count = reinterpret_cast<int*>(b + o_part + attn_b - 256);
   d->lm_val = reinterpret_cast<float*>(b + o_lmv);
@@ -603,6 +605,47 @@ vv_status vv_decoder_profile_init(vv_decoder* d, const int32_t* input_ids,
   }
   for (auto e : t.ev) cudaEventDestroy(e);
   return st;
+}
+
+vv_status vv_decoder_generate(vv_decoder* d, const int32_t* first_token, const int32_t* position,
+                              int32_t n_steps, const int32_t* stop_ids, int32_t n_stop,
+                              int32_t* tokens_out, int32_t* n_out, vv_stream stream) {
+  VV_CHECK_ARG(d && first_token && position && tokens_out && n_out,
+               "vv_decoder_generate: null pointer");
+  VV_CHECK_ARG(n_stop >= 0 && n_stop <= vv::kMaxStopIds && (n_stop == 0 || stop_ids),
+               "vv_decoder_generate: n_stop %d (0..%d)", n_stop, vv::kMaxStopIds);
+  VV_CHECK_ARG(d->persistent, "vv_decoder_generate needs the persistent step kernel");
+  if (n_steps < 1) return set_error(VV_ERR_SHAPE, "n_steps=%d", n_steps);
+  if (d->len_host + n_steps > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "%d + %d steps exceed the KV capacity %d", d->len_host,
+                     n_steps, d->cfg.kv_capacity);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* done = d->d_gen;
+  int32_t* count = d->d_gen + 1;
+  int32_t* gpos = d->d_gen + 2;
+  VV_CUDA(cudaMemsetAsync(d->d_gen, 0, 2 * sizeof(int32_t), s));
+  VV_CUDA(cudaMemcpyAsync(gpos, position, sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  vv::StepParams p = d->step;
+  p.input_embeds = nullptr;
+  p.position = gpos;
+  p.logits = nullptr;
+  p.trace = d->trace;
+  p.gen_done = done;
+  p.gen_count = count;
+  p.gen_pos = gpos;
+  p.n_stop = n_stop;
+  for (int j = 0; j < n_stop; ++j) p.stop_ids[j] = stop_ids[j];
+  for (int i = 0; i < n_steps; ++i) {
+    p.token = i == 0 ? first_token : tokens_out + (i - 1);
+    p.argmax = tokens_out + i;
+    VV_CUDA(vv::launch_step(p, s));
+  }
+  int32_t n = 0;
+  VV_CUDA(cudaMemcpyAsync(&n, count, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  VV_CUDA(cudaStreamSynchronize(s));
+  d->len_host += n;
+  *n_out = n;
+  return VV_OK;
 }
 
 vv_status vv_decoder_sync_status(vv_decoder* d, vv_stream stream) {

@@ -28,6 +28,7 @@ struct vv_decoder {
   float* rope_sin = nullptr;
   int32_t* d_length = nullptr;
   int32_t* d_argmax = nullptr;
+  int32_t* d_gen = nullptr;  // [done, count, position] of vv_decoder_generate
   float* attn_part = nullptr;
   int* attn_count = nullptr;
   int attn_chunks = 1;

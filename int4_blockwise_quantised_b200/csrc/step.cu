@@ -917,6 +917,9 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   __shared__ int s_idx[NW];
   __shared__ int s_last;
 
+  // generation stopped by an earlier step of the same vv_decoder_generate call: every CTA sees
+  // the same word (written by the previous launch) and leaves before touching anything
+  if (p.gen_done && __ldcg(p.gen_done) != 0) return;
   const int past = *p.length;
   if (tid == 0) {
     for (int i = 0; i < p.nstages; ++i) {
@@ -1171,10 +1174,17 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       }
     }
     if (lane == 0) {
-      *p.argmax = bi == 0x7fffffff ? 0 : bi;
+      const int tok = bi == 0x7fffffff ? 0 : bi;
+      *p.argmax = tok;
       *p.head_count = 0;
       *p.bar_count = 0u;  // every CTA has passed every barrier of this launch
       *p.length = past + 1;
+      if (p.gen_done) {  // every CTA read the position at its start, long before this point
+        *p.gen_count += 1;
+        *p.gen_pos += 1;
+        for (int j = 0; j < p.n_stop; ++j)
+          if (tok == p.stop_ids[j]) *p.gen_done = 1;
+      }
     }
   }
 }

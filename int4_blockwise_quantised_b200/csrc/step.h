@@ -49,6 +49,14 @@ struct StepParams {
   int32_t* length;
   unsigned* bar_count;
   unsigned* bar_gen;
+  // greedy generation (vv_decoder_generate), all null otherwise: a launch finding *gen_done set
+  // returns at once; else its last CTA counts the token (*gen_count), advances *position (which
+  // then points at the generation's own position word) and sets *gen_done on a stop id.
+  int32_t* gen_done;
+  int32_t* gen_count;
+  int32_t* gen_pos;
+  int32_t stop_ids[8];
+  int n_stop;
   uint64_t* stamps;   // timeline tap [grid][max_stamps] (globaltimer ns) or nullptr
   int max_stamps;
   // launch shape
@@ -65,5 +73,6 @@ int step_max_tiles(int cap);
 cudaError_t step_configure(StepParams& p, int* blocks_per_sm);
 void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_bytes);
 cudaError_t launch_step(const StepParams& p, cudaStream_t s);
+constexpr int kMaxStopIds = 8;
 
 }  // namespace vv

@@ -182,3 +182,14 @@ class Decoder:
                                               ptr(audio_features), N, audio_offset, ptr(logits),
                                               ptr(argmax), ms, n, stream_handle(stream)))
         return dict(zip(self.PREFILL_KINDS, list(ms))), dict(zip(self.PREFILL_KINDS, list(n)))
+
+    def generate(self, first_token, position, n_steps, stop_ids=(), tokens_out=None, stream=None):
+        """Greedy generation on the device; returns (tokens int32 device tensor [n_steps], n)."""
+        toks = tokens_out if tokens_out is not None else torch.zeros(
+            n_steps, dtype=torch.int32, device=first_token.device)
+        ids = (ctypes.c_int32 * max(len(stop_ids), 1))(*stop_ids)
+        n = ctypes.c_int32()
+        check(_vv.lib.vv_decoder_generate(self.handle, ptr(first_token), ptr(position), n_steps,
+                                          ids, len(stop_ids), ptr(toks), ctypes.byref(n),
+                                          stream_handle(stream)))
+        return toks, n.value

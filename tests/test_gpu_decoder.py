@@ -281,3 +281,62 @@ def test_prefill_full_length_one_layer():
     assert normwise(dec.k_cache[:, 0, :, :S].cpu().numpy(), ora["k"]) <= TOL
     assert normwise(dec.v_cache[:, 0, :, :S].cpu().numpy(), ora["v"]) <= TOL
     assert torch.count_nonzero(dec.k_cache[:, 0, :, S:]).item() == 0
+
+
+# --------------------------------------------------------------------------- greedy generate
+def test_generate_greedy_loop_on_device():
+    """vv_decoder_generate: each step's argmax feeds the next step on the device; the tokens are
+    the oracle's greedy choices (teacher-forced with the GPU's own tokens: equal wherever the
+    oracle's top-2 margin exceeds 1e-2, else one of its top two), equal to step-by-step decoding,
+    and a stop id ends the generation early with the rest of the output untouched."""
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape = synth.SHAPE_TINY
+    cfg = ocfg(shape)
+    W = oracle_model(shape, "int4")
+    model = gpu_model(shape, "int4")
+    P, N = 9, 6
+    dec = Decoder(model, P + N + 4)
+    kp, vp = synth.past_kv(shape, P)
+    fill_cache(dec, kp, vp)
+    first = torch.tensor([17], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([P], dtype=torch.int32, device="cuda")
+    toks, n = dec.generate(first, pos, N)
+    dec.sync_status()
+    assert n == N and dec.length == P + N
+    gen = toks.cpu().numpy().tolist()
+    # oracle, teacher-forced with the generated tokens
+    kc = [kp[l].copy() for l in range(shape.layers)]
+    vc = [vp[l].copy() for l in range(shape.layers)]
+    tok = 17
+    for i in range(N):
+        ora = odec.decoder_step(cfg, W, W["embed"][tok], P + i, kc, vc)
+        order = np.argsort(ora["logits"])
+        if ora["logits"][order[-1]] - ora["logits"][order[-2]] > 1e-2:
+            assert gen[i] == ora["argmax"], (i, gen[i], ora["argmax"])
+        else:
+            assert gen[i] in (order[-1], order[-2])
+        for l in range(shape.layers):
+            kc[l] = np.concatenate([kc[l], ora["k_new"][l][:, None, :]], axis=1)
+            vc[l] = np.concatenate([vc[l], ora["v_new"][l][:, None, :]], axis=1)
+        tok = gen[i]
+    # step-by-step decoding from the same state gives the same tokens
+    dec.set_length(P)
+    t = first.clone()
+    p2 = pos.clone()
+    seq = []
+    for i in range(N):
+        dec.step(p2, token=t, argmax=t)
+        p2 += 1
+        seq.append(int(t.item()))
+    assert seq == gen
+    # a stop id ends the generation; later entries stay as they were
+    stop = gen[2]
+    n_exp = gen.index(stop) + 1
+    dec.set_length(P)
+    out = torch.full((N,), -1, dtype=torch.int32, device="cuda")
+    toks2, n2 = dec.generate(first, pos, N, stop_ids=(stop, 151645), tokens_out=out)
+    dec.sync_status()
+    assert n2 == n_exp and dec.length == P + n_exp
+    got = toks2.cpu().numpy().tolist()
+    assert got[:n_exp] == gen[:n_exp] and all(v == -1 for v in got[n_exp:])
