@@ -68,7 +68,10 @@ def peaks():
 # ----------------------------------------------------------------------------------- bytes
 def phase_bytes(shape, P):
     """Algorithmic bytes per launch of each decode phase at past length P (per layer, except
-    the lm_head which is per step)."""
+    the lm_head which is per step): the bytes the method must move from HBM -- packed weights
+    (16 code bytes + 2 scale bytes per 32 weights), fp16 biases and RMSNorm gammas, the KV read
+    (P positions) and write (1 position), the fp16 lm_head, the fp32 logits and the fp16 input
+    embedding.  Activations between phases stay on chip / in L2 and are not counted."""
     H, D, Hq, Hkv, I, V = shape.hidden, shape.head_dim, shape.n_q, shape.n_kv, shape.inter, shape.vocab
 
     def packed(N, K):
@@ -76,12 +79,12 @@ def phase_bytes(shape, P):
 
     qkv_rows = (Hq + 2 * Hkv) * D
     return {
-        "qkv": packed(qkv_rows, H) + 2 * qkv_rows + 2 * H + 4 * H + 4 * qkv_rows,
-        "attn": 2 * Hkv * (P + 1) * D * 2 + 4 * qkv_rows + 4 * Hq * D,
-        "o_proj": packed(H, Hq * D) + 4 * Hq * D + 8 * H,
-        "gate_up": 2 * packed(I, H) + 2 * H + 4 * H + 4 * I,
-        "down": packed(H, I) + 4 * I + 8 * H,
-        "lm_head": V * H * 2 + 2 * H + 4 * H + 4 * V,
+        "qkv": packed(qkv_rows, H) + 2 * qkv_rows + 2 * H,
+        "attn": 2 * Hkv * (P + 1) * D * 2,
+        "o_proj": packed(H, Hq * D),
+        "gate_up": 2 * packed(I, H) + 2 * H,
+        "down": packed(H, I),
+        "lm_head": V * H * 2 + 2 * H + 4 * V + 2 * H,
     }
 
 
@@ -126,7 +129,9 @@ class ClockSampler:
     def __init__(self, device_index):
         self.proc = None
         self.dev = device_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        import tempfile
+
+        self.path = os.path.join(tempfile.gettempdir(), f"vv_clocks_rank{device_index}.csv")
 
     def start(self):
         try:

@@ -40,6 +40,13 @@ def test_host_side_argument_checks():
     code, text = vv.last_error()
     assert code == vv.VV_ERR_INVALID_ARG and "null" in text
 
+    n = ctypes.c_int32()
+    ids = (ctypes.c_int32 * 9)()
+    assert lib.vv_decoder_generate(None, fake, fake, 4, ids, 0, fake, ctypes.byref(n),
+                                   None) == vv.VV_ERR_INVALID_ARG
+    assert lib.vv_decoder_generate(fake, fake, fake, 4, ids, 9, fake, ctypes.byref(n),
+                                   None) == vv.VV_ERR_INVALID_ARG  # more than 8 stop ids
+
 
 def test_decoder_create_rejects_bad_config():
     cfg = vv.vv_config(1536, 1, 12, 5, 128, 8960, 1000, 1e-6, 1e6, 16, 16, 0)  # 12 % 5 != 0
