@@ -15,16 +15,23 @@
 // phase's input is an activation vector produced by every CTA), stage that vector in shared
 // memory / registers (with the fused RMSNorm where the layer has one), then consume the phase's
 // stages.  Phases per layer:
-//   QKV  : y = [Wq;Wk;Wv] . RMSNorm(x) + b              -> qkv (fp32)
+//   QKV  : y = [Wq;Wk;Wv] . RMSNorm(x) + b              -> qkv (fp32); the CTA's q/k/v rows
+//          form one stream of stages even where they straddle two matrices
 //   ATTN : per (kv head, 64-position tile): RoPE(q), RoPE(k_new) + append at slot `length`,
-//          online-softmax partial; the last CTA of a head merges the partials -> attn (fp32)
+//          online-softmax partial (m, l, o); up to 32 tiles per head the O staging of every CTA
+//          merges the partials, beyond that the last CTA of a head merges them -> attn (fp32)
 //   O    : x += Wo . attn
 //   GU   : h = silu(Wg . RMSNorm(x)) * (Wu . RMSNorm(x))
 //   DOWN : x += Wd . h
 // then HEAD: logits = W_lm . RMSNorm(x), argmax (last CTA reduces), length += 1.
+// GEMV stages run in one of three modes: x in registers (K <= 1536), whole rows per warp with x
+// in shared memory (larger K, many rows), or each row split over three warps (larger K, few
+// rows).  In greedy generation (StepParams::gen_done set) a launch after a stop token returns
+// at once, and the last CTA advances the generation's position and token count.
 //
-// The grid barrier is an arrival counter plus a generation word in global memory; every wait is
-// bounded (VV_ERR_TIMEOUT in the device error word after 2 s, then the kernel carries on).  The
+// The grid barrier is a monotonic arrival counter in global memory (barrier k completes at
+// (k + 1) x grid arrivals; the last CTA of the launch resets it); every wait is bounded
+// (VV_ERR_TIMEOUT in the device error word after 2 s, then the kernel carries on).  The
 // cooperative launch guarantees that all CTAs are resident.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
