@@ -257,6 +257,10 @@ vv_status vv_decoder_step(vv_decoder* dec, const uint16_t* input_embeds, const i
  * replaced by audio_features; causal attention over the S positions; writes present K/V at
  * slots 0..S-1, sets length = S, and emits the last position's logits / argmax.
  *   input_ids, position_ids: device int32 [S]; audio_features: device fp16 [N, H] or NULL (N=0)
+ * All S positions go through tensor-core GEMMs at once (each packed matrix is dequantised to an
+ * fp16 operand, rounded once: exact for ternary weights, within 2^-12 relative for int4), with
+ * fp32 accumulation and an fp32 residual.  The first call allocates a prefill workspace sized
+ * for max_prefill (kept until vv_decoder_destroy).  Asynchronous on `stream`.
  * Errors: VV_ERR_RANGE (audio_offset + N > S, negative offset), VV_ERR_CAPACITY (S > cap or
  * S > max_prefill), VV_ERR_INVALID_ARG. */
 vv_status vv_decoder_init(vv_decoder* dec, const int32_t* input_ids, const int32_t* position_ids,
