@@ -81,22 +81,25 @@ def final_logits(cfg, weights, x):
     return ops.lm_head_logits(xn, weights["lm_head"])
 
 
-def decoder_step(cfg, weights, input_embeds, position, k_cache, v_cache):
+def decoder_step(cfg, weights, input_embeds, position, k_cache, v_cache, kv_dtype=np.float16):
     """One decode step at batch 1.
 
-    input_embeds float16 [H]; position int; k_cache/v_cache: per layer float16 [Hkv, P, D]
-    (the P past positions).  Returns dict with logits float64 [V], argmax, layer_out float64
-    [L, H] (the residual after each layer), k_new/v_new float16 [L, Hkv, D].
+    input_embeds float16 [H]; position int; k_cache/v_cache: per layer [Hkv, P, D] (the P past
+    positions) of the cache's storage type kv_dtype.  Returns dict with logits float64 [V],
+    argmax, layer_out float64 [L, H] (the residual after each layer), k_new/v_new [L, Hkv, D]
+    rounded to kv_dtype.  The contract stores K/V in float16 ("vibevoice-asr-bitnet-onnx",
+    decoder_step I/O); kv_dtype=np.float32 is the fp32-cache variant of "VibeVoice-ASR — ONNX
+    export for Vernacula" (Highlights), where only the storage rounding differs.
     """
     x = np.asarray(input_embeds, dtype=np.float16).astype(np.float64)[None, :]
     scale = 1.0 / math.sqrt(cfg.head_dim)
     outs, k_new, v_new = [], [], []
     for li, lw in enumerate(weights["layers"]):
         q, k, v = _attn_in(cfg, lw, x, [position])
-        k16 = k[0].astype(np.float16)
-        v16 = v[0].astype(np.float16)
-        K = np.concatenate([np.asarray(k_cache[li], np.float16), k16[:, None, :]], axis=1)
-        V = np.concatenate([np.asarray(v_cache[li], np.float16), v16[:, None, :]], axis=1)
+        k16 = k[0].astype(kv_dtype)
+        v16 = v[0].astype(kv_dtype)
+        K = np.concatenate([np.asarray(k_cache[li], kv_dtype), k16[:, None, :]], axis=1)
+        V = np.concatenate([np.asarray(v_cache[li], kv_dtype), v16[:, None, :]], axis=1)
         o = ops.gqa_decode_attention(q[0], K.astype(np.float64), V.astype(np.float64), scale)
         x = _mlp_out(cfg, lw, x, o.reshape(1, -1))
         outs.append(x[0].copy())

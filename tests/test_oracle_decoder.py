@@ -158,3 +158,33 @@ def test_audio_splice_rows():
     assert np.array_equal(e[:2], embed[[1, 2]])
     assert np.array_equal(e[2:5], feats)
     assert np.array_equal(e[5], embed[3])
+
+
+def test_fp32_kv_cache_variant_differs_only_by_storage_rounding():
+    """kv_dtype=float32 keeps the new K/V at fp32; with the k/v projections zero and position 0
+    (RoPE = identity) the new K/V are the fp16 biases themselves, so both storage types give
+    identical results; in general the fp32 K/V rounds to the fp16 K/V within half an ulp."""
+    W = build_model(TINY_SHAPE, TINY)
+    kp, vp = synth.past_kv(TINY_SHAPE, 5)
+    emb = W["embed"][11]
+    a = decoder.decoder_step(TINY, W, emb, 5, list(kp), list(vp))
+    b = decoder.decoder_step(TINY, W, emb, 5, [k.astype(np.float32) for k in kp],
+                             [v.astype(np.float32) for v in vp], kv_dtype=np.float32)
+    assert b["k_new"].dtype == np.float32 and a["k_new"].dtype == np.float16
+    k16 = a["k_new"].astype(np.float64)
+    assert np.all(np.abs(b["k_new"].astype(np.float16).astype(np.float64) - k16)
+                  <= np.spacing(np.abs(a["k_new"])).astype(np.float64))
+    assert not np.array_equal(a["logits"], b["logits"])  # the storage type does take effect
+    assert np.max(np.abs(a["logits"] - b["logits"])) <= 1e-2 * np.max(np.abs(a["logits"]))
+    # zero k/v projections at position 0: new k = bk, v = bv exactly -> identical results
+    Z = dict(W, layers=[dict(lw) for lw in W["layers"]])
+    zero = pack.pack_sym_int4(np.zeros((TINY.n_kv * TINY.head_dim, TINY.hidden), np.float32))
+    for lw in Z["layers"]:
+        lw["wk"] = zero
+        lw["wv"] = zero
+    e16 = [np.zeros((TINY.n_kv, 0, TINY.head_dim), np.float16)] * TINY.layers
+    e32 = [np.zeros((TINY.n_kv, 0, TINY.head_dim), np.float32)] * TINY.layers
+    c = decoder.decoder_step(TINY, Z, emb, 0, e16, e16)
+    d = decoder.decoder_step(TINY, Z, emb, 0, e32, e32, kv_dtype=np.float32)
+    assert np.array_equal(c["logits"], d["logits"])
+    assert np.array_equal(c["k_new"].astype(np.float32), d["k_new"])
