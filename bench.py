@@ -313,10 +313,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    extra = 0
+    seq_starts = 0
     for i in range(args.steps):
         if i % seq == 0:
-            extra += 3  # set_length kernel + pos fill + (pos add counted below)
+            seq_starts += 1  # vv_decoder_set_length: one set_int_kernel
         one_step(i % seq)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -328,7 +328,9 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(ms, dist, "cuda")
     ms_per_step = ms / args.steps
     tok_s = whole_job_rate(args.steps, world, ms)
-    gpu_launches = args.steps * (n_launch + 1) + extra  # + the position increment per step
+    # this library's kernels only: one step launch per step (persistent kernel) plus the length
+    # reset at each sequence start; torch's position fill / increment are not counted
+    gpu_launches = args.steps * n_launch + seq_starts
 
     # -------------------------------------- per-step distribution (one sequence, not timed above)
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(seq + 1)]
@@ -548,7 +550,8 @@ def measure_prefill(model, shape, S, N, steps, warmup, dist=None, world=1):
         "e2e_tok_s": world * S / (e2e_ms * 1e-3), "e2e_ms": e2e_ms,
         "h2d_bytes": ids.nbytes + pos.nbytes + feats.nbytes, "d2h_bytes": 4,
         "tflops_whole": total_fl / (ms_per * 1e-3) / 1e12, "roofline": roof, "clocks": clk,
-        "launches": sum(kind_n.values()),
+        # kernels of one prefill: the profiled marks minus the per-layer bias copies
+        "launches": sum(kind_n.values()) - shape.layers,
     }
 
 
