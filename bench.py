@@ -254,29 +254,45 @@ def blas_threads():
 
 
 # ------------------------------------------------------------------------------------ ours
-def run_ours(args, rank, world, local_rank):
+def init_dist(world, local_rank):
     import torch
 
-    from int4_blockwise_quantised_b200 import _vv
-    from int4_blockwise_quantised_b200.model import Decoder, PackedModel
-
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist_mod
-        import datetime
+    if world <= 1:
+        return None
+    import datetime
 
-        dist = dist_mod
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+    import torch.distributed as dist_mod
+
+    dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    return dist_mod
 
-    shape, mode, P, seq, desc = CONFIGS[args.config]
+
+def build_model(shape, mode):
+    from int4_blockwise_quantised_b200 import _vv
+    from int4_blockwise_quantised_b200.model import PackedModel
+
     std = std_for(shape)
     vmode = _vv.VV_TERNARY if mode == "ternary" else _vv.VV_SYM_INT4
+    return PackedModel(shape, vmode, lambda li, m: synth.master(shape, m, li, std),
+                       lambda li: synth.layer_vectors(shape, li), synth.model_tables(shape),
+                       "cuda")
+
+
+def measure_decode(config, steps, warmup, dist, world, local_rank, model=None):
+    """Device-timed decode steps of one config (inputs resident, greedy token fed back on the
+    device), the per-step distribution over one sequence, the end-to-end variant through the
+    public API with host buffers, the roofline of the step kernel and its timeline breakdown.
+    Returns (record, model)."""
+    import torch
+
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape, mode, P, seq, desc = CONFIGS[config]
     t0 = time.time()
-    model = PackedModel(shape, vmode, lambda li, m: synth.master(shape, m, li, std),
-                        lambda li: synth.layer_vectors(shape, li), synth.model_tables(shape),
-                        "cuda")
+    if model is None:
+        model = build_model(shape, mode)
     setup_s = time.time() - t0
     cap = P + max(seq, 64) + 8
     dec = Decoder(model, cap)
@@ -302,7 +318,7 @@ def run_ours(args, rank, world, local_rank):
 
     n_launch = dec.step_launches
     # warm-up (also captures the graph)
-    for i in range(args.warmup):
+    for i in range(warmup):
         one_step(i % seq)
     dec.sync_status()
 
@@ -314,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     seq_starts = 0
-    for i in range(args.steps):
+    for i in range(steps):
         if i % seq == 0:
             seq_starts += 1  # vv_decoder_set_length: one set_int_kernel
         one_step(i % seq)
@@ -326,11 +342,11 @@ def run_ours(args, rank, world, local_rank):
     dec.sync_status()
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, dist, "cuda")
-    ms_per_step = ms / args.steps
-    tok_s = whole_job_rate(args.steps, world, ms)
+    ms_per_step = ms / steps
+    tok_s = whole_job_rate(steps, world, ms)
     # this library's kernels only: one step launch per step (persistent kernel) plus the length
     # reset at each sequence start; torch's position fill / increment are not counted
-    gpu_launches = args.steps * n_launch + seq_starts
+    gpu_launches = steps * n_launch + seq_starts
 
     # -------------------------------------- per-step distribution (one sequence, not timed above)
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(seq + 1)]
@@ -353,7 +369,7 @@ def run_ours(args, rank, world, local_rank):
     emb_dev = torch.empty(shape.hidden, dtype=torch.float16, device="cuda")
     pos_dev = torch.empty(1, dtype=torch.int32, device="cuda")
     am_dev = torch.empty(1, dtype=torch.int32, device="cuda")
-    e2e_steps = min(args.steps, 256)
+    e2e_steps = min(steps, 256)
     for i in range(3):  # capture the e2e graph (different pointers) outside the timed region
         dec.set_length(P)
         emb_dev.copy_(emb_host, non_blocking=True)
@@ -391,7 +407,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "hbm", "kernel": "step_kernel (persistent decode step, 1 launch/step)",
                 "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                 "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "traffic": traffic_for("step_kernel"),
+                "traffic": traffic_for("step_kernel", config),
                 "algorithmic_bytes_per_launch": sb, "avg_launch_us": round(ms_per_step * 1e3, 2)}
     # per-phase breakdown from the kernel's timeline tap (one extra step, not timed)
     try:
@@ -401,21 +417,18 @@ def run_ours(args, rank, world, local_rank):
         roofline["phases_us"] = phase_breakdown(stamps.astype(np.int64), shape.layers)
     except Exception as e:  # the tap is diagnostics only
         roofline["phases_us"] = {"error": str(e)[:200]}
-
-    result = {
-        "metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "config": {"workload": args.config, "description": desc, "batch": 1, "past_P": P,
+    dec.close()
+    rec = {
+        "value": round(tok_s, 2), "unit": "tok/s", "ms_per_step": round(ms_per_step, 5),
+        "config": {"workload": config, "description": desc, "batch": 1, "past_P": P,
                    "steps_per_sequence": seq, "weights": f"{mode} block-32",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (weights %.0f MB, L2 126 MB); no flush" % (
                        sb / 1e6)},
         "step_us": round(ms_per_step * 1e3, 2),
         "step_us_percentiles": pct,
-        "hbm_gbs": round(sb / (ms_per_step * 1e-3) / 1e9, 1),
-        "hbm_frac_of_measured": round(sb / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "hbm_gbs": round(achieved, 1),
+        "hbm_frac_of_measured": round(achieved / peak, 4),
         "hbm_frac_of_8tbs": round(sb / (ms_per_step * 1e-3) / 8e12, 4),
         "algorithmic_bytes_per_step": sb,
         "roofline": roofline,
@@ -428,18 +441,42 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "setup_s": round(setup_s, 1),
     }
+    return rec, model
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    dist = init_dist(world, local_rank)
+    rec, model = measure_decode(args.config, args.steps, args.warmup, dist, world, local_rank)
+    result = {"metric": METRIC, "value": rec["value"], "unit": "tok/s", "n_gpus": world,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec["ms_per_step"],
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+              "data": "synthetic"}
+    result.update({k: v for k, v in rec.items() if k not in result})
     if args.config == "decode-1p5b" and not args.no_prefill:
         # decoder_init at S = 4530 on the same int4 1.5B weights (the ASR prefill workload)
         pshape, _, pS, pN, _ = PREFILL_CONFIGS["prefill-asr-1p5b"]
-        dec.close()
         pr = measure_prefill(model, pshape, pS, pN, 10, 3, dist, world)
         result["prefill"] = {"workload": "prefill-asr-1p5b", "value": round(pr["tok_s"], 1),
                              "unit": "tok/s", "ms": round(pr["ms"], 3),
                              "tflops_whole_prefill": round(pr["tflops_whole"], 1),
-                             "e2e_tok_s": round(pr["e2e_tok_s"], 1), "roofline": pr["roofline"]}
+                             "e2e_tok_s": round(pr["e2e_tok_s"], 1), "roofline": pr["roofline"],
+                             "clocks": pr["clocks"]}
         result["gpu_launches_prefill"] = pr["launches"] * 10
-        dec = None
+    del model
+    torch.cuda.empty_cache()
+    if args.config == "decode-1p5b" and not args.no_extra:
+        # the metric's other model size and the long-context decode, each a sub-record with its
+        # own roofline, e2e and clocks (same timing protocol, fewer steps)
+        for sub in ("decode-7b", "decode-asr-1p5b"):
+            r2, m2 = measure_decode(sub, min(args.steps, 64), args.warmup, dist, world, local_rank)
+            del m2
+            torch.cuda.empty_cache()
+            r2["steps"] = min(args.steps, 64)
+            result[sub.replace("-", "_")] = r2
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        shape, mode, P, _, _ = CONFIGS[args.config]
         st, sample, thr = oracle_sample_time(shape, mode, P)
         result["cpu_baseline"] = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr,
                                   "kind": "oracle", "sample": sample,
@@ -450,8 +487,6 @@ def run_ours(args, rank, world, local_rank):
                                                     "cores": 1, "sample": sample1}
         except Exception as e:  # threadpoolctl missing: report the all-cores figure only
             result["cpu_baseline"]["one_thread"] = {"error": str(e)[:200]}
-    if dec is not None:
-        dec.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -651,45 +686,57 @@ def run_prefill(args, rank, world, local_rank):
         print(json.dumps(result), flush=True)
 
 
+PHASES = ("qkv", "attn", "o", "gu_down")
+
+
+def timeline_names(L):
+    """Stamp names of one CTA's row, in the step kernel's order: kernel start; per layer the
+    barrier before each phase (arrive, exit; none before layer 0's q/k/v), then the point where
+    the phase's input is staged (q/k/v, gate/up) or its work is done (attention, o-proj), and the
+    layer end; then the lm_head barrier, its staged input and the end."""
+    names = ["start"]
+    for l in range(L):
+        if l > 0:
+            names += [f"L{l}.qkv.arrive", f"L{l}.qkv.exit"]
+        names += [f"L{l}.qkv.staged"]
+        names += [f"L{l}.attn.arrive", f"L{l}.attn.exit", f"L{l}.attn.done"]
+        names += [f"L{l}.o.arrive", f"L{l}.o.exit", f"L{l}.o.done"]
+        names += [f"L{l}.gu_down.arrive", f"L{l}.gu_down.exit", f"L{l}.gu_down.staged", f"L{l}.end"]
+    names += ["head.arrive", "head.exit", "head.staged", "end"]
+    return names
+
+
 def phase_breakdown(st, L):
     """Critical-path time per phase summed over layers (us) from the timeline stamps: a phase
-    runs from its barrier exit to the last CTA's arrival at the next barrier; barrier = release
-    latency after the last arrival."""
-    names = ["start", "L0.qkv.staged"]
-    for ph in ("attn", "o", "gu", "down"):
-        names += [f"L0.{ph}.arrive", f"L0.{ph}.exit"] + ([] if ph == "attn" else [f"L0.{ph}.staged"])
-    for l in range(1, L):
-        names += [f"L{l}.qkv.arrive", f"L{l}.qkv.exit", f"L{l}.qkv.staged"]
-        for ph in ("attn", "o", "gu", "down"):
-            names += [f"L{l}.{ph}.arrive", f"L{l}.{ph}.exit"] + ([] if ph == "attn" else [f"L{l}.{ph}.staged"])
-    names += ["head.arrive", "head.exit", "head.staged", "end"]
+    runs from the last CTA's exit of its barrier (kernel start for layer 0's q/k/v) to the last
+    CTA's arrival at the next barrier; barrier = release latency after the last arrival."""
+    names = timeline_names(L)
     if st.shape[1] != len(names):
         return {"error": f"{st.shape[1]} stamps, expected {len(names)}"}
     ix = {k: i for i, k in enumerate(names)}
     st = st - st[:, 0].min()
     out = {}
-    phs = ("qkv", "attn", "o", "gu", "down")
     for l in range(L):
-        for j, ph in enumerate(phs):
-            b = ix.get(f"L{l}.{ph}.exit", ix["start"])
-            nxt = f"L{l}.{phs[j + 1]}.arrive" if j + 1 < len(phs) else (
-                f"L{l + 1}.qkv.arrive" if l + 1 < L else "head.arrive")
-            e = ix[nxt]
+        for j, ph in enumerate(PHASES):
+            b = ix["start"] if (l == 0 and j == 0) else ix[f"L{l}.{ph}.exit"]
+            nxt = f"L{l}.{PHASES[j + 1]}" if j + 1 < len(PHASES) else (
+                f"L{l + 1}.qkv" if l + 1 < L else "head")
+            e = ix[nxt + ".arrive"]
             out[ph] = out.get(ph, 0) + (st[:, e].max() - st[:, b].max())
-            out["barriers"] = out.get("barriers", 0) + (
-                st[:, ix[nxt.replace("arrive", "exit")]].max() - st[:, e].max())
+            out["barriers"] = out.get("barriers", 0) + (st[:, ix[nxt + ".exit"]].max() - st[:, e].max())
     out["lm_head"] = st[:, ix["end"]].max() - st[:, ix["head.exit"]].max()
     out["total"] = st[:, ix["end"]].max()
     return {k: round(v / 1e3, 1) for k, v in out.items()}
 
 
-def traffic_for(kernel):
-    """DRAM bytes per launch from the committed ncu summary, or None when the kernel's source
-    changed since the counters were taken."""
+def traffic_for(kernel, workload=None):
+    """DRAM bytes per launch from the committed ncu summary (entry "kernel/workload", else
+    "kernel"), or None when the kernel's source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(kernel)
+    tab = json.load(open(p))
+    d = tab.get(f"{kernel}/{workload}") or tab.get(kernel)
     if not d:
         return None
     src = os.path.join(ROOT, d["source"])
@@ -698,34 +745,74 @@ def traffic_for(kernel):
 
 
 # ------------------------------------------------------------------------------ reference arm
+class OracleFullStep:
+    """The oracle (as it stands) running whole decode steps: every layer (each packed matrix
+    dequantised inside the call, as the oracle always does) and the full lm_head."""
+
+    def __init__(self, shape, mode, P):
+        from oracle import decoder as odec
+        from oracle import pack as opack
+
+        std = std_for(shape)
+        self.shape, self.P = shape, P
+        layers = []
+        for li in range(shape.layers):
+            lw = dict(synth.layer_vectors(shape, li))
+            for m in synth.MATRICES:
+                W = synth.master(shape, m, li, std)
+                lw[m] = (opack.pack_ternary(W, opack.ternary_scale(W)) if mode == "ternary"
+                         else opack.pack_sym_int4(W))
+            layers.append(lw)
+        self.W = dict(synth.model_tables(shape), layers=layers)
+        self.kp, self.vp = synth.past_kv(shape, P)
+        self.emb = synth.input_embeds(shape)[0]
+        self.cfg = odec.Config(shape.hidden, shape.layers, shape.n_q, shape.n_kv,
+                               shape.head_dim, shape.inter, shape.vocab, shape.eps, shape.theta)
+
+    def run(self):
+        from oracle import decoder as odec
+
+        t0 = time.perf_counter()
+        r = odec.decoder_step(self.cfg, self.W, self.emb, self.P, list(self.kp), list(self.vp))
+        dt = time.perf_counter() - t0
+        assert np.isfinite(r["logits"]).all()
+        return dt
+
+
 def run_reference(args, rank):
-    """The oracle as the reference arm: every step is one bounded oracle sample (one layer +
-    1/L of the lm_head, scaled by L), on this arm's config, metric and unit."""
+    """The oracle as the reference arm: whole decode steps (all layers + lm_head) of this arm's
+    config, metric and unit; at most 1 warm-up and 3 timed steps (each is seconds of CPU work).
+    Under torchrun only rank 0 runs."""
     if rank != 0:
         return
     if args.config in PREFILL_CONFIGS:
         run_reference_prefill(args)
         return
     shape, mode, P, seq, desc = CONFIGS[args.config]
-    o = OracleSample(shape, mode, P)
-    for _ in range(args.warmup):
+    t0 = time.perf_counter()
+    o = OracleFullStep(shape, mode, P)
+    setup_s = time.perf_counter() - t0
+    warm, steps = min(args.warmup, 1), min(args.steps, 3)
+    for _ in range(warm):
         o.run()
     t0 = time.perf_counter()
-    est = [o.run() for _ in range(args.steps)]
+    ts = [o.run() for _ in range(steps)]
     wall = time.perf_counter() - t0
-    st = statistics.median(est)
+    st = statistics.median(ts)
     value = 1.0 / st
     result = {
         "metric": METRIC, "value": round(value, 4), "unit": "tok/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(st * 1e3, 3),
+        "steps": steps, "warmup": warm, "ms_per_step": round(st * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": args.config, "description": desc, "batch": 1, "past_P": P},
         "cpu_baseline": {"value": round(value, 4), "unit": "tok/s", "cores": blas_threads(),
-                         "kind": "oracle", "sample": o.describe(args.steps)},
+                         "kind": "oracle",
+                         "sample": f"{steps} whole oracle decode steps ({shape.layers} layers, "
+                                   f"dequantised per call, full lm_head) at P={P}; median"},
         "e2e": {"value": round(value, 4), "unit": "tok/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
-        "wall_s": round(wall, 2),
+        "wall_s": round(wall, 2), "setup_s": round(setup_s, 1),
     }
     print(json.dumps(result), flush=True)
 
@@ -767,6 +854,8 @@ def main():
                     choices=sorted(CONFIGS) + sorted(PREFILL_CONFIGS))
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill measurement added to the default decode line")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the 7B and long-context decode sub-records of the default line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

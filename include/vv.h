@@ -62,6 +62,16 @@ vv_status vv_last_error(char* buf, size_t n);
 /* Synchronise `stream` and return (and clear) the device error word of the current device. */
 vv_status vv_sync_status(vv_stream stream);
 
+/* Self-test of the bounded device waits (no counterpart in the pages: a property of this
+ * library).  Launches one CTA on `stream` that waits, through the same helpers the kernels use,
+ * for a signal that never comes -- which = 0: an mbarrier phase nobody completes (the stage-ring
+ * wait); which = 1: a global counter nobody increments (the grid-barrier wait; scratch: device,
+ * 16 bytes, 16-byte aligned, zeroed by the call) -- and gives up after limit_ns, recording
+ * VV_ERR_TIMEOUT in the device error word, which the next vv_sync_status returns.  The kernel
+ * then exits normally; the context stays usable.  limit_ns in [1e3, 1e8].
+ * Errors: VV_ERR_INVALID_ARG. */
+vv_status vv_wait_selftest(int32_t which, int64_t limit_ns, void* scratch, vv_stream stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Packing ([BITNET] ternarisation and MatMulNBits paragraphs; [STATUS] "Done": int4 build).
  *
@@ -143,7 +153,8 @@ vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cache, const u
  * 256 KiB that every GPU loading this library holds until the process exits.  No counterpart in
  * the pages: this is a property of this library, not of the method.
  *  - The first call on a device looks up the array's device address with that device current;
- *    make that first call before any stream capture.
+ *    make that first call before any stream capture.  `stream` must belong to the current device
+ *    (VV_ERR_INVALID_ARG otherwise: the array's address differs per device).
  *  - The call allocates nothing (no cudaMalloc/cudaFree); it clears the arrival counters with
  *    cudaMemsetAsync on `stream` and then launches the kernel.
  *  - All calls share the one array, which keeps the previous call's partials: calls that overlap
@@ -279,15 +290,6 @@ vv_status vv_decoder_set_graph(vv_decoder* dec, int32_t enable);
 /* Synchronise `stream` and return (and clear) the device error word. */
 vv_status vv_decoder_sync_status(vv_decoder* dec, vv_stream stream);
 
-/* Profiling tap: run one step with plain launches (no graph, no launch overlap) and CUDA events
- * around every launch on `stream`; phase_ms (HOST float[6]) receives the device time summed over
- * layers of [qkv, attention, o-proj, gate/up, down, lm_head].  Appends a position like
- * vv_decoder_step.  Synchronous.  Errors as vv_decoder_step. */
-vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
-                                  const int32_t* token_id, const int32_t* position_id,
-                                  float* logits, int32_t* argmax_out, float* phase_ms,
-                                  vv_stream stream);
-
 /* Greedy generation on the device ("vibevoice-asr-bitnet-onnx": the driver's greedy decode
  * with stop tokens): up to n_steps decode steps, the token of step i being the argmax of step
  * i - 1 (step 0: *first_token), positions *position, *position + 1, ...; each step appends to
@@ -298,7 +300,9 @@ vv_status vv_decoder_profile_step(vv_decoder* dec, const uint16_t* input_embeds,
  * steps run (the stop token included).  Needs the persistent step kernel.  Synchronous: one host
  * synchronisation for the whole generation.
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (n_steps < 1), VV_ERR_CAPACITY (length + n_steps >
- * capacity); device-side range errors as vv_decoder_step. */
+ * capacity); a device-side error recorded during the generation (VV_ERR_RANGE for a token or
+ * position out of range, VV_ERR_TIMEOUT) is returned by this call itself (and cleared), with
+ * *n_out still set. */
 vv_status vv_decoder_generate(vv_decoder* dec, const int32_t* first_token, const int32_t* position,
                               int32_t n_steps, const int32_t* stop_ids, int32_t n_stop,
                               int32_t* tokens_out, int32_t* n_out, vv_stream stream);
@@ -331,8 +335,8 @@ vv_status vv_decoder_step_timeline(vv_decoder* dec, const uint16_t* input_embeds
                                    uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,
                                    int32_t* per_cta_out, vv_stream stream);
 
-/* Number of kernel launches one vv_decoder_step enqueues (for launch accounting): 1 for the
- * persistent step kernel (default), 5 per layer + 1 with VV_STEP=kernels in the environment. */
+/* Number of kernel launches one vv_decoder_step enqueues (for launch accounting): 1 (the
+ * persistent step kernel). */
 int32_t vv_decoder_step_launches(const vv_decoder* dec);
 
 #ifdef __cplusplus

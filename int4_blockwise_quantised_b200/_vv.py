@@ -91,11 +91,11 @@ def _load():
         "vv_decoder_set_graph": (S, [P, c_int32]),
         "vv_decoder_sync_status": (S, [P, P]),
         "vv_decoder_step_launches": (c_int32, [P]),
-        "vv_decoder_profile_step": (S, [P, P, P, P, P, P, POINTER(c_float), P]),
         "vv_decoder_generate": (S, [P, P, P, c_int32, POINTER(c_int32), c_int32, P,
                                     POINTER(c_int32), P]),
         "vv_decoder_profile_init": (S, [P, P, P, c_int64, P, c_int64, c_int64, P, P,
                                         POINTER(c_float), POINTER(c_int32), P]),
+        "vv_wait_selftest": (S, [c_int32, c_int64, P, P]),
         "vv_decoder_step_timeline": (S, [P, P, P, P, P, c_int32, POINTER(c_int32),
                                          POINTER(c_int32), P]),
     }
@@ -150,6 +150,12 @@ def vv_version():
 
 def vv_sync_status(stream=None):
     check(lib.vv_sync_status(stream_handle(stream)))
+
+
+def vv_wait_selftest(which, limit_ns, scratch=None, stream=None):
+    """Launch the bounded-wait self-test (which 0: mbarrier, 1: global counter; scratch: device
+    tensor of >= 16 bytes for which = 1)."""
+    check(lib.vv_wait_selftest(which, int(limit_ns), ptr(scratch), stream_handle(stream)))
 
 
 def vv_ternary_scale(w, stream=None):

@@ -44,6 +44,22 @@ int sm_count() {
   return cached[dev];
 }
 
+namespace {
+// Self-test of the bounded waits: one CTA waits, through the same helpers the kernels use, on a
+// signal that never comes (an mbarrier nobody arrives at; a counter nobody increments).
+__global__ void wait_selftest_kernel(int which, uint64_t limit_ns, unsigned* counter) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  if (which == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, limit_ns);
+  } else {
+    wait_counter_geq(counter, 1u, limit_ns);
+  }
+}
+}  // namespace
+
 }  // namespace vv
 
 extern "C" {
@@ -56,6 +72,20 @@ vv_status vv_last_error(char* buf, size_t n) {
     buf[n - 1] = '\0';
   }
   return vv::t_last_code;
+}
+
+vv_status vv_wait_selftest(int32_t which, int64_t limit_ns, void* scratch, vv_stream stream) {
+  VV_CHECK_ARG(which == 0 || which == 1, "vv_wait_selftest: which %d (0 or 1)", which);
+  VV_CHECK_ARG(limit_ns >= 1000 && limit_ns <= 100000000, "vv_wait_selftest: limit %lld ns",
+               (long long)limit_ns);
+  VV_CHECK_ARG(which == 0 || (scratch && vv::aligned16(scratch)),
+               "vv_wait_selftest: counter scratch null or misaligned");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (which == 1) VV_CUDA(cudaMemsetAsync(scratch, 0, 16, s));
+  vv::wait_selftest_kernel<<<1, 32, 0, s>>>(which, (uint64_t)limit_ns,
+                                            static_cast<unsigned*>(scratch));
+  VV_CUDA(cudaGetLastError());
+  return VV_OK;
 }
 
 vv_status vv_sync_status(vv_stream stream) {

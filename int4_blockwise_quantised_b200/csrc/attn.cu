@@ -46,7 +46,6 @@ struct AttnSmem {
   int is_last;
 };
 
-template <bool FUSED>
 __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw);
@@ -54,9 +53,8 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.Hq / a.Hkv;
 
-  // Past positions: standalone len, fused *length (stable: set a whole step earlier).
-  const int past = FUSED ? *a.length : a.len;
-  const int npos = FUSED ? past + 1 : past;
+  const int past = a.len;
+  const int npos = past;
   const int ntiles = (npos + TT - 1) / TT;
   const int tpc = (ntiles + nchunks - 1) / nchunks;
   const int t_begin = c * tpc;
@@ -97,48 +95,12 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
 
   pdl_wait();
 
-  // ---- q of the group (rotated, scaled into the log2 domain) and, fused, the new k/v.
-  int pos = 0;
-  if (FUSED) {
-    pos = *a.position;
-    if (pos < 0 || pos >= a.max_position) {
-      if (tid == 0) set_device_error(VV_ERR_RANGE);
-      pos = min(max(pos, 0), a.max_position - 1);
-    }
-  }
+  // ---- q of the group, scaled into the log2 domain
   const float qscale = a.scale * kLog2e;
   for (int i = tid; i < G * D; i += kThreads) {
     const int h = i / D, d = i % D;
-    float qv;
-    if (FUSED) {
-      const float* qh = a.qkv + (size_t)(g * G + h) * D;
-      const int fi = d & (D / 2 - 1);
-      const float cs = a.rope_cos[(size_t)pos * (D / 2) + fi];
-      const float sn = a.rope_sin[(size_t)pos * (D / 2) + fi];
-      const float x1 = __ldcg(qh + fi), x2 = __ldcg(qh + fi + D / 2);
-      qv = d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
-    } else {
-      qv = __half2float(reinterpret_cast<const __half*>(a.q_f16)[(size_t)(g * G + h) * D + d]);
-    }
+    const float qv = __half2float(reinterpret_cast<const __half*>(a.q_f16)[(size_t)(g * G + h) * D + d]);
     sm.q[h][d] = qv * qscale;
-  }
-  // The CTA owning the last tile rotates the new key, rounds k/v to fp16 and stores them at
-  // slot `past`; the row enters shared memory when that tile is processed (the bulk copies of
-  // every tile cover only rows < past, and an earlier tile may still occupy the buffer).
-  const bool owns_new = FUSED && (t_end == ntiles);
-  __half my_kn = __float2half_rn(0.f), my_vn = __float2half_rn(0.f);
-  if (owns_new && tid < D) {
-    const int d = tid;
-    const float* kh = a.qkv + (size_t)(a.Hq + g) * D;
-    const float* vh = a.qkv + (size_t)(a.Hq + a.Hkv + g) * D;
-    const int fi = d & (D / 2 - 1);
-    const float cs = a.rope_cos[(size_t)pos * (D / 2) + fi];
-    const float sn = a.rope_sin[(size_t)pos * (D / 2) + fi];
-    const float x1 = __ldcg(kh + fi), x2 = __ldcg(kh + fi + D / 2);
-    my_kn = __float2half_rn(d < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn);
-    my_vn = __float2half_rn(__ldcg(vh + d));
-    a.k_cache[((size_t)g * a.cap + past) * D + d] = __half_as_ushort(my_kn);
-    a.v_cache[((size_t)g * a.cap + past) * D + d] = __half_as_ushort(my_vn);
   }
   if (tid < kMaxG) {
     sm.m[tid] = -INFINITY;
@@ -163,13 +125,6 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
     mbar_wait(&sm.bar[b], ((t - t_begin) >> 1) & 1);
     const int p0 = t * TT;
     const int n = min(TT, npos - p0);
-    if (owns_new && t == ntiles - 1) {
-      if (tid < D) {
-        sm.k[b][(past - p0) * D + tid] = my_kn;
-        sm.v[b][(past - p0) * D + tid] = my_vn;
-      }
-      __syncthreads();
-    }
 
     // scores: warp w -> positions w, w+8, ...
     for (int p = warp; p < n; p += 2 * (kThreads / 32)) {
@@ -249,8 +204,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
       if (h < G) {
         const float r = o[j] / sm.l[h];
         const size_t idx = (size_t)(g * G + h) * D + od;
-        if (FUSED) a.out_f32[idx] = r;
-        else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(r);
+        reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(r);
       }
     }
     return;
@@ -316,8 +270,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const AttnArgs a)
         acc = fmaf(sm.mw[cc][h], __ldcg(base + ((size_t)cc * kMaxG + h) * kPartStride + 4 + od),
                    acc);
       const size_t idx = (size_t)(g * G + h) * D + od;
-      if (FUSED) a.out_f32[idx] = acc;
-      else reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(acc);
+      reinterpret_cast<__half*>(a.out_f16)[idx] = __float2half_rn(acc);
     }
   }
   if (tid == 0) a.ws_count[g] = 0;
@@ -338,19 +291,13 @@ size_t attn_workspace_bytes(int Hq, int Hkv, int nchunks) {
   return (size_t)Hkv * nchunks * kMaxG * kPartStride * sizeof(float) + 256;
 }
 
-cudaError_t launch_attn(const AttnArgs& a, bool fused, cudaStream_t s, bool pdl) {
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(AttnSmem);
   dim3 grid(a.nchunks, a.Hkv);
-  if (fused) {
-    auto k = attn_decode_kernel<true>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch(k, grid, dim3(kThreads), smem, s, pdl, a);
-  }
-  auto k = attn_decode_kernel<false>;
+  auto k = attn_decode_kernel;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch(k, grid, dim3(kThreads), smem, s, pdl, a);
+  return launch(k, grid, dim3(kThreads), smem, s, false, a);
 }
 
 }  // namespace vv
@@ -394,7 +341,7 @@ extern "C" vv_status vv_gqa_decode_attn(const uint16_t* q, const uint16_t* k_cac
   a.ws_part = static_cast<float*>(ws);
   a.ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + need - 256);
   a.nchunks = nch;
-  return vv::cuda_check(vv::launch_attn(a, false, static_cast<cudaStream_t>(stream), false),
+  return vv::cuda_check(vv::launch_attn(a, static_cast<cudaStream_t>(stream)),
                         "attention launch");
 }
 
@@ -441,6 +388,13 @@ extern "C" vv_status vv_gqa_decode_attn_noalloc(const uint16_t* q, const uint16_
   int dev = 0;
   VV_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return vv::set_error(VV_ERR_INVALID_ARG, "device ordinal %d", dev);
+  // The array's address is per device: the stream must belong to the current device.
+  int sdev = dev;
+  VV_CUDA(cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev));
+  if (sdev != dev)
+    return vv::set_error(VV_ERR_INVALID_ARG,
+                         "vv_gqa_decode_attn_noalloc: stream of device %d, current device %d",
+                         sdev, dev);
   void* base = nullptr;
   {
     // First call on a device: look up the array's device address with that device current.
@@ -469,5 +423,5 @@ extern "C" vv_status vv_gqa_decode_attn_noalloc(const uint16_t* q, const uint16_
   a.ws_part = reinterpret_cast<float*>(ws);
   a.ws_count = reinterpret_cast<int*>(ws + need - 256);
   a.nchunks = nch;
-  return vv::cuda_check(vv::launch_attn(a, false, s, false), "attention (no-alloc) launch");
+  return vv::cuda_check(vv::launch_attn(a, s), "attention (no-alloc) launch");
 }

@@ -39,134 +39,15 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
                          const int32_t* position, float* logits, int32_t* argmax,
-                         cudaStream_t s, bool head, cudaEvent_t* ev) {
-  if (d->persistent && ev == nullptr && head) {
-    StepParams p = d->step;
-    p.input_embeds = reinterpret_cast<const __half*>(embeds);
-    p.token = token;
-    p.position = position;
-    p.logits = logits;
-    p.argmax = argmax ? argmax : d->d_argmax;
-    p.trace = d->trace;
-    return launch_step(p, s);
-  }
-  // ev (profiling): 2 events per launch, recorded around each kernel; PDL off so the events
-  // bracket exactly one kernel.
-  const bool pdl = ev == nullptr && d->use_pdl;
-  int evi = 0;
-  auto mark = [&]() {
-    if (ev) cudaEventRecord(ev[evi++], s);
-  };
-  const vv_config& c = d->cfg;
-  const int H = c.hidden, D = c.head_dim, Hq = c.n_q, Hkv = c.n_kv, I = c.inter;
-  const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
-  cudaError_t e;
-  for (int l = 0; l < c.layers; ++l) {
-    const vv_layer_weights& w = d->layers[l];
-    QkvArgs qa = {};
-    qa.w[0] = GemvWeights{w.wq.q, w.wq.scales};
-    qa.w[1] = GemvWeights{w.wk.q, w.wk.scales};
-    qa.w[2] = GemvWeights{w.wv.q, w.wv.scales};
-    qa.rows[0] = Hq * D;
-    qa.rows[1] = Hkv * D;
-    qa.rows[2] = Hkv * D;
-    qa.bias[0] = w.bq;
-    qa.bias[1] = w.bk;
-    qa.bias[2] = w.bv;
-    qa.K = H;
-    qa.x_resid_in = d->x_resid;
-    if (l == 0) {
-      qa.embeds = embeds;
-      qa.embed_table = embeds ? nullptr : d->embed;
-      qa.token = token;
-      qa.vocab = c.vocab;
-      qa.x_resid_out = d->x_resid;
-    }
-    qa.gamma = w.input_norm;
-    qa.eps = c.eps;
-    qa.out = d->qkv;
-    // The first kernel of a step is not overlapped with the previous step (it reads the
-    // caller's inputs and the length written by the previous step's last kernel).
-    mark();
-    if ((e = launch_qkv(qa, s, pdl && l > 0)) != cudaSuccess) return e;
-    mark();
-
-    AttnArgs aa = {};
-    aa.qkv = d->qkv;
-    aa.position = position;
-    aa.length = d->d_length;
-    aa.rope_cos = d->rope_cos;
-    aa.rope_sin = d->rope_sin;
-    aa.max_position = c.max_position;
-    aa.k_cache = d->k_cache + (size_t)l * layer_kv;
-    aa.v_cache = d->v_cache + (size_t)l * layer_kv;
-    aa.cap = c.kv_capacity;
-    aa.Hq = Hq;
-    aa.Hkv = Hkv;
-    aa.scale = 1.0f / sqrtf((float)D);
-    aa.out_f32 = d->o;
-    aa.ws_part = d->attn_part;
-    aa.ws_count = d->attn_count;
-    aa.nchunks = d->attn_chunks;
-    mark();
-    if ((e = launch_attn(aa, true, s, pdl)) != cudaSuccess) return e;
-    mark();
-
-    ResidArgs ro = {};
-    ro.w = GemvWeights{w.wo.q, w.wo.scales};
-    ro.N = H;
-    ro.K = Hq * D;
-    ro.x = d->o;
-    ro.x_resid = d->x_resid;
-    mark();
-    if ((e = launch_resid(ro, s, pdl)) != cudaSuccess) return e;
-    mark();
-
-    GateUpArgs ga = {};
-    ga.wg = GemvWeights{w.wgate.q, w.wgate.scales};
-    ga.wu = GemvWeights{w.wup.q, w.wup.scales};
-    ga.N = I;
-    ga.K = H;
-    ga.x_resid = d->x_resid;
-    ga.gamma = w.post_norm;
-    ga.eps = c.eps;
-    ga.h = d->h;
-    mark();
-    if ((e = launch_gateup(ga, s, pdl)) != cudaSuccess) return e;
-    mark();
-
-    ResidArgs rd = {};
-    rd.w = GemvWeights{w.wdown.q, w.wdown.scales};
-    rd.N = H;
-    rd.K = I;
-    rd.x = d->h;
-    rd.x_resid = d->x_resid;
-    rd.trace = d->trace ? d->trace + (size_t)l * H : nullptr;
-    mark();
-    if ((e = launch_resid(rd, s, pdl)) != cudaSuccess) return e;
-    mark();
-  }
-  if (!head) {
-    add_int_kernel<<<1, 1, 0, s>>>(d->d_length, 1);
-    return cudaGetLastError();
-  }
-  LmHeadArgs la = {};
-  la.x = d->x_resid;
-  la.gamma = d->final_norm;
-  la.w = d->lm_head;
-  la.V = c.vocab;
-  la.H = H;
-  la.eps = c.eps;
-  la.logits = logits;
-  la.idx = argmax ? argmax : d->d_argmax;
-  la.ws_val = d->lm_val;
-  la.ws_idx = d->lm_idx;
-  la.ws_count = d->lm_count;
-  la.length = d->d_length;
-  mark();
-  e = launch_lm_head(la, s, pdl);
-  mark();
-  return e;
+                         cudaStream_t s) {
+  StepParams p = d->step;
+  p.input_embeds = reinterpret_cast<const __half*>(embeds);
+  p.token = token;
+  p.position = position;
+  p.logits = logits;
+  p.argmax = argmax ? argmax : d->d_argmax;
+  p.trace = d->trace;
+  return launch_step(p, s);
 }
 
 }  // namespace vv
@@ -183,11 +64,10 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   VV_CHECK_SHAPE(c.head_dim == 128, "head_dim %d (only 128)", c.head_dim);
   VV_CHECK_SHAPE(c.n_kv >= 1 && c.n_kv <= 64 && c.n_q % c.n_kv == 0 && c.n_q / c.n_kv <= 8,
                  "n_q %d / n_kv %d", c.n_q, c.n_kv);
-  VV_CHECK_SHAPE(c.hidden >= 256 && c.hidden % 256 == 0 && c.hidden <= 16384, "hidden %d",
+  VV_CHECK_SHAPE(c.hidden >= 256 && c.hidden % 256 == 0 && c.hidden <= 7680, "hidden %d",
                  c.hidden);
-  VV_CHECK_SHAPE(c.inter >= 256 && c.inter % 256 == 0 && c.inter <= 32768, "inter %d", c.inter);
-  VV_CHECK_SHAPE((c.n_q * c.head_dim) % 256 == 0 && c.n_q * c.head_dim <= 16384, "n_q*D %d",
-                 c.n_q * c.head_dim);
+  VV_CHECK_SHAPE(c.inter >= 64 && c.inter % 256 == 0 && c.inter <= 65536, "inter %d", c.inter);
+  VV_CHECK_SHAPE(c.n_q * c.head_dim <= 7680, "n_q*D %d", c.n_q * c.head_dim);
   VV_CHECK_SHAPE(c.layers >= 1 && c.vocab >= 1 && c.kv_capacity >= 1 && c.max_position >= 1 &&
                      c.max_prefill >= 0,
                  "layers/vocab/capacity/max_position");
@@ -214,42 +94,39 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   d->k_cache = k_cache;
   d->v_cache = v_cache;
   cudaGetDevice(&d->device);
-  // VV_PDL=0 launches the step without programmatic dependent launch (diagnostics).
-  if (const char* e = getenv("VV_PDL")) d->use_pdl = atoi(e) != 0;
 
   const int H = c.hidden, D = c.head_dim;
-  d->attn_chunks = vv::attn_default_chunks(c.n_kv, c.kv_capacity);
-  const int lm_grid = vv::lm_head_grid(c.vocab);
+  const int grid = vv::sm_count();
+  const int max_tiles = vv::step_max_tiles(c.kv_capacity);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = vv::align_up(off + bytes, 256);
     return o;
   };
-  const size_t o_x = take((size_t)H * 4);
+  const size_t o_x = take((size_t)H * 8);
   const size_t o_qkv = take((size_t)(c.n_q + 2 * c.n_kv) * D * 4);
-  const size_t o_o = take((size_t)c.n_q * D * 4);
-  const size_t o_h = take((size_t)c.inter * 4);
   const size_t o_cos = take((size_t)c.max_position * (D / 2) * 4);
   const size_t o_sin = take((size_t)c.max_position * (D / 2) * 4);
   const size_t o_len = take(16);
   const size_t o_arg = take(16);
   const size_t o_gen = take(16);  // generation: done flag, token count, position
-  const size_t attn_b = vv::attn_workspace_bytes(c.n_q, c.n_kv, d->attn_chunks);
-  const size_t o_part = take(attn_b);
-  const size_t o_lmv = take((size_t)lm_grid * 4);
-  const size_t o_lmi = take((size_t)lm_grid * 4);
-  const size_t o_lmc = take(16);
-  // persistent step kernel
-  const int grid = vv::sm_count();
-  const int max_tiles = vv::step_max_tiles(c.kv_capacity);
-  const size_t o_spart = take(vv::step_attn_part_floats(c.n_kv, max_tiles) * 4);
-  const size_t o_scnt = take((size_t)c.n_kv * 4);
+  const size_t o_part = take(vv::step_attn_part_floats(c.n_kv, max_tiles) * 4);
   const size_t o_hval = take((size_t)grid * 4);
   const size_t o_hidx = take((size_t)grid * 4);
   const size_t o_hcnt = take(16);
   const size_t o_bar = take(16);
   const size_t o_layers = take(sizeof(vv::StepLayer) * c.layers);
+  const int lm_grid = vv::lm_head_grid(c.vocab);
+  const size_t o_xl = take((size_t)H * 4);
+  const size_t o_lmv = take((size_t)lm_grid * 4);
+  const size_t o_lmi = take((size_t)lm_grid * 4);
+  const size_t o_lmc = take(16);
+  // column images of Wo and Wd (the o-proj and down phases read column blocks)
+  const size_t wo_b = vv::step_wo_image_bytes(H, c.n_q);
+  const size_t wd_b = vv::step_wd_image_bytes(H, c.inter, grid);
+  const size_t o_wo = take(wo_b * c.layers);
+  const size_t o_wd = take(wd_b * c.layers);
   d->ws_bytes = off;
   vv_status st = vv::cuda_check(cudaMalloc(&d->ws, d->ws_bytes), "cudaMalloc(decoder workspace)");
   if (st) {
@@ -258,17 +135,12 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   }
   st = vv::cuda_check(cudaMemset(d->ws, 0, d->ws_bytes), "cudaMemset");
   unsigned char* b = d->ws;
-  d->x_resid = reinterpret_cast<float*>(b + o_x);
-  d->qkv = reinterpret_cast<float*>(b + o_qkv);
-  d->o = reinterpret_cast<float*>(b + o_o);
-  d->h = reinterpret_cast<float*>(b + o_h);
   d->rope_cos = reinterpret_cast<float*>(b + o_cos);
   d->rope_sin = reinterpret_cast<float*>(b + o_sin);
   d->d_length = reinterpret_cast<int32_t*>(b + o_len);
   d->d_argmax = reinterpret_cast<int32_t*>(b + o_arg);
   d->d_gen = reinterpret_cast<int32_t*>(b + o_gen);
-  d->attn_part = reinterpret_cast<float*>(b + o_part);
-  d->attn_count = reinterpret_cast<int*>(b + o_part + attn_b - 256);
+  d->x_last = reinterpret_cast<float*>(b + o_xl);
   d->lm_val = reinterpret_cast<float*>(b + o_lmv);
   d->lm_idx = reinterpret_cast<int*>(b + o_lmi);
   d->lm_count = reinterpret_cast<int*>(b + o_lmc);
@@ -294,23 +166,19 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
     p.rope_cos = d->rope_cos;
     p.rope_sin = d->rope_sin;
     p.max_position = c.max_position;
-    p.x_resid = d->x_resid;
-    p.qkv = d->qkv;
-    p.attn_out = d->o;
-    p.h = d->h;
-    p.attn_part = reinterpret_cast<float*>(b + o_spart);
-    p.attn_count = reinterpret_cast<int*>(b + o_scnt);
+    p.x_acc = reinterpret_cast<unsigned long long*>(b + o_x);
+    p.qkv = reinterpret_cast<float*>(b + o_qkv);
+    p.attn_part = reinterpret_cast<float*>(b + o_part);
     p.max_tiles = max_tiles;
     p.head_val = reinterpret_cast<float*>(b + o_hval);
     p.head_idx = reinterpret_cast<int*>(b + o_hidx);
     p.head_count = reinterpret_cast<int*>(b + o_hcnt);
     p.length = d->d_length;
     p.bar_count = reinterpret_cast<unsigned*>(b + o_bar);
-    p.bar_gen = reinterpret_cast<unsigned*>(b + o_bar + 4);
     p.grid = grid;
     p.nstages = 4;
-    p.x_floats = std::max(std::max(H, c.n_q * D), c.inter);
-    const size_t fixed = vv::step_smem_bytes(0, p.nstages, p.x_floats);
+    p.stage_bytes = 0;
+    const size_t fixed = vv::step_smem_bytes(p);
     int smem_max = 0;
     cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, d->device);
     if (smem_max <= 0) smem_max = 232448;
@@ -329,27 +197,29 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
       hl[l].bias[0] = reinterpret_cast<const __half*>(L.bq);
       hl[l].bias[1] = reinterpret_cast<const __half*>(L.bk);
       hl[l].bias[2] = reinterpret_cast<const __half*>(L.bv);
+      hl[l].wo_img = b + o_wo + (size_t)l * wo_b;
+      hl[l].wd_img = b + o_wd + (size_t)l * wd_b;
     }
     if (!st)
       st = vv::cuda_check(cudaMemcpy(d->d_layers, hl.data(), sizeof(vv::StepLayer) * c.layers,
                                      cudaMemcpyHostToDevice),
                           "copy layer table");
+    if (!st)
+      st = vv::cuda_check(vv::step_build_images(p, hl.data(), b + o_wo, b + o_wd, nullptr),
+                          "build column images");
+    if (!st) st = vv::cuda_check(cudaDeviceSynchronize(), "build column images");
     int nb = 0;
-    if (!st && H > 32 * grid)
-      st = set_error(VV_ERR_SHAPE, "hidden %d > 32 x SM count (persistent step)", H);
     if (!st) st = vv::cuda_check(vv::step_configure(p, &nb), "step kernel configuration");
     if (!st && nb < 1) {
       int regs = 0, mt = 0, ss = 0, lb = 0;
       vv::step_func_info(&regs, &mt, &ss, &lb);
       st = set_error(VV_ERR_SHAPE,
-                     "persistent step: no stage size >= 32 KB fits one CTA per SM (regs %d, "
-                     "max threads %d, static smem %d, local %d, threads %d, smem optin %d)",
+                     "persistent step: no stage size that holds an attention tile fits one CTA "
+                     "per SM (regs %d, max threads %d, static smem %d, local %d, threads %d, "
+                     "smem optin %d)",
                      regs, mt, ss, lb, vv::step_threads(), smem_max);
     }
-    if (!st && max_tiles > 256)
-      st = set_error(VV_ERR_SHAPE, "kv_capacity %d > 16384 (persistent step)", c.kv_capacity);
   }
-  if (const char* e = getenv("VV_STEP")) d->persistent = strcmp(e, "kernels") != 0;
 
   // RoPE tables: angle = pos * theta^(-2i/D) in float64, cos/sin rounded once to fp32.
   if (!st) {
@@ -417,10 +287,7 @@ vv_status vv_decoder_set_graph(vv_decoder* d, int32_t enable) {
   return VV_OK;
 }
 
-int32_t vv_decoder_step_launches(const vv_decoder* d) {
-  if (!d) return 0;
-  return d->persistent ? 1 : d->cfg.layers * 5 + 1;
-}
+int32_t vv_decoder_step_launches(const vv_decoder* d) { return d ? 1 : 0; }
 
 vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int32_t* token_id,
                           const int32_t* position_id, float* logits, int32_t* argmax_out,
@@ -433,7 +300,7 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
                      d->cfg.kv_capacity);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!d->use_graph) {
-    VV_CUDA(vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s, true, nullptr));
+    VV_CUDA(vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s));
     d->len_host += 1;
     return VV_OK;
   }
@@ -453,7 +320,7 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
     cudaGraph_t g = nullptr;
     VV_CUDA(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
     cudaError_t le =
-        vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, cs, true, nullptr);
+        vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, cs);
     cudaError_t ee = cudaStreamEndCapture(cs, &g);
     if (le != cudaSuccess) {
       if (g) cudaGraphDestroy(g);
@@ -470,47 +337,13 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
   return VV_OK;
 }
 
-vv_status vv_decoder_profile_step(vv_decoder* d, const uint16_t* input_embeds,
-                                  const int32_t* token_id, const int32_t* position_id,
-                                  float* logits, int32_t* argmax_out, float* phase_ms,
-                                  vv_stream stream) {
-  VV_CHECK_ARG(d && position_id && phase_ms, "vv_decoder_profile_step: null pointer");
-  VV_CHECK_ARG(input_embeds || token_id, "vv_decoder_profile_step: need input_embeds or token");
-  if (d->len_host + 1 > d->cfg.kv_capacity)
-    return set_error(VV_ERR_CAPACITY, "KV cache full (%d of %d)", d->len_host,
-                     d->cfg.kv_capacity);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int n = 2 * (d->cfg.layers * 5 + 1);
-  std::vector<cudaEvent_t> ev(n, nullptr);
-  vv_status st = VV_OK;
-  for (int i = 0; i < n && !st; ++i) st = vv::cuda_check(cudaEventCreate(&ev[i]), "event");
-  if (!st)
-    st = vv::cuda_check(vv::enqueue_step(d, input_embeds, token_id, position_id, logits,
-                                         argmax_out, s, true, ev.data()),
-                        "profile step");
-  if (!st) st = vv::cuda_check(cudaStreamSynchronize(s), "sync");
-  if (!st) {
-    for (int i = 0; i < 6; ++i) phase_ms[i] = 0.f;
-    for (int k = 0; k < n / 2; ++k) {
-      float ms = 0.f;
-      cudaEventElapsedTime(&ms, ev[2 * k], ev[2 * k + 1]);
-      const int phase = (k == n / 2 - 1) ? 5 : (k % 5);
-      phase_ms[phase] += ms;
-    }
-    d->len_host += 1;
-  }
-  for (auto e : ev)
-    if (e) cudaEventDestroy(e);
-  return st;
-}
-
 vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
                                    const int32_t* token_id, const int32_t* position_id,
                                    uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,
                                    int32_t* per_cta_out, vv_stream stream) {
   VV_CHECK_ARG(d && position_id && stamps && grid_out && per_cta_out, "null pointer");
   VV_CHECK_ARG(input_embeds || token_id, "need input_embeds or token_id");
-  const int need = 14 * d->cfg.layers + 11;
+  const int need = vv::step_timeline_stamps(d->cfg.layers);
   if (max_per_cta < need)
     return set_error(VV_ERR_CAPACITY, "max_per_cta %d < %d", max_per_cta, need);
   if (d->len_host + 1 > d->cfg.kv_capacity)
@@ -539,7 +372,7 @@ vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
   cudaFree(dst);
   if (st) return st;
   int n = 0;
-  while (n < max_per_cta - 3 && stamps[n] != 0) ++n;
+  while (n < max_per_cta - 8 && stamps[n] != 0) ++n;
   *grid_out = grid;
   *per_cta_out = n;
   d->len_host += 1;
@@ -614,7 +447,6 @@ vv_status vv_decoder_generate(vv_decoder* d, const int32_t* first_token, const i
                "vv_decoder_generate: null pointer");
   VV_CHECK_ARG(n_stop >= 0 && n_stop <= vv::kMaxStopIds && (n_stop == 0 || stop_ids),
                "vv_decoder_generate: n_stop %d (0..%d)", n_stop, vv::kMaxStopIds);
-  VV_CHECK_ARG(d->persistent, "vv_decoder_generate needs the persistent step kernel");
   if (n_steps < 1) return set_error(VV_ERR_SHAPE, "n_steps=%d", n_steps);
   if (d->len_host + n_steps > d->cfg.kv_capacity)
     return set_error(VV_ERR_CAPACITY, "%d + %d steps exceed the KV capacity %d", d->len_host,
@@ -645,7 +477,9 @@ vv_status vv_decoder_generate(vv_decoder* d, const int32_t* first_token, const i
   VV_CUDA(cudaStreamSynchronize(s));
   d->len_host += n;
   *n_out = n;
-  return VV_OK;
+  // a device-side error during the generation (a bounded wait that ran out, a token or position
+  // out of range) is this call's result
+  return vv_sync_status(stream);
 }
 
 vv_status vv_decoder_sync_status(vv_decoder* d, vv_stream stream) {

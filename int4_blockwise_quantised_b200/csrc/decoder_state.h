@@ -20,18 +20,13 @@ struct vv_decoder {
 
   unsigned char* ws = nullptr;
   size_t ws_bytes = 0;
-  float* x_resid = nullptr;
-  float* qkv = nullptr;
-  float* o = nullptr;
-  float* h = nullptr;
   float* rope_cos = nullptr;
   float* rope_sin = nullptr;
   int32_t* d_length = nullptr;
   int32_t* d_argmax = nullptr;
   int32_t* d_gen = nullptr;  // [done, count, position] of vv_decoder_generate
-  float* attn_part = nullptr;
-  int* attn_count = nullptr;
-  int attn_chunks = 1;
+  // prefill's final norm + lm_head: fp32 residual of the last position and argmax partials
+  float* x_last = nullptr;
   float* lm_val = nullptr;
   int* lm_idx = nullptr;
   int* lm_count = nullptr;
@@ -42,8 +37,6 @@ struct vv_decoder {
   int32_t len_host = 0;
   float* trace = nullptr;
   bool use_graph = true;
-  bool use_pdl = true;
-  bool persistent = true;          // one cooperative kernel per step (default)
   vv::StepParams step = {};        // persistent-kernel parameters (per-call pointers patched)
   vv::StepLayer* d_layers = nullptr;
   cudaGraphExec_t gexec = nullptr;
@@ -62,11 +55,9 @@ struct PrefillTimer {
 };
 __global__ void set_int_kernel(int32_t* p, int32_t v);
 __global__ void add_int_kernel(int32_t* p, int32_t v);
-// Enqueue one decode step (plain launches).  head=false skips the lm_head and only advances the
-// device length (used by the token-by-token prefill).
+// Enqueue one decode step: one launch of the persistent step kernel.
 cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
-                         const int32_t* position, float* logits, int32_t* argmax, cudaStream_t s,
-                         bool head, cudaEvent_t* events = nullptr);
+                         const int32_t* position, float* logits, int32_t* argmax, cudaStream_t s);
 cudaError_t prefill_run(vv_decoder* dec, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
                         cudaStream_t s, PrefillTimer* timer = nullptr);

@@ -113,93 +113,6 @@ __device__ void stage_x(float* xs, const float* __restrict__ src32, const __half
 // Each op describes: number of segments (matrices read per stage), the CTA -> rows mapping, the
 // x source, and what happens to a finished row group.
 
-struct OpQkv {  // [Wq; Wk; Wv] . RMSNorm(x) + bias -> out fp32
-  static constexpr int NSEG = 1;
-  static constexpr bool NORM = true;
-  QkvArgs a;
-  int cta_split[3];  // CTAs per matrix
-  __device__ void rows(int cta, const uint8_t** q, const __half** s, int& r0, int& r1,
-                       int& mat) const {
-    int c = cta, m = 0;
-    while (m < 2 && c >= cta_split[m]) c -= cta_split[m++];
-    const int n = a.rows[m], per = cta_split[m];
-    r0 = (int)((int64_t)n * c / per);
-    r1 = (int)((int64_t)n * (c + 1) / per);
-    q[0] = a.w[m].q;
-    s[0] = reinterpret_cast<const __half*>(a.w[m].scales);
-    mat = m;
-  }
-  __device__ void load_x(float* xs, int tid, int nthreads, float* red) const {
-    const __half* e16 = nullptr;
-    if (a.embeds) {
-      e16 = reinterpret_cast<const __half*>(a.embeds);
-    } else if (a.embed_table) {
-      int tok = __ldcg(a.token);
-      if (tok < 0 || tok >= a.vocab) {
-        if (tid == 0) set_device_error(VV_ERR_RANGE);
-        tok = min(max(tok, 0), a.vocab - 1);
-      }
-      e16 = reinterpret_cast<const __half*>(a.embed_table) + (int64_t)tok * a.K;
-    }
-    if (e16 && a.x_resid_out && blockIdx.x == 0) {
-      for (int k = tid; k < a.K; k += nthreads) a.x_resid_out[k] = __half2float(e16[k]);
-    }
-    stage_x<true>(xs, e16 ? nullptr : a.x_resid_in, e16,
-                  reinterpret_cast<const __half*>(a.gamma), a.eps, a.K, tid, nthreads, red);
-  }
-  __device__ void finish(int mat, int row, float y) const {
-    int off = 0;
-    for (int m = 0; m < mat; ++m) off += a.rows[m];
-    const __half* b = reinterpret_cast<const __half*>(a.bias[mat]);
-    a.out[off + row] = y + (b ? __half2float(b[row]) : 0.f);
-  }
-};
-
-struct OpResid {  // x_resid[n] += W[n] . x
-  static constexpr int NSEG = 1;
-  static constexpr bool NORM = false;
-  ResidArgs a;
-  __device__ void rows(int cta, const uint8_t** q, const __half** s, int& r0, int& r1,
-                       int& mat) const {
-    r0 = (int)((int64_t)a.N * cta / gridDim.x);
-    r1 = (int)((int64_t)a.N * (cta + 1) / gridDim.x);
-    q[0] = a.w.q;
-    s[0] = reinterpret_cast<const __half*>(a.w.scales);
-    mat = 0;
-  }
-  __device__ void load_x(float* xs, int tid, int nthreads, float* red) const {
-    stage_x<false>(xs, a.x, nullptr, nullptr, 0.f, a.K, tid, nthreads, red);
-  }
-  __device__ void finish(int, int row, float y) const {
-    const float v = __ldcg(a.x_resid + row) + y;
-    a.x_resid[row] = v;
-    if (a.trace) a.trace[row] = v;
-  }
-};
-
-struct OpGateUp {  // h[n] = silu(Wg[n] . xn) * (Wu[n] . xn)
-  static constexpr int NSEG = 2;
-  static constexpr bool NORM = true;
-  GateUpArgs a;
-  __device__ void rows(int cta, const uint8_t** q, const __half** s, int& r0, int& r1,
-                       int& mat) const {
-    r0 = (int)((int64_t)a.N * cta / gridDim.x);
-    r1 = (int)((int64_t)a.N * (cta + 1) / gridDim.x);
-    q[0] = a.wg.q;
-    s[0] = reinterpret_cast<const __half*>(a.wg.scales);
-    q[1] = a.wu.q;
-    s[1] = reinterpret_cast<const __half*>(a.wu.scales);
-    mat = 0;
-  }
-  __device__ void load_x(float* xs, int tid, int nthreads, float* red) const {
-    stage_x<true>(xs, a.x_resid, nullptr, reinterpret_cast<const __half*>(a.gamma), a.eps, a.K,
-                  tid, nthreads, red);
-  }
-  __device__ void finish2(int row, float g, float u) const {
-    a.h[row] = g / (1.f + __expf(-g)) * u;
-  }
-};
-
 struct MatmulArgs {
   const uint16_t* x;
   GemvWeights w;
@@ -407,43 +320,6 @@ int grid_for_rows(int N, int rows_per_cta_min) {
 }
 
 }  // namespace
-
-// ------------------------------------------------------------------------------- launchers
-// Tile choices by K (the reduction length): K = 1536/3584 -> one warp spans the row (WK = 1),
-// eight row groups per stage; larger K -> warps split K.
-cudaError_t launch_qkv(const QkvArgs& a, cudaStream_t s, bool pdl) {
-  OpQkv op;
-  op.a = a;
-  const int total = a.rows[0] + a.rows[1] + a.rows[2];
-  int grid = grid_for_rows(total, 8);
-  int assigned = 0;
-  for (int m = 0; m < 3; ++m) {
-    int c = (int)((int64_t)grid * a.rows[m] / total);
-    if (c < 1) c = 1;
-    op.cta_split[m] = c;
-    assigned += c;
-  }
-  grid = assigned;
-  if (a.K <= 2048) return launch_gemv<OpQkv, GemvCfg<4, 1, 8, 2, 1>>(op, a.K, grid, s, pdl);
-  return launch_gemv<OpQkv, GemvCfg<2, 2, 4, 2, 1>>(op, a.K, grid, s, pdl);
-}
-
-cudaError_t launch_resid(const ResidArgs& a, cudaStream_t s, bool pdl) {
-  OpResid op;
-  op.a = a;
-  const int grid = grid_for_rows(a.N, 4);
-  if (a.K <= 2048) return launch_gemv<OpResid, GemvCfg<4, 3, 2, 2, 1>>(op, a.K, grid, s, pdl);
-  if (a.K <= 4096) return launch_gemv<OpResid, GemvCfg<4, 4, 2, 3, 1>>(op, a.K, grid, s, pdl);
-  return launch_gemv<OpResid, GemvCfg<4, 6, 1, 3, 1>>(op, a.K, grid, s, pdl);
-}
-
-cudaError_t launch_gateup(const GateUpArgs& a, cudaStream_t s, bool pdl) {
-  OpGateUp op;
-  op.a = a;
-  const int grid = grid_for_rows(a.N, 2);
-  if (a.K <= 2048) return launch_gemv<OpGateUp, GemvCfg<4, 1, 8, 3, 2>>(op, a.K, grid, s, pdl);
-  return launch_gemv<OpGateUp, GemvCfg<4, 2, 4, 3, 2>>(op, a.K, grid, s, pdl);
-}
 
 // Generic fallback GEMV for any K % 32 == 0 and M <= 8: one warp per output row, x read from
 // global (L2-resident), plain loads.  Used by vv_matmul_nbits when the TMA path does not apply.

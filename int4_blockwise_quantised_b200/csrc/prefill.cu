@@ -12,8 +12,6 @@
 //   X  += Hm . Wd^T                                   tcgen05 GEMM, residual epilogue
 // Each packed int4 matrix is first dequantised to an fp16 copy ((code - 8) * scale, rounded once)
 // in a reused workspace buffer.  The last row then goes through the final RMSNorm + lm_head.
-// VV_PREFILL=steps in the environment selects the token-by-token path (one decode step per
-// position), kept as a cross-check of the tensor-core path.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -139,10 +137,6 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const float* __restrict__ 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-cudaError_t prefill_steps(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
-                          const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
-                          cudaStream_t s);
-
 }  // namespace
 
 cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
@@ -162,9 +156,6 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   do {                                               \
     if ((e = mark(k)) != cudaSuccess) return e;      \
   } while (0)
-  const char* mode = getenv("VV_PREFILL");
-  if (mode && strcmp(mode, "steps") == 0)
-    return prefill_steps(d, ids, pos, S, audio, N, off, logits, argmax, s);
   const vv_config& c = d->cfg;
   const int H = c.hidden, Hq = c.n_q, Hkv = c.n_kv, I = c.inter, HQD = Hq * D;
   const int NQKV = (Hq + 2 * Hkv) * D;
@@ -313,11 +304,11 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     }
   }
   // ---- last position: final norm + lm_head + argmax; the residual row feeds later steps
-  if ((e = cudaMemcpyAsync(d->x_resid, X + (size_t)(S - 1) * H, (size_t)H * 4,
+  if ((e = cudaMemcpyAsync(d->x_last, X + (size_t)(S - 1) * H, (size_t)H * 4,
                            cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
     return e;
   LmHeadArgs la = {};
-  la.x = d->x_resid;
+  la.x = d->x_last;
   la.gamma = d->final_norm;
   la.w = d->lm_head;
   la.V = c.vocab;
@@ -337,57 +328,5 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   return cudaSuccess;
 #undef VV_MARK
 }
-
-namespace {
-// Token-by-token prefill: one decode step per prompt position (cross-check path).
-__global__ void __launch_bounds__(256) splice_kernel(const int32_t* __restrict__ ids, int S,
-                                                     const uint16_t* __restrict__ embed, int V,
-                                                     int H, const uint16_t* __restrict__ audio,
-                                                     int N, int off, uint16_t* __restrict__ out) {
-  const int row = blockIdx.x;
-  if (row >= S) return;
-  const uint4* src;
-  if (row >= off && row < off + N) {
-    src = reinterpret_cast<const uint4*>(audio + (size_t)(row - off) * H);
-  } else {
-    int id = ids[row];
-    if (id < 0 || id >= V) {
-      if (threadIdx.x == 0) set_device_error(VV_ERR_RANGE);
-      id = min(max(id, 0), V - 1);
-    }
-    src = reinterpret_cast<const uint4*>(embed + (size_t)id * H);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * H);
-  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = src[i];
-}
-
-cudaError_t prefill_steps(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
-                          const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
-                          cudaStream_t s) {
-  const vv_config& c = d->cfg;
-  const size_t need = (size_t)c.max_prefill * c.hidden * 2;
-  if (d->pws_bytes < need) {
-    if (d->pws) cudaFree(d->pws);
-    d->pws = nullptr;
-    d->pws_bytes = 0;
-    cudaError_t e = cudaMalloc(&d->pws, need);
-    if (e != cudaSuccess) return e;
-    d->pws_bytes = need;
-  }
-  uint16_t* embeds = reinterpret_cast<uint16_t*>(d->pws);
-  splice_kernel<<<S, 256, 0, s>>>(ids, S, d->embed, c.vocab, c.hidden, audio, N, off, embeds);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  set_int_kernel<<<1, 1, 0, s>>>(d->d_length, 0);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  for (int i = 0; i < S; ++i) {
-    const bool last = i == S - 1;
-    e = enqueue_step(d, embeds + (size_t)i * c.hidden, nullptr, pos + i, last ? logits : nullptr,
-                     last ? argmax : nullptr, s, last, nullptr);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
-}
-}  // namespace
 
 }  // namespace vv

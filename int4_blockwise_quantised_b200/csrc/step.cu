@@ -3,31 +3,34 @@
 // export for Vernacula", section "Highlights": the step's ~1950 launches are the overhead to
 // remove).
 //
-// One CTA per SM.  Warp 0..NW-1 compute, warp NW is the producer.
+// One CTA per SM.  Warps 0..NW-1 compute, warp NW is the producer.
 //
-// The producer walks a static per-CTA schedule of everything the step streams from HBM -- for each
-// layer: its rows of [Wq;Wk;Wv], its K/V tiles, its rows of Wo, of Wgate+Wup, of Wdown; then its
-// rows of the lm_head -- and moves it with cp.async.bulk into a ring of shared-memory stages.
-// Weights and past K/V do not depend on the step's activations, so the producer never waits for
-// them: HBM keeps streaming across phase boundaries, limited only by the ring's depth.
+// Producer: walks a static per-CTA schedule of everything the step streams from HBM and moves it
+// with cp.async.bulk into a ring of shared-memory stages.  Weights and past K/V do not depend on
+// the step's activations, so HBM keeps streaming across phase boundaries, limited only by the
+// ring's depth.
 //
-// Compute warps walk the same schedule.  Before each phase they pass a grid-wide barrier (the
-// phase's input is an activation vector produced by every CTA), stage that vector in shared
-// memory / registers (with the fused RMSNorm where the layer has one), then consume the phase's
-// stages.  Phases per layer:
-//   QKV  : y = [Wq;Wk;Wv] . RMSNorm(x) + b              -> qkv (fp32); the CTA's q/k/v rows
-//          form one stream of stages even where they straddle two matrices
-//   ATTN : per (kv head, 64-position tile): RoPE(q), RoPE(k_new) + append at slot `length`,
-//          online-softmax partial (m, l, o); up to 32 tiles per head the O staging of every CTA
-//          merges the partials, beyond that the last CTA of a head merges them -> attn (fp32)
-//   O    : x += Wo . attn
-//   GU   : h = silu(Wg . RMSNorm(x)) * (Wu . RMSNorm(x))
-//   DOWN : x += Wd . h
+// Compute warps, per layer (four dependent phases, a grid barrier before each but the first):
+//   QKV  : xn = RMSNorm(x); this CTA's rows of [Wq;Wk;Wv] . xn + b  -> qkv (fp32)
+//   ATTN : items (kv head g, 64-position tile): RoPE(q), RoPE(k_new) + append at slot `length`,
+//          online-softmax partial (m, l, o) per head
+//   O    : items (head h, 128-row block): merge head h's partials -> o_h, then the 128 columns
+//          of Wo that multiply o_h, for the block's rows; the products are added into x
+//   GU+D : xn = RMSNorm(x); for each of this CTA's 64-channel slices: gate/up rows -> h =
+//          silu(g) u; then the slice's 64 columns of Wd for all H rows, added into x
 // then HEAD: logits = W_lm . RMSNorm(x), argmax (last CTA reduces), length += 1.
-// GEMV stages run in one of three modes: x in registers (K <= 1536), whole rows per warp with x
-// in shared memory (larger K, many rows), or each row split over three warps (larger K, few
-// rows).  In greedy generation (StepParams::gen_done set) a launch after a stop token returns
-// at once, and the last CTA advances the generation's position and token count.
+//
+// The residual x lives in global memory as 64-bit fixed point (units of 2^-32): the o-proj and
+// down partial products of many CTAs are added with integer atomics, so the sum does not depend
+// on their order (bit-reproducible), and each phase that needs x reads it back after a barrier.
+//
+// int4 GEMV arithmetic (every packed matrix): the activation vector is written once per phase in
+// 16-bit block fixed point, X_k = round(x_k 2^(15 - E_b)) with 2^E_b > max|x| over the 32-block b
+// (|X| <= 32767); dp2a multiplies int16 pairs of X with the unsigned 4-bit codes c (unpacked to
+// bytes), so sum_k (c_k - 8) X_k over a half-block is exact in int32 (the -8 X term is folded
+// into the accumulator's start value); each half-block sum becomes one fp32 value, multiplied by
+// the block's fp16 scale and 2^(E_b - 15), and accumulated in fp32.  The lm_head (fp16 weights)
+// uses exact fp16 x fp16 products with fp32 accumulation (fma.rn.f32.f16).
 //
 // The grid barrier is a monotonic arrival counter in global memory (barrier k completes at
 // (k + 1) x grid arrivals; the last CTA of the launch resets it); every wait is bounded
@@ -45,6 +48,7 @@ namespace {
 
 constexpr int NW = 15;                 // compute warps (+1 producer: 512 threads, 4-warp register granules)
 constexpr int kThreads = (NW + 1) * 32;
+constexpr int NT = NW * 32;            // compute threads
 constexpr int D = 128;
 constexpr int TT = 64;                 // attention tile (positions)
 constexpr int kRowH = D + 8;           // halves per K/V row in a stage: 272 bytes, so consecutive
@@ -52,14 +56,13 @@ constexpr int kRowH = D + 8;           // halves per K/V row in a stage: 272 byt
 constexpr int kMaxG = 8;
 constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kRegHB = 3;              // half-blocks per lane held in registers (K <= 1536)
-constexpr int kMergeInO = 32;          // up to this many tiles per head, every CTA merges the
-                                       // attention partials while staging the o-projection input
-
-enum Phase { PH_QKV = 0, PH_ATTN, PH_O, PH_GU, PH_DOWN, PH_HEAD };
+constexpr int kMaxK = 16384;           // largest GEMV input length (hidden, n_q * D)
+constexpr int kHeadRegHB = 3;          // lm_head: x chunks per lane held in registers (H <= 1536)
+constexpr float kFix = 4294967296.f;   // residual fixed point: 2^32 units per 1.0
+constexpr float kUnfix = 2.3283064365386963e-10f;  // 2^-32
 
 __device__ __forceinline__ void cbar() {  // compute warps only
-  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
 __device__ __forceinline__ void cta_range(int n, int cta, int ncta, int& r0, int& r1) {
@@ -67,21 +70,38 @@ __device__ __forceinline__ void cta_range(int n, int cta, int ncta, int& r0, int
   r1 = (int)((int64_t)n * (cta + 1) / ncta);
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void st_release_u32(unsigned* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Timeline tap: thread 0 of each CTA records %globaltimer at fixed points of the schedule
-// (barrier arrival, barrier exit, x staged, end) when p.stamps is set.
+// Residual fixed point: value -> 2^-32 units (two's complement in the 64-bit word) and back.
+__device__ __forceinline__ unsigned long long to_fix(float v) {
+  return (unsigned long long)__float2ll_rn(v * kFix);
+}
+__device__ __forceinline__ float from_fix(unsigned long long v) {
+  return __ll2float_rn((long long)v) * kUnfix;
+}
+
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Timeline tap: thread 0 of each CTA records %globaltimer at fixed points of the schedule when
+// p.stamps is set.
 __device__ __forceinline__ void stamp(const StepParams& p, int& k) {
   if (p.stamps && threadIdx.x == 0) {
-    if (k < p.max_stamps) p.stamps[(size_t)blockIdx.x * p.max_stamps + k] = globaltimer_ns();
+    if (k < p.max_stamps - 8) p.stamps[(size_t)blockIdx.x * p.max_stamps + k] = globaltimer_ns();
     ++k;
   }
 }
@@ -89,55 +109,20 @@ __device__ __forceinline__ void stamp(const StepParams& p, int& k) {
 // Grid-wide barrier among the compute warps of all CTAs.  The arrival counter only grows during
 // a launch (barrier k completes when it reaches (k + 1) * gridDim.x) and the last CTA of the
 // lm_head phase resets it, so an arrival is one fire-and-forget release-add and the wait one
-// acquire poll.  Bounded wait.
-__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
+// acquire poll.  Bounded wait.  Stamps: arrival, exit.
 __device__ void grid_barrier(const StepParams& p, unsigned& nbar, int& sk) {
   cbar();
   stamp(p, sk);
   if (threadIdx.x == 0) {
-    const unsigned target = (nbar + 1) * gridDim.x;
     red_release_add(p.bar_count, 1u);
-    if (ld_acquire_u32(p.bar_count) < target) {
-      const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_u32(p.bar_count) < target) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          set_device_error(VV_ERR_TIMEOUT);
-          break;
-        }
-      }
-    }
+    wait_counter_geq(p.bar_count, (nbar + 1) * gridDim.x);
   }
   ++nbar;
   stamp(p, sk);
   cbar();
 }
 
-// --------------------------------------------------------------------------------- schedule
-// Rows per stage of a packed matrix with K columns (codes + scales per row), nseg matrices per
-// stage (gate/up share a stage).
-__device__ __forceinline__ int packed_row_bytes(int K) { return (K >> 5) * 18; }
-__device__ __forceinline__ int rows_per_stage(int row_bytes, int nseg, int stage_bytes) {
-  int r = stage_bytes / (row_bytes * nseg);
-  return r > 64 ? 64 : r;
-}
-
-// Rows per stage of a phase: bounded by the stage size, and for the split-K (large K, few rows)
-// path by kSplitRows so that kSplitRows x kSplitW = NW warps share a stage.  `rows` is the
-// CTA's row count for the phase: with x in shared memory and at least 2 NW units, warps take
-// whole rows instead (row mode) and stages are filled.  Producer and consumers compute the same.
-constexpr int kSplitW = 3;                // warps per row when K is large
-constexpr int kSplitRows = NW / kSplitW;  // 5 rows per stage
-__device__ __forceinline__ bool row_mode(int K, int nseg, int rows) {
-  return K > 32 * kRegHB * 16 && rows * nseg >= 2 * NW;
-}
-__device__ __forceinline__ int phase_rps(int K, int nseg, int stage_bytes, int rows) {
-  const int r = rows_per_stage((K >> 5) * 18, nseg, stage_bytes);
-  return (K > 32 * kRegHB * 16 && !row_mode(K, nseg, rows)) ? min(r, kSplitRows) : r;
-}
-
+// ------------------------------------------------------------------------------ stage ring
 struct Ring {
   uint64_t wait_ns;  // time this thread spent blocked in ring waits (timeline tap)
   unsigned char* base;
@@ -145,20 +130,17 @@ struct Ring {
   uint64_t* empty;
   int stage_bytes;
   int nstages;
-  int idx;  // running stage counter
+  int idx;         // running stage counter
   int ph;          // phase kind of the stages being consumed (timeline tap)
   uint64_t* tapw;  // timeline tap: per-phase-kind ring wait of compute thread 0 (else null)
-  __device__ unsigned char* slot_ptr(int i) const { return base + (size_t)(i % nstages) * stage_bytes; }
 };
 
-// Producer side of one stage: wait for the slot, post the byte count, issue the copies.
 struct Copy {
   const void* src;
   uint32_t bytes;
   uint32_t dst_off;
 };
 
-// Ring wait with wait-time accounting.
 __device__ __forceinline__ void ring_wait(Ring& r, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
@@ -197,6 +179,27 @@ __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t 
     if (c[i].bytes) bulk_g2s_stream(dst + c[i].dst_off, c[i].src, c[i].bytes, &r.full[slot], pol);
 }
 
+// Consumer side: wait for the next stage, return its base.
+__device__ __forceinline__ const unsigned char* consume_begin(Ring& r, int& slot) {
+  const int s = r.idx++;
+  slot = s % r.nstages;
+  ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
+  return r.base + (size_t)slot * r.stage_bytes;
+}
+__device__ __forceinline__ void consume_end(Ring& r, int slot) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&r.empty[slot]);
+}
+
+// --------------------------------------------------------------------------- stage geometry
+// Row phases (QKV, gate/up): stage = [seg0 codes rps rows][seg1 codes][seg0 scales][seg1 scales],
+// rows of K/32 x 16 code bytes and K/32 x 2 scale bytes.  Column phases (o-proj, down): stage =
+// [codes rps rows x nb x 16][scales rps rows x nb x 2] of a column image.
+__device__ __forceinline__ int rows_per_stage(int row_bytes, int stage_bytes) {
+  int r = stage_bytes / row_bytes;
+  return r & ~7;  // a multiple of 8 rows keeps every scale run 16-byte aligned
+}
+
 // One attention tile: `rows` past K rows and V rows (256 bytes each) into the padded row layout
 // (kRowH halves per row; V after TT K rows).
 __device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int rows, uint64_t pol) {
@@ -211,17 +214,16 @@ __device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int r
   }
 }
 
-// Stream rows [r0, r1) of a packed matrix (and optionally the same rows of a second one).
-__device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, const uint8_t* q1,
-                               const __half* s1, int K, int r0, int r1, uint64_t pol) {
+// Rows [r0, r1) of a packed matrix, and the same rows of a second one (gate/up).
+__device__ void produce_rows(Ring& r, const uint8_t* q0, const __half* s0, const uint8_t* q1,
+                             const __half* s1, int K, int r0, int r1, uint64_t pol) {
   const int nseg = q1 ? 2 : 1;
   const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
-  const int rps = phase_rps(K, nseg, r.stage_bytes, r1 - r0);
+  const int rps = rows_per_stage((rq + rs) * nseg, r.stage_bytes);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     Copy c[4];
     int k = 0;
-    // layout: [seg0 codes (rps rows)][seg1 codes][seg0 scales][seg1 scales]
     c[k++] = Copy{q0 + (size_t)a * rq, (uint32_t)(n * rq), 0u};
     if (q1) c[k++] = Copy{q1 + (size_t)a * rq, (uint32_t)(n * rq), (uint32_t)(rps * rq)};
     c[k++] = Copy{reinterpret_cast<const unsigned char*>(s0) + (size_t)a * rs, (uint32_t)(n * rs),
@@ -233,12 +235,12 @@ __device__ void produce_packed(Ring& r, const uint8_t* q0, const __half* s0, con
   }
 }
 
-// Stream logical rows [r0, r1) of [Wq; Wk; Wv] (bounds: first row of each matrix); a stage may
-// hold rows of two matrices, laid out as one matrix of consecutive rows.
+// Logical rows [r0, r1) of [Wq; Wk; Wv] (bounds: first row of each matrix); a stage may hold
+// rows of two matrices, laid out as one matrix of consecutive rows.
 __device__ void produce_qkv(Ring& r, const StepLayer& w, int K, int r0, int r1,
                             const int (&bounds)[4], uint64_t pol) {
   const int rq = (K >> 5) * 16, rs = (K >> 5) * 2;
-  const int rps = phase_rps(K, 1, r.stage_bytes, r1 - r0);
+  const int rps = rows_per_stage(rq + rs, r.stage_bytes);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     Copy c[6];
@@ -255,35 +257,57 @@ __device__ void produce_qkv(Ring& r, const StepLayer& w, int K, int r0, int r1,
   }
 }
 
-// Tiles (kv head g, tile t) owned by this CTA: items i = cta + k * ncta < Hkv * ntiles.
+// A column image of `rows` rows x nb blocks: [codes rows x nb x 16][scales rows x nb x 2].
+__device__ void produce_cols(Ring& r, const unsigned char* img, int rows, int nb, uint64_t pol) {
+  const int rps = rows_per_stage(nb * 18, r.stage_bytes);
+  const unsigned char* sc = img + (size_t)rows * nb * 16;
+  for (int a = 0; a < rows; a += rps) {
+    const int n = min(rps, rows - a);
+    Copy c[2] = {Copy{img + (size_t)a * nb * 16, (uint32_t)(n * nb * 16), 0u},
+                 Copy{sc + (size_t)a * nb * 2, (uint32_t)(n * nb * 2), (uint32_t)(rps * nb * 16)}};
+    produce(r, c, 2, pol);
+  }
+}
+
 __device__ __forceinline__ int ntiles_for(int past) { return (past + 1 + TT - 1) / TT; }
+__device__ __forceinline__ int n_slices(const StepParams& p) { return p.I / kSlice; }
+__device__ __forceinline__ int slices_of(const StepParams& p, int cta) {
+  const int ns = n_slices(p);
+  return ns > cta ? (ns - 1 - cta) / (int)gridDim.x + 1 : 0;
+}
+__device__ __forceinline__ size_t wd_cta_stride(const StepParams& p) {
+  const int nsl_max = (n_slices(p) + gridDim.x - 1) / gridDim.x;
+  return (size_t)p.H * nsl_max * 2 * 18;
+}
 
 __device__ void producer(const StepParams& p, Ring& r, int past) {
   const uint64_t pol = policy_evict_first();
   const int cta = blockIdx.x, ncta = gridDim.x;
-  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv, I = p.I;
+  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv;
   const int nqkv = (Hq + 2 * Hkv) * D;
   const int nt = ntiles_for(past);
+  const int nrb = H / kORows;
+  const int nsl = slices_of(p, cta);
+  const int ns = n_slices(p);
+  int o0, o1;
+  cta_range(Hq * nrb, cta, ncta, o0, o1);
   for (int l = 0; l < p.L; ++l) {
     const StepLayer& w = p.layers[l];
-    // QKV: logical rows [0, nqkv) over the three matrices
     int r0, r1;
     cta_range(nqkv, cta, ncta, r0, r1);
     const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
     produce_qkv(r, w, H, r0, r1, bounds, pol);
-    // ATTN: past K/V rows of the tiles
     for (int it = cta; it < Hkv * nt; it += ncta) {
       const int g = it / nt, t = it % nt;
       const int p0 = t * TT, p1 = min(p0 + TT, past);
       const size_t off = ((size_t)(l * Hkv + g) * p.cap + p0) * D;
       produce_kv_rows(r, p.k_cache + off, p.v_cache + off, max(p1 - p0, 0), pol);
     }
-    cta_range(H, cta, ncta, r0, r1);
-    produce_packed(r, w.q[3], w.s[3], nullptr, nullptr, Hq * D, r0, r1, pol);
-    cta_range(I, cta, ncta, r0, r1);
-    produce_packed(r, w.q[4], w.s[4], w.q[5], w.s[5], H, r0, r1, pol);
-    cta_range(H, cta, ncta, r0, r1);
-    produce_packed(r, w.q[6], w.s[6], nullptr, nullptr, I, r0, r1, pol);
+    for (int i = o0; i < o1; ++i)
+      produce_cols(r, w.wo_img + (size_t)i * kORows * 4 * 18, kORows, 4, pol);
+    for (int s = cta; s < ns; s += ncta)
+      produce_rows(r, w.q[4], w.s[4], w.q[5], w.s[5], H, s * kSlice, (s + 1) * kSlice, pol);
+    if (nsl > 0) produce_cols(r, w.wd_img + (size_t)cta * wd_cta_stride(p), H, 2 * nsl, pol);
   }
   // HEAD: fp16 rows of the lm_head
   int r0, r1;
@@ -297,374 +321,234 @@ __device__ void producer(const StepParams& p, Ring& r, int past) {
   }
 }
 
-// ------------------------------------------------------------------------ compute helpers
-// x staging.  Source fp32 (or fp16 embedding row), optional RMSNorm with fp16 gamma; the result
-// is rounded once to fp16 (the GEMV's activation type) and stored in the half2-pair layout of the
-// dequant-dot: element k (hb = k/16, word = (k/8)%2, j = k%8) goes to uint4 (word * NHB + hb),
-// component j%4, half j/4, i.e. the pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7) of each word.  A warp
-// reading half-blocks hb = lane + 32i touches consecutive 16-byte chunks (no bank conflicts).
-// All compute threads; ends with a compute barrier.
-__device__ __forceinline__ int xh_slot(int k, int nhb) {
-  const int hb = k >> 4, word = (k >> 3) & 1, j = k & 7;
-  return ((word * nhb + hb) * 4 + (j & 3)) * 2 + (j >> 2);
+// ------------------------------------------------------------------ GEMV operand (X) staging
+// The activation operand of the int4 GEMVs, in shared memory:
+//   xq   uint4 [2][NHB]: half-block hb, code word w (elements 8w..8w+7 of the half-block) ->
+//        int16 pairs (X0,X2) (X4,X6) (X1,X3) (X5,X7) in the dp2a order of the unpacked codes
+//        (low nibbles = even elements, high nibbles = odd elements);
+//   corr int [NHB]: -8 * sum of X over the half-block;
+//   fb   float [NHB/2]: 2^(E_b - 15) per 32-block.
+struct XOp {
+  uint4* xq;
+  int* corr;
+  float* fb;
+};
+
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
+// Write X of the 4 consecutive elements k..k+3 (k % 4 == 0) held by this thread.  Every thread
+// of the compute group calls this for chunk slots in lockstep (the 32-block of k is spread over
+// 8 consecutive threads, the half-block over 4); `valid` false for padding slots.
+__device__ __forceinline__ void put_x4(const XOp& xo, int NHB, int k, float4 y, bool valid) {
+  float m = valid ? fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))) : 0.f;
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  // 2^E > m: E = unbiased exponent of m + 1 (denormals and zero -> the smallest normal)
+  int E = max((__float_as_int(m) >> 23) & 0xFF, 1) - 126;
+  E = max(E, -100);
+  const float sc = pow2f(15 - E);
+  auto q = [&](float v) { return min(max(__float2int_rn(v * sc), -32767), 32767); };
+  const int X0 = q(y.x), X1 = q(y.y), X2 = q(y.z), X3 = q(y.w);
+  int sx = valid ? X0 + X1 + X2 + X3 : 0;
+  sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+  sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+  if (!valid) return;
+  const int hb = k >> 4, w = (k >> 3) & 1, j0 = k & 7;  // j0 in {0, 4}
+  uint32_t* dst = reinterpret_cast<uint32_t*>(xo.xq) + (size_t)(w * NHB + hb) * 4;
+  auto pk = [](int a, int b) { return (uint32_t)(uint16_t)(int16_t)a | ((uint32_t)(uint16_t)(int16_t)b << 16); };
+  dst[j0 >> 2] = pk(X0, X2);
+  dst[2 + (j0 >> 2)] = pk(X1, X3);
+  if ((k & 15) == 0) xo.corr[hb] = -8 * sx;
+  if ((k & 31) == 0) xo.fb[k >> 5] = pow2f(E - 15);
 }
 
-__device__ void stage_x(__half* xs, float* red, const float* src32, const __half* src16,
-                        const __half* gamma, float eps, int K, float* copy_out) {
+// Stage a K-vector (K % 32 == 0, K <= 4 * 4 * NT) as the GEMV operand: y = src (* rsqrt(mean
+// src^2 + eps) * gamma when gamma is set).  load(k) returns elements k..k+3 as fp32.  Optional
+// fp32 copy of src (trace).  All compute threads; ends with a compute barrier.
+template <class Load>
+__device__ void stage_idp(const XOp& xo, Load load, const __half* gamma, float eps, int K,
+                          float* red, float* copy_out) {
   const int tid = threadIdx.x;
-  constexpr int NT = NW * 32;
-  constexpr int kReg = 5;  // float4 chunks per thread kept in registers (K <= 4 * 5 * NT = 9600)
-  const int nhb = K >> 4;
-  auto load4 = [&](int k) -> float4 {
-    if (src32) return __ldcg(reinterpret_cast<const float4*>(src32 + k));
-    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(src16 + k));
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-  };
-  auto put = [&](int k, float4 t, float inv) {
-    float y[4] = {t.x, t.y, t.z, t.w};
+  constexpr int kC = 4;  // chunks of 4 per thread
+  const int NHB = K >> 4;
+  float4 v[kC];
+  float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float u = y[e];
-      if (gamma) u = u * inv * __half2float(gamma[k + e]);
-      xs[xh_slot(k + e, nhb)] = __float2half_rn(u);
-    }
-  };
-  auto norm_inv = [&](float ss) {
+  for (int i = 0; i < kC; ++i) {
+    const int k = (tid + i * NT) * 4;
+    v[i] = k < K ? load(k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (k < K && copy_out) *reinterpret_cast<float4*>(copy_out + k) = v[i];
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+  }
+  if (gamma) {
     ss = warp_sum(ss);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
     cbar();
     float tot = 0.f;
 #pragma unroll
     for (int i = 0; i < NW; ++i) tot += red[i];
-    return rsqrtf(tot / (float)K + eps);
-  };
-  if (K > kReg * 4 * NT) {  // large K (7B down projection): two passes over the source
-    float ss = 0.f;
-    for (int k = tid * 4; k < K; k += NT * 4) {
-      const float4 t = load4(k);
-      if (copy_out) *reinterpret_cast<float4*>(copy_out + k) = t;
-      ss += t.x * t.x + t.y * t.y + t.z * t.z + t.w * t.w;
-    }
-    const float inv = gamma ? norm_inv(ss) : 1.f;
-    for (int k = tid * 4; k < K; k += NT * 4) put(k, load4(k), inv);
-    cbar();
-    return;
-  }
-  float4 v[kReg];
-  uint2 gv[kReg];  // gamma halves, loaded with x so their latency overlaps
-  float ss = 0.f;
+    const float inv = rsqrtf(tot / (float)K + eps);
 #pragma unroll
-  for (int i = 0; i < kReg; ++i) {
-    const int k = (tid + i * NT) * 4;
-    if (k < K) {
-      if (gamma) gv[i] = *reinterpret_cast<const uint2*>(gamma + k);
-      v[i] = load4(k);
-      if (copy_out) *reinterpret_cast<float4*>(copy_out + k) = v[i];
-      ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
-    } else {
-      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
-  const float inv = gamma ? norm_inv(ss) : 1.f;
-#pragma unroll
-  for (int i = 0; i < kReg; ++i) {
-    const int k = (tid + i * NT) * 4;
-    if (k < K) {
-      float y[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      if (gamma) {
-        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].x));
-        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].y));
-        y[0] *= inv * g01.x;
-        y[1] *= inv * g01.y;
-        y[2] *= inv * g23.x;
-        y[3] *= inv * g23.y;
+    for (int i = 0; i < kC; ++i) {
+      const int k = (tid + i * NT) * 4;
+      if (k < K) {
+        const uint2 gv = *reinterpret_cast<const uint2*>(gamma + k);
+        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&gv.x));
+        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&gv.y));
+        v[i].x *= inv * g01.x;
+        v[i].y *= inv * g01.y;
+        v[i].z *= inv * g23.x;
+        v[i].w *= inv * g23.y;
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) xs[xh_slot(k + e, nhb)] = __float2half_rn(y[e]);
     }
+  }
+#pragma unroll
+  for (int i = 0; i < kC; ++i) {
+    const int k = (tid + i * NT) * 4;
+    if (i * NT * 4 < K) put_x4(xo, NHB, k, v[i], k < K);  // warp-uniform slot condition
   }
   cbar();
 }
 
-// Dot of one half-block (8 bytes of codes = 16 columns) with its two x words (half2 pairs).
-__device__ __forceinline__ float hb_doth(uint2 wv, uint4 xa, uint4 xb) {
-  return dot8_h(wv.x, xa) + dot8_h(wv.y, xb);
+// ----------------------------------------------------------------------------- int4 GEMV
+// One half-block (16 weights: two code words) against its X pairs: exact int32 sum of
+// (c - 8) X, starting from corr = -8 sum X.
+__device__ __forceinline__ int hb_dot(uint2 wv, uint4 xa, uint4 xb, int corr) {
+  const uint32_t l0 = wv.x & 0x0F0F0F0Fu, h0 = (wv.x >> 4) & 0x0F0F0F0Fu;
+  const uint32_t l1 = wv.y & 0x0F0F0F0Fu, h1 = (wv.y >> 4) & 0x0F0F0F0Fu;
+  int s = corr;
+  s = dp2a_lo(xa.x, l0, s);
+  s = dp2a_hi(xa.y, l0, s);
+  s = dp2a_lo(xa.z, h0, s);
+  s = dp2a_hi(xa.w, h0, s);
+  s = dp2a_lo(xb.x, l1, s);
+  s = dp2a_hi(xb.y, l1, s);
+  s = dp2a_lo(xb.z, h1, s);
+  s = dp2a_hi(xb.w, h1, s);
+  return s;
 }
 
-// One stage with x in shared memory and whole rows per warp (large K, rows plentiful): warp w
-// takes units [w R, w R + R), lanes stride the half-blocks, one shuffle reduction per unit; no
-// cross-warp reduction, so no barrier inside the stage.
-template <int R, class RowQ, class RowS, class Fin>
-__device__ __forceinline__ void smemx_pass(RowQ rowq, RowS rows, const uint4* xs4, int K, int units,
-                                           int nseg, int a, Fin fin) {
+// Rows of one stage against the staged X.  Units are (row, segment) pairs, u -> (u / nseg,
+// u % nseg); LPR lanes share a unit (lane % LPR strides the half-blocks), a warp takes 32/LPR x R
+// units per pass.  rowq(u) / rows(u): code and scale bytes of unit u's row.  fin(u, y) is called
+// once per unit by the group's first lane; with PAIR (nseg == 2, R even) fin2(row, y0, y1) once
+// per row instead.
+template <int LPR, int R, bool PAIR, class RowQ, class RowS, class Fin>
+__device__ __forceinline__ void idp_pass(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows,
+                                         Fin fin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NHB = K >> 4;
-  for (int u0 = warp * R; u0 < units; u0 += NW * R) {
-    const unsigned char* wq[R];
-    const __half* ws[R];
-    int lr[R];
-    bool ok[R];
+  constexpr int GPW = 32 / LPR;  // unit groups per warp
+  const int sub = lane % LPR, grp = lane / LPR;
+  const uint4* xq = xo.xq;
+  for (int u0 = (warp * GPW + grp) * R; u0 < units; u0 += NW * GPW * R) {
+    const unsigned char* q[R];
+    const __half* sc[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      const int u = u0 + k;
-      ok[k] = u < units;
-      const int uu = ok[k] ? u : u0;
-      const int sg = nseg == 2 ? (uu & 1) : 0;
-      lr[k] = nseg == 2 ? (uu >> 1) : uu;
-      wq[k] = rowq(sg, lr[k]);
-      ws[k] = rows(sg, lr[k]);
+      const int u = min(u0 + k, units - 1);
+      q[k] = rowq(u);
+      sc[k] = rows(u);
     }
     float acc[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) acc[k] = 0.f;
-#pragma unroll 2
-    for (int hb = lane; hb < NHB; hb += 32) {
-      const uint4 xa = xs4[hb], xb = xs4[NHB + hb];
+    for (int hb = sub; hb < NHB; hb += LPR) {
+      const uint4 xa = xq[hb], xb = xq[NHB + hb];
+      const int cr = xo.corr[hb];
+      const float f = xo.fb[hb >> 1];
 #pragma unroll
       for (int k = 0; k < R; ++k) {
-        const uint2 wv = *reinterpret_cast<const uint2*>(wq[k] + hb * 8);
-        acc[k] = fmaf(__half2float(ws[k][hb >> 1]), hb_doth(wv, xa, xb), acc[k]);
+        const uint2 wv = *reinterpret_cast<const uint2*>(q[k] + hb * 8);
+        const float s = __half2float(sc[k][hb >> 1]) * f;
+        acc[k] = fmaf(s, (float)hb_dot(wv, xa, xb, cr), acc[k]);
       }
     }
-#pragma unroll
-    for (int k = 0; k < R; ++k) acc[k] = warp_sum(acc[k]);
-    if (lane == 0) {
-      if (nseg == 2) {
-#pragma unroll
-        for (int k = 0; k + 1 < R; k += 2)
-          if (ok[k]) fin(a + lr[k], acc[k], acc[k + 1]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < R; ++k)
-          if (ok[k]) fin(a + lr[k], acc[k], 0.f);
-      }
-    }
-  }
-}
-
-// One stage of the register-x path: warp w takes units [w R, w R + R), then [w R + NW R, ...);
-// unit u is (segment, row) = (u & 1, u >> 1) for gate/up pairs, else (0, u).  Lanes stride the
-// half-blocks; one shuffle reduction per unit; lane 0 finishes the rows.
-template <int R, class RowQ, class RowS, class Fin>
-__device__ __forceinline__ void regx_pass(RowQ rowq, RowS rows, const uint4 (&xr)[kRegHB][2], int K,
-                                          int units, int nseg, int a, Fin fin) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NHB = K >> 4;
-  for (int u0 = warp * R; u0 < units; u0 += NW * R) {
-    int sg[R], lr[R];
-    bool ok[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      const int u = u0 + k;
-      ok[k] = u < units;
-      const int uu = ok[k] ? u : u0;
-      sg[k] = nseg == 2 ? (uu & 1) : 0;
-      lr[k] = nseg == 2 ? (uu >> 1) : uu;
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
     }
-    float acc[R];
-#pragma unroll
-    for (int k = 0; k < R; ++k) acc[k] = 0.f;
-#pragma unroll
-    for (int j = 0; j < kRegHB; ++j) {
-      const int hb = lane + 32 * j;
-      if (hb < NHB) {
-#pragma unroll
-        for (int k = 0; k < R; ++k) {
-          const uint2 wv = *reinterpret_cast<const uint2*>(rowq(sg[k], lr[k]) + hb * 8);
-          const float sc = __half2float(rows(sg[k], lr[k])[hb >> 1]);
-          acc[k] = fmaf(sc, hb_doth(wv, xr[j][0], xr[j][1]), acc[k]);
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < R; ++k) acc[k] = warp_sum(acc[k]);
-    if (lane == 0) {
-      if (nseg == 2) {
+    if (sub == 0) {
+      if (PAIR) {
 #pragma unroll
         for (int k = 0; k + 1 < R; k += 2)
-          if (ok[k]) fin(a + lr[k], acc[k], acc[k + 1]);
+          if (u0 + k < units) fin(u0 + k, acc[k], acc[k + 1]);
       } else {
 #pragma unroll
         for (int k = 0; k < R; ++k)
-          if (ok[k]) fin(a + lr[k], acc[k], 0.f);
+          if (u0 + k < units) fin(u0 + k, acc[k], 0.f);
       }
     }
   }
 }
 
-// Consume the stages of a packed-matrix phase.  fin(row, y0, y1) is called once per output row
-// (y1: the up value of a gate/up pair, nseg = 2).
-//  * K <= 1536 (x in registers xr): each warp takes 4 rows per pass (or 2 gate/up pairs) for
-//    instruction-level parallelism; lanes stride the half-blocks; shuffle reduction.
-//  * larger K (x in shared memory, interleaved): each row is split over kSplitW warps, partial
-//    sums meet in shared memory (red2) and the first warp of the row finishes it.
-template <class Fin>
-__device__ __forceinline__ void consume_packed(Ring& r, const __half* xs, const uint4 (&xr)[kRegHB][2],
-                                               bool regx, int K, int r0, int r1, int nseg,
-                                               float* red2, Fin fin) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+template <int LPR, int R, bool PAIR, class RowQ, class RowS, class Fin>
+__device__ __forceinline__ void idp_dispatch(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows, Fin fin) {
+  idp_pass<LPR, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+}
+
+// Pick lanes per unit from the half-block count: 32 (long rows) down to 4 (short rows).
+template <int R, bool PAIR, class RowQ, class RowS, class Fin>
+__device__ __forceinline__ void idp_any(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows, Fin fin) {
+  if (NHB >= 32) idp_pass<32, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+  else if (NHB >= 16) idp_pass<16, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+  else if (NHB >= 8) idp_pass<8, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+  else idp_pass<4, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+}
+
+// Row phase: consume the stages of rows [r0, r1) (nseg matrices per stage).  fin(row, y0, y1).
+template <bool PAIR, class Fin>
+__device__ void consume_rows(Ring& r, const XOp& xo, int K, int r0, int r1, int nseg, Fin fin) {
   const int KB = K >> 5, NHB = K >> 4;
   const int rq = KB * 16, rs = KB * 2;
-  const int rps = phase_rps(K, nseg, r.stage_bytes, r1 - r0);
-  const bool rowmode = row_mode(K, nseg, r1 - r0);
-  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+  const int rps = rows_per_stage((rq + rs) * nseg, r.stage_bytes);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
-    const int s = r.idx++;
-    const int slot = s % r.nstages;
-    ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
-    const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
+    int slot;
+    const unsigned char* st = consume_begin(r, slot);
     const unsigned char* scb = st + (size_t)nseg * rps * rq;
-    auto rowq = [&](int sg, int lr) { return st + (size_t)(sg * rps + lr) * rq; };
-    auto rows = [&](int sg, int lr) {
-      return reinterpret_cast<const __half*>(scb + (size_t)(sg * rps + lr) * rs);
+    auto rowq = [&](int u) { return st + (size_t)((u % nseg) * rps + u / nseg) * rq; };
+    auto rows = [&](int u) {
+      return reinterpret_cast<const __half*>(scb + (size_t)((u % nseg) * rps + u / nseg) * rs);
     };
-    if (regx) {
-      // R row slots per warp pass: as many as keep every warp busy (R = 1 for the small
-      // phases, up to 4 for instruction-level parallelism when rows are plentiful); gate/up
-      // pairs stay inside one warp (R >= 2).
-      const int units = n * nseg;
-      if (nseg == 1 && units <= NW)
-        regx_pass<1>(rowq, rows, xr, K, units, nseg, a, fin);
-      else if (units <= 2 * NW)
-        regx_pass<2>(rowq, rows, xr, K, units, nseg, a, fin);
-      else
-        regx_pass<4>(rowq, rows, xr, K, units, nseg, a, fin);
-    } else if (rowmode) {
-      smemx_pass<2>(rowq, rows, xs4, K, n * nseg, nseg, a, fin);
-    } else {
-      // split-K: warp w -> row w / kSplitW, slice w % kSplitW
-      const int lrow = warp / kSplitW, slice = warp % kSplitW;
-      float acc0 = 0.f, acc1 = 0.f;
-      if (lrow < n) {
-        const unsigned char* q0 = rowq(0, lrow);
-        const __half* sc0 = rows(0, lrow);
-        const unsigned char* q1 = rowq(nseg - 1, lrow);
-        const __half* sc1 = rows(nseg - 1, lrow);
-        for (int hb = lane + 32 * slice; hb < NHB; hb += 32 * kSplitW) {
-          const uint4 xa = xs4[hb], xb = xs4[NHB + hb];
-          const uint2 w0 = *reinterpret_cast<const uint2*>(q0 + hb * 8);
-          acc0 = fmaf(__half2float(sc0[hb >> 1]), hb_doth(w0, xa, xb), acc0);
-          if (nseg == 2) {
-            const uint2 w1 = *reinterpret_cast<const uint2*>(q1 + hb * 8);
-            acc1 = fmaf(__half2float(sc1[hb >> 1]), hb_doth(w1, xa, xb), acc1);
-          }
-        }
-      }
-      acc0 = warp_sum(acc0);
-      acc1 = warp_sum(acc1);
-      if (lane == 0) {
-        red2[warp * 2 + 0] = acc0;
-        red2[warp * 2 + 1] = acc1;
-      }
-      cbar();
-      if (lane == 0 && slice == 0 && lrow < n) {
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < kSplitW; ++k) {
-          y0 += red2[(warp + k) * 2 + 0];
-          y1 += red2[(warp + k) * 2 + 1];
-        }
-        fin(a + lrow, y0, y1);
-      }
-      cbar();
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&r.empty[slot]);
+    auto f = [&](int u, float y0, float y1) { fin(a + u / nseg, y0, y1); };
+    if (PAIR) idp_any<2, true>(xo, NHB, n * nseg, rowq, rows, f);
+    else if (n >= 4 * NW) idp_any<4, false>(xo, NHB, n, rowq, rows, f);
+    else idp_any<1, false>(xo, NHB, n, rowq, rows, f);
+    consume_end(r, slot);
   }
 }
 
-// Preload the lane's half-blocks of x (fp16 pair layout in xs) into registers.
-__device__ __forceinline__ void load_xr(const __half* xs, uint4 (&xr)[kRegHB][2], int K) {
-  const int lane = threadIdx.x & 31;
-  const int NHB = K >> 4;
-  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
-#pragma unroll
-  for (int j = 0; j < kRegHB; ++j) {
-    const int hb = lane + 32 * j;
-    xr[j][0] = hb < NHB ? xs4[hb] : make_uint4(0u, 0u, 0u, 0u);
-    xr[j][1] = hb < NHB ? xs4[NHB + hb] : make_uint4(0u, 0u, 0u, 0u);
+// Column phase: consume the stages of a column image of `rows` rows x nb blocks (K = 32 nb).
+template <class Fin>
+__device__ void consume_cols(Ring& r, const XOp& xo, int rows_total, int nb, Fin fin) {
+  const int NHB = nb * 2;
+  const int rps = rows_per_stage(nb * 18, r.stage_bytes);
+  for (int a = 0; a < rows_total; a += rps) {
+    const int n = min(rps, rows_total - a);
+    int slot;
+    const unsigned char* st = consume_begin(r, slot);
+    const unsigned char* scb = st + (size_t)rps * nb * 16;
+    auto rowq = [&](int u) { return st + (size_t)u * nb * 16; };
+    auto rows = [&](int u) { return reinterpret_cast<const __half*>(scb + (size_t)u * nb * 2); };
+    auto f = [&](int u, float y0, float) { fin(a + u, y0); };
+    idp_any<2, false>(xo, NHB, n, rowq, rows, f);
+    consume_end(r, slot);
   }
 }
 
+// ------------------------------------------------------------------------------- attention
 struct AttnScratch {
   float cs[D / 2], sn[D / 2];  // RoPE cos/sin at this step's position
   float q[kMaxG][D];
   float s[kMaxG][TT];
   float m[kMaxG], l[kMaxG];
-  float mw[256][kMaxG];
   float pv[4][kMaxG][D];  // P.V partial sums per position quarter
-  int is_last;
 };
 
-__device__ __forceinline__ bool merge_in_o(const StepParams& p, int nt) {
-  return nt <= kMergeInO && p.Hkv * nt * (p.Hq / p.Hkv) <= 256 * kMaxG;
-}
-
-// Stage the o-projection input straight from the attention partials (merge_in_o case): per head
-// M = max_t m_t, L = sum_t l_t 2^(m_t - M), o[h][d] = sum_t 2^(m_t - M) o_t[h][d] / L; rounded to
-// fp16 into the GEMV layout.  Each thread merges its 4 dims online over batches of 6 tiles, the
-// batch's m, l and o loads all in flight together.  Ends with a compute barrier.
-__device__ void stage_attn_merged(const StepParams& p, __half* xs, int nt) {
-  const int tid = threadIdx.x;
-  const int G = p.Hq / p.Hkv, K = p.Hq * D, nhb = K >> 4;
-  constexpr int kB = 6;
-  for (int k4 = tid; k4 < K / 4; k4 += NW * 32) {
-    const int k = k4 * 4;
-    const int hh = k >> 7, d = k & (D - 1);
-    const int g = hh / G, h = hh % G;
-    const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + h) * kPart;
-    float M = -INFINITY, L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int t0 = 0; t0 < nt; t0 += kB) {
-      float4 v[kB];
-      float mt[kB], lt[kB];
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        if (t0 + u < nt) {
-          const float* pt = base + (size_t)(t0 + u) * kMaxG * kPart;
-          mt[u] = __ldcg(pt);
-          lt[u] = __ldcg(pt + 1);
-          v[u] = __ldcg(reinterpret_cast<const float4*>(pt + 4 + d));
-        } else {
-          mt[u] = -INFINITY;
-          lt[u] = 0.f;
-          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      float bm = M;
-#pragma unroll
-      for (int u = 0; u < kB; ++u) bm = fmaxf(bm, mt[u]);
-      const float c = exp2f(M - bm);  // 0 on the first batch (M = -inf)
-      L *= c;
-      acc.x *= c;
-      acc.y *= c;
-      acc.z *= c;
-      acc.w *= c;
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const float e = exp2f(mt[u] - bm);
-        L = fmaf(lt[u], e, L);
-        acc.x = fmaf(e, v[u].x, acc.x);
-        acc.y = fmaf(e, v[u].y, acc.y);
-        acc.z = fmaf(e, v[u].z, acc.z);
-        acc.w = fmaf(e, v[u].w, acc.w);
-      }
-      M = bm;
-    }
-    const float inv = 1.f / L;
-    xs[xh_slot(k + 0, nhb)] = __float2half_rn(acc.x * inv);
-    xs[xh_slot(k + 1, nhb)] = __float2half_rn(acc.y * inv);
-    xs[xh_slot(k + 2, nhb)] = __float2half_rn(acc.z * inv);
-    xs[xh_slot(k + 3, nhb)] = __float2half_rn(acc.w * inv);
-  }
-  cbar();
-}
-
 __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
-                          int past, int pos) {
+                          int past) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.Hq / p.Hkv;
   const int nt = ntiles_for(past);
@@ -676,11 +560,11 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   // position, the new k/v: every global load is issued before any is used (one L2 round trip).
   const float qscale = p.scale * kLog2e;
   const bool newpos = t == nt - 1;
-  constexpr int kQPer = (kMaxG * D + NW * 32 - 1) / (NW * 32);  // q element pairs per thread
+  constexpr int kQPer = (kMaxG * D + NT - 1) / NT;  // q element pairs per thread
   float qa[kQPer], qb[kQPer];
 #pragma unroll
   for (int j = 0; j < kQPer; ++j) {
-    const int i = tid + j * NW * 32;
+    const int i = tid + j * NT;
     qa[j] = qb[j] = 0.f;
     if (i < G * D) {
       const int h = i / D, d = i % D;
@@ -700,7 +584,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   }
 #pragma unroll
   for (int j = 0; j < kQPer; ++j) {
-    const int i = tid + j * NW * 32;
+    const int i = tid + j * NT;
     if (i < G * D) {
       const int h = i / D, d = i % D;
       const int fi = d & (D / 2 - 1);
@@ -708,10 +592,8 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
       as.q[h][d] = (d < D / 2 ? qa[j] * cs - qb[j] * sn : qb[j] * cs + qa[j] * sn) * qscale;
     }
   }
-  const int s = r.idx++;
-  const int slot = s % r.nstages;
-  ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
-  __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
+  int slot;
+  __half* kt = reinterpret_cast<__half*>(const_cast<unsigned char*>(consume_begin(r, slot)));
   __half* vt = kt + TT * kRowH;
   if (newpos && tid < D) {  // this tile holds the new position: rotate k, append k/v
     const int d = tid, fi = d & (D / 2 - 1);
@@ -729,26 +611,23 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   // order, so the q reads are broadcasts; the padded K rows keep the k reads conflict-free.
   for (int item = warp; item < 2 * G; item += NW) {
     const int h = item >> 1, pp = (item & 1) * 32 + lane;
-    {
-      float sc = -INFINITY;
-      if (pp < n) {
-        const __half* kr = kt + pp * kRowH;
-        float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
+    float sc = -INFINITY;
+    if (pp < n) {
+      const __half* kr = kt + pp * kRowH;
+      float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-          const int cc = c;
-          const uint4 kv = *reinterpret_cast<const uint4*>(kr + cc * 8);
-          const float4 qa = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
-          const float4 qb = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
-          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa.x, qa.y), acc);
-          acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa.z, qa.w), acc2);
-          acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb.x, qb.y), acc);
-          acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb.z, qb.w), acc2);
-        }
-        sc = (acc.x + acc.y) + (acc2.x + acc2.y);
+      for (int c = 0; c < 16; ++c) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(kr + c * 8);
+        const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][c * 8]);
+        const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][c * 8 + 4]);
+        acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa4.x, qa4.y), acc);
+        acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa4.z, qa4.w), acc2);
+        acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb4.x, qb4.y), acc);
+        acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb4.z, qb4.w), acc2);
       }
-      as.s[h][pp] = sc;
+      sc = (acc.x + acc.y) + (acc2.x + acc2.y);
     }
+    as.s[h][pp] = sc;
   }
   cbar();
   if (warp < G) {  // softmax statistics of this tile, per head
@@ -771,7 +650,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
   // memory (as.pv), then written as the tile's partial.
   {
     const int units = G * 16 * 4;
-    for (int u = tid; u < units; u += NW * 32) {
+    for (int u = tid; u < units; u += NT) {
       const int o = u & 15, q = (u >> 4) & 3, h = u >> 6;
       float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
       const float* ph = as.s[h];
@@ -791,7 +670,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     }
     cbar();
     float* part = p.attn_part + ((size_t)(g * p.max_tiles + t) * kMaxG) * kPart;
-    for (int idx = tid; idx < G * D; idx += NW * 32) {
+    for (int idx = tid; idx < G * D; idx += NT) {
       const int h = idx >> 7, d = idx & (D - 1);
       part[h * kPart + 4 + d] = (as.pv[0][h][d] + as.pv[1][h][d]) + (as.pv[2][h][d] + as.pv[3][h][d]);
     }
@@ -800,97 +679,68 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
       part[tid * kPart + 1] = as.l[tid];
     }
   }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&r.empty[slot]);
-  // Short caches: the partials are merged by every CTA when it stages the o-projection input
-  // (after the grid barrier, which orders these stores).  Long caches: the last tile of head g to
-  // finish merges g's partials here.
-  if (merge_in_o(p, nt)) return;
-  __threadfence();
+  consume_end(r, slot);
+  cbar();  // as.s / as.pv are reused by the next item
+}
+
+// Merge head h's partials over the nt tiles: M = max_t m_t, L = sum_t l_t 2^(m_t - M),
+// o[d] = sum_t 2^(m_t - M) o_t[d] / L.  Threads (d4, tile slice): 32 float4 columns x up to
+// 15 tile slices, combined through shared memory.  Result in out[128] (fp32, shared).
+__device__ void merge_head(const StepParams& p, int h, int nt, float* scratch, float* out) {
+  const int tid = threadIdx.x;
+  const int G = p.Hq / p.Hkv, g = h / G, hh = h % G;
+  const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + hh) * kPart;
+  const int d4 = tid & 31, ts = tid >> 5;  // ts in [0, NW)
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int t = ts; t < nt; t += NW) {
+    const float* pt = base + (size_t)t * kMaxG * kPart;
+    const float mt = __ldcg(pt), lt = __ldcg(pt + 1);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(pt + 4) + d4);
+    const float bm = fmaxf(M, mt);
+    const float c = exp2f(M - bm), e = exp2f(mt - bm);
+    L = L * c + lt * e;
+    acc.x = acc.x * c + e * v.x;
+    acc.y = acc.y * c + e * v.y;
+    acc.z = acc.z * c + e * v.z;
+    acc.w = acc.w * c + e * v.w;
+    M = bm;
+  }
+  // scratch: [NW][32][6]
+  float* sp = scratch + (ts * 32 + d4) * 6;
+  sp[0] = M;
+  sp[1] = L;
+  sp[2] = acc.x;
+  sp[3] = acc.y;
+  sp[4] = acc.z;
+  sp[5] = acc.w;
   cbar();
-  if (tid == 0) {
-    const int prev = atomicAdd(&p.attn_count[g], 1);
-    as.is_last = prev == nt - 1;
+  if (tid < 32) {
+    float Mx = -INFINITY;
+    for (int s = 0; s < NW; ++s) Mx = fmaxf(Mx, scratch[(s * 32 + tid) * 6]);
+    float Lt = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < NW; ++s) {
+      const float* q = scratch + (s * 32 + tid) * 6;
+      const float e = q[0] == -INFINITY ? 0.f : exp2f(q[0] - Mx);
+      Lt = fmaf(q[1], e, Lt);
+      a.x = fmaf(q[2], e, a.x);
+      a.y = fmaf(q[3], e, a.y);
+      a.z = fmaf(q[4], e, a.z);
+      a.w = fmaf(q[5], e, a.w);
+    }
+    const float inv = 1.f / Lt;
+    reinterpret_cast<float4*>(out)[tid] = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
   }
   cbar();
-  if (!as.is_last) return;
-  __threadfence();
-  const float* base = p.attn_part + (size_t)g * p.max_tiles * kMaxG * kPart;
-  if (warp < G) {  // merge weights of head h: every m, l load in flight at once
-    const int h = warp;
-    constexpr int kPer = 256 / 32;  // nt <= max_tiles <= 256
-    float mv[kPer], lv[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int c = lane + 32 * j;
-      mv[j] = -INFINITY;
-      lv[j] = 0.f;
-      if (c < nt) {
-        const float* pp = base + ((size_t)c * kMaxG + h) * kPart;
-        mv[j] = __ldcg(pp);
-        lv[j] = __ldcg(pp + 1);
-      }
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) mx = fmaxf(mx, mv[j]);
-    mx = warp_max(mx);
-    float L = 0.f;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      mv[j] = exp2f(mv[j] - mx);  // 0 for absent tiles
-      L = fmaf(lv[j], mv[j], L);
-    }
-    L = warp_sum(L);
-    const float inv = 1.f / L;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-      if (lane + 32 * j < nt) as.mw[lane + 32 * j][h] = mv[j] * inv;
-  }
-  cbar();
-  // o merge: (head, 4-dim column) x tile half -> partial sums in as.pv, then the halves add up
-  const int cols = G * (D / 4);
-  const int halves = (NW * 32) / cols >= 2 ? 2 : 1;
-  const int tsplit = (nt + halves - 1) / halves;
-  for (int idx = tid; idx < cols * halves; idx += NW * 32) {
-    const int col = idx % cols, part = idx / cols;
-    const int h = col / (D / 4), d4 = col % (D / 4);
-    const int t0 = part * tsplit, t1 = min(nt, t0 + tsplit);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = t0; c0 < t1; c0 += 8) {
-      const int m = min(8, t1 - c0);
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = u < m ? __ldcg(reinterpret_cast<const float4*>(base + ((size_t)(c0 + u) * kMaxG + h) * kPart + 4) + d4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (u < m) {
-          const float w = as.mw[c0 + u][h];
-          acc.x = fmaf(w, v[u].x, acc.x);
-          acc.y = fmaf(w, v[u].y, acc.y);
-          acc.z = fmaf(w, v[u].z, acc.z);
-          acc.w = fmaf(w, v[u].w, acc.w);
-        }
-      }
-    }
-    *reinterpret_cast<float4*>(&as.pv[part][h][4 * d4]) = acc;
-  }
-  cbar();
-  for (int idx = tid; idx < cols; idx += NW * 32) {
-    const int h = idx / (D / 4), d4 = idx % (D / 4);
-    float4 acc = *reinterpret_cast<const float4*>(&as.pv[0][h][4 * d4]);
-    if (halves == 2) {
-      const float4 b2 = *reinterpret_cast<const float4*>(&as.pv[1][h][4 * d4]);
-      acc.x += b2.x;
-      acc.y += b2.y;
-      acc.z += b2.z;
-      acc.w += b2.w;
-    }
-    *reinterpret_cast<float4*>(p.attn_out + (size_t)(g * G + h) * D + 4 * d4) = acc;
-  }
-  if (tid == 0) p.attn_count[g] = 0;
+}
+
+// --------------------------------------------------------------------------- lm_head x
+// fp16 x in the half2-pair layout of the fp16 head dot: element k (hb = k/16, word = (k/8)%2,
+// j = k%8) at uint4 (word * NHB + hb), component j%4, half j/4.
+__device__ __forceinline__ int xh_slot(int k, int nhb) {
+  const int hb = k >> 4, word = (k >> 3) & 1, j = k & 7;
+  return ((word * nhb + hb) * 4 + (j & 3)) * 2 + (j >> 2);
 }
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
@@ -900,6 +750,7 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv;
   Ring r;
   r.wait_ns = 0;
   r.ph = 0;
@@ -912,9 +763,23 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   r.stage_bytes = p.stage_bytes;
   r.nstages = p.nstages;
   r.idx = 0;
-  __half* xs = reinterpret_cast<__half*>(smem + (size_t)p.nstages * p.stage_bytes);
-  AttnScratch& as = *reinterpret_cast<AttnScratch*>(smem + (size_t)p.nstages * p.stage_bytes +
-                                                     (size_t)p.x_floats * 2);
+  // shared layout after the ring: xq [2][kMaxK/16] uint4 | corr [kMaxK/16] | fb [kMaxK/32] |
+  // hbuf [kMaxK/...] | AttnScratch | red[64] | mbarriers
+  unsigned char* sp = smem + (size_t)p.nstages * p.stage_bytes;
+  const int maxK = max(H, Hq * D);
+  const int nhb_max = maxK / 16;
+  XOp xo;
+  xo.xq = reinterpret_cast<uint4*>(sp);
+  sp += (size_t)nhb_max * 2 * 16;
+  xo.corr = reinterpret_cast<int*>(sp);
+  sp += (size_t)nhb_max * 4;
+  xo.fb = reinterpret_cast<float*>(sp);
+  sp += (size_t)nhb_max * 2;
+  const int nsl = slices_of(p, blockIdx.x);
+  float* hbuf = reinterpret_cast<float*>(sp);  // h of this CTA's slices, then o_h of an o-item
+  sp += (size_t)max(nsl * kSlice, D) * 4;
+  sp = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sp) + 15) & ~uintptr_t(15));
+  AttnScratch& as = *reinterpret_cast<AttnScratch*>(sp);
   float* red = reinterpret_cast<float*>(&as + 1);  // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 64) + 15) &
                                                ~uintptr_t(15));
@@ -954,124 +819,158 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   int sk = 0;        // timeline stamp index
   stamp(p, sk);
   const int cta = blockIdx.x, ncta = gridDim.x;
-  const int H = p.H, Hq = p.Hq, Hkv = p.Hkv, I = p.I;
   const int nqkv = (Hq + 2 * Hkv) * D;
   const int nt = ntiles_for(past);
+  const int nrb = H / kORows;
+  const int ns = n_slices(p);
   int pos = *p.position;
   if (pos < 0 || pos >= p.max_position) {
     if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
     pos = min(max(pos, 0), p.max_position - 1);
   }
-  uint4 xr[kRegHB][2];
-  for (int i = tid; i < D / 2; i += NW * 32) {
+  for (int i = tid; i < D / 2; i += NT) {
     as.cs[i] = p.rope_cos[(size_t)pos * (D / 2) + i];
     as.sn[i] = p.rope_sin[(size_t)pos * (D / 2) + i];
   }
-  // This CTA's rows of the residual (the o-proj and down phases update exactly these rows).
-  int hr0, hr1;
-  cta_range(H, cta, ncta, hr0, hr1);
-  float* xown = red + 32;  // up to 32 rows (H <= 32 * gridDim.x)
+  const __half* e16 = p.input_embeds;
+  if (!e16) {
+    int tok = __ldcg(p.token);
+    if (tok < 0 || tok >= p.V) {
+      if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
+      tok = min(max(tok, 0), p.V - 1);
+    }
+    e16 = p.embed + (size_t)tok * H;
+  }
+  auto load_emb = [&](int k) -> float4 {
+    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(e16 + k));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  };
+  auto load_x = [&](int k) -> float4 {
+    const ulonglong2 a = __ldcg(reinterpret_cast<const ulonglong2*>(p.x_acc + k));
+    const ulonglong2 b = __ldcg(reinterpret_cast<const ulonglong2*>(p.x_acc + k + 2));
+    return make_float4(from_fix(a.x), from_fix(a.y), from_fix(b.x), from_fix(b.y));
+  };
+  // residual = embedding: this CTA's share of rows, before the first barrier (the o-phase adds
+  // come after two more barriers)
+  {
+    int hr0, hr1;
+    cta_range(H / 4, cta, ncta, hr0, hr1);
+    for (int i = hr0 + tid; i < hr1; i += NT) {
+      const float4 v = load_emb(4 * i);
+      reinterpret_cast<ulonglong2*>(p.x_acc + 4 * i)[0] = make_ulonglong2(to_fix(v.x), to_fix(v.y));
+      reinterpret_cast<ulonglong2*>(p.x_acc + 4 * i)[1] = make_ulonglong2(to_fix(v.z), to_fix(v.w));
+    }
+  }
+  int o0, o1;
+  cta_range(Hq * nrb, cta, ncta, o0, o1);
 
   for (int l = 0; l < p.L; ++l) {
     const StepLayer& w = p.layers[l];
     // ---------------------------------------------------------------- QKV
     r.ph = 0;
     if (l == 0) {
-      const __half* e16 = p.input_embeds;
-      if (!e16) {
-        int tok = __ldcg(p.token);
-        if (tok < 0 || tok >= p.V) {
-          if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
-          tok = min(max(tok, 0), p.V - 1);
-        }
-        e16 = p.embed + (size_t)tok * H;
-      }
-      for (int i = tid; i < hr1 - hr0; i += NW * 32) xown[i] = __half2float(e16[hr0 + i]);
-      stage_x(xs, red, nullptr, e16, w.in_norm, p.eps, H, cta == 0 ? p.x_resid : nullptr);
-      stamp(p, sk);
+      stage_idp(xo, load_emb, w.in_norm, p.eps, H, red, nullptr);
     } else {
       grid_barrier(p, gen, sk);
-      stage_x(xs, red, p.x_resid, nullptr, w.in_norm, p.eps, H, nullptr);
-      stamp(p, sk);
+      float* tr = (p.trace && cta == 0) ? p.trace + (size_t)(l - 1) * H : nullptr;
+      stage_idp(xo, load_x, w.in_norm, p.eps, H, red, tr);
     }
-    const bool regH = H <= 32 * kRegHB * 16;
+    stamp(p, sk);
     {
       int r0, r1;
       cta_range(nqkv, cta, ncta, r0, r1);
       const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
       // this CTA's q/k/v biases -> shared memory (as.q is free until the attention phase)
       float* bias_s = &as.q[0][0];
-      for (int i = tid; i < r1 - r0; i += NW * 32) {
+      for (int i = tid; i < r1 - r0; i += NT) {
         const int row = r0 + i;
         const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
         const __half* b = w.bias[m];
         bias_s[i] = b ? __half2float(b[row - bounds[m]]) : 0.f;
       }
-      if (regH) load_xr(xs, xr, H);
       cbar();
-      // [Wq; Wk; Wv] as one matrix of nqkv rows (the producer joins the segments)
       const float* bs = bias_s - r0;
-      consume_packed(r, xs, xr, regH, H, r0, r1, 1, &as.s[0][0],
-                     [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
+      consume_rows<false>(r, xo, H, r0, r1, 1,
+                          [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
     }
     // ---------------------------------------------------------------- ATTN
     r.ph = 1;
     grid_barrier(p, gen, sk);
-    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, pos);
+    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past);
+    stamp(p, sk);
     // ---------------------------------------------------------------- O
     r.ph = 2;
     grid_barrier(p, gen, sk);
-    if (merge_in_o(p, nt)) {
-      stage_attn_merged(p, xs, nt);
-    } else {
-      stage_x(xs, red, p.attn_out, nullptr, nullptr, 0.f, Hq * D, nullptr);
+    {
+      int cur_h = -1;
+      for (int i = o0; i < o1; ++i) {
+        const int h = i / nrb, rb = i % nrb;
+        if (h != cur_h) {
+          merge_head(p, h, nt, &as.pv[0][0][0], hbuf);
+          stage_idp(xo, [&](int k) { return *reinterpret_cast<const float4*>(hbuf + k); },
+                    nullptr, 0.f, D, red, nullptr);
+          cur_h = h;
+        }
+        unsigned long long* xr = p.x_acc + (size_t)rb * kORows;
+        consume_cols(r, xo, kORows, 4, [&](int row, float y) { red_add_u64(xr + row, to_fix(y)); });
+      }
     }
     stamp(p, sk);
-    const bool regO = Hq * D <= 32 * kRegHB * 16;
-    if (regO) load_xr(xs, xr, Hq * D);
-    {
-      int r0, r1;
-      cta_range(H, cta, ncta, r0, r1);
-      consume_packed(r, xs, xr, regO, Hq * D, r0, r1, 1, &as.s[0][0], [&](int row, float y, float) {
-        const float v = xown[row - hr0] + y;
-        xown[row - hr0] = v;
-        p.x_resid[row] = v;
-      });
-    }
-    // ---------------------------------------------------------------- GU
+    // ---------------------------------------------------------------- GU + DOWN
     r.ph = 3;
     grid_barrier(p, gen, sk);
-    stage_x(xs, red, p.x_resid, nullptr, w.post_norm, p.eps, H, nullptr);
-    stamp(p, sk);
-    if (regH) load_xr(xs, xr, H);
-    {
-      int r0, r1;
-      cta_range(I, cta, ncta, r0, r1);
-      consume_packed(r, xs, xr, regH, H, r0, r1, 2, &as.s[0][0], [&](int row, float g, float u) {
-        p.h[row] = g / (1.f + __expf(-g)) * u;
-      });
+    if (nsl > 0) {
+      stage_idp(xo, load_x, w.post_norm, p.eps, H, red, nullptr);
+      stamp(p, sk);
+      int j = 0;
+      for (int s = cta; s < ns; s += ncta, ++j) {
+        float* hs = hbuf + j * kSlice - s * kSlice;
+        consume_rows<true>(r, xo, H, s * kSlice, (s + 1) * kSlice, 2, [&](int row, float g, float u) {
+          hs[row] = g / (1.f + __expf(-g)) * u;
+        });
+      }
+      cbar();
+      r.ph = 4;
+      stage_idp(xo, [&](int k) { return *reinterpret_cast<const float4*>(hbuf + k); }, nullptr,
+                0.f, nsl * kSlice, red, nullptr);
+      consume_cols(r, xo, H, 2 * nsl, [&](int row, float y) { red_add_u64(p.x_acc + row, to_fix(y)); });
+    } else {
+      stamp(p, sk);
     }
-    // ---------------------------------------------------------------- DOWN
-    r.ph = 4;
-    grid_barrier(p, gen, sk);
-    stage_x(xs, red, p.h, nullptr, nullptr, 0.f, I, nullptr);
     stamp(p, sk);
-    {
-      int r0, r1;
-      cta_range(H, cta, ncta, r0, r1);
-      float* tr = p.trace ? p.trace + (size_t)l * H : nullptr;
-      consume_packed(r, xs, xr, false, I, r0, r1, 1, &as.s[0][0], [&](int row, float y, float) {
-        const float v = xown[row - hr0] + y;
-        xown[row - hr0] = v;
-        p.x_resid[row] = v;
-        if (tr) tr[row] = v;
-      });
-    }
   }
   // ------------------------------------------------------------------------------ HEAD
   r.ph = 5;
   grid_barrier(p, gen, sk);
-  stage_x(xs, red, p.x_resid, nullptr, p.final_norm, p.eps, H, nullptr);
+  __half* xs = reinterpret_cast<__half*>(xo.xq);
+  {
+    // final RMSNorm, x rounded once to fp16 in the pair layout of the fp16 head dot
+    const int nhb = H >> 4;
+    float* tr = (p.trace && cta == 0) ? p.trace + (size_t)(p.L - 1) * H : nullptr;
+    float ss = 0.f;
+    for (int k = tid * 4; k < H; k += NT * 4) {
+      const float4 v = load_x(k);
+      if (tr) *reinterpret_cast<float4*>(tr + k) = v;
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    cbar();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) tot += red[i];
+    const float inv = rsqrtf(tot / (float)H + p.eps);
+    for (int k = tid * 4; k < H; k += NT * 4) {
+      const float4 v = load_x(k);
+      const float y[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        xs[xh_slot(k + e, nhb)] = __float2half_rn(y[e] * inv * __half2float(p.final_norm[k + e]));
+    }
+    cbar();
+  }
   stamp(p, sk);
   float best = -INFINITY;
   int best_i = 0x7fffffff;
@@ -1085,20 +984,19 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     // held in registers for c = lane + 32 j when the row fits (H <= 1536)
     const int nhb = H >> 4;
     const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
-    const bool regHead = nch <= 32 * 2 * kRegHB;
+    const bool regHead = nch <= 32 * 2 * kHeadRegHB;
+    uint4 xr[2 * kHeadRegHB];
     if (regHead) {
 #pragma unroll
-      for (int j = 0; j < 2 * kRegHB; ++j) {
+      for (int j = 0; j < 2 * kHeadRegHB; ++j) {
         const int c = lane + 32 * j;
-        xr[j >> 1][j & 1] = c < nch ? xs4[(c & 1) * nhb + (c >> 1)] : make_uint4(0u, 0u, 0u, 0u);
+        xr[j] = c < nch ? xs4[(c & 1) * nhb + (c >> 1)] : make_uint4(0u, 0u, 0u, 0u);
       }
     }
     for (int a = r0; a < r1; a += rps) {
       const int n = min(rps, r1 - a);
-      const int s = r.idx++;
-      const int slot = s % r.nstages;
-      ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
-      const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
+      int slot;
+      const unsigned char* st = consume_begin(r, slot);
       for (int i = warp; i < n; i += NW) {
         const unsigned char* row = st + (size_t)i * rb;
         float acc = 0.f;
@@ -1116,9 +1014,9 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
         };
         if (regHead) {
 #pragma unroll
-          for (int j = 0; j < 2 * kRegHB; ++j) {
+          for (int j = 0; j < 2 * kHeadRegHB; ++j) {
             const int c = lane + 32 * j;
-            if (c < nch) chunk(*reinterpret_cast<const uint4*>(row + c * 16), xr[j >> 1][j & 1]);
+            if (c < nch) chunk(*reinterpret_cast<const uint4*>(row + c * 16), xr[j]);
           }
         } else {
           for (int c = lane; c < nch; c += 32)
@@ -1134,8 +1032,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&r.empty[slot]);
+      consume_end(r, slot);
     }
   }
   if (lane == 0) {
@@ -1196,12 +1093,86 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   }
 }
 
+// ------------------------------------------------------------------------ column images
+// Wo (rows H, columns Hq * D): item i = (h, rb) -> rows [kORows rb, +kORows) x blocks
+// [4h, 4h + 4): codes [kORows][4][16] then scales [kORows][4].
+__global__ void wo_image_kernel(const uint8_t* __restrict__ q, const __half* __restrict__ s, int H,
+                                int Hq, unsigned char* __restrict__ img) {
+  const int KB = Hq * D / 32;
+  const int nrb = H / kORows;
+  const int64_t total = (int64_t)Hq * nrb * kORows * 4;  // (item, row, block) triples
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int b = (int)(t & 3);
+    const int rr = (int)((t >> 2) % kORows);
+    const int i = (int)((t >> 2) / kORows);
+    const int h = i / nrb, rb = i % nrb;
+    const int row = rb * kORows + rr, blk = 4 * h + b;
+    unsigned char* it = img + (size_t)i * kORows * 4 * 18;
+    reinterpret_cast<uint4*>(it)[rr * 4 + b] =
+        *reinterpret_cast<const uint4*>(q + ((size_t)row * KB + blk) * 16);
+    reinterpret_cast<__half*>(it + kORows * 4 * 16)[rr * 4 + b] = s[(size_t)row * KB + blk];
+  }
+}
+
+// Wd (rows H, columns I): CTA c's image holds its slices c, c + grid, ... (64 columns = 2 blocks
+// each): codes [H][2 nsl][16] then scales [H][2 nsl]; CTA images `stride` bytes apart.
+__global__ void wd_image_kernel(const uint8_t* __restrict__ q, const __half* __restrict__ s, int H,
+                                int I, int grid, size_t stride, unsigned char* __restrict__ img) {
+  const int KB = I / 32;
+  const int ns = I / kSlice;
+  const int64_t total = (int64_t)H * KB;  // (row, block)
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int row = (int)(t / KB), blk = (int)(t % KB);
+    const int sl = blk / 2, c = sl % grid, j = sl / grid;
+    const int nsl = (ns - 1 - c) / grid + 1;
+    const int nb = 2 * nsl;
+    const int col = 2 * j + (blk & 1);
+    unsigned char* ci = img + (size_t)c * stride;
+    reinterpret_cast<uint4*>(ci)[(size_t)row * nb + col] =
+        *reinterpret_cast<const uint4*>(q + ((size_t)row * KB + blk) * 16);
+    reinterpret_cast<__half*>(ci + (size_t)H * nb * 16)[(size_t)row * nb + col] =
+        s[(size_t)row * KB + blk];
+  }
+}
+
 }  // namespace
 
-size_t step_smem_bytes(int stage_bytes, int nstages, int x_floats) {
-  // x is staged in fp16: x_floats halves
-  return (size_t)nstages * stage_bytes + (size_t)x_floats * 2 + sizeof(AttnScratch) + 64 * 4 +
-         2 * nstages * 8 + 64;
+size_t step_wo_image_bytes(int H, int Hq) { return (size_t)Hq * (H / kORows) * kORows * 4 * 18; }
+
+size_t step_wd_image_bytes(int H, int I, int grid) {
+  const int ns = I / kSlice;
+  const int nsl_max = (ns + grid - 1) / grid;
+  return (size_t)grid * H * nsl_max * 2 * 18;
+}
+
+cudaError_t step_build_images(const StepParams& p, const StepLayer* hl, unsigned char* wo_img,
+                              unsigned char* wd_img, cudaStream_t s) {
+  const size_t wo_b = step_wo_image_bytes(p.H, p.Hq);
+  const size_t wd_b = step_wd_image_bytes(p.H, p.I, p.grid);
+  const int ns = p.I / kSlice;
+  const size_t stride = (size_t)p.H * ((ns + p.grid - 1) / p.grid) * 2 * 18;
+  for (int l = 0; l < p.L; ++l) {
+    wo_image_kernel<<<p.grid * 4, 256, 0, s>>>(hl[l].q[3], hl[l].s[3], p.H, p.Hq,
+                                               wo_img + (size_t)l * wo_b);
+    wd_image_kernel<<<p.grid * 4, 256, 0, s>>>(hl[l].q[6], hl[l].s[6], p.H, p.I, p.grid, stride,
+                                               wd_img + (size_t)l * wd_b);
+  }
+  return cudaGetLastError();
+}
+
+size_t step_smem_bytes(const StepParams& p) {
+  const int maxK = std::max(p.H, p.Hq * D);
+  const int nhb_max = maxK / 16;
+  const int ns = p.I / kSlice;
+  const int nsl_max = (ns + p.grid - 1) / p.grid;
+  size_t b = (size_t)p.nstages * p.stage_bytes;
+  b += (size_t)nhb_max * 2 * 16 + (size_t)nhb_max * 4 + (size_t)nhb_max * 2;
+  b += (size_t)std::max(nsl_max * kSlice, D) * 4;
+  b = (b + 15) & ~size_t(15);
+  b += sizeof(AttnScratch) + 64 * 4 + 16 + 2 * p.nstages * 8 + 64;
+  return b;
 }
 
 int step_threads() { return kThreads; }
@@ -1212,15 +1183,15 @@ size_t step_attn_part_floats(int Hkv, int max_tiles) {
 
 int step_max_tiles(int cap) { return (cap + TT - 1) / TT; }
 
-// Pick the largest stage size (>= 32 KB, 1 KB steps) for which one CTA per SM is resident.
+// Pick the largest stage size (>= one attention tile, 1 KB steps) for which one CTA per SM is
+// resident.
 cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
   cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                        (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   *blocks_per_sm = 0;
-  // a stage must hold one attention tile: 2 x TT padded rows of kRowH halves (34 KB)
   for (; p.stage_bytes >= 2 * TT * kRowH * 2; p.stage_bytes -= 1024) {
-    const size_t smem = step_smem_bytes(p.stage_bytes, p.nstages, p.x_floats);
+    const size_t smem = step_smem_bytes(p);
     e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -1247,7 +1218,7 @@ void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_by
 }
 
 cudaError_t launch_step(const StepParams& p, cudaStream_t s) {
-  const size_t smem = step_smem_bytes(p.stage_bytes, p.nstages, p.x_floats);
+  const size_t smem = step_smem_bytes(p);
   cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

@@ -95,12 +95,35 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; bounded (see kWaitLimitNs).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; gives up after limit_ns (default
+// kWaitLimitNs), records VV_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait_hint(bar, parity, 20000u)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_device_error(VV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until the global counter *p reaches `target` (acquire); gives up after limit_ns, records
+// VV_ERR_TIMEOUT and returns false.  The grid barriers of the step kernel wait through this.
+__device__ __forceinline__ bool wait_counter_geq(const unsigned* p, unsigned target,
+                                                 uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_u32(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_u32(p) < target) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_device_error(VV_ERR_TIMEOUT);
       return false;
     }

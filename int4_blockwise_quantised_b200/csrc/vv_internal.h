@@ -62,78 +62,26 @@ struct GemvWeights {
   const uint16_t* scales;
 };
 
-// y[n] = W[n, :] . xn + bias, W = [Wq; Wk; Wv] as three matrices (rows nq, nk, nv), K = H,
-// xn = RMSNorm(x) with gamma. x source: x_f32 (residual) or, when embed != nullptr, the fp16
-// embedding row (input_embeds, or embed_table[*token]); in that case the kernel also writes
-// the residual x_resid = row.
-struct QkvArgs {
-  GemvWeights w[3];
-  int rows[3];
-  const uint16_t* bias[3];
-  int K;
-  const float* x_resid_in;      // fp32 [K] or nullptr when reading the embedding
-  const uint16_t* embeds;       // fp16 [K] input_embeds, or nullptr
-  const uint16_t* embed_table;  // fp16 [V, K] with token, or nullptr
-  const int32_t* token;
-  int vocab;
-  float* x_resid_out;  // written when the embedding is the source
-  const uint16_t* gamma;
-  float eps;
-  float* out;  // fp32 [rows0 + rows1 + rows2]
-};
-cudaError_t launch_qkv(const QkvArgs& a, cudaStream_t s, bool pdl);
-
-// x_resid[n] += W[n, :] . x  (x fp32 [K], no norm).  Optional trace copy of the updated rows.
-struct ResidArgs {
-  GemvWeights w;
-  int N, K;
-  const float* x;
-  float* x_resid;
-  float* trace;  // fp32 [N] or nullptr: receives the updated residual rows
-};
-cudaError_t launch_resid(const ResidArgs& a, cudaStream_t s, bool pdl);
-
-// h[n] = silu(Wg[n,:] . xn) * (Wu[n,:] . xn),  xn = RMSNorm(x_resid) with gamma.
-struct GateUpArgs {
-  GemvWeights wg, wu;
-  int N, K;
-  const float* x_resid;
-  const uint16_t* gamma;
-  float eps;
-  float* h;  // fp32 [N]
-};
-cudaError_t launch_gateup(const GateUpArgs& a, cudaStream_t s, bool pdl);
-
 // Standalone MatMulNBits GEMV: y[m, n] = x[m, :] . W[n, :] (+bias) in fp16, M <= 8.
 cudaError_t launch_matmul_nbits_gemv(const uint16_t* x, GemvWeights w, const uint16_t* bias,
                                      int M, int N, int K, uint16_t* y, cudaStream_t s);
 
 // Attention (attn.cu) ------------------------------------------------------------------------
 struct AttnArgs {
-  // standalone: q fp16 [Hq, D] rotated, all `len` positions in the cache.
-  const uint16_t* q_f16;
-  // fused decoder mode: q/k/v fp32 pre-RoPE from the QKV GEMV ([Hq*D | Hkv*D | Hkv*D]);
-  // rotates q and k at *position, appends k/v at slot *length, attends over *length + 1.
-  const float* qkv;
-  const int32_t* position;
-  const int32_t* length;
-  const float* rope_cos;  // [max_position, D/2]
-  const float* rope_sin;
-  int max_position;
-  uint16_t* k_cache;  // [Hkv, cap, D] of this layer
+  const uint16_t* q_f16;  // fp16 [Hq, D], already rotated
+  uint16_t* k_cache;      // [Hkv, cap, D]
   uint16_t* v_cache;
-  int len;  // standalone: valid positions
+  int len;                // valid positions
   int cap, Hq, Hkv;
   float scale;
-  uint16_t* out_f16;  // standalone output [Hq, D]
-  float* out_f32;     // fused output [Hq*D]
+  uint16_t* out_f16;  // [Hq, D]
   float* ws_part;     // partials
   int* ws_count;      // per kv-head arrival counters
   int nchunks;
 };
 size_t attn_workspace_bytes(int Hq, int Hkv, int nchunks);
 int attn_default_chunks(int Hkv, int cap);
-cudaError_t launch_attn(const AttnArgs& a, bool fused, cudaStream_t s, bool pdl);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t s);
 
 // lm_head (lmhead.cu) ---------------------------------------------------------------------
 struct LmHeadArgs {

@@ -136,20 +136,9 @@ class Decoder:
         check(_vv.lib.vv_decoder_step(self.handle, ptr(input_embeds), ptr(token), ptr(position),
                                       ptr(logits), ptr(argmax), stream_handle(stream)))
 
-    PHASES = ("qkv", "attn", "o_proj", "gate_up", "down", "lm_head")
-
-    def profile_step(self, position, input_embeds=None, token=None, logits=None, argmax=None,
-                     stream=None):
-        """One step with CUDA events around every launch; returns {phase: ms summed over layers}."""
-        out = (ctypes.c_float * 6)()
-        check(_vv.lib.vv_decoder_profile_step(self.handle, ptr(input_embeds), ptr(token),
-                                              ptr(position), ptr(logits), ptr(argmax), out,
-                                              stream_handle(stream)))
-        return dict(zip(self.PHASES, list(out)))
-
     def step_timeline(self, position, input_embeds=None, token=None, stream=None):
         """One persistent step with the timeline tap; returns uint64 ns array [grid, stamps]."""
-        maxn = 14 * self.model.shape.layers + 16
+        maxn = 13 * self.model.shape.layers + 3 + 8
         grid_max = 1024
         buf = np.zeros(grid_max * maxn, dtype=np.uint64)
         g = ctypes.c_int32()

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import synth
-from helpers import TOL, gpu_model, normwise, ocfg, oracle_model
+from helpers import TOL, dev, fill_cache, gpu_model, normwise, ocfg, oracle_model, run_steps
 from oracle import decoder as odec
 
 pytestmark = pytest.mark.gpu
@@ -20,73 +20,6 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def need_gpu():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-
-
-def dev(a):
-    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-
-def fill_cache(dec, kp, vp):
-    P = kp.shape[2]
-    dec.k_cache[:, 0, :, :P] = dev(kp)
-    dec.v_cache[:, 0, :, :P] = dev(vp)
-    dec.set_length(P)
-
-
-def run_steps(shape, mode, P, steps, cap=None, graph=True, check_kv=True, layers_oracle=None):
-    from int4_blockwise_quantised_b200.model import Decoder
-
-    cfg = ocfg(shape)
-    W = oracle_model(shape, mode)
-    model = gpu_model(shape, mode)
-    cap = cap or P + steps + 5
-    dec = Decoder(model, cap)
-    dec.set_graph(graph)
-    kp, vp = synth.past_kv(shape, P)
-    fill_cache(dec, kp, vp)
-    kc = [kp[l].copy() for l in range(shape.layers)]
-    vc = [vp[l].copy() for l in range(shape.layers)]
-    trace = torch.zeros((shape.layers, shape.hidden), dtype=torch.float32, device="cuda")
-    dec.set_trace(trace)
-    emb = synth.input_embeds(shape, steps)
-    pos_t = torch.zeros(1, dtype=torch.int32, device="cuda")
-    emb_t = torch.zeros(shape.hidden, dtype=torch.float16, device="cuda")
-    logits = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
-    amax = torch.zeros(1, dtype=torch.int32, device="cuda")
-    worst = 0.0
-    for s in range(steps):
-        pos = P + s
-        pos_t.fill_(pos)
-        emb_t.copy_(dev(emb[s]))
-        dec.step(pos_t, input_embeds=emb_t, logits=logits, argmax=amax)
-        dec.sync_status()
-        ora = odec.decoder_step(cfg, W, emb[s], pos, kc, vc)
-        lo = trace.cpu().numpy()
-        for l in range(shape.layers):
-            e = normwise(lo[l], ora["layer_out"][l])
-            worst = max(worst, e)
-            assert e <= TOL, f"step {s} layer {l}: {e}"
-        e = normwise(logits.cpu().numpy(), ora["logits"])
-        assert e <= TOL, f"step {s} logits: {e}"
-        ref = ora["logits"]
-        top2 = np.sort(ref)[-2:]
-        if top2[1] - top2[0] > 1e-2:
-            assert int(amax.item()) == ora["argmax"]
-        if check_kv:
-            # appended K/V: floating point -> contract tolerance; the slot is checked exactly below
-            slot = P + s
-            kg = dec.k_cache[:, 0, :, slot].cpu().numpy()
-            vg = dec.v_cache[:, 0, :, slot].cpu().numpy()
-            assert normwise(kg, ora["k_new"]) <= TOL and normwise(vg, ora["v_new"]) <= TOL
-        for l in range(shape.layers):
-            kc[l] = np.concatenate([kc[l], ora["k_new"][l][:, None, :]], axis=1)
-            vc[l] = np.concatenate([vc[l], ora["v_new"][l][:, None, :]], axis=1)
-    # untouched slots: past positions bit-identical, beyond length still zero
-    n = P + steps
-    assert np.array_equal(dec.k_cache[:, 0, :, :P].cpu().numpy(), kp)
-    assert torch.count_nonzero(dec.k_cache[:, 0, :, n:]).item() == 0
-    assert dec.length == n
-    return worst
 
 
 def test_single_layer_ternary_config():
@@ -111,16 +44,17 @@ def test_small_ternary_long_context():
     run_steps(synth.SHAPE_SMALL, "ternary", 4530, 2)
 
 
-def test_wide_hidden_row_mode():
-    """hidden 2048 > 1536: x no longer fits in registers; gate/up (38 pairs per CTA) runs whole
-    rows per warp with x in shared memory, the other phases split K over warps."""
+def test_wide_hidden_uneven_slices():
+    """hidden 2048, 16/2 heads, intermediate 5632: 88 gate/up slices over the SMs (most CTAs
+    without one), 16 x 16 o-proj items, and a GEMV input longer than 1536."""
     shape = synth.Shape("wide", 2048, 2, 16, 2, 128, 5632, 4099, tied=True)
     run_steps(shape, "int4", 300, 2)
 
 
 def test_single_layer_7b_shapes():
     """One decoder layer at 7B shapes (hidden 3584, 28/4 heads, intermediate 18944, untied
-    152064-row head): q/k/v (31 rows per CTA) and gate/up in row mode, o-proj and down split-K."""
+    152064-row head): ~31 q/k/v rows per CTA, two gate/up slices per CTA (so the down columns of
+    a CTA span two slices), several o-proj items per CTA over two heads."""
     shape = synth.Shape("layer7b", 3584, 1, 28, 4, 128, 18944, 152064, tied=False)
     run_steps(shape, "int4", 128, 1)
 

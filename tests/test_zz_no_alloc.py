@@ -4,7 +4,8 @@ vv_gqa_decode_attn_noalloc serves callers that cannot allocate device memory whe
 attention; it keeps its split-K scratch in a static device array instead of a caller workspace.
 This file is collected last so that a failure here never hides the other tests; it must pass on
 its own in a fresh process as well as after them.  Two calls in a row (different lengths, so the
-second reuses the array the first one left behind) are compared with vv_gqa_decode_attn.
+second reuses the array the first one left behind) are compared with vv_gqa_decode_attn and
+directly with the oracle's grouped-query attention.
 """
 
 import math
@@ -15,6 +16,7 @@ import torch
 
 import synth
 from helpers import TOL, normwise
+from oracle import ops
 
 pytestmark = pytest.mark.gpu
 
@@ -35,12 +37,18 @@ def test_noalloc_attention_matches_workspace_entry_point():
         _vv.vv_sync_status()
         e = normwise(got.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64))
         assert e <= TOL, f"call {call}: normwise difference {e}"
+        ora = ops.gqa_decode_attention(q.cpu().numpy(), K[:, :length].cpu().numpy(),
+                                       V[:, :length].cpu().numpy(), 1 / math.sqrt(D))
+        e = normwise(got.cpu().numpy().astype(np.float64), ora)
+        assert e <= TOL, f"call {call}: normwise error against the oracle {e}"
 
 
 def test_noalloc_attention_rejects_oversized_scratch():
     from int4_blockwise_quantised_b200 import _vv
 
-    # a 4800-position cache with 2 KV heads needs 2 x 74 chunks of partials (> 256 KiB)
+    # a 4800-position cache with 2 KV heads needs more split-K partials than the 256 KiB array
+    # holds (the chunk count depends on the SM count; the workspace size says how many)
+    assert _vv.vv_gqa_decode_attn_workspace_size(12, 2, 128, 4800) > 256 * 1024
     q = torch.zeros((12, 128), dtype=torch.float16, device="cuda")
     kv = torch.zeros((2, 4800, 128), dtype=torch.float16, device="cuda")
     with pytest.raises(_vv.VVError) as e:
