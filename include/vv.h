@@ -59,7 +59,9 @@ const char* vv_version(void);
  * Returns the last error code. */
 vv_status vv_last_error(char* buf, size_t n);
 
-/* Synchronise `stream` and return (and clear) the device error word of the current device. */
+/* Synchronise `stream` and return (and clear) the device error word of the current device.
+ * While the word holds VV_ERR_TIMEOUT, every bounded wait of later kernels gives up at once (a
+ * kernel whose schedule went wrong ends quickly); clear it with this call. */
 vv_status vv_sync_status(vv_stream stream);
 
 /* Self-test of the bounded device waits (no counterpart in the pages: a property of this
@@ -106,26 +108,19 @@ vv_status vv_pack_nbits(const float* w, int64_t N, int64_t K, int32_t block, int
  * MatMulNBits ([STATUS] "Done": com.microsoft::MatMulNBits, 5 per layer).
  *   y[m, n] = sum_k x[m, k] * (code[n, k] - 8) * scale[n, k / 32]  (+ bias[n])
  * x device fp16 [M, K]; q/scales as produced by vv_pack_nbits for [N, K]; bias device fp16 [N]
- * or NULL; y device fp16 [M, N].  Products and sums in fp32, one rounding to fp16 at the end.
- * 1 <= M <= 8 runs the dequant-fused GEMV (each weight byte read once for all M rows).
- * Requirements: K % 32 == 0, block == 32, all pointers 16-byte aligned.
- * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (K % 32, M outside [1, 8], N < 1). */
+ * or NULL; y device fp16 [M, N].  One launch, no scratch:
+ *   1 <= M <= 8: dequant-fused GEMV (each weight byte read once for all M rows); products and
+ *                sums in fp32, one rounding to fp16 at the end.  K % 32 == 0.
+ *   M > 8:       tcgen05 tensor-core GEMM; the int4 codes are expanded inside the kernel, in
+ *                shared memory, to the fp16 operand fp16((code - 8) * scale) (rounded once:
+ *                exact for ternary weights, within 2^-12 relative for int4) and multiplied with
+ *                fp32 accumulation in tensor memory (the prefill's projections, [BITNET]
+ *                decoder_init contract).  N % 128 == 0, K % 256 == 0, M < 2^24.
+ * Requirements: block == 32, all pointers 16-byte aligned.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (K % 32, N < 1, the M > 8 shape rules). */
 vv_status vv_matmul_nbits(const uint16_t* x, const uint8_t* q, const uint16_t* scales,
                           const uint16_t* bias, int64_t M, int64_t N, int64_t K, int32_t block,
                           uint16_t* y, vv_stream stream);
-
-/* MatMulNBits for many rows (the prefill's projections: decoder_init runs every layer's five
- * MatMulNBits over all S prompt positions at once, [BITNET] decoder_init contract).
- *   y[m, n] = fp16( sum_k x[m, k] * w16[n, k]  (+ bias[n]) ),  w16 = fp16((code - 8) * scale)
- * Two launches: W is dequantised into w_f16 (caller's device scratch, fp16 [N, K], overwritten),
- * then a tcgen05 tensor-core GEMM (fp16 operands, fp32 accumulation in tensor memory) writes y.
- * Same operands as vv_matmul_nbits; any M >= 1.  Requirements: N % 128 == 0 or N % 192 == 0, K % 64 == 0,
- * block == 32, all pointers 16-byte aligned, M < 2^24.  The fp16 rounding of each dequantised
- * weight is the only difference from vv_matmul_nbits' arithmetic.
- * Errors: VV_ERR_INVALID_ARG (null, misaligned), VV_ERR_SHAPE (N, K, M out of range). */
-vv_status vv_matmul_nbits_tc(const uint16_t* x, const uint8_t* q, const uint16_t* scales,
-                             const uint16_t* bias, int64_t M, int64_t N, int64_t K,
-                             int32_t block, uint16_t* w_f16, uint16_t* y, vv_stream stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Grouped-query decode attention ([STATUS] "Done": com.microsoft::GroupQueryAttention, one per
@@ -284,6 +279,12 @@ vv_status vv_decoder_init(vv_decoder* dec, const int32_t* input_ids, const int32
  * off.  Changing it re-captures the step graph. */
 vv_status vv_decoder_set_trace(vv_decoder* dec, float* layer_out);
 
+/* Bound of every device-side wait of the step kernel (grid barriers, the stage ring), in ns;
+ * default 2e9.  A wait that runs out records VV_ERR_TIMEOUT (reported by
+ * vv_decoder_sync_status) and lets the kernel finish; once one wait has timed out, all others
+ * give up at once.  limit_ns in [1e5, 1e10].  Errors: VV_ERR_INVALID_ARG. */
+vv_status vv_decoder_set_wait_limit(vv_decoder* dec, int64_t limit_ns);
+
 /* Turn CUDA-graph replay of the step on (default) or off (plain launches every call). */
 vv_status vv_decoder_set_graph(vv_decoder* dec, int32_t enable);
 
@@ -312,7 +313,8 @@ vv_status vv_decoder_generate(vv_decoder* dec, const int32_t* first_token, const
  * float [5] and launches: HOST int32 [5] receive the device time and the number of launches (or
  * copies) of each kind: [0] embedding splice, RMSNorm, RoPE/KV write, bias and trace copies;
  * [1] weight dequantisation to fp16; [2] tensor-core GEMMs; [3] causal attention; [4] final
- * norm + lm_head + argmax.  Errors as vv_decoder_init. */
+ * norm + lm_head + argmax.  Kind [1] stays 0 ms / 0 launches: the GEMMs expand the int4 weights
+ * in shared memory, no separate dequantisation runs.  Errors as vv_decoder_init. */
 vv_status vv_decoder_profile_init(vv_decoder* dec, const int32_t* input_ids,
                                   const int32_t* position_ids, int64_t S,
                                   const uint16_t* audio_features, int64_t N, int64_t audio_offset,

@@ -72,7 +72,6 @@ def _load():
         "vv_ternary_scale": (S, [P, c_int64, POINTER(c_float), P]),
         "vv_pack_nbits": (S, [P, c_int64, c_int64, c_int32, c_int32, c_float, P, P, P]),
         "vv_matmul_nbits": (S, [P, P, P, P, c_int64, c_int64, c_int64, c_int32, P, P]),
-    "vv_matmul_nbits_tc": (S, [P, P, P, P, c_int64, c_int64, c_int64, c_int32, P, P, P]),
         "vv_gqa_decode_attn_workspace_size": (c_size_t, [c_int32, c_int32, c_int32, c_int32]),
         "vv_gqa_decode_attn": (S, [P, P, P, c_int32, c_int32, c_int32, c_int32, c_int32, c_float,
                                    P, P, c_size_t, P]),
@@ -89,6 +88,7 @@ def _load():
         "vv_decoder_init": (S, [P, P, P, c_int64, P, c_int64, c_int64, P, P, P]),
         "vv_decoder_set_trace": (S, [P, P]),
         "vv_decoder_set_graph": (S, [P, c_int32]),
+        "vv_decoder_set_wait_limit": (S, [P, c_int64]),
         "vv_decoder_sync_status": (S, [P, P]),
         "vv_decoder_step_launches": (c_int32, [P]),
         "vv_decoder_generate": (S, [P, P, P, c_int32, POINTER(c_int32), c_int32, P,
@@ -190,20 +190,6 @@ def vv_matmul_nbits(x, q, scales, bias=None, stream=None, out=None):
     y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
     check(lib.vv_matmul_nbits(ptr(x2), ptr(q), ptr(scales), ptr(bias), M, N, K, 32, ptr(y),
                               stream_handle(stream)))
-    return y
-
-
-def vv_matmul_nbits_tc(x, q, scales, bias=None, stream=None, out=None, w_scratch=None):
-    """Tensor-core MatMulNBits for many rows: y fp16 [M, N] = x . fp16(dequant(q, scales))^T."""
-    assert x.dtype == torch.float16
-    x2 = x.reshape(-1, x.shape[-1])
-    M, K = x2.shape
-    N = q.shape[0]
-    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
-    w = w_scratch if w_scratch is not None else torch.empty((N, K), dtype=torch.float16,
-                                                            device=x.device)
-    check(lib.vv_matmul_nbits_tc(ptr(x2), ptr(q), ptr(scales), ptr(bias), M, N, K, 32, ptr(w),
-                                 ptr(y), stream_handle(stream)))
     return y
 
 

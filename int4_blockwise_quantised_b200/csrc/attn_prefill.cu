@@ -3,13 +3,27 @@
 //
 //   O[i, h] = sum_{j <= i} softmax_j(scale * Q[i, h] . K[j, g]) V[j, g]
 //
-// One CTA = 64 queries x one query head, 4 warps of 16 queries.  Key/value blocks of 64
-// positions stream global -> shared with cp.async (16-byte chunks XOR-swizzled by row so the
-// ldmatrix reads are bank-conflict free), double-buffered.  S = Q K^T and O += P V run on
-// mma.sync m16n8k16 (fp16 in, fp32 accumulate); the online softmax lives in registers (exp2 of
-// scores pre-scaled by log2 e); P is re-packed from the S accumulators into A fragments.
+// Flash attention on the 5th-generation tensor cores.  One CTA = 128 queries x one query head;
+// key/value blocks of 128 positions up to the diagonal.
+//   warp 0      : TMA producer: the Q tile once, then K and V tiles (128 x 128 fp16, 128-byte
+//                 swizzle, two 64-column boxes each) into a two-stage ring;
+//   warp 1      : allocates TMEM (two S buffers + O), one thread issues the MMAs:
+//                 S_j = Q K_j^T  (kind::f16, A = Q and B = K_j from shared memory, K-major) into
+//                 S buffer j % 2, and O += P_j V_j (A = P_j from tensor memory, B = V_j from
+//                 shared memory read MN-major, i.e. straight from the row-major cache tile);
+//   warps 2..5  : softmax, one thread per query row (TMEM lane): reads S_j, applies the scale
+//                 (log2 domain) and the causal mask, exponentiates against the row's running
+//                 maximum and writes P_j (fp16) over S_j in tensor memory; O is rescaled only when
+//                 a block's maximum exceeds the running one by more than 2^8 (the exponentials
+//                 stay below 2^8, and the final division uses the same maxima); at the end O / l
+//                 is rounded to fp16 and stored.
+// Every mbarrier wait is bounded; TMEM is released before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "vv_device.cuh"
 #include "vv_internal.h"
@@ -19,232 +33,369 @@ namespace vv {
 namespace {
 
 constexpr int D = 128;
-constexpr int QB = 64;  // queries per CTA
-constexpr int KB = 64;  // keys per block
-constexpr int kThreads = 128;
+constexpr int BQ = 128;   // queries per CTA (TMEM lanes)
+constexpr int BKV = 128;  // keys per block
+constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;  // log2 headroom before O is rescaled
+constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 tile: two 64-column atoms
+constexpr uint32_t kAtom = 128 * 128;      // 128 rows x 128 bytes
 
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {  // byte offset inside a tile
-  return (uint32_t)(row * (D * 2) + ((chunk ^ (row & 7)) << 4));
+// instruction descriptors (kind::f16, D f32, M = 128, N = 128): S (both K-major); PV (B MN-major)
+constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kIdescPV = kIdescS | (1u << 16);
+
+// K-major, 128-byte swizzle: SBO = 1024 (8 rows x 128 B)
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// MN-major, 128-byte swizzle: LBO = next 64 N-elements (the second 64-column atom), SBO = next 8
+// K-rows (1024 B)
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(kAtom >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;  // zero-fill past the end of the sequence
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-constexpr int kTile = KB * D * 2;  // 16 KB
-constexpr int kSmem = 4 * kTile;     // K and V, double-buffered
+struct Maps {
+  CUtensorMap q;   // fp16 [S, Hq * D], box {64, 128}
+  CUtensorMap kv[2];  // fp16 [Hkv][S][D] (K, V): dims {D, S, Hkv}, box {64, 128, 1}
+};
 
-__global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const AttnPrefillArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_dyn[];
-  unsigned char* sK[2] = {smem_dyn, smem_dyn + kTile};
-  unsigned char* sV[2] = {smem_dyn + 2 * kTile, smem_dyn + 3 * kTile};
-  const int qb = blockIdx.x, h = blockIdx.y;
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_prefill_tc_kernel(const __grid_constant__ Maps mp, const AttnPrefillArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = smem;
+  unsigned char* sK = smem + kTile;           // 2 stages
+  unsigned char* sV = smem + 3 * kTile;       // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTile);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* pv_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = a.Hq / a.Hkv, g = h / G;
   const int S = a.S;
-  const int q0 = qb * QB;
-  const __half* kc = reinterpret_cast<const __half*>(a.k_cache) + (size_t)g * a.cap * D;
-  const __half* vc = reinterpret_cast<const __half*>(a.v_cache) + (size_t)g * a.cap * D;
-  const float sl2 = a.scale * kLog2e;
+  const int nqb = (S + BQ - 1) / BQ;
+  // heaviest work first: block index -> (query block from the end, head)
+  const int qb = nqb - 1 - (int)blockIdx.x / a.Hq;
+  const int h = (int)blockIdx.x % a.Hq;
+  const int g = h / (a.Hq / a.Hkv);
+  const int q0 = qb * BQ;
+  const int nkb = qb + 1;  // key blocks up to the diagonal
 
-  // ---- Q fragments of this warp's 16 rows (A operand, row-major), straight from global
-  const int gq = lane >> 2, tq = lane & 3;
-  const int r_lo = q0 + warp * 16 + gq, r_hi = r_lo + 8;
-  uint32_t qf[8][4];
-  {
-    const __half* q = reinterpret_cast<const __half*>(a.q);
-    const size_t ld = (size_t)a.Hq * D;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(pv_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, kTile);
+      tma_load_2d(sQ, &mp.q, h * D, q0, q_full);
+      tma_load_2d(sQ + kAtom, &mp.q, h * D + 64, q0, q_full);
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j & 1;
+        if (j >= 2) mbar_wait(&kv_empty[st], ((j >> 1) - 1) & 1);
+        unsigned char* kt = sK + st * kTile;
+        unsigned char* vt = sV + st * kTile;
+        mbar_arrive_expect_tx(&k_full[st], kTile);
+        tma_load_3d(kt, &mp.kv[0], 0, j * BKV, g, &k_full[st]);
+        tma_load_3d(kt + kAtom, &mp.kv[0], 64, j * BKV, g, &k_full[st]);
+        mbar_arrive_expect_tx(&v_full[st], kTile);
+        tma_load_3d(vt, &mp.kv[1], 0, j * BKV, g, &v_full[st]);
+        tma_load_3d(vt + kAtom, &mp.kv[1], 64, j * BKV, g, &v_full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      mbar_wait(q_full, 0);
+      const uint32_t qa = smem_u32(sQ);
+      // S_j into buffer j % 2: 8 K-steps of 16 (32 bytes inside a 128-byte row, atom per 64)
+      auto issue_s = [&](int j) {
+        const int st = j & 1;
+        mbar_wait(&k_full[st], (j >> 1) & 1);
+        tc_after();
+        const uint32_t kb = smem_u32(sK + st * kTile);
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int c0 = ks * 16 + 2 * tq;
-      auto ld2 = [&](int r, int c) -> uint32_t {
-        if (r >= S) return 0u;
-        return *reinterpret_cast<const uint32_t*>(q + (size_t)r * ld + (size_t)h * D + c);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * kAtom + (uint32_t)(k & 3) * 32;
+          mma_ss(tS[st], desc_k_sw128(qa + off), desc_k_sw128(kb + off), kIdescS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[st]);
       };
-      qf[ks][0] = ld2(r_lo, c0);
-      qf[ks][1] = ld2(r_hi, c0);
-      qf[ks][2] = ld2(r_lo, c0 + 8);
-      qf[ks][3] = ld2(r_hi, c0 + 8);
+      issue_s(0);
+      if (nkb > 1) issue_s(1);
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j & 1;
+        mbar_wait(&p_full[st], (j >> 1) & 1);
+        mbar_wait(&v_full[st], (j >> 1) & 1);
+        tc_after();
+        const uint32_t vb = smem_u32(sV + st * kTile);
+        // O += P_j V_j: K = keys, 16 per step (8 TMEM columns of fp16 pairs; 2 x 8 rows of V)
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          mma_ts(tO, tS[st] + (uint32_t)(k * 8), desc_mn_sw128(vb + (uint32_t)k * 2048), kIdescPV,
+                 (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&kv_empty[st]);
+        mma_commit(pv_done);
+        if (j + 2 < nkb) {
+          // S_{j+2} overwrites P_j: after PV_j has read it
+          mbar_wait(pv_done, j & 1);
+          issue_s(j + 2);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // softmax / epilogue: TMEM lane quarter = warp % 4; row = query q0 + lane quarter * 32 + lane
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qi = q0 + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float c = a.scale * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < nkb; ++j) {
+      const int st = j & 1;
+      mbar_wait(&s_full[st], (j >> 1) & 1);
+      tc_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS[st] + lane_off + (uint32_t)(cc * 32), sr[cc]);
+      tmem_wait_ld();
+      const int k0 = j * BKV;
+      const bool diag = j == nkb - 1;
+      float mb = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          float v = __uint_as_float(sr[cc][t]) * c;
+          if (diag && k0 + cc * 32 + t > qi) v = -INFINITY;
+          sr[cc][t] = __float_as_uint(v);
+          mb = fmaxf(mb, v);
+        }
+      }
+      // lazy rescale: move the reference maximum only when this block's exceeds it by > 2^8
+      const bool move = mb > m_used + kRescale;
+      const float m_new = move ? mb : m_used;
+      const float corr = move ? exp2f(m_used - m_new) : 1.f;  // 0 on the first block
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // O holds sum over blocks < j: wait until PV_{j-1} has written it, then rescale
+        mbar_wait(pv_done, (j - 1) & 1);
+        tc_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + (uint32_t)(cc * 32), o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * corr);
+          tmem_st32(tO + lane_off + (uint32_t)(cc * 32), o);
+        }
+      }
+      l *= corr;
+      m_used = m_new;
+      // P_j = 2^(s - m_used) as fp16 pairs into columns 0..63 of the S buffer
+      uint32_t pp[2][32];
+      float ls = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+          const float e0 = exp2f(__uint_as_float(sr[cc][t]) - m_used);
+          const float e1 = exp2f(__uint_as_float(sr[cc][t + 1]) - m_used);
+          ls += e0 + e1;
+          pp[cc >> 1][(cc & 1) * 16 + (t >> 1)] = pack_h2(e0, e1);
+        }
+      }
+      l += ls;
+      tmem_st32(tS[st] + lane_off, pp[0]);
+      tmem_st32(tS[st] + lane_off + 32, pp[1]);
+      tmem_wait_st();
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[st]);
+    }
+    // epilogue: O / l -> fp16
+    mbar_wait(pv_done, (nkb - 1) & 1);
+    tc_after();
+    const float il = l > 0.f ? 1.f / l : 0.f;
+    __half* out = reinterpret_cast<__half*>(a.out) + (size_t)qi * a.Hq * D + (size_t)h * D;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tO + lane_off + (uint32_t)(cc * 32), o);
+      tmem_wait_ld();
+      if (qi < S) {
+#pragma unroll
+        for (int t = 0; t < 32; t += 8) {
+          uint4 v;
+          v.x = pack_h2(__uint_as_float(o[t + 0]) * il, __uint_as_float(o[t + 1]) * il);
+          v.y = pack_h2(__uint_as_float(o[t + 2]) * il, __uint_as_float(o[t + 3]) * il);
+          v.z = pack_h2(__uint_as_float(o[t + 4]) * il, __uint_as_float(o[t + 5]) * il);
+          v.w = pack_h2(__uint_as_float(o[t + 6]) * il, __uint_as_float(o[t + 7]) * il);
+          *reinterpret_cast<uint4*>(out + cc * 32 + t) = v;
+        }
+      }
     }
   }
-
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-
-  const int nkb = min((q0 + QB - 1) / KB, (S - 1) / KB) + 1;  // causal: blocks up to the diagonal
-  auto load_kv = [&](int kb, int buf) {
-    const int k0 = kb * KB;
-    for (int i = threadIdx.x; i < KB * (D / 8); i += kThreads) {
-      const int r = i >> 4, c = i & 15;
-      const bool ok = k0 + r < S;
-      const size_t off = (size_t)(ok ? k0 + r : 0) * D + c * 8;
-      cp_async16(smem_u32(sK[buf]) + swz(r, c), kc + off, ok);
-      cp_async16(smem_u32(sV[buf]) + swz(r, c), vc + off, ok);
-    }
-    cp_async_commit();
-  };
-  load_kv(0, 0);
-
-  for (int kb = 0; kb < nkb; ++kb) {
-    const int buf = kb & 1;
-    if (kb + 1 < nkb) {
-      load_kv(kb + 1, buf ^ 1);
-      cp_async_wait1();
-    } else {
-      cp_async_wait0();
-    }
-    __syncthreads();
-    const uint32_t kbase = smem_u32(sK[buf]), vbase = smem_u32(sV[buf]);
-    // ---- S = Q K^T : 16 rows x 64 keys per warp (8 n-tiles of 8 keys)
-    float sc[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-      for (int jp = 0; jp < 4; ++jp) {  // pairs of n-tiles: keys 16jp .. 16jp+15
-        // matrices: (keys 16jp+0..7, d 16ks+0..7), (same keys, d +8..15),
-        //           (keys 16jp+8..15, d 16ks+0..7), (keys +8..15, d +8..15)
-        const int mi = lane >> 3, rr = lane & 7;
-        const int key = jp * 16 + ((mi >> 1) << 3) + rr;
-        const int chunk = ks * 2 + (mi & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + swz(key, chunk), b0, b1, b2, b3);
-        mma16816(sc[2 * jp], qf[ks], b0, b1);
-        mma16816(sc[2 * jp + 1], qf[ks], b2, b3);
-      }
-    }
-    // ---- scale, causal mask, online softmax (rows lo = gq, hi = gq + 8 of this warp)
-    const int k0 = kb * KB;
-    float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = k0 + j * 8 + 2 * tq + (e & 1);
-        const int row = (e < 2) ? r_lo : r_hi;
-        float v = sc[j][e] * sl2;
-        if (key > row || key >= S) v = -INFINITY;
-        sc[j][e] = v;
-      }
-      mx_lo = fmaxf(mx_lo, fmaxf(sc[j][0], sc[j][1]));
-      mx_hi = fmaxf(mx_hi, fmaxf(sc[j][2], sc[j][3]));
-    }
-#pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
-      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
-    }
-    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-    // rows with no valid key yet keep -inf; use 0 as the reference to avoid inf - inf
-    const float ref_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
-    const float ref_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
-    const float cr_lo = exp2f(m_lo - ref_lo), cr_hi = exp2f(m_hi - ref_hi);
-    m_lo = mn_lo;
-    m_hi = mn_hi;
-    float sum_lo = 0.f, sum_hi = 0.f;
-    uint32_t pf[4][4];  // P as A fragments, 4 k-steps of 16 keys
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float p0 = exp2f(sc[j][0] - ref_lo), p1 = exp2f(sc[j][1] - ref_lo);
-      const float p2 = exp2f(sc[j][2] - ref_hi), p3 = exp2f(sc[j][3] - ref_hi);
-      sum_lo += p0 + p1;
-      sum_hi += p2 + p3;
-      const int s = j >> 1, half = j & 1;
-      pf[s][half * 2 + 0] = pack_h2(p0, p1);  // a0 / a2: row lo
-      pf[s][half * 2 + 1] = pack_h2(p2, p3);  // a1 / a3: row hi
-    }
-#pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-      sum_lo += __shfl_xor_sync(0xffffffffu, sum_lo, off);
-      sum_hi += __shfl_xor_sync(0xffffffffu, sum_hi, off);
-    }
-    l_lo = l_lo * cr_lo + sum_lo;
-    l_hi = l_hi * cr_hi + sum_hi;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= cr_lo;
-      o[i][1] *= cr_lo;
-      o[i][2] *= cr_hi;
-      o[i][3] *= cr_hi;
-    }
-    // ---- O += P V : 16 d n-tiles of 8, 4 key k-steps of 16
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-#pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {  // pairs of d n-tiles: d 16dp .. 16dp+15
-        // .trans matrices: (keys 16s+0..7, d 16dp+0..7), (keys 16s+8..15, d 16dp+0..7),
-        //                  (keys 16s+0..7, d 16dp+8..15), (keys +8..15, d +8..15)
-        const int mi = lane >> 3, rr = lane & 7;
-        const int key = s * 16 + ((mi & 1) << 3) + rr;
-        const int chunk = dp * 2 + (mi >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vbase + swz(key, chunk), b0, b1, b2, b3);
-        mma16816(o[2 * dp], pf[s], b0, b1);
-        mma16816(o[2 * dp + 1], pf[s], b2, b3);
-      }
-    }
-    __syncthreads();  // buffer `buf` is reloaded two iterations later
-  }
-  // ---- normalise and store O [S, Hq * D] fp16
-  const float il_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, il_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
-  __half* out = reinterpret_cast<__half*>(a.out);
-  const size_t ld = (size_t)a.Hq * D;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int d = i * 8 + 2 * tq;
-    if (r_lo < S)
-      *reinterpret_cast<uint32_t*>(out + (size_t)r_lo * ld + (size_t)h * D + d) =
-          pack_h2(o[i][0] * il_lo, o[i][1] * il_lo);
-    if (r_hi < S)
-      *reinterpret_cast<uint32_t*>(out + (size_t)r_hi * ld + (size_t)h * D + d) =
-          pack_h2(o[i][2] * il_hi, o[i][3] * il_hi);
+  tc_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
   }
 }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+constexpr size_t kSmem = 5 * kTile + 16 * 8 + 1024;
 
 }  // namespace
 
 cudaError_t launch_attn_prefill(const AttnPrefillArgs& a, cudaStream_t s) {
-  cudaError_t e =
-      cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  auto fn = encode_fn();
+  if (!fn || a.S < 1 || a.Hq % a.Hkv != 0) return cudaErrorInvalidValue;
+  Maps mp;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.Hq * D, (cuuint64_t)a.S};
+    cuuint64_t strides[1] = {(cuuint64_t)a.Hq * D * 2};
+    cuuint32_t box[2] = {64, BQ};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&mp.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  for (int t = 0; t < 2; ++t) {
+    // rows past S read as zeros (the cache may hold anything there)
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.S, (cuuint64_t)a.Hkv};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.cap * D * 2};
+    cuuint32_t box[3] = {64, BKV, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const uint16_t* base = t == 0 ? a.k_cache : a.v_cache;
+    if (fn(&mp.kv[t], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims,
+           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.S + QB - 1) / QB, a.Hq);
-  attn_prefill_kernel<<<grid, kThreads, kSmem, s>>>(a);
+  const int nqb = (a.S + BQ - 1) / BQ;
+  attn_prefill_tc_kernel<<<nqb * a.Hq, kThreads, kSmem, s>>>(mp, a);
   return cudaGetLastError();
 }
 

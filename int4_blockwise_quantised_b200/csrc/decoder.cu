@@ -176,6 +176,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
     p.length = d->d_length;
     p.bar_count = reinterpret_cast<unsigned*>(b + o_bar);
     p.grid = grid;
+    p.wait_ns = vv::kWaitLimitNs;
     p.nstages = 4;
     p.stage_bytes = 0;
     const size_t fixed = vv::step_smem_bytes(p);
@@ -278,6 +279,18 @@ int32_t vv_decoder_length(const vv_decoder* d) { return d ? d->len_host : -1; }
 vv_status vv_decoder_set_trace(vv_decoder* d, float* layer_out) {
   VV_CHECK_ARG(d, "null decoder");
   d->trace = layer_out;
+  return VV_OK;
+}
+
+vv_status vv_decoder_set_wait_limit(vv_decoder* d, int64_t limit_ns) {
+  VV_CHECK_ARG(d, "null decoder");
+  VV_CHECK_ARG(limit_ns >= 100000 && limit_ns <= 10000000000ll,
+               "vv_decoder_set_wait_limit: %lld ns (1e5 .. 1e10)", (long long)limit_ns);
+  d->step.wait_ns = (uint64_t)limit_ns;
+  if (d->gexec) {  // the captured graph holds the old parameters
+    cudaGraphExecDestroy(d->gexec);
+    d->gexec = nullptr;
+  }
   return VV_OK;
 }
 

@@ -268,6 +268,243 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------- packed int4 B operand
+// The same GEMM with B given as MatMulNBits codes + fp16 scales (up to three row segments of one
+// matrix stack, or two segments interleaved row by row): the int4 weights are dequantised into
+// the fp16 B tile in shared memory, never written to global memory.
+//   warp 0      : TMA producer: per 64-wide k block, the A tile (fp16 128 x 64), the codes
+//                 (BN rows x 32 bytes) and the scales (BN rows x 8 blocks, the 256-wide group
+//                 holding this k block) into a ring of raw stages;
+//   warp 1      : TMEM allocation, one thread issues tcgen05.mma kind::f16 from the A stage and
+//                 the converted B stage; commits release both;
+//   warps 2..5  : epilogue (as above);
+//   warps 6..9  : converters: codes + scale -> fp16((code - 8) * scale) (one rounding, as the
+//                 fp32 product rounded to fp16) written in the 128-byte-swizzled K-major layout
+//                 of a B stage (a second, smaller ring).
+constexpr int kQThreads = 320;
+template <int BN>
+struct QCfg {
+  static constexpr uint32_t kCodes = BN * 32;     // codes of one k block (64 columns)
+  static constexpr uint32_t kScales = BN * 16;    // scales of 8 blocks (256 columns)
+  static constexpr uint32_t kRaw = kStageA + kCodes + kScales;
+  static constexpr int kRawStages = 4;
+  static constexpr uint32_t kStageB = BN * BK * 2;
+  static constexpr int kBStages = 2;
+  static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;
+  static constexpr uint32_t kIdesc = Cfg<BN>::kIdesc;
+};
+
+struct PackedMaps {
+  CUtensorMap q[3];  // uint8 [rows_m, K/2], box {32, BN (or BN/2 interleaved)}
+  CUtensorMap s[3];  // fp16 [rows_m, K/32], box {8, BN (or BN/2)}
+  int row0[4];       // first output row of each segment (non-interleaved), row0[nseg] = N
+  int nseg;
+  int interleave;
+};
+
+__device__ __forceinline__ void tma_load_2d_u(void* dst, const CUtensorMap* tm, int c0, int c1,
+                                              uint64_t* bar) {
+  tma_load_2d(dst, tm, c0, c1, bar);
+}
+
+// (code - 8) * scale for the 8 elements of one code word, natural order, as 4 fp16 pairs.
+__device__ __forceinline__ uint4 dequant8_f16(uint32_t w, uint32_t s2) {
+  uint32_t o[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    uint32_t y, h, d;
+    // byte t of w into bytes 0 and 2; low nibble -> low half, high nibble -> high half mantissa
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(w), "r"((uint32_t)(t | 0x40 | (t << 8) | 0x4000)));
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(y), "r"(0x00F0000Fu), "r"(0x64006400u));
+    // (1024 + c) - 1032 = c - 8; (1024 + 16 c) / 16 - 72 = c - 8  (exact in fp16)
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(h), "r"(0x2C003C00u), "r"(0xD480E408u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[t]) : "r"(d), "r"(s2));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int EPI, int BN>
+__global__ void __launch_bounds__(kQThreads, 1)
+    gemm_q4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ PackedMaps pm,
+                   const GemmEpilogue e, const int M, const int N, const int K) {
+  using C = QCfg<BN>;
+  constexpr int RS = C::kRawStages, BS = C::kBStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sB = smem;                       // BS x kStageB (1024-aligned)
+  unsigned char* sRaw = smem + BS * C::kStageB;    // RS x kRaw (A first: 1024-aligned)
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(sRaw + RS * C::kRaw);
+  uint64_t* raw_empty = raw_full + RS;
+  uint64_t* b_full = raw_empty + RS;
+  uint64_t* b_empty = b_full + BS;
+  uint64_t* acc_full = b_empty + BS;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = N / BN;
+  const int tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int kblocks = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < RS; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 1 + 4);  // the MMA commit (A read) + 4 converter warps (codes)
+    }
+    for (int i = 0; i < BS; ++i) {
+      mbar_init(&b_full[i], 4);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+        const int n0 = n_blk * BN;
+        // segment and its first row of this tile (tiles never straddle segments)
+        int sg = 0, r0 = 0;
+        if (!pm.interleave) {
+          while (sg + 1 < pm.nseg && n0 >= pm.row0[sg + 1]) ++sg;
+          r0 = n0 - pm.row0[sg];
+        } else {
+          r0 = n0 / 2;
+        }
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % RS;
+          if (g >= RS) mbar_wait(&raw_empty[s], ((g / RS) - 1) & 1);
+          mbar_arrive_expect_tx(&raw_full[s], C::kRaw);
+          unsigned char* st = sRaw + s * C::kRaw;
+          tma_load_2d(st, &tmA, kb * BK, m_blk * BM, &raw_full[s]);
+          const int sx = (kb * 2) & ~7;  // first of the 8 scale blocks holding this k block
+          if (!pm.interleave) {
+            tma_load_2d(st + kStageA, &pm.q[sg], kb * 32, r0, &raw_full[s]);
+            tma_load_2d(st + kStageA + C::kCodes, &pm.s[sg], sx, r0, &raw_full[s]);
+          } else {
+            tma_load_2d(st + kStageA, &pm.q[0], kb * 32, r0, &raw_full[s]);
+            tma_load_2d(st + kStageA + C::kCodes / 2, &pm.q[1], kb * 32, r0, &raw_full[s]);
+            tma_load_2d(st + kStageA + C::kCodes, &pm.s[0], sx, r0, &raw_full[s]);
+            tma_load_2d(st + kStageA + C::kCodes + C::kScales / 2, &pm.s[1], sx, r0, &raw_full[s]);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int g = 0, i = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2) mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1);
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % RS, sb = g % BS;
+          mbar_wait(&raw_full[s], (g / RS) & 1);
+          mbar_wait(&b_full[sb], (g / BS) & 1);
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sRaw + s * C::kRaw), b0 = smem_u32(sB + sb * C::kStageB);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), C::kIdesc,
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&raw_empty[s]);
+          umma_commit(&b_empty[sb]);
+        }
+        umma_commit(&acc_full[buf]);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    const int q = warp & 3;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+      const int buf = i & 1;
+      const int row = m_blk * BM + q * 32 + lane;
+      mbar_wait(&acc_full[buf], (i >> 1) & 1);
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(base + (uint32_t)c, v);
+        if (row < M) epilogue_chunk<EPI, BN>(e, v, row, n_blk * BN + c);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  } else {
+    // converters: thread ct owns B rows ct, ct + 128 (< BN)
+    const int ct = threadIdx.x - 6 * 32;
+    int g = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb, ++g) {
+        const int s = g % RS, sb = g % BS;
+        mbar_wait(&raw_full[s], (g / RS) & 1);
+        if (g >= BS) mbar_wait(&b_empty[sb], ((g / BS) - 1) & 1);
+        const unsigned char* codes = sRaw + s * C::kRaw + kStageA;
+        const __half* scl = reinterpret_cast<const __half*>(codes + C::kCodes);
+        unsigned char* bt = sB + sb * C::kStageB;
+        const int sj = (kb * 2) & 7;  // this k block's first scale within the 8 loaded
+#pragma unroll
+        for (int rr = 0; rr < (BN + 127) / 128; ++rr) {
+          const int n = ct + rr * 128;
+          if (n < BN) {
+            // source row of output row n in the codes / scales tiles
+            const int src = pm.interleave ? (n & 1) * (BN / 2) + (n >> 1) : n;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint4 cw = *reinterpret_cast<const uint4*>(codes + src * 32 + j * 16);
+              const uint16_t sh = reinterpret_cast<const uint16_t*>(scl)[src * 8 + sj + j];
+              const uint32_t s2 = (uint32_t)sh | ((uint32_t)sh << 16);
+              const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int chunk = 4 * j + c;  // 16-byte chunk of the 128-byte row
+                *reinterpret_cast<uint4*>(bt + n * 128 + ((chunk ^ (n & 7)) << 4)) =
+                    dequant8_f16(w4[c], s2);
+              }
+            }
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&b_full[sb]);
+          mbar_arrive(&raw_empty[s]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------------------ tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -381,13 +618,119 @@ cudaError_t launch_bn(const uint16_t* A, const uint16_t* B, int M, int N, int K,
 
 }  // namespace
 
-size_t gemm_tc_smem() { return smem_bytes<256>(); }
-
 // Wave efficiency of a tile count on the SMs: tiles / (waves * SMs).
 static double wave_eff(long tiles, int sms) {
   const long waves = (tiles + sms - 1) / sms;
   return (double)tiles / (double)(waves * sms);
 }
+
+namespace {
+
+// Generic 2D tensor map: [rows, cols] of `dtype` elements of `esize` bytes, box {bc, br}.
+bool make_map2(CUtensorMap* tm, CUtensorMapDataType dtype, int esize, const void* base, int rows,
+               int cols, int bc, int br) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+  cuuint32_t box[2] = {(cuuint32_t)bc, (cuuint32_t)br};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+size_t q4_smem_bytes() {
+  using C = QCfg<BN>;
+  return C::kBStages * C::kStageB + C::kRawStages * C::kRaw + (2 * C::kRawStages + 2 * C::kBStages + 4) * 8 +
+         16 + 1024;
+}
+
+template <int EPI, int BN>
+cudaError_t run_q4(const CUtensorMap& ta, const PackedMaps& pm, const GemmEpilogue& e, int M,
+                   int N, int K, int grid, cudaStream_t s) {
+  const size_t smem = q4_smem_bytes<BN>();
+  cudaError_t err = cudaFuncSetAttribute(gemm_q4_kernel<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  gemm_q4_kernel<EPI, BN><<<grid, kQThreads, smem, s>>>(ta, pm, e, M, N, K);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_q4_bn(const uint16_t* A, const PackedB& B, int M, int N, int K, int epi,
+                         const GemmEpilogue& e, cudaStream_t s) {
+  CUtensorMap ta;
+  if (!make_map(&ta, A, M, K, BM)) return cudaErrorInvalidValue;
+  PackedMaps pm = {};
+  pm.nseg = B.nseg;
+  pm.interleave = B.interleave;
+  const int br = B.interleave ? BN / 2 : BN;
+  int r = 0;
+  for (int g = 0; g < B.nseg; ++g) {
+    if (!make_map2(&pm.q[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B.q[g], B.rows[g], K / 2, 32, br) ||
+        !make_map2(&pm.s[g], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, B.s[g], B.rows[g], K / 32, 8, br))
+      return cudaErrorInvalidValue;
+    pm.row0[g] = r;
+    r += B.rows[g];
+  }
+  pm.row0[B.nseg] = r;
+  const int tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  switch (epi) {
+    case kEpiBias: return run_q4<kEpiBias, BN>(ta, pm, e, M, N, K, grid, s);
+    case kEpiResid: return run_q4<kEpiResid, BN>(ta, pm, e, M, N, K, grid, s);
+    case kEpiSwiglu: return run_q4<kEpiSwiglu, BN>(ta, pm, e, M, N, K, grid, s);
+    case kEpiF16: return run_q4<kEpiF16, BN>(ta, pm, e, M, N, K, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+bool gemm_q4_supported(const PackedB& B, int N, int K) {
+  if (K < 256 || K % 256 != 0 || B.nseg < 1 || B.nseg > 3) return false;
+  if (B.interleave) return B.nseg == 2 && B.rows[0] == B.rows[1] && N == 2 * B.rows[0] && N % 128 == 0;
+  int tot = 0;
+  for (int g = 0; g < B.nseg; ++g) {
+    if (B.rows[g] % 128 != 0) return false;
+    tot += B.rows[g];
+  }
+  return tot == N;
+}
+
+cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s) {
+  if (M < 1 || !gemm_q4_supported(B, N, K) || !aligned16(A)) return cudaErrorInvalidValue;
+  for (int g = 0; g < B.nseg; ++g)
+    if (!aligned16(B.q[g]) || !aligned16(B.s[g])) return cudaErrorInvalidValue;
+  const int sms = sm_count();
+  const long mt = (M + BM - 1) / BM;
+  // tile width: segments (or interleaved pairs) must hold whole tiles; among the widths that
+  // fit, the widest whose wave efficiency is within 0.1 of the best
+  auto fits = [&](int w) {
+    if (N % w != 0) return false;
+    if (B.interleave) return (w / 2) % 8 == 0;
+    for (int g = 0; g < B.nseg; ++g)
+      if (B.rows[g] % w != 0) return false;
+    return true;
+  };
+  const int widths[3] = {256, 192, 128};
+  double best = 0.0;
+  for (int w : widths)
+    if (fits(w)) best = std::max(best, wave_eff(mt * (N / w), sms));
+  for (int w : widths) {
+    if (!fits(w) || wave_eff(mt * (N / w), sms) < best - 0.1) continue;
+    if (w == 256) return launch_q4_bn<256>(A, B, M, N, K, epi, e, s);
+    if (w == 192) return launch_q4_bn<192>(A, B, M, N, K, epi, e, s);
+    return launch_q4_bn<128>(A, B, M, N, K, epi, e, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t gemm_tc_smem() { return smem_bytes<256>(); }
+
 
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
@@ -410,34 +753,3 @@ cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, i
 }
 
 }  // namespace vv
-
-extern "C" vv_status vv_matmul_nbits_tc(const uint16_t* x, const uint8_t* q,
-                                        const uint16_t* scales, const uint16_t* bias, int64_t M,
-                                        int64_t N, int64_t K, int32_t block, uint16_t* w_f16,
-                                        uint16_t* y, vv_stream stream) {
-  VV_CHECK_ARG(x && q && scales && w_f16 && y, "vv_matmul_nbits_tc: null pointer");
-  VV_CHECK_ARG(vv::aligned16(x) && vv::aligned16(q) && vv::aligned16(scales) &&
-                   vv::aligned16(w_f16) && vv::aligned16(y) && (!bias || vv::aligned16(bias)),
-               "vv_matmul_nbits_tc: pointers must be 16-byte aligned");
-  VV_CHECK_SHAPE(block == 32, "vv_matmul_nbits_tc: block %d (only 32)", block);
-  VV_CHECK_SHAPE(K >= 64 && K % 64 == 0 && K < (1 << 24), "vv_matmul_nbits_tc: K=%lld",
-                 (long long)K);
-  VV_CHECK_SHAPE(N >= 128 && (N % 128 == 0 || N % 192 == 0) && N < (1 << 24),
-                 "vv_matmul_nbits_tc: N=%lld",
-                 (long long)N);
-  VV_CHECK_SHAPE(M >= 1 && M < (1 << 24), "vv_matmul_nbits_tc: M=%lld", (long long)M);
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  vv::DequantSrc src = {};
-  src.q[0] = q;
-  src.s[0] = scales;
-  src.rows[0] = (int)N;
-  src.nseg = 1;
-  __half* w = reinterpret_cast<__half*>(w_f16);
-  VV_CUDA(vv::launch_dequant_f16(src, (int)N, (int)K, w, s));
-  vv::GemmEpilogue e = {};
-  e.out_f16 = reinterpret_cast<__half*>(y);
-  e.bias = reinterpret_cast<const __half*>(bias);
-  e.ldo = (int)N;
-  VV_CUDA(vv::launch_gemm_tc(x, w_f16, (int)M, (int)N, (int)K, vv::kEpiF16, e, s));
-  return VV_OK;
-}

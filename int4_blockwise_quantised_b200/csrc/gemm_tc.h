@@ -37,4 +37,18 @@ struct DequantSrc {
 cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
                                cudaStream_t s);
 
+// B operand as packed MatMulNBits matrices, dequantised inside the GEMM (no fp16 copy in global
+// memory): up to three row segments (N = sum of rows, each a multiple of 128), or two segments
+// of equal rows interleaved row by row (interleave = 1, N = 2 * rows).  K % 256 == 0.
+struct PackedB {
+  const uint8_t* q[3];
+  const uint16_t* s[3];
+  int rows[3];
+  int nseg;
+  int interleave;
+};
+bool gemm_q4_supported(const PackedB& B, int N, int K);
+cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s);
+
 }  // namespace vv

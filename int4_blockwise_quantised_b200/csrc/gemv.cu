@@ -25,6 +25,7 @@
 
 #include "vv_device.cuh"
 #include "vv_internal.h"
+#include "gemm_tc.h"
 
 namespace vv {
 namespace {
@@ -411,9 +412,25 @@ extern "C" vv_status vv_matmul_nbits(const uint16_t* x, const uint8_t* q, const 
   VV_CHECK_SHAPE(block == 32, "vv_matmul_nbits: block %d (only 32)", block);
   VV_CHECK_SHAPE(K >= 32 && K % 32 == 0 && K < (1 << 30), "vv_matmul_nbits: K=%lld", (long long)K);
   VV_CHECK_SHAPE(N >= 1 && N < (1 << 30), "vv_matmul_nbits: N=%lld", (long long)N);
-  VV_CHECK_SHAPE(M >= 1 && M <= 8, "vv_matmul_nbits: M=%lld (1..8)", (long long)M);
-  return vv::cuda_check(
-      vv::launch_matmul_nbits_gemv(x, vv::GemvWeights{q, scales}, bias, (int)M, (int)N, (int)K, y,
-                                   static_cast<cudaStream_t>(stream)),
-      "matmul_nbits launch");
+  VV_CHECK_SHAPE(M >= 1 && M < (1 << 24), "vv_matmul_nbits: M=%lld", (long long)M);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= 8)
+    return vv::cuda_check(vv::launch_matmul_nbits_gemv(x, vv::GemvWeights{q, scales}, bias, (int)M,
+                                                       (int)N, (int)K, y, s),
+                          "matmul_nbits GEMV launch");
+  // many rows: tcgen05 GEMM with the int4 operand dequantised in shared memory
+  vv::PackedB pb = {};
+  pb.q[0] = q;
+  pb.s[0] = scales;
+  pb.rows[0] = (int)N;
+  pb.nseg = 1;
+  VV_CHECK_SHAPE(vv::gemm_q4_supported(pb, (int)N, (int)K),
+                 "vv_matmul_nbits: M=%lld > 8 needs N %% 128 == 0 and K %% 256 == 0 (N=%lld K=%lld)",
+                 (long long)M, (long long)N, (long long)K);
+  vv::GemmEpilogue e = {};
+  e.out_f16 = reinterpret_cast<__half*>(y);
+  e.bias = reinterpret_cast<const __half*>(bias);
+  e.ldo = (int)N;
+  return vv::cuda_check(vv::launch_gemm_q4(x, pb, (int)M, (int)N, (int)K, vv::kEpiF16, e, s),
+                        "matmul_nbits tensor-core launch");
 }

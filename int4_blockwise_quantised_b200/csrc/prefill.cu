@@ -10,8 +10,9 @@
 //   X  += O . Wo^T                                    tcgen05 GEMM, residual epilogue
 //   Hm  = silu(Xn Wg^T) * (Xn Wu^T), Xn = RMSNorm(X)  tcgen05 GEMM over interleaved gate/up rows
 //   X  += Hm . Wd^T                                   tcgen05 GEMM, residual epilogue
-// Each packed int4 matrix is first dequantised to an fp16 copy ((code - 8) * scale, rounded once)
-// in a reused workspace buffer.  The last row then goes through the final RMSNorm + lm_head.
+// The GEMMs read the packed int4 matrices as they are: converter warps inside the GEMM expand each
+// 64-column block of codes to fp16 ((code - 8) * scale, rounded once) in shared memory, right
+// before the tensor cores read it.  The last row then goes through the final RMSNorm + lm_head.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -172,11 +173,6 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   const size_t o_qkv = take((size_t)SM * NQKV * 4);
   const size_t o_q = take((size_t)SM * HQD * 2);
   const size_t o_h = take((size_t)SM * I * 2);
-  size_t wmax = (size_t)NQKV * H;
-  if ((size_t)2 * I * H > wmax) wmax = (size_t)2 * I * H;
-  if ((size_t)H * I > wmax) wmax = (size_t)H * I;
-  if ((size_t)H * HQD > wmax) wmax = (size_t)H * HQD;
-  const size_t o_w = take(wmax * 2);
   const size_t o_bias = take((size_t)NQKV * 2);
   const size_t need = off_b;
   if (d->pws_bytes < need) {
@@ -193,7 +189,6 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   float* QKV = reinterpret_cast<float*>(b + o_qkv);
   __half* Q = reinterpret_cast<__half*>(b + o_q);
   __half* Hm = reinterpret_cast<__half*>(b + o_h);
-  __half* W = reinterpret_cast<__half*>(b + o_w);
   __half* Bqkv = reinterpret_cast<__half*>(b + o_bias);
   const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
   cudaError_t e;
@@ -210,13 +205,11 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     // ---- QKV
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.input_norm), c.eps, Xn);
     VV_MARK(kPfMisc);
-    DequantSrc dq = {};
-    dq.q[0] = w.wq.q; dq.s[0] = w.wq.scales; dq.rows[0] = HQD;
-    dq.q[1] = w.wk.q; dq.s[1] = w.wk.scales; dq.rows[1] = Hkv * D;
-    dq.q[2] = w.wv.q; dq.s[2] = w.wv.scales; dq.rows[2] = Hkv * D;
-    dq.nseg = 3;
-    if ((e = launch_dequant_f16(dq, NQKV, H, W, s)) != cudaSuccess) return e;
-    VV_MARK(kPfDequant);
+    PackedB pb = {};
+    pb.q[0] = w.wq.q; pb.s[0] = w.wq.scales; pb.rows[0] = HQD;
+    pb.q[1] = w.wk.q; pb.s[1] = w.wk.scales; pb.rows[1] = Hkv * D;
+    pb.q[2] = w.wv.q; pb.s[2] = w.wv.scales; pb.rows[2] = Hkv * D;
+    pb.nseg = 3;
     const uint16_t* bsrc[3] = {w.bq, w.bk, w.bv};
     const int brows[3] = {HQD, Hkv * D, Hkv * D};
     int boff = 0;
@@ -233,8 +226,8 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     ep.out_f32 = QKV;
     ep.bias = Bqkv;
     ep.ldo = NQKV;
-    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
-                            S, NQKV, H, kEpiBias, ep, s)) != cudaSuccess)
+    if ((e = launch_gemm_q4(reinterpret_cast<const uint16_t*>(Xn), pb, S, NQKV, H, kEpiBias, ep,
+                            s)) != cudaSuccess)
       return e;
     VV_MARK(kPfGemm);
     rope_kv_kernel<<<S, 256, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
@@ -254,46 +247,40 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     if ((e = launch_attn_prefill(aa, s)) != cudaSuccess) return e;
     VV_MARK(kPfAttn);
     // ---- O projection + residual
-    dq = {};
-    dq.q[0] = w.wo.q; dq.s[0] = w.wo.scales; dq.rows[0] = H;
-    dq.nseg = 1;
-    if ((e = launch_dequant_f16(dq, H, HQD, W, s)) != cudaSuccess) return e;
-    VV_MARK(kPfDequant);
+    pb = {};
+    pb.q[0] = w.wo.q; pb.s[0] = w.wo.scales; pb.rows[0] = H;
+    pb.nseg = 1;
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;
-    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
-                            S, H, HQD, kEpiResid, ep, s)) != cudaSuccess)
+    if ((e = launch_gemm_q4(reinterpret_cast<const uint16_t*>(Xn), pb, S, H, HQD, kEpiResid, ep,
+                            s)) != cudaSuccess)
       return e;
     VV_MARK(kPfGemm);
     // ---- gate/up + SwiGLU
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.post_norm), c.eps, Xn);
     VV_MARK(kPfMisc);
-    dq = {};
-    dq.q[0] = w.wgate.q; dq.s[0] = w.wgate.scales; dq.rows[0] = I;
-    dq.q[1] = w.wup.q; dq.s[1] = w.wup.scales; dq.rows[1] = I;
-    dq.nseg = 2;
-    dq.interleave = 1;
-    if ((e = launch_dequant_f16(dq, 2 * I, H, W, s)) != cudaSuccess) return e;
-    VV_MARK(kPfDequant);
+    pb = {};
+    pb.q[0] = w.wgate.q; pb.s[0] = w.wgate.scales; pb.rows[0] = I;
+    pb.q[1] = w.wup.q; pb.s[1] = w.wup.scales; pb.rows[1] = I;
+    pb.nseg = 2;
+    pb.interleave = 1;
     ep = {};
     ep.out_f16 = Hm;
     ep.ldo = I;
-    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Xn), reinterpret_cast<const uint16_t*>(W),
-                            S, 2 * I, H, kEpiSwiglu, ep, s)) != cudaSuccess)
+    if ((e = launch_gemm_q4(reinterpret_cast<const uint16_t*>(Xn), pb, S, 2 * I, H, kEpiSwiglu, ep,
+                            s)) != cudaSuccess)
       return e;
     VV_MARK(kPfGemm);
     // ---- down + residual
-    dq = {};
-    dq.q[0] = w.wdown.q; dq.s[0] = w.wdown.scales; dq.rows[0] = H;
-    dq.nseg = 1;
-    if ((e = launch_dequant_f16(dq, H, I, W, s)) != cudaSuccess) return e;
-    VV_MARK(kPfDequant);
+    pb = {};
+    pb.q[0] = w.wdown.q; pb.s[0] = w.wdown.scales; pb.rows[0] = H;
+    pb.nseg = 1;
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;
-    if ((e = launch_gemm_tc(reinterpret_cast<const uint16_t*>(Hm), reinterpret_cast<const uint16_t*>(W),
-                            S, H, I, kEpiResid, ep, s)) != cudaSuccess)
+    if ((e = launch_gemm_q4(reinterpret_cast<const uint16_t*>(Hm), pb, S, H, I, kEpiResid, ep,
+                            s)) != cudaSuccess)
       return e;
     VV_MARK(kPfGemm);
     if (d->trace) {

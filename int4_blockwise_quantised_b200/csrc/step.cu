@@ -115,7 +115,7 @@ __device__ void grid_barrier(const StepParams& p, unsigned& nbar, int& sk) {
   stamp(p, sk);
   if (threadIdx.x == 0) {
     red_release_add(p.bar_count, 1u);
-    wait_counter_geq(p.bar_count, (nbar + 1) * gridDim.x);
+    wait_counter_geq(p.bar_count, (nbar + 1) * gridDim.x, p.wait_ns);
   }
   ++nbar;
   stamp(p, sk);
@@ -125,6 +125,7 @@ __device__ void grid_barrier(const StepParams& p, unsigned& nbar, int& sk) {
 // ------------------------------------------------------------------------------ stage ring
 struct Ring {
   uint64_t wait_ns;  // time this thread spent blocked in ring waits (timeline tap)
+  uint64_t wait_limit;  // bound of every wait (StepParams::wait_ns)
   unsigned char* base;
   uint64_t* full;
   uint64_t* empty;
@@ -144,7 +145,7 @@ struct Copy {
 __device__ __forceinline__ void ring_wait(Ring& r, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
-  mbar_wait(bar, parity);
+  mbar_wait(bar, parity, r.wait_limit);
   const uint64_t dt = globaltimer_ns() - t0;
   r.wait_ns += dt;
   if (r.tapw) r.tapw[r.ph] += dt;
@@ -159,7 +160,7 @@ __device__ __forceinline__ void producer_wait(Ring& r, uint64_t* bar, uint32_t p
   for (unsigned it = 1;; ++it) {
     __nanosleep(256);
     if (mbar_try_wait(bar, parity)) break;
-    if ((it & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63) == 0 && wait_expired(t0, r.wait_limit)) {
       set_device_error(VV_ERR_TIMEOUT);
       break;
     }
@@ -373,11 +374,17 @@ __device__ void stage_idp(const XOp& xo, Load load, const __half* gamma, float e
   constexpr int kC = 4;  // chunks of 4 per thread
   const int NHB = K >> 4;
   float4 v[kC];
+  uint2 gv[kC];  // gamma halves, loaded with x so that both arrive in one round trip
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < kC; ++i) {
     const int k = (tid + i * NT) * 4;
+    if (gamma && k < K) gv[i] = *reinterpret_cast<const uint2*>(gamma + k);
     v[i] = k < K ? load(k) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < kC; ++i) {
+    const int k = (tid + i * NT) * 4;
     if (k < K && copy_out) *reinterpret_cast<float4*>(copy_out + k) = v[i];
     ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
@@ -393,9 +400,8 @@ __device__ void stage_idp(const XOp& xo, Load load, const __half* gamma, float e
     for (int i = 0; i < kC; ++i) {
       const int k = (tid + i * NT) * 4;
       if (k < K) {
-        const uint2 gv = *reinterpret_cast<const uint2*>(gamma + k);
-        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&gv.x));
-        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&gv.y));
+        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].x));
+        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&gv[i].y));
         v[i].x *= inv * g01.x;
         v[i].y *= inv * g01.y;
         v[i].z *= inv * g23.x;
@@ -441,7 +447,10 @@ __device__ __forceinline__ void idp_pass(const XOp& xo, int NHB, int units, RowQ
   constexpr int GPW = 32 / LPR;  // unit groups per warp
   const int sub = lane % LPR, grp = lane / LPR;
   const uint4* xq = xo.xq;
-  for (int u0 = (warp * GPW + grp) * R; u0 < units; u0 += NW * GPW * R) {
+  // the loop bound is warp-uniform (every lane runs the same iterations, as the full-mask
+  // shuffles below require); lane groups past the last unit work on a clamped row and skip fin
+  for (int ub = warp * GPW * R; ub < units; ub += NW * GPW * R) {
+    const int u0 = ub + grp * R;
     const unsigned char* q[R];
     const __half* sc[R];
 #pragma unroll
@@ -753,6 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   const int H = p.H, Hq = p.Hq, Hkv = p.Hkv;
   Ring r;
   r.wait_ns = 0;
+  r.wait_limit = p.wait_ns;
   r.ph = 0;
   // timeline tap: the last 8 stamps of a CTA's row hold thread 0's ring wait per phase kind
   // (QKV, ATTN, O, GU, DOWN, HEAD at max-8 .. max-3), then the producer's done time and its
@@ -870,6 +880,20 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     const StepLayer& w = p.layers[l];
     // ---------------------------------------------------------------- QKV
     r.ph = 0;
+    int r0, r1;
+    cta_range(nqkv, cta, ncta, r0, r1);
+    // this CTA's q/k/v biases -> shared memory before the barrier (they do not depend on x;
+    // as.q is free until the attention phase; stage_idp's barriers order the stores)
+    {
+      const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
+      float* bias_s = &as.q[0][0];
+      for (int i = tid; i < r1 - r0; i += NT) {
+        const int row = r0 + i;
+        const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
+        const __half* b = w.bias[m];
+        bias_s[i] = b ? __half2float(b[row - bounds[m]]) : 0.f;
+      }
+    }
     if (l == 0) {
       stage_idp(xo, load_emb, w.in_norm, p.eps, H, red, nullptr);
     } else {
@@ -879,19 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     }
     stamp(p, sk);
     {
-      int r0, r1;
-      cta_range(nqkv, cta, ncta, r0, r1);
-      const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
-      // this CTA's q/k/v biases -> shared memory (as.q is free until the attention phase)
-      float* bias_s = &as.q[0][0];
-      for (int i = tid; i < r1 - r0; i += NT) {
-        const int row = r0 + i;
-        const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
-        const __half* b = w.bias[m];
-        bias_s[i] = b ? __half2float(b[row - bounds[m]]) : 0.f;
-      }
-      cbar();
-      const float* bs = bias_s - r0;
+      const float* bs = &as.q[0][0] - r0;
       consume_rows<false>(r, xo, H, r0, r1, 1,
                           [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
     }

@@ -63,6 +63,7 @@ struct StepParams {
   int32_t* gen_pos;
   int32_t stop_ids[8];
   int n_stop;
+  uint64_t wait_ns;   // bound of every device-side wait (ns)
   uint64_t* stamps;   // timeline tap [grid][max_stamps] (globaltimer ns) or nullptr
   int max_stamps;
   // launch shape

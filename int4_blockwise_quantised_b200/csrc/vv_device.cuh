@@ -29,8 +29,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Limit for any single wait: far above any legitimate wait inside one kernel.
+// Default limit for any single wait: far above any legitimate wait inside one kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// A wait gives up once its own limit has passed, or as soon as another wait anywhere on the
+// device has already timed out (so a kernel whose schedule went wrong finishes quickly instead
+// of letting every later wait run out its own limit).
+__device__ __forceinline__ bool wait_expired(uint64_t t0, uint64_t limit_ns) {
+  if (globaltimer_ns() - t0 > limit_ns) return true;
+  return *reinterpret_cast<volatile int*>(&g_device_error) == VV_ERR_TIMEOUT;
+}
 
 // ----------------------------------------------------------------------------------------------
 // Programmatic dependent launch (PDL).  griddepcontrol.wait blocks until the preceding kernel in
@@ -102,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait_hint(bar, parity, 20000u)) {
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (wait_expired(t0, limit_ns)) {
       set_device_error(VV_ERR_TIMEOUT);
       return false;
     }
@@ -123,7 +131,7 @@ __device__ __forceinline__ bool wait_counter_geq(const unsigned* p, unsigned tar
   if (ld_acquire_u32(p) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire_u32(p) < target) {
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (wait_expired(t0, limit_ns)) {
       set_device_error(VV_ERR_TIMEOUT);
       return false;
     }

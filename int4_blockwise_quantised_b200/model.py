@@ -124,6 +124,9 @@ class Decoder:
         self._trace = buf
         check(_vv.lib.vv_decoder_set_trace(self.handle, ptr(buf)))
 
+    def set_wait_limit(self, ns):
+        check(_vv.lib.vv_decoder_set_wait_limit(self.handle, int(ns)))
+
     def set_graph(self, enable):
         check(_vv.lib.vv_decoder_set_graph(self.handle, 1 if enable else 0))
 

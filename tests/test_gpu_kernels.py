@@ -123,8 +123,10 @@ def test_gemv_multirow(vv, M):
 
 # ------------------------------------------------------------- tensor-core MatMulNBits (many rows)
 def test_gemm_tc_one_hot_layout_exact(vv):
-    """Row m of x is one-hot at column k_m: y[m] must be the fp16 dequantised column k_m exactly
-    (single product, fp32 accumulate, one rounding).  Columns span swizzle chunks and K blocks."""
+    """Row m of x is one-hot at column k_m (M = 14 > 8: the tensor-core path, int4 expanded in
+    shared memory): y[m] must be the fp16 dequantised column k_m exactly (single product, fp32
+    accumulate, one rounding).  Columns span swizzle chunks, 64-column k blocks and the 256-column
+    scale groups."""
     N, K = 512, 1536
     W = synth.normal_f32((N, K), 0.02, 19)
     q, sc = opack.pack_sym_int4(W)
@@ -133,15 +135,15 @@ def test_gemm_tc_one_hot_layout_exact(vv):
     X = np.zeros((len(cols), K), np.float16)
     for i, k in enumerate(cols):
         X[i, k] = 1.0
-    Y = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc)).cpu().numpy()
+    Y = vv.vv_matmul_nbits(dev(X), dev(q), dev(sc)).cpu().numpy()
     for i, k in enumerate(cols):
         assert np.array_equal(Y[i], deq[:, k].astype(np.float16)), (i, k)
 
 
 # 256-, 192- and 128-wide tiles, a single tile, ragged M tails, and enough tiles (4530 rows) that
-# every CTA of the persistent grid cycles through both accumulators
-GEMM_TC_SHAPES = [(1, 256, 64), (37, 1024, 1536), (128, 2048, 1536), (129, 512, 8960),
-                  (300, 1536, 8960), (513, 256, 3584), (600, 128, 64), (1000, 1536, 512),
+# every CTA of the persistent grid cycles through both accumulators (M > 8: tensor-core path)
+GEMM_TC_SHAPES = [(9, 256, 256), (37, 1024, 1536), (128, 2048, 1536), (129, 512, 8960),
+                  (300, 1536, 8960), (513, 256, 3584), (600, 128, 256), (1000, 1536, 512),
                   (4530, 2048, 1536), (4530, 1536, 1536)]
 
 
@@ -154,29 +156,39 @@ def test_gemm_tc_random(vv, M, N, K):
     X = synth.normal_f16((M, K), 1.0, 21)
     b = synth.normal_f16((N,), 0.02, 22)
     ref = oops.matmul_nbits(X.astype(np.float64), q, sc, K, b)
-    Y = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc), dev(b))
+    Y = vv.vv_matmul_nbits(dev(X), dev(q), dev(sc), dev(b))
     assert normwise(Y.cpu().numpy().astype(np.float64), ref) <= 1e-3
 
 
 def test_gemm_tc_ternary_matches_gemv(vv):
-    """Ternary weights: the tensor-core path and the GEMV path agree row by row (M = 8)."""
+    """Ternary weights: the tensor-core path (M = 16) and the GEMV path (two calls of M = 8)
+    agree row by row."""
     N, K = 1536, 1536
     W = synth.normal_f32((N, K), 0.02, 23)
     s = opack.ternary_scale(W)
     q, sc = opack.pack_ternary(W, s)
-    X = synth.normal_f16((8, K), 1.0, 24)
-    a = vv.vv_matmul_nbits_tc(dev(X), dev(q), dev(sc)).cpu().numpy().astype(np.float64)
-    g = vv.vv_matmul_nbits(dev(X), dev(q), dev(sc)).cpu().numpy().astype(np.float64)
+    X = synth.normal_f16((16, K), 1.0, 24)
+    a = vv.vv_matmul_nbits(dev(X), dev(q), dev(sc)).cpu().numpy().astype(np.float64)
+    g = np.concatenate([vv.vv_matmul_nbits(dev(X[i:i + 8]), dev(q), dev(sc)).cpu().numpy()
+                        for i in (0, 8)]).astype(np.float64)
     assert normwise(a, g) <= 1e-3
 
 
 def test_gemm_tc_rejects_bad_shapes(vv):
+    """M > 8 needs N % 128 == 0 and K % 256 == 0 (the GEMV path, M <= 8, does not)."""
     q = torch.zeros((100, 2, 16), dtype=torch.uint8, device="cuda")
     sc = torch.zeros((100, 2), dtype=torch.float16, device="cuda")
-    x = torch.zeros((4, 64), dtype=torch.float16, device="cuda")
+    x = torch.zeros((12, 64), dtype=torch.float16, device="cuda")
     with pytest.raises(vv.VVError) as e:
-        vv.vv_matmul_nbits_tc(x, q, sc)
+        vv.vv_matmul_nbits(x, q, sc)
     assert e.value.code == vv.VV_ERR_SHAPE
+    q2 = torch.zeros((128, 2, 16), dtype=torch.uint8, device="cuda")
+    sc2 = torch.zeros((128, 2), dtype=torch.float16, device="cuda")
+    with pytest.raises(vv.VVError) as e:
+        vv.vv_matmul_nbits(x, q2, sc2)  # K = 64
+    assert e.value.code == vv.VV_ERR_SHAPE
+    vv.vv_matmul_nbits(x[:8], q, sc)  # M <= 8: any N, K % 32
+    vv.vv_sync_status()
 
 
 # ---------------------------------------------------------------------------------- attention
