@@ -692,8 +692,9 @@ PHASES = ("qkv", "attn", "o", "gu_down")
 def timeline_names(L):
     """Stamp names of one CTA's row, in the step kernel's order: kernel start; per layer the
     barrier before each phase (arrive, exit; none before layer 0's q/k/v), then the point where
-    the phase's input is staged (q/k/v, gate/up) or its work is done (attention, o-proj), and the
-    layer end; then the lm_head barrier, its staged input and the end."""
+    the phase's input is staged (q/k/v, gate/up) or its work is done (attention, o-proj); in the
+    gate/up + down phase also the end of gate/up and the staged h; the layer end; then the lm_head
+    barrier, its staged input and the end."""
     names = ["start"]
     for l in range(L):
         if l > 0:
@@ -701,7 +702,8 @@ def timeline_names(L):
         names += [f"L{l}.qkv.staged"]
         names += [f"L{l}.attn.arrive", f"L{l}.attn.exit", f"L{l}.attn.done"]
         names += [f"L{l}.o.arrive", f"L{l}.o.exit", f"L{l}.o.done"]
-        names += [f"L{l}.gu_down.arrive", f"L{l}.gu_down.exit", f"L{l}.gu_down.staged", f"L{l}.end"]
+        names += [f"L{l}.gu_down.arrive", f"L{l}.gu_down.exit", f"L{l}.gu_down.staged",
+                  f"L{l}.gu_down.gu_done", f"L{l}.gu_down.h_staged", f"L{l}.end"]
     names += ["head.arrive", "head.exit", "head.staged", "end"]
     return names
 

@@ -39,6 +39,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "vv_device.cuh"
 #include "vv_internal.h"
 #include "step.h"
@@ -51,8 +53,6 @@ constexpr int kThreads = (NW + 1) * 32;
 constexpr int NT = NW * 32;            // compute threads
 constexpr int D = 128;
 constexpr int TT = 64;                 // attention tile (positions)
-constexpr int kRowH = D + 8;           // halves per K/V row in a stage: 272 bytes, so consecutive
-                                       // rows start 4 banks apart (conflict-free 16-byte reads)
 constexpr int kMaxG = 8;
 constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
@@ -127,14 +127,30 @@ struct Ring {
   uint64_t wait_ns;  // time this thread spent blocked in ring waits (timeline tap)
   uint64_t wait_limit;  // bound of every wait (StepParams::wait_ns)
   unsigned char* base;
+  uint32_t base_a;   // shared-space address of base
   uint64_t* full;
   uint64_t* empty;
   int stage_bytes;
   int nstages;
-  int idx;         // running stage counter
-  int ph;          // phase kind of the stages being consumed (timeline tap)
-  uint64_t* tapw;  // timeline tap: per-phase-kind ring wait of compute thread 0 (else null)
+  int slot;          // slot of the next stage (running counter modulo nstages)
+  uint32_t par;      // parity of the next stage's round (stage index / nstages, low bit)
+  bool wrapped;      // at least one full round of the ring done (producer: slots need freeing)
+  int ph;            // phase kind of the stages being consumed (timeline tap)
+  uint64_t* tapw;    // timeline tap: per-phase-kind ring wait of compute thread 0 (else null)
 };
+
+// Advance the ring position by one stage; returns the slot taken.
+__device__ __forceinline__ int ring_next(Ring& r, uint32_t& par, bool& wrapped) {
+  const int slot = r.slot;
+  par = r.par;
+  wrapped = r.wrapped;
+  if (++r.slot == r.nstages) {
+    r.slot = 0;
+    r.par ^= 1u;
+    r.wrapped = true;
+  }
+  return slot;
+}
 
 struct Copy {
   const void* src;
@@ -168,24 +184,33 @@ __device__ __forceinline__ void producer_wait(Ring& r, uint64_t* bar, uint32_t p
   r.wait_ns += globaltimer_ns() - t0;
 }
 
+// Producer side: take the next slot (waiting until the consumers have freed it, from the second
+// round on) and arm its full barrier for `tx_bytes`; returns the slot.
+__device__ __forceinline__ int produce_begin(Ring& r, uint32_t tx_bytes) {
+  uint32_t par;
+  bool wrapped;
+  const int slot = ring_next(r, par, wrapped);
+  if (wrapped) producer_wait(r, &r.empty[slot], par ^ 1u);
+  mbar_arrive_expect_tx(&r.full[slot], tx_bytes);
+  return slot;
+}
+
 __device__ __forceinline__ void produce(Ring& r, const Copy* c, int n, uint64_t pol) {
-  const int s = r.idx++;
-  const int slot = s % r.nstages;
-  if (s >= r.nstages) producer_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
   uint32_t tot = 0;
   for (int i = 0; i < n; ++i) tot += c[i].bytes;
-  mbar_arrive_expect_tx(&r.full[slot], tot);
+  const int slot = produce_begin(r, tot);
   unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
   for (int i = 0; i < n; ++i)
     if (c[i].bytes) bulk_g2s_stream(dst + c[i].dst_off, c[i].src, c[i].bytes, &r.full[slot], pol);
 }
 
-// Consumer side: wait for the next stage, return its base.
-__device__ __forceinline__ const unsigned char* consume_begin(Ring& r, int& slot) {
-  const int s = r.idx++;
-  slot = s % r.nstages;
-  ring_wait(r, &r.full[slot], (s / r.nstages) & 1);
-  return r.base + (size_t)slot * r.stage_bytes;
+// Consumer side: wait for the next stage; returns its shared-space address (and the slot).
+__device__ __forceinline__ uint32_t consume_begin(Ring& r, int& slot) {
+  uint32_t par;
+  bool wrapped;
+  slot = ring_next(r, par, wrapped);
+  ring_wait(r, &r.full[slot], par);
+  return r.base_a + (uint32_t)(slot * r.stage_bytes);
 }
 __device__ __forceinline__ void consume_end(Ring& r, int slot) {
   __syncwarp();
@@ -201,17 +226,15 @@ __device__ __forceinline__ int rows_per_stage(int row_bytes, int stage_bytes) {
   return r & ~7;  // a multiple of 8 rows keeps every scale run 16-byte aligned
 }
 
-// One attention tile: `rows` past K rows and V rows (256 bytes each) into the padded row layout
-// (kRowH halves per row; V after TT K rows).
+// One attention tile: `rows` past K rows and V rows (256 bytes each, consecutive in the cache)
+// with one copy each: K rows at the stage base, V rows TT rows after them.
 __device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int rows, uint64_t pol) {
-  const int s = r.idx++;
-  const int slot = s % r.nstages;
-  if (s >= r.nstages) producer_wait(r, &r.empty[slot], ((s / r.nstages) - 1) & 1);
-  mbar_arrive_expect_tx(&r.full[slot], (uint32_t)rows * D * 2 * 2);
+  const uint32_t bytes = (uint32_t)rows * D * 2;
+  const int slot = produce_begin(r, 2 * bytes);
   unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
-  for (int i = 0; i < rows; ++i) {
-    bulk_g2s_stream(dst + (size_t)i * kRowH * 2, k + (size_t)i * D, D * 2, &r.full[slot], pol);
-    bulk_g2s_stream(dst + (size_t)(TT + i) * kRowH * 2, v + (size_t)i * D, D * 2, &r.full[slot], pol);
+  if (bytes) {
+    bulk_g2s_stream(dst, k, bytes, &r.full[slot], pol);
+    bulk_g2s_stream(dst + (size_t)TT * D * 2, v, bytes, &r.full[slot], pol);
   }
 }
 
@@ -270,7 +293,13 @@ __device__ void produce_cols(Ring& r, const unsigned char* img, int rows, int nb
   }
 }
 
-__device__ __forceinline__ int ntiles_for(int past) { return (past + 1 + TT - 1) / TT; }
+// Attention tile size of a launch: 32 positions when doubling the tiles of 64 still gives every
+// item its own CTA, else 64.  Producer and consumers compute the same.
+__device__ __forceinline__ int tile_for(int past, int Hkv) {
+  const int n64 = (past + 1 + TT - 1) / TT;
+  return 2 * Hkv * n64 <= (int)gridDim.x ? TT / 2 : TT;
+}
+__device__ __forceinline__ int ntiles_for(int past, int tt) { return (past + 1 + tt - 1) / tt; }
 __device__ __forceinline__ int n_slices(const StepParams& p) { return p.I / kSlice; }
 __device__ __forceinline__ int slices_of(const StepParams& p, int cta) {
   const int ns = n_slices(p);
@@ -281,12 +310,19 @@ __device__ __forceinline__ size_t wd_cta_stride(const StepParams& p) {
   return (size_t)p.H * nsl_max * 2 * 18;
 }
 
+// CTA c's down-column image stores row (i + wd_rot) mod H at position i: the CTAs walk x from
+// different rows, so their residual additions reach different L2 lines at the same time.
+__host__ __device__ __forceinline__ int wd_rot(int H, int c, int grid) {
+  return (int)((((long long)c * H) / grid) & ~31LL) % H;
+}
+
 __device__ void producer(const StepParams& p, Ring& r, int past) {
   const uint64_t pol = policy_evict_first();
   const int cta = blockIdx.x, ncta = gridDim.x;
   const int H = p.H, Hq = p.Hq, Hkv = p.Hkv;
   const int nqkv = (Hq + 2 * Hkv) * D;
-  const int nt = ntiles_for(past);
+  const int tt = tile_for(past, Hkv);
+  const int nt = ntiles_for(past, tt);
   const int nrb = H / kORows;
   const int nsl = slices_of(p, cta);
   const int ns = n_slices(p);
@@ -300,7 +336,7 @@ __device__ void producer(const StepParams& p, Ring& r, int past) {
     produce_qkv(r, w, H, r0, r1, bounds, pol);
     for (int it = cta; it < Hkv * nt; it += ncta) {
       const int g = it / nt, t = it % nt;
-      const int p0 = t * TT, p1 = min(p0 + TT, past);
+      const int p0 = t * tt, p1 = min(p0 + tt, past);
       const size_t off = ((size_t)(l * Hkv + g) * p.cap + p0) * D;
       produce_kv_rows(r, p.k_cache + off, p.v_cache + off, max(p1 - p0, 0), pol);
     }
@@ -333,6 +369,7 @@ struct XOp {
   uint4* xq;
   int* corr;
   float* fb;
+  uint32_t xq_a, corr_a, fb_a;  // the same, as shared-space addresses
 };
 
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
@@ -418,58 +455,103 @@ __device__ void stage_idp(const XOp& xo, Load load, const __half* gamma, float e
 }
 
 // ----------------------------------------------------------------------------- int4 GEMV
+// Shared-memory loads by 32-bit shared-space address.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_half(uint32_t a) {
+  unsigned short h;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(a));
+  return __half2float(__ushort_as_half(h));
+}
+
 // One half-block (16 weights: two code words) against its X pairs: exact int32 sum of
-// (c - 8) X, starting from corr = -8 sum X.
+// (c - 8) X, starting from corr = -8 sum X (two independent dp2a chains).
 __device__ __forceinline__ int hb_dot(uint2 wv, uint4 xa, uint4 xb, int corr) {
   const uint32_t l0 = wv.x & 0x0F0F0F0Fu, h0 = (wv.x >> 4) & 0x0F0F0F0Fu;
   const uint32_t l1 = wv.y & 0x0F0F0F0Fu, h1 = (wv.y >> 4) & 0x0F0F0F0Fu;
-  int s = corr;
+  int s = corr, t = 0;
   s = dp2a_lo(xa.x, l0, s);
+  t = dp2a_lo(xb.x, l1, t);
   s = dp2a_hi(xa.y, l0, s);
+  t = dp2a_hi(xb.y, l1, t);
   s = dp2a_lo(xa.z, h0, s);
+  t = dp2a_lo(xb.z, h1, t);
   s = dp2a_hi(xa.w, h0, s);
-  s = dp2a_lo(xb.x, l1, s);
-  s = dp2a_hi(xb.y, l1, s);
-  s = dp2a_lo(xb.z, h1, s);
-  s = dp2a_hi(xb.w, h1, s);
-  return s;
+  t = dp2a_hi(xb.w, h1, t);
+  return s + t;
 }
 
-// Rows of one stage against the staged X.  Units are (row, segment) pairs, u -> (u / nseg,
-// u % nseg); LPR lanes share a unit (lane % LPR strides the half-blocks), a warp takes 32/LPR x R
-// units per pass.  rowq(u) / rows(u): code and scale bytes of unit u's row.  fin(u, y) is called
-// once per unit by the group's first lane; with PAIR (nseg == 2, R even) fin2(row, y0, y1) once
-// per row instead.
-template <int LPR, int R, bool PAIR, class RowQ, class RowS, class Fin>
-__device__ __forceinline__ void idp_pass(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows,
-                                         Fin fin) {
+// The units of one stage: unit u = (row u / NSEG, matrix u % NSEG); the code bytes of (row, m)
+// start at q0 + (m rps + row) rq, its scales at s0 + (m rps + row) rs (shared-space addresses).
+struct UnitMap {
+  uint32_t q0, s0;
+  int rps, rq, rs;
+};
+
+// Rows per pass (R) for `units` units with `gpw` lane groups per warp: the R in {1, 2, 4} ({2, 4}
+// for pairs) that minimises the busiest warp's share (R x its passes), the larger R on ties.
+__device__ __forceinline__ int pick_r(int units, int gpw, bool pair) {
+  int best = pair ? 2 : 1, cost_best = 1 << 30;
+  for (int R = best; R <= 4; R *= 2) {
+    const int passes = (units + gpw * R - 1) / (gpw * R);
+    const int cost = R * ((passes + NW - 1) / NW);
+    if (cost <= cost_best) {
+      best = R;
+      cost_best = cost;
+    }
+  }
+  return best;
+}
+
+// The units of one stage against the staged X: LPR lanes per unit (lane % LPR strides the
+// half-blocks), R units per lane group and pass.  fin(u, y0, y1) is called by the group's first
+// lane once per unit (y1 = 0), or with NSEG == 2 once per row with both matrices' results.
+template <int LPR, int R, int NSEG, class Fin>
+__device__ __forceinline__ void gemv_pass(const XOp& xo, int NHB, int units, const UnitMap& m,
+                                          Fin fin) {
+  static_assert(NSEG == 1 || R % NSEG == 0, "pairs need an even R");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int GPW = 32 / LPR;  // unit groups per warp
+  constexpr int GPW = 32 / LPR;
   const int sub = lane % LPR, grp = lane / LPR;
-  const uint4* xq = xo.xq;
   // the loop bound is warp-uniform (every lane runs the same iterations, as the full-mask
-  // shuffles below require); lane groups past the last unit work on a clamped row and skip fin
+  // shuffles below require); lane groups past the last unit work on a clamped unit, skip fin
   for (int ub = warp * GPW * R; ub < units; ub += NW * GPW * R) {
     const int u0 = ub + grp * R;
-    const unsigned char* q[R];
-    const __half* sc[R];
+    uint32_t qa[R], sa[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
       const int u = min(u0 + k, units - 1);
-      q[k] = rowq(u);
-      sc[k] = rows(u);
+      const int idx = NSEG == 1 ? u : (u % NSEG) * m.rps + u / NSEG;
+      qa[k] = m.q0 + (uint32_t)(idx * m.rq);
+      sa[k] = m.s0 + (uint32_t)(idx * m.rs);
     }
     float acc[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) acc[k] = 0.f;
+#pragma unroll 2
     for (int hb = sub; hb < NHB; hb += LPR) {
-      const uint4 xa = xq[hb], xb = xq[NHB + hb];
-      const int cr = xo.corr[hb];
-      const float f = xo.fb[hb >> 1];
+      const uint4 xa = lds128(xo.xq_a + hb * 16), xb = lds128(xo.xq_a + (NHB + hb) * 16);
+      const int cr = (int)lds32(xo.corr_a + hb * 4);
+      const float f = __uint_as_float(lds32(xo.fb_a + (hb >> 1) * 4));
 #pragma unroll
       for (int k = 0; k < R; ++k) {
-        const uint2 wv = *reinterpret_cast<const uint2*>(q[k] + hb * 8);
-        const float s = __half2float(sc[k][hb >> 1]) * f;
+        const uint2 wv = lds64(qa[k] + hb * 8);
+        const float s = lds_half(sa[k] + (hb >> 1) * 2) * f;
         acc[k] = fmaf(s, (float)hb_dot(wv, xa, xb, cr), acc[k]);
       }
     }
@@ -479,57 +561,64 @@ __device__ __forceinline__ void idp_pass(const XOp& xo, int NHB, int units, RowQ
       for (int o = LPR / 2; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
     }
     if (sub == 0) {
-      if (PAIR) {
 #pragma unroll
-        for (int k = 0; k + 1 < R; k += 2)
-          if (u0 + k < units) fin(u0 + k, acc[k], acc[k + 1]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < R; ++k)
-          if (u0 + k < units) fin(u0 + k, acc[k], 0.f);
-      }
+      for (int k = 0; k < R; k += NSEG)
+        if (u0 + k < units) fin(u0 + k, acc[k], NSEG == 2 ? acc[k + NSEG - 1] : 0.f);
     }
   }
 }
 
-template <int LPR, int R, bool PAIR, class RowQ, class RowS, class Fin>
-__device__ __forceinline__ void idp_dispatch(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows, Fin fin) {
-  idp_pass<LPR, R, PAIR>(xo, NHB, units, rowq, rows, fin);
+// One stage: lanes per unit from the row length (a lane takes about 4 half-blocks of short rows;
+// rows longer than 16 half-blocks take a whole warp), rows per pass from the unit count.
+template <int NSEG, class Fin>
+__device__ __forceinline__ void gemv_stage(const XOp& xo, int NHB, int units, const UnitMap& m,
+                                           Fin fin) {
+  auto go = [&](auto lpr_c) {
+    constexpr int LPR = decltype(lpr_c)::value;
+    const int R = pick_r(units, 32 / LPR, NSEG == 2);
+    if constexpr (NSEG == 1) {
+      if (R == 1) {
+        gemv_pass<LPR, 1, NSEG>(xo, NHB, units, m, fin);
+        return;
+      }
+    }
+    if (R == 2)
+      gemv_pass<LPR, 2, NSEG>(xo, NHB, units, m, fin);
+    else
+      gemv_pass<LPR, 4, NSEG>(xo, NHB, units, m, fin);
+  };
+  if (NHB > 16) {
+    go(std::integral_constant<int, 32>());
+  } else if (NHB > 8) {
+    go(std::integral_constant<int, 4>());
+  } else if constexpr (NSEG == 1) {
+    if (NHB > 4)
+      go(std::integral_constant<int, 2>());
+    else
+      go(std::integral_constant<int, 1>());
+  } else {
+    go(std::integral_constant<int, 4>());
+  }
 }
 
-// Pick lanes per unit from the half-block count: 32 (long rows) down to 4 (short rows).
-template <int R, bool PAIR, class RowQ, class RowS, class Fin>
-__device__ __forceinline__ void idp_any(const XOp& xo, int NHB, int units, RowQ rowq, RowS rows, Fin fin) {
-  if (NHB >= 32) idp_pass<32, R, PAIR>(xo, NHB, units, rowq, rows, fin);
-  else if (NHB >= 16) idp_pass<16, R, PAIR>(xo, NHB, units, rowq, rows, fin);
-  else if (NHB >= 8) idp_pass<8, R, PAIR>(xo, NHB, units, rowq, rows, fin);
-  else idp_pass<4, R, PAIR>(xo, NHB, units, rowq, rows, fin);
-}
-
-// Row phase: consume the stages of rows [r0, r1) (nseg matrices per stage).  fin(row, y0, y1).
-template <bool PAIR, class Fin>
-__device__ void consume_rows(Ring& r, const XOp& xo, int K, int r0, int r1, int nseg, Fin fin) {
+// Row phase: the stages of rows [r0, r1) of NSEG matrices.  fin(row, y0, y1).
+template <int NSEG, class Fin>
+__device__ void consume_rows(Ring& r, const XOp& xo, int K, int r0, int r1, Fin fin) {
   const int KB = K >> 5, NHB = K >> 4;
   const int rq = KB * 16, rs = KB * 2;
-  const int rps = rows_per_stage((rq + rs) * nseg, r.stage_bytes);
+  const int rps = rows_per_stage((rq + rs) * NSEG, r.stage_bytes);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     int slot;
-    const unsigned char* st = consume_begin(r, slot);
-    const unsigned char* scb = st + (size_t)nseg * rps * rq;
-    auto rowq = [&](int u) { return st + (size_t)((u % nseg) * rps + u / nseg) * rq; };
-    auto rows = [&](int u) {
-      return reinterpret_cast<const __half*>(scb + (size_t)((u % nseg) * rps + u / nseg) * rs);
-    };
-    auto f = [&](int u, float y0, float y1) { fin(a + u / nseg, y0, y1); };
-    if (PAIR) idp_any<2, true>(xo, NHB, n * nseg, rowq, rows, f);
-    else if (n >= 4 * NW) idp_any<4, false>(xo, NHB, n, rowq, rows, f);
-    else idp_any<1, false>(xo, NHB, n, rowq, rows, f);
+    const uint32_t st = consume_begin(r, slot);
+    const UnitMap m{st, st + (uint32_t)(NSEG * rps * rq), rps, rq, rs};
+    gemv_stage<NSEG>(xo, NHB, n * NSEG, m,
+                     [&](int u, float y0, float y1) { fin(a + u / NSEG, y0, y1); });
     consume_end(r, slot);
   }
 }
 
-// Column phase: consume the stages of a column image of `rows` rows x nb blocks (K = 32 nb).
+// Column phase: the stages of a column image of `rows_total` rows x nb blocks (K = 32 nb).
 template <class Fin>
 __device__ void consume_cols(Ring& r, const XOp& xo, int rows_total, int nb, Fin fin) {
   const int NHB = nb * 2;
@@ -537,12 +626,9 @@ __device__ void consume_cols(Ring& r, const XOp& xo, int rows_total, int nb, Fin
   for (int a = 0; a < rows_total; a += rps) {
     const int n = min(rps, rows_total - a);
     int slot;
-    const unsigned char* st = consume_begin(r, slot);
-    const unsigned char* scb = st + (size_t)rps * nb * 16;
-    auto rowq = [&](int u) { return st + (size_t)u * nb * 16; };
-    auto rows = [&](int u) { return reinterpret_cast<const __half*>(scb + (size_t)u * nb * 2); };
-    auto f = [&](int u, float y0, float) { fin(a + u, y0); };
-    idp_any<2, false>(xo, NHB, n, rowq, rows, f);
+    const uint32_t st = consume_begin(r, slot);
+    const UnitMap m{st, st + (uint32_t)(rps * nb * 16), rps, nb * 16, nb * 2};
+    gemv_stage<1>(xo, NHB, n, m, [&](int u, float y0, float) { fin(a + u, y0); });
     consume_end(r, slot);
   }
 }
@@ -557,13 +643,13 @@ struct AttnScratch {
 };
 
 __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
-                          int past) {
+                          int past, int tt) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.Hq / p.Hkv;
-  const int nt = ntiles_for(past);
+  const int nt = ntiles_for(past, tt);
   const int npos = past + 1;
-  const int p0 = t * TT;
-  const int n = min(TT, npos - p0);
+  const int p0 = t * tt;
+  const int n = min(tt, npos - p0);
   const float* qkv = p.qkv;
   // q of the group (rotated, scaled into the log2 domain) and, on the tile holding the new
   // position, the new k/v: every global load is issued before any is used (one L2 round trip).
@@ -602,8 +688,9 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     }
   }
   int slot;
-  __half* kt = reinterpret_cast<__half*>(const_cast<unsigned char*>(consume_begin(r, slot)));
-  __half* vt = kt + TT * kRowH;
+  consume_begin(r, slot);
+  __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
+  __half* vt = kt + TT * D;
   if (newpos && tid < D) {  // this tile holds the new position: rotate k, append k/v
     const int d = tid, fi = d & (D / 2 - 1);
     const float cs = as.cs[fi], sn = as.sn[fi];
@@ -612,23 +699,25 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     const size_t off = ((size_t)(l * p.Hkv + g) * p.cap + past) * D + d;
     p.k_cache[off] = kn;
     p.v_cache[off] = vn;
-    kt[(past - p0) * kRowH + d] = kn;
-    vt[(past - p0) * kRowH + d] = vn;
+    kt[(past - p0) * D + d] = kn;
+    vt[(past - p0) * D + d] = vn;
   }
   cbar();
-  // scores: warp w -> head w/2, positions (w%2)*32 + lane.  All lanes walk the chunks in the same
-  // order, so the q reads are broadcasts; the padded K rows keep the k reads conflict-free.
+  // scores: warp w -> head w/2, positions (w%2)*32 + lane.  K rows are 256 bytes apart, so each
+  // lane walks the 16 chunks of its row starting at chunk `lane % 16`: the 8 lanes of a 16-byte
+  // load phase then read 8 different K chunks (distinct banks; the q reads are 2-way).
   for (int item = warp; item < 2 * G; item += NW) {
     const int h = item >> 1, pp = (item & 1) * 32 + lane;
     float sc = -INFINITY;
     if (pp < n) {
-      const __half* kr = kt + pp * kRowH;
+      const __half* kr = kt + pp * D;
       float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(kr + c * 8);
-        const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][c * 8]);
-        const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][c * 8 + 4]);
+        const int cc = (c + lane) & 15;
+        const uint4 kv = *reinterpret_cast<const uint4*>(kr + cc * 8);
+        const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
+        const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
         acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa4.x, qa4.y), acc);
         acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa4.z, qa4.w), acc2);
         acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb4.x, qb4.y), acc);
@@ -665,7 +754,7 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
       const float* ph = as.s[h];
       const int p_end = min(n, q * 16 + 16);
       for (int pp = q * 16; pp < p_end; ++pp) {
-        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * kRowH + o * 8);
+        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * D + o * 8);
         const float w = ph[pp];
         const float2 ww = make_float2(w, w);
         a0 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.x)), ww, a0);
@@ -702,18 +791,32 @@ __device__ void merge_head(const StepParams& p, int h, int nt, float* scratch, f
   const int d4 = tid & 31, ts = tid >> 5;  // ts in [0, NW)
   float M = -INFINITY, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int t = ts; t < nt; t += NW) {
-    const float* pt = base + (size_t)t * kMaxG * kPart;
-    const float mt = __ldcg(pt), lt = __ldcg(pt + 1);
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(pt + 4) + d4);
-    const float bm = fmaxf(M, mt);
-    const float c = exp2f(M - bm), e = exp2f(mt - bm);
-    L = L * c + lt * e;
-    acc.x = acc.x * c + e * v.x;
-    acc.y = acc.y * c + e * v.y;
-    acc.z = acc.z * c + e * v.z;
-    acc.w = acc.w * c + e * v.w;
-    M = bm;
+  // up to 4 tiles per thread per round: all their loads are issued before the first is used
+  for (int t0 = ts; t0 < nt; t0 += 4 * NW) {
+    float mt[4], lt[4];
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * NW;
+      if (t < nt) {
+        const float* pt = base + (size_t)t * kMaxG * kPart;
+        mt[j] = __ldcg(pt);
+        lt[j] = __ldcg(pt + 1);
+        v[j] = __ldcg(reinterpret_cast<const float4*>(pt + 4) + d4);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (t0 + j * NW >= nt) break;
+      const float bm = fmaxf(M, mt[j]);
+      const float c = exp2f(M - bm), e = exp2f(mt[j] - bm);
+      L = L * c + lt[j] * e;
+      acc.x = acc.x * c + e * v[j].x;
+      acc.y = acc.y * c + e * v[j].y;
+      acc.z = acc.z * c + e * v[j].z;
+      acc.w = acc.w * c + e * v[j].w;
+      M = bm;
+    }
   }
   // scratch: [NW][32][6]
   float* sp = scratch + (ts * 32 + d4) * 6;
@@ -772,7 +875,10 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   r.base = smem;
   r.stage_bytes = p.stage_bytes;
   r.nstages = p.nstages;
-  r.idx = 0;
+  r.base_a = smem_u32(smem);
+  r.slot = 0;
+  r.par = 0;
+  r.wrapped = false;
   // shared layout after the ring: xq [2][kMaxK/16] uint4 | corr [kMaxK/16] | fb [kMaxK/32] |
   // hbuf [kMaxK/...] | AttnScratch | red[64] | mbarriers
   unsigned char* sp = smem + (size_t)p.nstages * p.stage_bytes;
@@ -785,6 +891,9 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   sp += (size_t)nhb_max * 4;
   xo.fb = reinterpret_cast<float*>(sp);
   sp += (size_t)nhb_max * 2;
+  xo.xq_a = smem_u32(xo.xq);
+  xo.corr_a = smem_u32(xo.corr);
+  xo.fb_a = smem_u32(xo.fb);
   const int nsl = slices_of(p, blockIdx.x);
   float* hbuf = reinterpret_cast<float*>(sp);  // h of this CTA's slices, then o_h of an o-item
   sp += (size_t)max(nsl * kSlice, D) * 4;
@@ -830,7 +939,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   stamp(p, sk);
   const int cta = blockIdx.x, ncta = gridDim.x;
   const int nqkv = (Hq + 2 * Hkv) * D;
-  const int nt = ntiles_for(past);
+  const int tt = tile_for(past, Hkv);
+  const int nt = ntiles_for(past, tt);
   const int nrb = H / kORows;
   const int ns = n_slices(p);
   int pos = *p.position;
@@ -882,35 +992,35 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     r.ph = 0;
     int r0, r1;
     cta_range(nqkv, cta, ncta, r0, r1);
-    // this CTA's q/k/v biases -> shared memory before the barrier (they do not depend on x;
-    // as.q is free until the attention phase; stage_idp's barriers order the stores)
-    {
+    // this CTA's q/k/v biases (at most NT rows): the load is issued before the barrier (the
+    // biases do not depend on x), the store to shared memory after it (as.q is free until the
+    // attention phase; stage_idp's barriers order the stores before the GEMV reads them)
+    float bias_v = 0.f;
+    if (tid < r1 - r0) {
       const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
-      float* bias_s = &as.q[0][0];
-      for (int i = tid; i < r1 - r0; i += NT) {
-        const int row = r0 + i;
-        const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
-        const __half* b = w.bias[m];
-        bias_s[i] = b ? __half2float(b[row - bounds[m]]) : 0.f;
-      }
+      const int row = r0 + tid;
+      const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
+      const __half* b = w.bias[m];
+      if (b) bias_v = __half2float(__ldg(b + (row - bounds[m])));
     }
+    if (l > 0) grid_barrier(p, gen, sk);
+    if (tid < r1 - r0) (&as.q[0][0])[tid] = bias_v;
     if (l == 0) {
       stage_idp(xo, load_emb, w.in_norm, p.eps, H, red, nullptr);
     } else {
-      grid_barrier(p, gen, sk);
       float* tr = (p.trace && cta == 0) ? p.trace + (size_t)(l - 1) * H : nullptr;
       stage_idp(xo, load_x, w.in_norm, p.eps, H, red, tr);
     }
     stamp(p, sk);
     {
       const float* bs = &as.q[0][0] - r0;
-      consume_rows<false>(r, xo, H, r0, r1, 1,
+      consume_rows<1>(r, xo, H, r0, r1,
                           [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
     }
     // ---------------------------------------------------------------- ATTN
     r.ph = 1;
     grid_barrier(p, gen, sk);
-    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past);
+    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, tt);
     stamp(p, sk);
     // ---------------------------------------------------------------- O
     r.ph = 2;
@@ -939,16 +1049,24 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       int j = 0;
       for (int s = cta; s < ns; s += ncta, ++j) {
         float* hs = hbuf + j * kSlice - s * kSlice;
-        consume_rows<true>(r, xo, H, s * kSlice, (s + 1) * kSlice, 2, [&](int row, float g, float u) {
+        consume_rows<2>(r, xo, H, s * kSlice, (s + 1) * kSlice, [&](int row, float g, float u) {
           hs[row] = g / (1.f + __expf(-g)) * u;
         });
       }
       cbar();
+      stamp(p, sk);
       r.ph = 4;
       stage_idp(xo, [&](int k) { return *reinterpret_cast<const float4*>(hbuf + k); }, nullptr,
                 0.f, nsl * kSlice, red, nullptr);
-      consume_cols(r, xo, H, 2 * nsl, [&](int row, float y) { red_add_u64(p.x_acc + row, to_fix(y)); });
+      stamp(p, sk);
+      const int rot = wd_rot(H, cta, ncta);
+      consume_cols(r, xo, H, 2 * nsl, [&](int i, float y) {
+        const int row = i + rot < H ? i + rot : i + rot - H;
+        red_add_u64(p.x_acc + row, to_fix(y));
+      });
     } else {
+      stamp(p, sk);
+      stamp(p, sk);
       stamp(p, sk);
     }
     stamp(p, sk);
@@ -1008,7 +1126,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     for (int a = r0; a < r1; a += rps) {
       const int n = min(rps, r1 - a);
       int slot;
-      const unsigned char* st = consume_begin(r, slot);
+      consume_begin(r, slot);
+      const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
       for (int i = warp; i < n; i += NW) {
         const unsigned char* row = st + (size_t)i * rb;
         float acc = 0.f;
@@ -1128,7 +1247,8 @@ __global__ void wo_image_kernel(const uint8_t* __restrict__ q, const __half* __r
 }
 
 // Wd (rows H, columns I): CTA c's image holds its slices c, c + grid, ... (64 columns = 2 blocks
-// each): codes [H][2 nsl][16] then scales [H][2 nsl]; CTA images `stride` bytes apart.
+// each): codes [H][2 nsl][16] then scales [H][2 nsl], rows rotated by wd_rot; CTA images
+// `stride` bytes apart.
 __global__ void wd_image_kernel(const uint8_t* __restrict__ q, const __half* __restrict__ s, int H,
                                 int I, int grid, size_t stride, unsigned char* __restrict__ img) {
   const int KB = I / 32;
@@ -1142,9 +1262,11 @@ __global__ void wd_image_kernel(const uint8_t* __restrict__ q, const __half* __r
     const int nb = 2 * nsl;
     const int col = 2 * j + (blk & 1);
     unsigned char* ci = img + (size_t)c * stride;
-    reinterpret_cast<uint4*>(ci)[(size_t)row * nb + col] =
+    const int rot = wd_rot(H, c, grid);
+    const int pos = row >= rot ? row - rot : row - rot + H;
+    reinterpret_cast<uint4*>(ci)[(size_t)pos * nb + col] =
         *reinterpret_cast<const uint4*>(q + ((size_t)row * KB + blk) * 16);
-    reinterpret_cast<__half*>(ci + (size_t)H * nb * 16)[(size_t)row * nb + col] =
+    reinterpret_cast<__half*>(ci + (size_t)H * nb * 16)[(size_t)pos * nb + col] =
         s[(size_t)row * KB + blk];
   }
 }
@@ -1193,7 +1315,7 @@ size_t step_attn_part_floats(int Hkv, int max_tiles) {
   return (size_t)Hkv * max_tiles * kMaxG * kPart;
 }
 
-int step_max_tiles(int cap) { return (cap + TT - 1) / TT; }
+int step_max_tiles(int cap) { return (cap + 1 + TT / 2 - 1) / (TT / 2); }
 
 // Pick the largest stage size (>= one attention tile, 1 KB steps) for which one CTA per SM is
 // resident.
@@ -1202,7 +1324,7 @@ cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
                                        (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   *blocks_per_sm = 0;
-  for (; p.stage_bytes >= 2 * TT * kRowH * 2; p.stage_bytes -= 1024) {
+  for (; p.stage_bytes >= 2 * TT * D * 2; p.stage_bytes -= 1024) {
     const size_t smem = step_smem_bytes(p);
     e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {

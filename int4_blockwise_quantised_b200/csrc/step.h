@@ -85,8 +85,8 @@ size_t step_wd_image_bytes(int H, int I, int grid);
 cudaError_t step_build_images(const StepParams& p, const StepLayer* host_layers,
                               unsigned char* wo_img, unsigned char* wd_img, cudaStream_t s);
 constexpr int kMaxStopIds = 8;
-// Entries per CTA the timeline tap needs for a model of L layers: 13 L + 3 stamps and 8 trailing
+// Entries per CTA the timeline tap needs for a model of L layers: 15 L + 3 stamps and 8 trailing
 // counters.
-inline int step_timeline_stamps(int L) { return 13 * L + 3 + 8; }
+inline int step_timeline_stamps(int L) { return 15 * L + 3 + 8; }
 
 }  // namespace vv

@@ -141,7 +141,7 @@ class Decoder:
 
     def step_timeline(self, position, input_embeds=None, token=None, stream=None):
         """One persistent step with the timeline tap; returns uint64 ns array [grid, stamps]."""
-        maxn = 13 * self.model.shape.layers + 3 + 8
+        maxn = 15 * self.model.shape.layers + 3 + 8
         grid_max = 1024
         buf = np.zeros(grid_max * maxn, dtype=np.uint64)
         g = ctypes.c_int32()

@@ -50,9 +50,9 @@ def test_phase_breakdown_recovers_known_durations():
 
 
 def test_timeline_names_match_the_kernel_stamp_count():
-    # 13 stamps per layer (11 for layer 0: no barrier before its q/k/v) + start + 4 for the head
+    # 15 stamps per layer (13 for layer 0: no barrier before its q/k/v) + start + 4 for the head
     for L in (1, 2, 28):
-        assert len(bench.timeline_names(L)) == 13 * L + 3
+        assert len(bench.timeline_names(L)) == 15 * L + 3
 
 
 def test_phase_breakdown_rejects_a_wrong_stamp_count():
