@@ -85,9 +85,10 @@ def decoder_step(cfg, weights, input_embeds, position, k_cache, v_cache, kv_dtyp
     """One decode step at batch 1.
 
     input_embeds float16 [H]; position int; k_cache/v_cache: per layer [Hkv, P, D] (the P past
-    positions) of the cache's storage type kv_dtype.  Returns dict with logits float64 [V],
-    argmax, layer_out float64 [L, H] (the residual after each layer), k_new/v_new [L, Hkv, D]
-    rounded to kv_dtype.  The contract stores K/V in float16 ("vibevoice-asr-bitnet-onnx",
+    positions) of the cache's storage type kv_dtype (np.float16, np.float32, "bf16", or np.float64
+    for a cache without storage rounding).  Returns dict with logits float64 [V], argmax,
+    layer_out float64 [L, H] (the residual after each layer), k_new/v_new [L, Hkv, D] rounded
+    to kv_dtype (arrays of kv_dtype; float64 holding bf16 values for "bf16").  The contract stores K/V in float16 ("vibevoice-asr-bitnet-onnx",
     decoder_step I/O); kv_dtype=np.float32 is the fp32-cache variant of "VibeVoice-ASR — ONNX
     export for Vernacula" (Highlights), where only the storage rounding differs.
     """
@@ -96,10 +97,10 @@ def decoder_step(cfg, weights, input_embeds, position, k_cache, v_cache, kv_dtyp
     outs, k_new, v_new = [], [], []
     for li, lw in enumerate(weights["layers"]):
         q, k, v = _attn_in(cfg, lw, x, [position])
-        k16 = k[0].astype(kv_dtype)
-        v16 = v[0].astype(kv_dtype)
-        K = np.concatenate([np.asarray(k_cache[li], kv_dtype), k16[:, None, :]], axis=1)
-        V = np.concatenate([np.asarray(v_cache[li], kv_dtype), v16[:, None, :]], axis=1)
+        k16 = ops.kv_round(k[0], kv_dtype)
+        v16 = ops.kv_round(v[0], kv_dtype)
+        K = np.concatenate([ops.kv_round(k_cache[li], kv_dtype), k16[:, None, :]], axis=1)
+        V = np.concatenate([ops.kv_round(v_cache[li], kv_dtype), v16[:, None, :]], axis=1)
         o = ops.gqa_decode_attention(q[0], K.astype(np.float64), V.astype(np.float64), scale)
         x = _mlp_out(cfg, lw, x, o.reshape(1, -1))
         outs.append(x[0].copy())

@@ -41,6 +41,27 @@ def rope(x, pos, theta):
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
+def round_bf16(x):
+    """Round to bfloat16 (8 significant bits, fp32 exponent range), nearest with ties to even;
+    returned as float64 values.  The storage rounding of the bf16 KV-cache variant (the fp16 /
+    fp32 cache trade-off of "VibeVoice-ASR — ONNX export for Vernacula", Highlights, with a
+    third storage type).  x = m 2^e with 0.5 <= |m| < 1 (frexp); m is rounded to a multiple of
+    2^-8.  Zero stays zero; the cache values here are far from bf16's subnormal and overflow
+    ranges, which are not modelled."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def kv_round(x, kv_dtype):
+    """A K/V value as stored in a cache of kv_dtype (np.float16, np.float32, "bf16", or
+    np.float64 for no storage rounding): an array of kv_dtype, float64 for "bf16"."""
+    if isinstance(kv_dtype, str):
+        assert kv_dtype == "bf16", kv_dtype
+        return round_bf16(x)
+    return np.asarray(x, dtype=np.float64).astype(kv_dtype)
+
+
 def repeat_kv(kv, group):
     """[Hkv, ...] -> [Hkv*group, ...]: query head h reads key/value head h // group."""
     return np.repeat(np.asarray(kv), group, axis=0)

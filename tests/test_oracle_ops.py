@@ -175,3 +175,42 @@ def test_frame_count_golden(seconds):
     _, rows = read_golden("asr_frame_count.txt")
     table = {r[0]: int(r[1]) for r in rows}
     assert synth.frames_for_audio(seconds) == table[float(seconds)]
+
+
+# ---------------------------------------------------------------- bf16 storage rounding
+def test_round_bf16_ties_to_even_at_eight_bits():
+    """bf16 keeps 8 significant bits: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 and goes to
+    the even neighbour 1; 1 + 3 2^-8 lies halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even)."""
+    cases = {1.0: 1.0, 1.0 + 2.0**-8: 1.0, 1.0 + 3 * 2.0**-8: 1.0 + 2.0**-6,
+             1.0 + 2.0**-7: 1.0 + 2.0**-7, -3.0: -3.0, 0.0: 0.0,
+             1.0 + 2.0**-8 + 2.0**-20: 1.0 + 2.0**-7, 255.5: 256.0, 254.5: 254.0}
+    for x, want in cases.items():
+        assert ops.round_bf16(np.array([x]))[0] == want, x
+
+
+def test_round_bf16_matches_torch_on_fp32_values():
+    """For values exactly representable in fp32, rounding straight from them is torch's
+    fp32 -> bfloat16 conversion (round to nearest even), an independent implementation."""
+    import torch
+
+    g = np.random.default_rng(5)
+    x = (g.standard_normal(20000) * np.exp(g.uniform(-20, 20, 20000))).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(ops.round_bf16(x.astype(np.float64)), want)
+
+
+def test_round_bf16_error_bound_and_idempotence():
+    g = np.random.default_rng(6)
+    x = g.standard_normal(10000) * 37.0
+    r = ops.round_bf16(x)
+    assert np.all(np.abs(r - x) <= np.abs(x) * 2.0**-8)
+    assert np.array_equal(ops.round_bf16(r), r)
+
+
+def test_kv_round_storage_types():
+    x = np.array([1.0 + 2.0**-12, -2.5 + 2.0**-30])
+    assert ops.kv_round(x, np.float16).dtype == np.float16
+    assert ops.kv_round(x, np.float16)[0] == 1.0  # 2^-12 is below fp16's half ulp at 1
+    assert ops.kv_round(x, np.float32)[1] == np.float32(-2.5 + 2.0**-30)
+    assert np.array_equal(ops.kv_round(x, np.float64), x)
+    assert np.array_equal(ops.kv_round(x, "bf16"), ops.round_bf16(x))
