@@ -40,6 +40,9 @@ CONFIGS = {
                   "28-layer decoder_step, 7B shapes, int4 sym block-32, P=4096, batch 1"),
     "decode-asr-1p5b": (synth.SHAPE_1P5B, "ternary", 4530, 256,
                         "ASR-shaped long decode, 1.5B ternary, P=4530 -> 4785, batch 1"),
+    "decode-0p5b": (synth.SHAPE_0P5B, "int4", 1024, 64,
+                    "20-layer decoder_step, Realtime-0.5B shapes (hidden 896, 7 q / 1 kv heads of "
+                    "128), int4 sym block-32, P=1024, batch 1"),
     "layer-1p5b": (synth.Shape("layer", 1536, 1, 12, 2, 128, 8960, 151936, tied=True), "ternary",
                    128, 64, "one decoder layer + lm_head, 1.5B shapes, ternary, P=128"),
 }
@@ -96,6 +99,19 @@ def prefill_flops(shape, S):
     gemm = 2 * S * (H * (Hq + 2 * Hkv) * D + Hq * D * H + H * 2 * I + I * H) * shape.layers
     attn = 2 * 2 * Hq * D * (S * (S + 1) // 2) * shape.layers
     return {"gemm": gemm, "attention": attn, "lm_head": 2 * V * H}
+
+
+def variant_step_bytes(shape, Ps, kv_bytes=2):
+    """Algorithmic bytes of one step of len(Ps) sequences stepped together: the weights and the
+    lm_head once, each sequence's KV read (P_b positions) and write in the cache's element size,
+    its logits and its input embedding."""
+    b = phase_bytes(shape, 0)
+    L, Hkv, D = shape.layers, shape.n_kv, shape.head_dim
+    weights = L * sum(v for k, v in b.items() if k not in ("lm_head", "attn"))
+    head_w = shape.vocab * shape.hidden * 2 + 2 * shape.hidden
+    per_seq = sum(L * 2 * Hkv * (P + 1) * D * kv_bytes + 4 * shape.vocab + 2 * shape.hidden
+                  for P in Ps)
+    return weights + head_w + per_seq
 
 
 def step_bytes(shape, P):
@@ -241,6 +257,39 @@ def oracle_sample_time_1thread(shape, mode, P, samples=3):
     return statistics.median(ts), o.describe(samples)
 
 
+def decode_cpu_baseline(shape, mode, P, samples=8):
+    """The oracle's decode step on the host cores (all BLAS threads) and at one thread."""
+    st, sample, thr = oracle_sample_time(shape, mode, P, samples)
+    rec = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr, "kind": "oracle",
+           "sample": sample, "host_cpus": os.cpu_count()}
+    try:
+        st1, sample1 = oracle_sample_time_1thread(shape, mode, P, min(samples, 3))
+        rec["one_thread"] = {"value": round(1.0 / st1, 4), "unit": "tok/s", "cores": 1,
+                             "sample": sample1}
+    except Exception as e:  # threadpoolctl missing: report the all-cores figure only
+        rec["one_thread"] = {"error": str(e)[:200]}
+    return rec
+
+
+def prefill_cpu_baseline(shape, mode, S, N):
+    """The oracle's prefill over S positions (one decoder layer, scaled by L) at all BLAS threads
+    and at one thread."""
+    o = OraclePrefillSample(shape, mode, S, N)
+    st = o.run()
+    rec = {"value": round(S / st, 3), "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": o.describe(1), "host_cpus": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            st1 = o.run()
+        rec["one_thread"] = {"value": round(S / st1, 3), "unit": "tok/s", "cores": 1,
+                             "sample": o.describe(1)}
+    except Exception as e:
+        rec["one_thread"] = {"error": str(e)[:200]}
+    return rec
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -278,6 +327,65 @@ def build_model(shape, mode):
     return PackedModel(shape, vmode, lambda li, m: synth.master(shape, m, li, std),
                        lambda li: synth.layer_vectors(shape, li), synth.model_tables(shape),
                        "cuda")
+
+
+def measure_variant(config, steps, warmup, local_rank, model, batch=1, kv=None):
+    """Device-timed decode steps of a variant of `config` on one GPU: `batch` sequences stepped
+    together (pasts P, P - 96, ...) and/or a KV cache of another element type (kv: "bf16" or
+    "f32").  Greedy tokens fed back on the device; the metric counts every sequence's token."""
+    import torch
+
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape, mode, P, seq, desc = CONFIGS[config]
+    tdt = {None: torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[kv]
+    eb = {None: 2, "bf16": 2, "f32": 4}[kv]
+    Ps = [P - 96 * b for b in range(batch)]
+    dec = Decoder(model, P + steps + warmup + 16, kv_dtype=tdt, batch=batch)
+    for b in range(batch):
+        kp, vp = synth.past_kv(shape, Ps[b], base=17 * b)
+        dec.k_cache[:, b, :, :Ps[b]] = torch.from_numpy(kp).cuda().to(tdt)
+        dec.v_cache[:, b, :, :Ps[b]] = torch.from_numpy(vp).cuda().to(tdt)
+        del kp, vp
+    stream = torch.cuda.current_stream()
+    tok = torch.full((batch,), 151643 % shape.vocab, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(Ps, dtype=torch.int32, device="cuda")
+    logits = torch.empty((batch, shape.vocab), dtype=torch.float32, device="cuda")
+    dec.set_lengths(Ps)
+    for i in range(warmup):
+        dec.step(pos, token=tok, logits=logits, argmax=tok)
+        pos.add_(1)
+    dec.sync_status()
+    dec.set_lengths(Ps)
+    pos.copy_(torch.tensor(Ps, dtype=torch.int32))
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(steps):
+        dec.step(pos, token=tok, logits=logits, argmax=tok)
+        pos.add_(1)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dec.sync_status()
+    ms = ev0.elapsed_time(ev1)
+    us = ms * 1e3 / steps
+    mean_Ps = [p_ + (steps - 1) / 2 for p_ in Ps]
+    byts = variant_step_bytes(shape, mean_Ps, eb)
+    peak, kind = peaks()
+    gbs = byts / (us * 1e-6) / 1e9
+    del dec
+    torch.cuda.empty_cache()
+    return {"workload": config + (f"-batch{batch}" if batch > 1 else "") + (f"-kv-{kv}" if kv else ""),
+            "value": round(batch * steps / (ms * 1e-3), 1), "unit": "tok/s",
+            "us_per_step": round(us, 2), "batch": batch, "pasts": Ps,
+            "kv_dtype": {None: "f16", "bf16": "bf16", "f32": "f32"}[kv],
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": kind,
+                         "bytes_per_step": int(byts)},
+            "clocks": clk}
 
 
 def measure_decode(config, steps, warmup, dist, world, local_rank, model=None):
@@ -464,12 +572,20 @@ def run_ours(args, rank, world, local_rank):
                              "e2e_tok_s": round(pr["e2e_tok_s"], 1), "roofline": pr["roofline"],
                              "clocks": pr["clocks"]}
         result["gpu_launches_prefill"] = pr["launches"] * 10
+    if args.config == "decode-1p5b" and not args.no_extra and world == 1:
+        # batch 2 (the CFG pair) and the bf16 / fp32 KV-cache variants of the same workload
+        variants = {}
+        for batch, kv in ((2, None), (1, "bf16"), (1, "f32")):
+            r3 = measure_variant(args.config, min(args.steps, 64), args.warmup, local_rank, model,
+                                 batch=batch, kv=kv)
+            variants[r3["workload"]] = r3
+        result["variants"] = variants
     del model
     torch.cuda.empty_cache()
     if args.config == "decode-1p5b" and not args.no_extra:
         # the metric's other model size and the long-context decode, each a sub-record with its
         # own roofline, e2e and clocks (same timing protocol, fewer steps)
-        for sub in ("decode-7b", "decode-asr-1p5b"):
+        for sub in ("decode-7b", "decode-asr-1p5b", "decode-0p5b"):
             r2, m2 = measure_decode(sub, min(args.steps, 64), args.warmup, dist, world, local_rank)
             del m2
             torch.cuda.empty_cache()
@@ -477,16 +593,13 @@ def run_ours(args, rank, world, local_rank):
             result[sub.replace("-", "_")] = r2
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         shape, mode, P, _, _ = CONFIGS[args.config]
-        st, sample, thr = oracle_sample_time(shape, mode, P)
-        result["cpu_baseline"] = {"value": round(1.0 / st, 4), "unit": "tok/s", "cores": thr,
-                                  "kind": "oracle", "sample": sample,
-                                  "host_cpus": os.cpu_count()}
-        try:
-            st1, sample1 = oracle_sample_time_1thread(shape, mode, P)
-            result["cpu_baseline"]["one_thread"] = {"value": round(1.0 / st1, 4), "unit": "tok/s",
-                                                    "cores": 1, "sample": sample1}
-        except Exception as e:  # threadpoolctl missing: report the all-cores figure only
-            result["cpu_baseline"]["one_thread"] = {"error": str(e)[:200]}
+        result["cpu_baseline"] = decode_cpu_baseline(shape, mode, P)
+        if "decode_7b" in result:  # the 7B decode (config 4) at all cores and one thread
+            s7, m7, P7, _, _ = CONFIGS["decode-7b"]
+            result["decode_7b"]["cpu_baseline"] = decode_cpu_baseline(s7, m7, P7, samples=3)
+        if "prefill" in result:  # the S = 4530 prefill (config 5) at one thread as well
+            pshape, pmode, pS, pN, _ = PREFILL_CONFIGS["prefill-asr-1p5b"]
+            result["prefill"]["cpu_baseline"] = prefill_cpu_baseline(pshape, pmode, pS, pN)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -171,7 +171,7 @@ vv_status vv_gqa_decode_attn_noalloc(const uint16_t* q, const uint16_t* k_cache,
  * x device fp32 [H] (the residual before the final norm); gamma device fp16 [H]; w_lm device
  * fp16 [V, H]; logits device fp32 [V] or NULL; idx device int32 [1].
  * ws: device workspace of vv_lm_head_argmax_workspace_size(V) bytes, zero-filled once before
- * its first use (left zeroed by every call).  Requirements: H % 256 == 0, H <= 16384.
+ * its first use (left zeroed by every call).  Requirements: H % 64 == 0, 64 <= H <= 16384.
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CAPACITY. */
 size_t vv_lm_head_argmax_workspace_size(int64_t V);
 vv_status vv_lm_head_argmax(const float* x, const uint16_t* gamma, const uint16_t* w_lm,
@@ -182,7 +182,10 @@ vv_status vv_lm_head_argmax(const float* x, const uint16_t* gamma, const uint16_
  * Decoder ([BITNET] decoder_init / decoder_step contracts; [ASR] "Highlights": KV cache kept
  * resident on the GPU, step replayed as one CUDA graph instead of ~1950 launches).
  *
- * The KV cache is the caller's: k_cache and v_cache are device fp16 [L, 1, Hkv, cap, D] each.
+ * The KV cache is the caller's: k_cache and v_cache are device [L, 1, Hkv, cap, D] each, of the
+ * storage type cfg.kv_dtype: fp16 (VV_KV_F16, the contract's type), or the variants bf16
+ * (VV_KV_BF16) and fp32 (VV_KV_F32) ("VibeVoice-ASR — ONNX export for Vernacula", Highlights:
+ * an fp32 cache against fp16 drift).  The pointers are passed as uint16_t* whatever the type.
  * "past K/V in, present K/V out" happens in place: after a call, positions 0..length-1 of the
  * cache are the present keys/values (viewed [L, 1, Hkv, length, D] with stride cap).
  * Keys are stored after RoPE.
@@ -200,7 +203,16 @@ typedef struct vv_config {
   int32_t kv_capacity; /* cap: slots per layer and head in the caller's cache */
   int32_t max_position;/* RoPE table length: position ids must lie in [0, max_position) */
   int32_t max_prefill; /* largest S accepted by vv_decoder_init (0 = no prefill workspace) */
+  int32_t kv_dtype;    /* VV_KV_F16 (0), VV_KV_BF16 (1) or VV_KV_F32 (2); the prefill needs F16 */
+  int32_t batch;       /* sequences stepped together, 1 or 2 (0 means 1); batch 2 is the
+                          CFG pair / two streams ("VibeVoice-1.5B — Current Status": the
+                          negative context stepped alongside the positive one); needs
+                          max_prefill == 0 */
 } vv_config;
+
+#define VV_KV_F16 0
+#define VV_KV_BF16 1
+#define VV_KV_F32 2
 
 typedef struct vv_packed_matrix {
   const uint8_t* q;       /* device uint8 [N, K/32, 16] */
@@ -233,25 +245,36 @@ typedef struct vv_decoder vv_decoder;
 
 /* Create a decoder on the current device.  All weight pointers are borrowed for the decoder's
  * lifetime; k_cache/v_cache likewise.  Allocates the decoder's workspace.  Length starts at 0.
- * Requirements: head_dim == 128, n_kv <= 64, n_q % n_kv == 0, n_q/n_kv <= 8, hidden and inter multiples of
- * 256 (inter <= 32768), 1 <= kv_capacity, 1 <= max_position.
+ * Requirements: head_dim == 128, n_kv <= 64, n_q % n_kv == 0, n_q/n_kv <= 8, hidden a multiple
+ * of 128 (<= 7680; 896 for the Realtime-0.5B backbone), inter a multiple of 256 (<= 65536),
+ * n_q * head_dim <= 7680, 1 <= kv_capacity, 1 <= max_position.  With max_prefill > 0, the
+ * scales of matrices whose K / 32 is not a multiple of 8 are copied once with a padded row
+ * pitch for the prefill GEMMs (the decoder owns the copy).
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CUDA (allocation). */
 vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* weights,
                             uint16_t* k_cache, uint16_t* v_cache, vv_decoder** out);
 vv_status vv_decoder_destroy(vv_decoder* dec);
 
-/* Set the number of valid cache positions (rewind / reset / adopt a cache filled elsewhere).
- * Enqueued on `stream`.  Errors: VV_ERR_CAPACITY if len > kv_capacity, VV_ERR_RANGE if < 0. */
+/* Set the number of valid cache positions (rewind / reset / adopt a cache filled elsewhere) of
+ * every sequence.  Enqueued on `stream`.  Errors: VV_ERR_CAPACITY if len > kv_capacity,
+ * VV_ERR_RANGE if < 0. */
 vv_status vv_decoder_set_length(vv_decoder* dec, int32_t len, vv_stream stream);
+/* The same per sequence: lens is a HOST int32 array of `batch` lengths. */
+vv_status vv_decoder_set_lengths(vv_decoder* dec, const int32_t* lens, vv_stream stream);
+/* Length of sequence 0 / of sequence `seq` (-1 for a bad handle or index); the batch size. */
 int32_t vv_decoder_length(const vv_decoder* dec);
+int32_t vv_decoder_sequence_length(const vv_decoder* dec, int32_t seq);
+int32_t vv_decoder_batch(const vv_decoder* dec);
 
-/* One decode step at batch 1 (decoder_step).
- *   input_embeds: device fp16 [H], or NULL to gather row *token_id of the embedding table
- *   token_id:     device int32 [1] (used only when input_embeds is NULL)
- *   position_id:  device int32 [1]; RoPE angle = position * theta^(-2i/D)
- *   logits:       device fp32 [V] or NULL
- *   argmax_out:   device int32 [1] or NULL (greedy token, lowest index on ties)
- * Appends this position's K/V at slot `length` of every layer, then length += 1.  The first
+/* One decode step (decoder_step) of the decoder's B = batch sequences; every weight byte is
+ * read once for all of them.  Arrays are sequence-major:
+ *   input_embeds: device fp16 [B, H], or NULL to gather rows token_id[b] of the embedding table
+ *   token_id:     device int32 [B] (used only when input_embeds is NULL)
+ *   position_id:  device int32 [B]; RoPE angle = position * theta^(-2i/D)
+ *   logits:       device fp32 [B, V] or NULL
+ *   argmax_out:   device int32 [B] or NULL (greedy token, lowest index on ties)
+ * Sequence b reads and appends cache [L, b, Hkv, ·, D] (the caches are [L, B, Hkv, cap, D]):
+ * its K/V go to slot length_b of every layer, then length_b += 1.  The first
  * call with a given set of pointers captures the step as a CUDA graph; later calls replay it.
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_CAPACITY (length == kv_capacity).  A position outside
  * [0, max_position) or a token outside [0, V) is reported by vv_decoder_sync_status. */
@@ -299,8 +322,8 @@ vv_status vv_decoder_sync_status(vv_decoder* dec, vv_stream stream);
  * at once.  first_token, position: device int32 [1]; tokens_out: device int32 [n_steps], entry i
  * = argmax of step i (entries past the stop are untouched); n_out: HOST int32, the number of
  * steps run (the stop token included).  Needs the persistent step kernel.  Synchronous: one host
- * synchronisation for the whole generation.
- * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (n_steps < 1), VV_ERR_CAPACITY (length + n_steps >
+ * synchronisation for the whole generation.  Batch 1 only.
+ * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE (n_steps < 1, batch > 1), VV_ERR_CAPACITY (length + n_steps >
  * capacity); a device-side error recorded during the generation (VV_ERR_RANGE for a token or
  * position out of range, VV_ERR_TIMEOUT) is returned by this call itself (and cleared), with
  * *n_out still set. */
@@ -323,15 +346,16 @@ vv_status vv_decoder_profile_init(vv_decoder* dec, const int32_t* input_ids,
 
 /* Timeline tap of the persistent step kernel: runs one step (appending a position like
  * vv_decoder_step, without graph capture) with every CTA recording the device clock
- * (%globaltimer, ns) at fixed points of its schedule: kernel start, then for each layer
- * [x staged (QKV)], barrier arrive/exit before attention, barrier arrive/exit before o-proj,
- * x staged, arrive/exit, x staged (gate/up), arrive/exit, x staged (down); layers > 0 start
- * with arrive/exit before QKV; then arrive/exit, x staged (lm_head), end.  stamps: HOST
- * uint64 [grid * max_per_cta]; *grid_out and *per_cta_out receive the CTA count and the number
- * of stamps each CTA wrote.  The last 8 entries of each CTA's row are not stamps: compute
- * thread 0's time blocked on the stage ring per phase kind (QKV, attention, o-proj, gate/up,
- * down, lm_head; ns), then the producer's finishing time and its time blocked on free slots.
- * Synchronous.  VV_ERR_CAPACITY when max_per_cta < 14 L + 11. */
+ * (%globaltimer, ns) at fixed points of its schedule: kernel start; for each layer (layers > 0
+ * first: barrier arrive / exit before q/k/v) x staged for q/k/v, arrive / exit / done of the
+ * attention phase, arrive / exit / done of the o-projection, arrive / exit of the gate/up +
+ * down phase, x staged, gate/up done, h staged, layer end (15 stamps per layer, 13 for layer
+ * 0); then arrive / exit / x staged of the lm_head and the end.  stamps: HOST uint64
+ * [grid * max_per_cta]; *grid_out and *per_cta_out receive the CTA count and the number of
+ * stamps each CTA wrote.  The last 8 entries of each CTA's row are not stamps: compute thread
+ * 0's time blocked on the stage ring per phase kind (QKV, attention, o-proj, gate/up, down,
+ * lm_head; ns), then the producer's finishing time and its time blocked on free slots.
+ * Synchronous.  VV_ERR_CAPACITY when max_per_cta < 15 L + 11. */
 vv_status vv_decoder_step_timeline(vv_decoder* dec, const uint16_t* input_embeds,
                                    const int32_t* token_id, const int32_t* position_id,
                                    uint64_t* stamps, int32_t max_per_cta, int32_t* grid_out,

@@ -26,6 +26,9 @@ VV_ERR_CUDA = 5
 VV_ERR_TIMEOUT = 6
 VV_SYM_INT4 = 0
 VV_TERNARY = 1
+VV_KV_F16 = 0
+VV_KV_BF16 = 1
+VV_KV_F32 = 2
 
 
 class VVError(RuntimeError):
@@ -38,7 +41,7 @@ class vv_config(Structure):
     _fields_ = [("hidden", c_int32), ("layers", c_int32), ("n_q", c_int32), ("n_kv", c_int32),
                 ("head_dim", c_int32), ("inter", c_int32), ("vocab", c_int32), ("eps", c_float),
                 ("rope_theta", c_float), ("kv_capacity", c_int32), ("max_position", c_int32),
-                ("max_prefill", c_int32)]
+                ("max_prefill", c_int32), ("kv_dtype", c_int32), ("batch", c_int32)]
 
 
 class vv_packed_matrix(Structure):
@@ -84,6 +87,9 @@ def _load():
         "vv_decoder_destroy": (S, [P]),
         "vv_decoder_set_length": (S, [P, c_int32, P]),
         "vv_decoder_length": (c_int32, [P]),
+        "vv_decoder_set_lengths": (S, [P, POINTER(c_int32), P]),
+        "vv_decoder_sequence_length": (c_int32, [P, c_int32]),
+        "vv_decoder_batch": (c_int32, [P]),
         "vv_decoder_step": (S, [P, P, P, P, P, P, P]),
         "vv_decoder_init": (S, [P, P, P, c_int64, P, c_int64, c_int64, P, P, P]),
         "vv_decoder_set_trace": (S, [P, P]),

@@ -62,9 +62,17 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   *out = nullptr;
   const vv_config& c = *cfg;
   VV_CHECK_SHAPE(c.head_dim == 128, "head_dim %d (only 128)", c.head_dim);
+  VV_CHECK_SHAPE(c.kv_dtype == VV_KV_F16 || c.kv_dtype == VV_KV_BF16 || c.kv_dtype == VV_KV_F32,
+                 "kv_dtype %d", c.kv_dtype);
+  VV_CHECK_SHAPE(c.batch >= 0 && c.batch <= vv::step_max_batch(), "batch %d (1 .. %d)", c.batch,
+                 vv::step_max_batch());
+  VV_CHECK_SHAPE(c.batch <= 1 || c.max_prefill == 0,
+                 "batch %d: the prefill (max_prefill > 0) runs one sequence", c.batch);
+  VV_CHECK_SHAPE(c.kv_dtype == VV_KV_F16 || c.max_prefill == 0,
+                 "kv_dtype %d: the prefill (max_prefill > 0) writes an fp16 cache only", c.kv_dtype);
   VV_CHECK_SHAPE(c.n_kv >= 1 && c.n_kv <= 64 && c.n_q % c.n_kv == 0 && c.n_q / c.n_kv <= 8,
                  "n_q %d / n_kv %d", c.n_q, c.n_kv);
-  VV_CHECK_SHAPE(c.hidden >= 256 && c.hidden % 256 == 0 && c.hidden <= 7680, "hidden %d",
+  VV_CHECK_SHAPE(c.hidden >= 128 && c.hidden % 128 == 0 && c.hidden <= 7680, "hidden %d",
                  c.hidden);
   VV_CHECK_SHAPE(c.inter >= 64 && c.inter % 256 == 0 && c.inter <= 65536, "inter %d", c.inter);
   VV_CHECK_SHAPE(c.n_q * c.head_dim <= 7680, "n_q*D %d", c.n_q * c.head_dim);
@@ -96,6 +104,8 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   cudaGetDevice(&d->device);
 
   const int H = c.hidden, D = c.head_dim;
+  const int NB = c.batch > 1 ? c.batch : 1;
+  d->nb = NB;
   const int grid = vv::sm_count();
   const int max_tiles = vv::step_max_tiles(c.kv_capacity);
   size_t off = 0;
@@ -104,16 +114,16 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
     off = vv::align_up(off + bytes, 256);
     return o;
   };
-  const size_t o_x = take((size_t)H * 8);
-  const size_t o_qkv = take((size_t)(c.n_q + 2 * c.n_kv) * D * 4);
+  const size_t o_x = take((size_t)NB * H * 8);
+  const size_t o_qkv = take((size_t)NB * (c.n_q + 2 * c.n_kv) * D * 4);
   const size_t o_cos = take((size_t)c.max_position * (D / 2) * 4);
   const size_t o_sin = take((size_t)c.max_position * (D / 2) * 4);
   const size_t o_len = take(16);
   const size_t o_arg = take(16);
   const size_t o_gen = take(16);  // generation: done flag, token count, position
-  const size_t o_part = take(vv::step_attn_part_floats(c.n_kv, max_tiles) * 4);
-  const size_t o_hval = take((size_t)grid * 4);
-  const size_t o_hidx = take((size_t)grid * 4);
+  const size_t o_part = take((size_t)NB * vv::step_attn_part_floats(c.n_kv, max_tiles) * 4);
+  const size_t o_hval = take((size_t)NB * grid * 4);
+  const size_t o_hidx = take((size_t)NB * grid * 4);
   const size_t o_hcnt = take(16);
   const size_t o_bar = take(16);
   const size_t o_layers = take(sizeof(vv::StepLayer) * c.layers);
@@ -148,6 +158,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
   {
     vv::StepParams& p = d->step;
     p.H = H;
+    p.nb = NB;
     p.L = c.layers;
     p.Hq = c.n_q;
     p.Hkv = c.n_kv;
@@ -160,8 +171,9 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
     p.embed = reinterpret_cast<const __half*>(w->embed);
     p.lm_head = reinterpret_cast<const __half*>(w->lm_head);
     p.final_norm = reinterpret_cast<const __half*>(w->final_norm);
-    p.k_cache = reinterpret_cast<__half*>(k_cache);
-    p.v_cache = reinterpret_cast<__half*>(v_cache);
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.kv_type = c.kv_dtype;
     p.cap = c.kv_capacity;
     p.rope_cos = d->rope_cos;
     p.rope_sin = d->rope_sin;
@@ -213,7 +225,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
     if (!st) st = vv::cuda_check(vv::step_configure(p, &nb), "step kernel configuration");
     if (!st && nb < 1) {
       int regs = 0, mt = 0, ss = 0, lb = 0;
-      vv::step_func_info(&regs, &mt, &ss, &lb);
+      vv::step_func_info(NB, &regs, &mt, &ss, &lb);
       st = set_error(VV_ERR_SHAPE,
                      "persistent step: no stage size that holds an attention tile fits one CTA "
                      "per SM (regs %d, max threads %d, static smem %d, local %d, threads %d, "
@@ -240,8 +252,10 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
           cudaMemcpy(d->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice),
           "copy rope sin");
   }
+  if (!st && c.max_prefill > 0) st = vv::cuda_check(vv::prefill_prepare(d), "prefill scales");
   if (st) {
     cudaFree(d->ws);
+    if (d->pf_pad) cudaFree(d->pf_pad);
     delete d;
     return st;
   }
@@ -258,6 +272,7 @@ vv_status vv_decoder_destroy(vv_decoder* d) {
   if (d->capture_stream) cudaStreamDestroy(d->capture_stream);
   if (d->ws) cudaFree(d->ws);
   if (d->pws) cudaFree(d->pws);
+  if (d->pf_pad) cudaFree(d->pf_pad);
   cudaSetDevice(cur);
   delete d;
   return VV_OK;
@@ -268,13 +283,37 @@ vv_status vv_decoder_set_length(vv_decoder* d, int32_t len, vv_stream stream) {
   if (len < 0) return set_error(VV_ERR_RANGE, "length %d < 0", len);
   if (len > d->cfg.kv_capacity)
     return set_error(VV_ERR_CAPACITY, "length %d > capacity %d", len, d->cfg.kv_capacity);
-  vv::set_int_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(d->d_length, len);
-  VV_CUDA(cudaGetLastError());
-  d->len_host = len;
+  for (int b = 0; b < d->nb; ++b) {
+    vv::set_int_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(d->d_length + b, len);
+    VV_CUDA(cudaGetLastError());
+    d->len_host[b] = len;
+  }
   return VV_OK;
 }
 
-int32_t vv_decoder_length(const vv_decoder* d) { return d ? d->len_host : -1; }
+vv_status vv_decoder_set_lengths(vv_decoder* d, const int32_t* lens, vv_stream stream) {
+  VV_CHECK_ARG(d && lens, "vv_decoder_set_lengths: null pointer");
+  for (int b = 0; b < d->nb; ++b) {
+    if (lens[b] < 0) return set_error(VV_ERR_RANGE, "sequence %d: length %d < 0", b, lens[b]);
+    if (lens[b] > d->cfg.kv_capacity)
+      return set_error(VV_ERR_CAPACITY, "sequence %d: length %d > capacity %d", b, lens[b],
+                       d->cfg.kv_capacity);
+  }
+  for (int b = 0; b < d->nb; ++b) {
+    vv::set_int_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(d->d_length + b, lens[b]);
+    VV_CUDA(cudaGetLastError());
+    d->len_host[b] = lens[b];
+  }
+  return VV_OK;
+}
+
+int32_t vv_decoder_length(const vv_decoder* d) { return d ? d->len_host[0] : -1; }
+
+int32_t vv_decoder_sequence_length(const vv_decoder* d, int32_t seq) {
+  return d && seq >= 0 && seq < d->nb ? d->len_host[seq] : -1;
+}
+
+int32_t vv_decoder_batch(const vv_decoder* d) { return d ? d->nb : 0; }
 
 vv_status vv_decoder_set_trace(vv_decoder* d, float* layer_out) {
   VV_CHECK_ARG(d, "null decoder");
@@ -308,13 +347,13 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
   VV_CHECK_ARG(d && position_id, "vv_decoder_step: null decoder or position");
   VV_CHECK_ARG(input_embeds || token_id, "vv_decoder_step: need input_embeds or token_id");
   VV_CHECK_ARG(!input_embeds || vv::aligned16(input_embeds), "input_embeds not 16-byte aligned");
-  if (d->len_host + 1 > d->cfg.kv_capacity)
-    return set_error(VV_ERR_CAPACITY, "KV cache full (%d of %d)", d->len_host,
+  if (d->max_len() + 1 > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "KV cache full (%d of %d)", d->max_len(),
                      d->cfg.kv_capacity);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!d->use_graph) {
     VV_CUDA(vv::enqueue_step(d, input_embeds, token_id, position_id, logits, argmax_out, s));
-    d->len_host += 1;
+    d->advance_lengths(1);
     return VV_OK;
   }
   const void* key[6] = {input_embeds, token_id, position_id, logits, argmax_out, d->trace};
@@ -346,7 +385,7 @@ vv_status vv_decoder_step(vv_decoder* d, const uint16_t* input_embeds, const int
     for (int i = 0; i < 6; ++i) d->gkey[i] = key[i];
   }
   VV_CUDA(cudaGraphLaunch(d->gexec, s));
-  d->len_host += 1;
+  d->advance_lengths(1);
   return VV_OK;
 }
 
@@ -359,7 +398,7 @@ vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
   const int need = vv::step_timeline_stamps(d->cfg.layers);
   if (max_per_cta < need)
     return set_error(VV_ERR_CAPACITY, "max_per_cta %d < %d", max_per_cta, need);
-  if (d->len_host + 1 > d->cfg.kv_capacity)
+  if (d->max_len() + 1 > d->cfg.kv_capacity)
     return set_error(VV_ERR_CAPACITY, "KV cache full");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int grid = d->step.grid;
@@ -388,7 +427,7 @@ vv_status vv_decoder_step_timeline(vv_decoder* d, const uint16_t* input_embeds,
   while (n < max_per_cta - 8 && stamps[n] != 0) ++n;
   *grid_out = grid;
   *per_cta_out = n;
-  d->len_host += 1;
+  d->advance_lengths(1);
   return VV_OK;
 }
 
@@ -409,7 +448,7 @@ vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t
   VV_CUDA(vv::prefill_run(d, input_ids, position_ids, (int)S, audio_features, (int)N,
                           (int)audio_offset, logits, argmax_out,
                           static_cast<cudaStream_t>(stream)));
-  d->len_host = (int32_t)S;
+  d->len_host[0] = (int32_t)S;
   return VV_OK;
 }
 
@@ -447,7 +486,7 @@ vv_status vv_decoder_profile_init(vv_decoder* d, const int32_t* input_ids,
       phase_ms[t.kind[i]] += ms;
       launches[t.kind[i]] += 1;
     }
-    d->len_host = (int32_t)S;
+    d->len_host[0] = (int32_t)S;
   }
   for (auto e : t.ev) cudaEventDestroy(e);
   return st;
@@ -461,8 +500,9 @@ vv_status vv_decoder_generate(vv_decoder* d, const int32_t* first_token, const i
   VV_CHECK_ARG(n_stop >= 0 && n_stop <= vv::kMaxStopIds && (n_stop == 0 || stop_ids),
                "vv_decoder_generate: n_stop %d (0..%d)", n_stop, vv::kMaxStopIds);
   if (n_steps < 1) return set_error(VV_ERR_SHAPE, "n_steps=%d", n_steps);
-  if (d->len_host + n_steps > d->cfg.kv_capacity)
-    return set_error(VV_ERR_CAPACITY, "%d + %d steps exceed the KV capacity %d", d->len_host,
+  if (d->nb != 1) return set_error(VV_ERR_SHAPE, "vv_decoder_generate: batch %d (only 1)", d->nb);
+  if (d->len_host[0] + n_steps > d->cfg.kv_capacity)
+    return set_error(VV_ERR_CAPACITY, "%d + %d steps exceed the KV capacity %d", d->len_host[0],
                      n_steps, d->cfg.kv_capacity);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* done = d->d_gen;
@@ -488,7 +528,7 @@ vv_status vv_decoder_generate(vv_decoder* d, const int32_t* first_token, const i
   int32_t n = 0;
   VV_CUDA(cudaMemcpyAsync(&n, count, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
   VV_CUDA(cudaStreamSynchronize(s));
-  d->len_host += n;
+  d->len_host[0] += n;
   *n_out = n;
   // a device-side error during the generation (a bounded wait that ran out, a token or position
   // out of range) is this call's result

@@ -33,8 +33,19 @@ struct vv_decoder {
   // prefill workspace (allocated lazily by the prefill path)
   unsigned char* pws = nullptr;
   size_t pws_bytes = 0;
+  // scales the prefill GEMMs read, [layer * 7 + matrix] (wq wk wv wo wgate wup wdown), with row
+  // pitch pf_pitch[matrix] in elements (0: K/32).  A matrix whose K/32 is not a multiple of 8
+  // reads a copy with the pitch padded to 8 blocks (pf_pad, owned).
+  std::vector<const uint16_t*> pf_scales;
+  int pf_pitch[7] = {0, 0, 0, 0, 0, 0, 0};
+  uint16_t* pf_pad = nullptr;
 
-  int32_t len_host = 0;
+  int nb = 1;                       // sequences stepped together (batch)
+  int32_t len_host[2] = {0, 0};     // host copy of each sequence's length
+  int32_t max_len() const { return nb > 1 && len_host[1] > len_host[0] ? len_host[1] : len_host[0]; }
+  void advance_lengths(int32_t n) {
+    for (int b = 0; b < nb; ++b) len_host[b] += n;
+  }
   float* trace = nullptr;
   bool use_graph = true;
   vv::StepParams step = {};        // persistent-kernel parameters (per-call pointers patched)
@@ -58,6 +69,8 @@ __global__ void add_int_kernel(int32_t* p, int32_t v);
 // Enqueue one decode step: one launch of the persistent step kernel.
 cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* token,
                          const int32_t* position, float* logits, int32_t* argmax, cudaStream_t s);
+// Prefill preparation at create: the pf_scales table (and padded scale copies where needed).
+cudaError_t prefill_prepare(vv_decoder* d);
 cudaError_t prefill_run(vv_decoder* dec, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
                         cudaStream_t s, PrefillTimer* timer = nullptr);

@@ -252,7 +252,7 @@ extern "C" vv_status vv_lm_head_argmax(const float* x, const uint16_t* gamma, co
   VV_CHECK_ARG(x && gamma && w_lm && idx && ws, "vv_lm_head_argmax: null pointer");
   VV_CHECK_ARG(vv::aligned16(x) && vv::aligned16(w_lm) && vv::aligned16(ws),
                "vv_lm_head_argmax: pointers must be 16-byte aligned");
-  VV_CHECK_SHAPE(H >= 256 && H % 256 == 0 && H <= 16384, "vv_lm_head_argmax: H=%lld",
+  VV_CHECK_SHAPE(H >= 64 && H % 64 == 0 && H <= 16384, "vv_lm_head_argmax: H=%lld",
                  (long long)H);
   VV_CHECK_SHAPE(V >= 1 && V < (int64_t(1) << 30), "vv_lm_head_argmax: V=%lld", (long long)V);
   const size_t need = vv::lm_head_workspace_bytes((int)V);

@@ -140,6 +140,55 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+namespace {
+// Rows of `kb` fp16 scales copied to a row pitch of `pitch` >= kb elements, zero-padded.
+__global__ void pad_scales_kernel(const uint16_t* __restrict__ src, int rows, int kb, int pitch,
+                                  uint16_t* __restrict__ dst) {
+  const int64_t n = (int64_t)rows * pitch;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / pitch), c = (int)(i % pitch);
+    dst[i] = c < kb ? src[(size_t)r * kb + c] : (uint16_t)0;
+  }
+}
+}  // namespace
+
+cudaError_t prefill_prepare(vv_decoder* d) {
+  const vv_config& c = d->cfg;
+  const int H = c.hidden, HQD = c.n_q * D, I = c.inter;
+  const int Km[7] = {H, H, H, HQD, H, H, I};
+  const int Nm[7] = {c.n_q * D, c.n_kv * D, c.n_kv * D, H, I, I, H};
+  size_t pad_elems = 0;
+  for (int m = 0; m < 7; ++m) {
+    const int kb = Km[m] / 32;
+    d->pf_pitch[m] = kb % 8 == 0 ? 0 : (kb + 7) & ~7;
+    if (d->pf_pitch[m]) pad_elems += (size_t)c.layers * Nm[m] * d->pf_pitch[m];
+  }
+  d->pf_scales.assign((size_t)c.layers * 7, nullptr);
+  if (pad_elems) {
+    cudaError_t e = cudaMalloc(&d->pf_pad, pad_elems * 2);
+    if (e != cudaSuccess) return e;
+  }
+  size_t off = 0;
+  for (int l = 0; l < c.layers; ++l) {
+    const vv_layer_weights& L = d->layers[l];
+    const vv_packed_matrix* mats[7] = {&L.wq, &L.wk, &L.wv, &L.wo, &L.wgate, &L.wup, &L.wdown};
+    for (int m = 0; m < 7; ++m) {
+      if (!d->pf_pitch[m]) {
+        d->pf_scales[(size_t)l * 7 + m] = mats[m]->scales;
+        continue;
+      }
+      uint16_t* dst = d->pf_pad + off;
+      off += (size_t)Nm[m] * d->pf_pitch[m];
+      pad_scales_kernel<<<256, 256>>>(mats[m]->scales, Nm[m], Km[m] / 32, d->pf_pitch[m], dst);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      d->pf_scales[(size_t)l * 7 + m] = dst;
+    }
+  }
+  return cudaDeviceSynchronize();
+}
+
 cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
                         cudaStream_t s, PrefillTimer* timer) {
@@ -206,10 +255,12 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.input_norm), c.eps, Xn);
     VV_MARK(kPfMisc);
     PackedB pb = {};
-    pb.q[0] = w.wq.q; pb.s[0] = w.wq.scales; pb.rows[0] = HQD;
-    pb.q[1] = w.wk.q; pb.s[1] = w.wk.scales; pb.rows[1] = Hkv * D;
-    pb.q[2] = w.wv.q; pb.s[2] = w.wv.scales; pb.rows[2] = Hkv * D;
+    const uint16_t* const* ps = &d->pf_scales[(size_t)l * 7];
+    pb.q[0] = w.wq.q; pb.s[0] = ps[0]; pb.rows[0] = HQD;
+    pb.q[1] = w.wk.q; pb.s[1] = ps[1]; pb.rows[1] = Hkv * D;
+    pb.q[2] = w.wv.q; pb.s[2] = ps[2]; pb.rows[2] = Hkv * D;
     pb.nseg = 3;
+    pb.s_pitch = d->pf_pitch[0];
     const uint16_t* bsrc[3] = {w.bq, w.bk, w.bv};
     const int brows[3] = {HQD, Hkv * D, Hkv * D};
     int boff = 0;
@@ -248,8 +299,9 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     VV_MARK(kPfAttn);
     // ---- O projection + residual
     pb = {};
-    pb.q[0] = w.wo.q; pb.s[0] = w.wo.scales; pb.rows[0] = H;
+    pb.q[0] = w.wo.q; pb.s[0] = ps[3]; pb.rows[0] = H;
     pb.nseg = 1;
+    pb.s_pitch = d->pf_pitch[3];
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;
@@ -261,10 +313,11 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.post_norm), c.eps, Xn);
     VV_MARK(kPfMisc);
     pb = {};
-    pb.q[0] = w.wgate.q; pb.s[0] = w.wgate.scales; pb.rows[0] = I;
-    pb.q[1] = w.wup.q; pb.s[1] = w.wup.scales; pb.rows[1] = I;
+    pb.q[0] = w.wgate.q; pb.s[0] = ps[4]; pb.rows[0] = I;
+    pb.q[1] = w.wup.q; pb.s[1] = ps[5]; pb.rows[1] = I;
     pb.nseg = 2;
     pb.interleave = 1;
+    pb.s_pitch = d->pf_pitch[4];
     ep = {};
     ep.out_f16 = Hm;
     ep.ldo = I;
@@ -274,8 +327,9 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     VV_MARK(kPfGemm);
     // ---- down + residual
     pb = {};
-    pb.q[0] = w.wdown.q; pb.s[0] = w.wdown.scales; pb.rows[0] = H;
+    pb.q[0] = w.wdown.q; pb.s[0] = ps[6]; pb.rows[0] = H;
     pb.nseg = 1;
+    pb.s_pitch = d->pf_pitch[6];
     ep = {};
     ep.out_f32 = X;
     ep.ldo = H;

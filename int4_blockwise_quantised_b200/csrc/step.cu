@@ -36,6 +36,7 @@
 // (k + 1) x grid arrivals; the last CTA of the launch resets it); every wait is bounded
 // (VV_ERR_TIMEOUT in the device error word after 2 s, then the kernel carries on).  The
 // cooperative launch guarantees that all CTAs are resident.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -53,7 +54,9 @@ constexpr int kThreads = (NW + 1) * 32;
 constexpr int NT = NW * 32;            // compute threads
 constexpr int D = 128;
 constexpr int TT = 64;                 // attention tile (positions)
+constexpr int kTileVOff = TT * D * 2;  // V rows of a tile start here: 64 rows of 2 bytes or 32 of 4
 constexpr int kMaxG = 8;
+constexpr int kMaxB = 2;               // sequences stepped together (batch)
 constexpr int kPart = 132;             // floats per (tile, head) partial: m, l, -, -, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxK = 16384;           // largest GEMV input length (hidden, n_q * D)
@@ -68,6 +71,15 @@ __device__ __forceinline__ void cbar() {  // compute warps only
 __device__ __forceinline__ void cta_range(int n, int cta, int ncta, int& r0, int& r1) {
   r0 = (int)((int64_t)n * cta / ncta);
   r1 = (int)((int64_t)n * (cta + 1) / ncta);
+}
+
+// This CTA's rows of the stacked [Wq; Wk; Wv] (n rows, n even): split in pairs of rows, so
+// that every run of scale rows a stage copies starts and ends on a 16-byte boundary (a row of
+// scales is K/16 bytes, a multiple of 8 for K % 128 == 0).
+__device__ __forceinline__ void qkv_range(int n, int cta, int ncta, int& r0, int& r1) {
+  cta_range(n / 2, cta, ncta, r0, r1);
+  r0 *= 2;
+  r1 *= 2;
 }
 
 __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
@@ -219,22 +231,25 @@ __device__ __forceinline__ void consume_end(Ring& r, int slot) {
 
 // --------------------------------------------------------------------------- stage geometry
 // Row phases (QKV, gate/up): stage = [seg0 codes rps rows][seg1 codes][seg0 scales][seg1 scales],
-// rows of K/32 x 16 code bytes and K/32 x 2 scale bytes.  Column phases (o-proj, down): stage =
+// rows of K/32 x 16 code bytes and K/32 x 2 scale bytes (K % 128 == 0: a scale row is a multiple
+// of 8 bytes, so runs of an even number of rows from an even row are 16-byte aligned).  Column phases (o-proj, down): stage =
 // [codes rps rows x nb x 16][scales rps rows x nb x 2] of a column image.
 __device__ __forceinline__ int rows_per_stage(int row_bytes, int stage_bytes) {
   int r = stage_bytes / row_bytes;
   return r & ~7;  // a multiple of 8 rows keeps every scale run 16-byte aligned
 }
 
-// One attention tile: `rows` past K rows and V rows (256 bytes each, consecutive in the cache)
-// with one copy each: K rows at the stage base, V rows TT rows after them.
-__device__ void produce_kv_rows(Ring& r, const __half* k, const __half* v, int rows, uint64_t pol) {
-  const uint32_t bytes = (uint32_t)rows * D * 2;
+// One attention tile: past K rows and V rows (D elements of elem_bytes each, consecutive in the
+// cache; `row_units` = rows x elem_bytes) with one copy each: K rows at the stage base, V rows
+// kTileVOff bytes after them.
+__device__ void produce_kv_rows(Ring& r, const unsigned char* k, const unsigned char* v,
+                                int row_units, uint64_t pol) {
+  const uint32_t bytes = (uint32_t)row_units * D;
   const int slot = produce_begin(r, 2 * bytes);
   unsigned char* dst = r.base + (size_t)slot * r.stage_bytes;
   if (bytes) {
     bulk_g2s_stream(dst, k, bytes, &r.full[slot], pol);
-    bulk_g2s_stream(dst + (size_t)TT * D * 2, v, bytes, &r.full[slot], pol);
+    bulk_g2s_stream(dst + kTileVOff, v, bytes, &r.full[slot], pol);
   }
 }
 
@@ -293,13 +308,36 @@ __device__ void produce_cols(Ring& r, const unsigned char* img, int rows, int nb
   }
 }
 
-// Attention tile size of a launch: 32 positions when doubling the tiles of 64 still gives every
-// item its own CTA, else 64.  Producer and consumers compute the same.
-__device__ __forceinline__ int tile_for(int past, int Hkv) {
-  const int n64 = (past + 1 + TT - 1) / TT;
-  return 2 * Hkv * n64 <= (int)gridDim.x ? TT / 2 : TT;
-}
+// The attention items of a launch: sequence b has nt[b] tiles of tt positions per KV head;
+// items are numbered sequence-major, (b, g, t) for b < nb, g < Hkv, t < nt[b].  Tiles of 32
+// positions when doubling the tiles of 64 still gives every item its own CTA (always for 4-byte
+// K/V, whose 32 rows fill kTileVOff), else 64.  Producer and consumers compute the same plan.
+struct AttnPlan {
+  int tt;
+  int nt[kMaxB];
+  int total;
+};
+__device__ __forceinline__ int kv_bytes(const StepParams& p) { return p.kv_type == 2 ? 4 : 2; }
 __device__ __forceinline__ int ntiles_for(int past, int tt) { return (past + 1 + tt - 1) / tt; }
+__device__ __forceinline__ AttnPlan attn_plan(const StepParams& p, const int* past) {
+  AttnPlan a;
+  int n64 = 0;
+  for (int b = 0; b < p.nb; ++b) n64 += ntiles_for(past[b], TT);
+  a.tt = (kv_bytes(p) == 4 || 2 * p.Hkv * n64 <= (int)gridDim.x) ? TT / 2 : TT;
+  a.total = 0;
+  for (int b = 0; b < kMaxB; ++b) {
+    a.nt[b] = b < p.nb ? ntiles_for(past[b], a.tt) : 0;
+    a.total += p.Hkv * a.nt[b];
+  }
+  return a;
+}
+__device__ __forceinline__ void attn_item_of(const AttnPlan& a, int Hkv, int it, int& b, int& g,
+                                             int& t) {
+  b = 0;
+  while (b + 1 < kMaxB && it >= Hkv * a.nt[b]) it -= Hkv * a.nt[b++];
+  g = it / a.nt[b];
+  t = it % a.nt[b];
+}
 __device__ __forceinline__ int n_slices(const StepParams& p) { return p.I / kSlice; }
 __device__ __forceinline__ int slices_of(const StepParams& p, int cta) {
   const int ns = n_slices(p);
@@ -316,13 +354,12 @@ __host__ __device__ __forceinline__ int wd_rot(int H, int c, int grid) {
   return (int)((((long long)c * H) / grid) & ~31LL) % H;
 }
 
-__device__ void producer(const StepParams& p, Ring& r, int past) {
+__device__ void producer(const StepParams& p, Ring& r, const int* past) {
   const uint64_t pol = policy_evict_first();
   const int cta = blockIdx.x, ncta = gridDim.x;
   const int H = p.H, Hq = p.Hq, Hkv = p.Hkv;
   const int nqkv = (Hq + 2 * Hkv) * D;
-  const int tt = tile_for(past, Hkv);
-  const int nt = ntiles_for(past, tt);
+  const AttnPlan plan = attn_plan(p, past);
   const int nrb = H / kORows;
   const int nsl = slices_of(p, cta);
   const int ns = n_slices(p);
@@ -331,14 +368,18 @@ __device__ void producer(const StepParams& p, Ring& r, int past) {
   for (int l = 0; l < p.L; ++l) {
     const StepLayer& w = p.layers[l];
     int r0, r1;
-    cta_range(nqkv, cta, ncta, r0, r1);
+    qkv_range(nqkv, cta, ncta, r0, r1);
     const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
     produce_qkv(r, w, H, r0, r1, bounds, pol);
-    for (int it = cta; it < Hkv * nt; it += ncta) {
-      const int g = it / nt, t = it % nt;
-      const int p0 = t * tt, p1 = min(p0 + tt, past);
-      const size_t off = ((size_t)(l * Hkv + g) * p.cap + p0) * D;
-      produce_kv_rows(r, p.k_cache + off, p.v_cache + off, max(p1 - p0, 0), pol);
+    for (int it = cta; it < plan.total; it += ncta) {
+      int b, g, t;
+      attn_item_of(plan, Hkv, it, b, g, t);
+      const int p0 = t * plan.tt, p1 = min(p0 + plan.tt, past[b]);
+      const size_t off = ((size_t)((l * p.nb + b) * Hkv + g) * p.cap + p0) * D;
+      const int eb = kv_bytes(p);
+      produce_kv_rows(r, static_cast<const unsigned char*>(p.k_cache) + off * eb,
+                      static_cast<const unsigned char*>(p.v_cache) + off * eb, max(p1 - p0, 0) * eb,
+                      pol);
     }
     for (int i = o0; i < o1; ++i)
       produce_cols(r, w.wo_img + (size_t)i * kORows * 4 * 18, kORows, 4, pol);
@@ -503,12 +544,17 @@ struct UnitMap {
   int rps, rq, rs;
 };
 
-// Rows per pass (R) for `units` units with `gpw` lane groups per warp: the R in {1, 2, 4} ({2, 4}
-// for pairs) that minimises the busiest warp's share (R x its passes), the larger R on ties.
-__device__ __forceinline__ int pick_r(int units, int gpw, bool pair) {
+// Rows per pass (R) for `units` units with 2^lg_gpw lane groups per warp: the R in {1, 2, 4}
+// ({2, 4} for pairs) that minimises the busiest warp's share (R x its passes), the larger R on
+// ties.  Shifts and a division by the constant NW only (this runs for every stage).
+__device__ __forceinline__ int pick_r(int units, int lg_gpw, bool pair) {
   int best = pair ? 2 : 1, cost_best = 1 << 30;
-  for (int R = best; R <= 4; R *= 2) {
-    const int passes = (units + gpw * R - 1) / (gpw * R);
+#pragma unroll
+  for (int lr = 0; lr <= 2; ++lr) {
+    const int R = 1 << lr;
+    if (R < best) continue;
+    const int sh = lg_gpw + lr;
+    const int passes = (units + (1 << sh) - 1) >> sh;
     const int cost = R * ((passes + NW - 1) / NW);
     if (cost <= cost_best) {
       best = R;
@@ -518,11 +564,12 @@ __device__ __forceinline__ int pick_r(int units, int gpw, bool pair) {
   return best;
 }
 
-// The units of one stage against the staged X: LPR lanes per unit (lane % LPR strides the
-// half-blocks), R units per lane group and pass.  fin(u, y0, y1) is called by the group's first
-// lane once per unit (y1 = 0), or with NSEG == 2 once per row with both matrices' results.
-template <int LPR, int R, int NSEG, class Fin>
-__device__ __forceinline__ void gemv_pass(const XOp& xo, int NHB, int units, const UnitMap& m,
+// The units of one stage against the staged X of NB sequences (the weights are read once for
+// all of them): LPR lanes per unit (lane % LPR strides the half-blocks), R units per lane group
+// and pass.  fin(u, y0, y1) is called by the group's first lane once per unit with y0[b] the
+// result of sequence b (y1 unused), or with NSEG == 2 once per row with both matrices' results.
+template <int LPR, int R, int NSEG, int NB, class Fin>
+__device__ __forceinline__ void gemv_pass(const XOp* xo, int NHB, int units, const UnitMap& m,
                                           Fin fin) {
   static_assert(NSEG == 1 || R % NSEG == 0, "pairs need an even R");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -540,52 +587,65 @@ __device__ __forceinline__ void gemv_pass(const XOp& xo, int NHB, int units, con
       qa[k] = m.q0 + (uint32_t)(idx * m.rq);
       sa[k] = m.s0 + (uint32_t)(idx * m.rs);
     }
-    float acc[R];
+    float acc[R][NB];
 #pragma unroll
-    for (int k = 0; k < R; ++k) acc[k] = 0.f;
+    for (int k = 0; k < R; ++k)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) acc[k][b] = 0.f;
 #pragma unroll 2
     for (int hb = sub; hb < NHB; hb += LPR) {
-      const uint4 xa = lds128(xo.xq_a + hb * 16), xb = lds128(xo.xq_a + (NHB + hb) * 16);
-      const int cr = (int)lds32(xo.corr_a + hb * 4);
-      const float f = __uint_as_float(lds32(xo.fb_a + (hb >> 1) * 4));
+      uint4 xa[NB], xb[NB];
+      int cr[NB];
+      float f[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        xa[b] = lds128(xo[b].xq_a + hb * 16);
+        xb[b] = lds128(xo[b].xq_a + (NHB + hb) * 16);
+        cr[b] = (int)lds32(xo[b].corr_a + hb * 4);
+        f[b] = __uint_as_float(lds32(xo[b].fb_a + (hb >> 1) * 4));
+      }
 #pragma unroll
       for (int k = 0; k < R; ++k) {
         const uint2 wv = lds64(qa[k] + hb * 8);
-        const float s = lds_half(sa[k] + (hb >> 1) * 2) * f;
-        acc[k] = fmaf(s, (float)hb_dot(wv, xa, xb, cr), acc[k]);
+        const float sc = lds_half(sa[k] + (hb >> 1) * 2);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          acc[k][b] = fmaf(sc * f[b], (float)hb_dot(wv, xa[b], xb[b], cr[b]), acc[k][b]);
       }
     }
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
+    for (int k = 0; k < R; ++k)
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
-    }
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) acc[k][b] += __shfl_xor_sync(0xffffffffu, acc[k][b], o);
     if (sub == 0) {
 #pragma unroll
       for (int k = 0; k < R; k += NSEG)
-        if (u0 + k < units) fin(u0 + k, acc[k], NSEG == 2 ? acc[k + NSEG - 1] : 0.f);
+        if (u0 + k < units) fin(u0 + k, acc[k], acc[k + NSEG - 1]);
     }
   }
 }
 
 // One stage: lanes per unit from the row length (a lane takes about 4 half-blocks of short rows;
 // rows longer than 16 half-blocks take a whole warp), rows per pass from the unit count.
-template <int NSEG, class Fin>
-__device__ __forceinline__ void gemv_stage(const XOp& xo, int NHB, int units, const UnitMap& m,
+template <int NSEG, int NB, class Fin>
+__device__ __forceinline__ void gemv_stage(const XOp* xo, int NHB, int units, const UnitMap& m,
                                            Fin fin) {
   auto go = [&](auto lpr_c) {
     constexpr int LPR = decltype(lpr_c)::value;
-    const int R = pick_r(units, 32 / LPR, NSEG == 2);
+    constexpr int kLgGpw = LPR == 32 ? 0 : LPR == 4 ? 3 : LPR == 2 ? 4 : 5;
+    const int R = pick_r(units, kLgGpw, NSEG == 2);
     if constexpr (NSEG == 1) {
       if (R == 1) {
-        gemv_pass<LPR, 1, NSEG>(xo, NHB, units, m, fin);
+        gemv_pass<LPR, 1, NSEG, NB>(xo, NHB, units, m, fin);
         return;
       }
     }
     if (R == 2)
-      gemv_pass<LPR, 2, NSEG>(xo, NHB, units, m, fin);
+      gemv_pass<LPR, 2, NSEG, NB>(xo, NHB, units, m, fin);
     else
-      gemv_pass<LPR, 4, NSEG>(xo, NHB, units, m, fin);
+      gemv_pass<LPR, 4, NSEG, NB>(xo, NHB, units, m, fin);
   };
   if (NHB > 16) {
     go(std::integral_constant<int, 32>());
@@ -601,9 +661,9 @@ __device__ __forceinline__ void gemv_stage(const XOp& xo, int NHB, int units, co
   }
 }
 
-// Row phase: the stages of rows [r0, r1) of NSEG matrices.  fin(row, y0, y1).
-template <int NSEG, class Fin>
-__device__ void consume_rows(Ring& r, const XOp& xo, int K, int r0, int r1, Fin fin) {
+// Row phase: the stages of rows [r0, r1) of NSEG matrices.  fin(row, y0, y1) with y0[b], y1[b].
+template <int NSEG, int NB, class Fin>
+__device__ void consume_rows(Ring& r, const XOp* xo, int K, int r0, int r1, Fin fin) {
   const int KB = K >> 5, NHB = K >> 4;
   const int rq = KB * 16, rs = KB * 2;
   const int rps = rows_per_stage((rq + rs) * NSEG, r.stage_bytes);
@@ -612,15 +672,16 @@ __device__ void consume_rows(Ring& r, const XOp& xo, int K, int r0, int r1, Fin 
     int slot;
     const uint32_t st = consume_begin(r, slot);
     const UnitMap m{st, st + (uint32_t)(NSEG * rps * rq), rps, rq, rs};
-    gemv_stage<NSEG>(xo, NHB, n * NSEG, m,
-                     [&](int u, float y0, float y1) { fin(a + u / NSEG, y0, y1); });
+    gemv_stage<NSEG, NB>(xo, NHB, n * NSEG, m,
+                         [&](int u, const float* y0, const float* y1) { fin(a + u / NSEG, y0, y1); });
     consume_end(r, slot);
   }
 }
 
 // Column phase: the stages of a column image of `rows_total` rows x nb blocks (K = 32 nb).
-template <class Fin>
-__device__ void consume_cols(Ring& r, const XOp& xo, int rows_total, int nb, Fin fin) {
+// fin(row, y) with y[b].
+template <int NB, class Fin>
+__device__ void consume_cols(Ring& r, const XOp* xo, int rows_total, int nb, Fin fin) {
   const int NHB = nb * 2;
   const int rps = rows_per_stage(nb * 18, r.stage_bytes);
   for (int a = 0; a < rows_total; a += rps) {
@@ -628,29 +689,71 @@ __device__ void consume_cols(Ring& r, const XOp& xo, int rows_total, int nb, Fin
     int slot;
     const uint32_t st = consume_begin(r, slot);
     const UnitMap m{st, st + (uint32_t)(rps * nb * 16), rps, nb * 16, nb * 2};
-    gemv_stage<1>(xo, NHB, n, m, [&](int u, float y0, float) { fin(a + u, y0); });
+    gemv_stage<1, NB>(xo, NHB, n, m, [&](int u, const float* y, const float*) { fin(a + u, y); });
     consume_end(r, slot);
   }
 }
 
 // ------------------------------------------------------------------------------- attention
+// K/V storage types of the cache (and of the attention tiles in shared memory): fp16 (the
+// contract), bf16 and fp32 (the variants).  load8 widens 8 consecutive elements to fp32 pairs.
+struct KvF16 {
+  using T = __half;
+  static constexpr int kBytes = 2;
+  __device__ static T from(float v) { return __float2half_rn(v); }
+  __device__ static void load8(const T* p, float2 (&f)[4]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    f[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+    f[1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+    f[2] = __half22float2(*reinterpret_cast<const __half2*>(&u.z));
+    f[3] = __half22float2(*reinterpret_cast<const __half2*>(&u.w));
+  }
+};
+struct KvBF16 {
+  using T = __nv_bfloat16;
+  static constexpr int kBytes = 2;
+  __device__ static T from(float v) { return __float2bfloat16_rn(v); }
+  __device__ static void load8(const T* p, float2 (&f)[4]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  }
+};
+struct KvF32 {
+  using T = float;
+  static constexpr int kBytes = 4;
+  __device__ static T from(float v) { return v; }
+  __device__ static void load8(const T* p, float2 (&f)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    f[0] = make_float2(a.x, a.y);
+    f[1] = make_float2(a.z, a.w);
+    f[2] = make_float2(b.x, b.y);
+    f[3] = make_float2(b.z, b.w);
+  }
+};
 struct AttnScratch {
-  float cs[D / 2], sn[D / 2];  // RoPE cos/sin at this step's position
+  float cs[kMaxB][D / 2], sn[kMaxB][D / 2];  // RoPE cos/sin at each sequence's position
   float q[kMaxG][D];
   float s[kMaxG][TT];
   float m[kMaxG], l[kMaxG];
   float pv[4][kMaxG][D];  // P.V partial sums per position quarter
 };
 
-__device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int g, int t,
-                          int past, int tt) {
+template <class KV>
+__device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, int b, int g,
+                          int t, int past, int tt) {
+  using T = typename KV::T;
+  const float* cs_b = as.cs[b];
+  const float* sn_b = as.sn[b];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.Hq / p.Hkv;
   const int nt = ntiles_for(past, tt);
   const int npos = past + 1;
   const int p0 = t * tt;
   const int n = min(tt, npos - p0);
-  const float* qkv = p.qkv;
+  const float* qkv = p.qkv + (size_t)b * (p.Hq + 2 * p.Hkv) * D;
   // q of the group (rotated, scaled into the log2 domain) and, on the tile holding the new
   // position, the new k/v: every global load is issued before any is used (one L2 round trip).
   const float qscale = p.scale * kLog2e;
@@ -683,22 +786,22 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     if (i < G * D) {
       const int h = i / D, d = i % D;
       const int fi = d & (D / 2 - 1);
-      const float cs = as.cs[fi], sn = as.sn[fi];
+      const float cs = cs_b[fi], sn = sn_b[fi];
       as.q[h][d] = (d < D / 2 ? qa[j] * cs - qb[j] * sn : qb[j] * cs + qa[j] * sn) * qscale;
     }
   }
   int slot;
   consume_begin(r, slot);
-  __half* kt = reinterpret_cast<__half*>(r.base + (size_t)slot * r.stage_bytes);
-  __half* vt = kt + TT * D;
+  T* kt = reinterpret_cast<T*>(r.base + (size_t)slot * r.stage_bytes);
+  T* vt = reinterpret_cast<T*>(r.base + (size_t)slot * r.stage_bytes + kTileVOff);
   if (newpos && tid < D) {  // this tile holds the new position: rotate k, append k/v
     const int d = tid, fi = d & (D / 2 - 1);
-    const float cs = as.cs[fi], sn = as.sn[fi];
-    const __half kn = __float2half_rn(d < D / 2 ? ka * cs - kb * sn : kb * cs + ka * sn);
-    const __half vn = __float2half_rn(vv);
-    const size_t off = ((size_t)(l * p.Hkv + g) * p.cap + past) * D + d;
-    p.k_cache[off] = kn;
-    p.v_cache[off] = vn;
+    const float cs = cs_b[fi], sn = sn_b[fi];
+    const T kn = KV::from(d < D / 2 ? ka * cs - kb * sn : kb * cs + ka * sn);
+    const T vn = KV::from(vv);
+    const size_t off = ((size_t)((l * p.nb + b) * p.Hkv + g) * p.cap + past) * D + d;
+    static_cast<T*>(p.k_cache)[off] = kn;
+    static_cast<T*>(p.v_cache)[off] = vn;
     kt[(past - p0) * D + d] = kn;
     vt[(past - p0) * D + d] = vn;
   }
@@ -710,18 +813,19 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     const int h = item >> 1, pp = (item & 1) * 32 + lane;
     float sc = -INFINITY;
     if (pp < n) {
-      const __half* kr = kt + pp * D;
+      const T* kr = kt + pp * D;
       float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {
         const int cc = (c + lane) & 15;
-        const uint4 kv = *reinterpret_cast<const uint4*>(kr + cc * 8);
+        float2 k8[4];
+        KV::load8(kr + cc * 8, k8);
         const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
         const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
-        acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.x)), make_float2(qa4.x, qa4.y), acc);
-        acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.y)), make_float2(qa4.z, qa4.w), acc2);
-        acc = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.z)), make_float2(qb4.x, qb4.y), acc);
-        acc2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&kv.w)), make_float2(qb4.z, qb4.w), acc2);
+        acc = __ffma2_rn(k8[0], make_float2(qa4.x, qa4.y), acc);
+        acc2 = __ffma2_rn(k8[1], make_float2(qa4.z, qa4.w), acc2);
+        acc = __ffma2_rn(k8[2], make_float2(qb4.x, qb4.y), acc);
+        acc2 = __ffma2_rn(k8[3], make_float2(qb4.z, qb4.w), acc2);
       }
       sc = (acc.x + acc.y) + (acc2.x + acc2.y);
     }
@@ -754,20 +858,21 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
       const float* ph = as.s[h];
       const int p_end = min(n, q * 16 + 16);
       for (int pp = q * 16; pp < p_end; ++pp) {
-        const uint4 v8 = *reinterpret_cast<const uint4*>(vt + pp * D + o * 8);
+        float2 v8[4];
+        KV::load8(vt + pp * D + o * 8, v8);
         const float w = ph[pp];
         const float2 ww = make_float2(w, w);
-        a0 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.x)), ww, a0);
-        a1 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.y)), ww, a1);
-        a2 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.z)), ww, a2);
-        a3 = __ffma2_rn(__half22float2(*reinterpret_cast<const __half2*>(&v8.w)), ww, a3);
+        a0 = __ffma2_rn(v8[0], ww, a0);
+        a1 = __ffma2_rn(v8[1], ww, a1);
+        a2 = __ffma2_rn(v8[2], ww, a2);
+        a3 = __ffma2_rn(v8[3], ww, a3);
       }
       float4* dst = reinterpret_cast<float4*>(&as.pv[q][h][o * 8]);
       dst[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
       dst[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
     }
     cbar();
-    float* part = p.attn_part + ((size_t)(g * p.max_tiles + t) * kMaxG) * kPart;
+    float* part = p.attn_part + (((size_t)b * p.Hkv + g) * p.max_tiles + t) * kMaxG * kPart;
     for (int idx = tid; idx < G * D; idx += NT) {
       const int h = idx >> 7, d = idx & (D - 1);
       part[h * kPart + 4 + d] = (as.pv[0][h][d] + as.pv[1][h][d]) + (as.pv[2][h][d] + as.pv[3][h][d]);
@@ -784,10 +889,11 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
 // Merge head h's partials over the nt tiles: M = max_t m_t, L = sum_t l_t 2^(m_t - M),
 // o[d] = sum_t 2^(m_t - M) o_t[d] / L.  Threads (d4, tile slice): 32 float4 columns x up to
 // 15 tile slices, combined through shared memory.  Result in out[128] (fp32, shared).
-__device__ void merge_head(const StepParams& p, int h, int nt, float* scratch, float* out) {
+__device__ void merge_head(const StepParams& p, int b, int h, int nt, float* scratch, float* out) {
   const int tid = threadIdx.x;
   const int G = p.Hq / p.Hkv, g = h / G, hh = h % G;
-  const float* base = p.attn_part + ((size_t)g * p.max_tiles * kMaxG + hh) * kPart;
+  const float* base =
+      p.attn_part + (((size_t)b * p.Hkv + g) * p.max_tiles * kMaxG + hh) * kPart;
   const int d4 = tid & 31, ts = tid >> 5;  // ts in [0, NW)
   float M = -INFINITY, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -859,6 +965,7 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+template <int NB>
 __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -879,39 +986,45 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   r.slot = 0;
   r.par = 0;
   r.wrapped = false;
-  // shared layout after the ring: xq [2][kMaxK/16] uint4 | corr [kMaxK/16] | fb [kMaxK/32] |
-  // hbuf [kMaxK/...] | AttnScratch | red[64] | mbarriers
+  // shared layout after the ring, per sequence b: xq [2][kMaxK/16] uint4 | corr [kMaxK/16] |
+  // fb [kMaxK/32] | hbuf; then AttnScratch | red[64] | mbarriers
   unsigned char* sp = smem + (size_t)p.nstages * p.stage_bytes;
   const int maxK = max(H, Hq * D);
   const int nhb_max = maxK / 16;
-  XOp xo;
-  xo.xq = reinterpret_cast<uint4*>(sp);
-  sp += (size_t)nhb_max * 2 * 16;
-  xo.corr = reinterpret_cast<int*>(sp);
-  sp += (size_t)nhb_max * 4;
-  xo.fb = reinterpret_cast<float*>(sp);
-  sp += (size_t)nhb_max * 2;
-  xo.xq_a = smem_u32(xo.xq);
-  xo.corr_a = smem_u32(xo.corr);
-  xo.fb_a = smem_u32(xo.fb);
   const int nsl = slices_of(p, blockIdx.x);
-  float* hbuf = reinterpret_cast<float*>(sp);  // h of this CTA's slices, then o_h of an o-item
-  sp += (size_t)max(nsl * kSlice, D) * 4;
-  sp = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sp) + 15) & ~uintptr_t(15));
+  XOp xo[NB];
+  float* hbuf[NB];  // h of this CTA's slices, then o_h of an o-item
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    xo[b].xq = reinterpret_cast<uint4*>(sp);
+    sp += (size_t)nhb_max * 2 * 16;
+    xo[b].corr = reinterpret_cast<int*>(sp);
+    sp += (size_t)nhb_max * 4;
+    xo[b].fb = reinterpret_cast<float*>(sp);
+    sp += (size_t)nhb_max * 2;
+    xo[b].xq_a = smem_u32(xo[b].xq);
+    xo[b].corr_a = smem_u32(xo[b].corr);
+    xo[b].fb_a = smem_u32(xo[b].fb);
+    hbuf[b] = reinterpret_cast<float*>(sp);
+    sp += (size_t)max(nsl * kSlice, D) * 4;
+    sp = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sp) + 15) & ~uintptr_t(15));
+  }
   AttnScratch& as = *reinterpret_cast<AttnScratch*>(sp);
   float* red = reinterpret_cast<float*>(&as + 1);  // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 64) + 15) &
                                                ~uintptr_t(15));
   r.full = bars;
   r.empty = bars + p.nstages;
-  __shared__ float s_val[NW];
-  __shared__ int s_idx[NW];
+  __shared__ float s_val[NB][NW];
+  __shared__ int s_idx[NB][NW];
   __shared__ int s_last;
 
   // generation stopped by an earlier step of the same vv_decoder_generate call: every CTA sees
   // the same word (written by the previous launch) and leaves before touching anything
   if (p.gen_done && __ldcg(p.gen_done) != 0) return;
-  const int past = *p.length;
+  int past[kMaxB];
+#pragma unroll
+  for (int b = 0; b < kMaxB; ++b) past[b] = b < NB ? p.length[b] : 0;
   if (tid == 0) {
     for (int i = 0; i < p.nstages; ++i) {
       mbar_init(&r.full[i], 1);
@@ -939,49 +1052,56 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   stamp(p, sk);
   const int cta = blockIdx.x, ncta = gridDim.x;
   const int nqkv = (Hq + 2 * Hkv) * D;
-  const int tt = tile_for(past, Hkv);
-  const int nt = ntiles_for(past, tt);
+  const AttnPlan plan = attn_plan(p, past);
   const int nrb = H / kORows;
   const int ns = n_slices(p);
-  int pos = *p.position;
-  if (pos < 0 || pos >= p.max_position) {
-    if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
-    pos = min(max(pos, 0), p.max_position - 1);
-  }
-  for (int i = tid; i < D / 2; i += NT) {
-    as.cs[i] = p.rope_cos[(size_t)pos * (D / 2) + i];
-    as.sn[i] = p.rope_sin[(size_t)pos * (D / 2) + i];
-  }
-  const __half* e16 = p.input_embeds;
-  if (!e16) {
-    int tok = __ldcg(p.token);
-    if (tok < 0 || tok >= p.V) {
+  const __half* e16[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    int pos = p.position[b];
+    if (pos < 0 || pos >= p.max_position) {
       if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
-      tok = min(max(tok, 0), p.V - 1);
+      pos = min(max(pos, 0), p.max_position - 1);
     }
-    e16 = p.embed + (size_t)tok * H;
+    for (int i = tid; i < D / 2; i += NT) {
+      as.cs[b][i] = p.rope_cos[(size_t)pos * (D / 2) + i];
+      as.sn[b][i] = p.rope_sin[(size_t)pos * (D / 2) + i];
+    }
+    e16[b] = p.input_embeds ? p.input_embeds + (size_t)b * H : nullptr;
+    if (!e16[b]) {
+      int tok = __ldcg(p.token + b);
+      if (tok < 0 || tok >= p.V) {
+        if (tid == 0 && cta == 0) set_device_error(VV_ERR_RANGE);
+        tok = min(max(tok, 0), p.V - 1);
+      }
+      e16[b] = p.embed + (size_t)tok * H;
+    }
   }
-  auto load_emb = [&](int k) -> float4 {
-    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(e16 + k));
+  auto load_emb = [&](int b, int k) -> float4 {
+    const uint2 hv = __ldcg(reinterpret_cast<const uint2*>(e16[b] + k));
     const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
-    return make_float4(a.x, a.y, b.x, b.y);
+    const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+    return make_float4(a.x, a.y, c.x, c.y);
   };
-  auto load_x = [&](int k) -> float4 {
-    const ulonglong2 a = __ldcg(reinterpret_cast<const ulonglong2*>(p.x_acc + k));
-    const ulonglong2 b = __ldcg(reinterpret_cast<const ulonglong2*>(p.x_acc + k + 2));
-    return make_float4(from_fix(a.x), from_fix(a.y), from_fix(b.x), from_fix(b.y));
+  auto load_x = [&](int b, int k) -> float4 {
+    const unsigned long long* xb = p.x_acc + (size_t)b * H;
+    const ulonglong2 a = __ldcg(reinterpret_cast<const ulonglong2*>(xb + k));
+    const ulonglong2 c = __ldcg(reinterpret_cast<const ulonglong2*>(xb + k + 2));
+    return make_float4(from_fix(a.x), from_fix(a.y), from_fix(c.x), from_fix(c.y));
   };
   // residual = embedding: this CTA's share of rows, before the first barrier (the o-phase adds
   // come after two more barriers)
   {
     int hr0, hr1;
     cta_range(H / 4, cta, ncta, hr0, hr1);
-    for (int i = hr0 + tid; i < hr1; i += NT) {
-      const float4 v = load_emb(4 * i);
-      reinterpret_cast<ulonglong2*>(p.x_acc + 4 * i)[0] = make_ulonglong2(to_fix(v.x), to_fix(v.y));
-      reinterpret_cast<ulonglong2*>(p.x_acc + 4 * i)[1] = make_ulonglong2(to_fix(v.z), to_fix(v.w));
-    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      for (int i = hr0 + tid; i < hr1; i += NT) {
+        const float4 v = load_emb(b, 4 * i);
+        unsigned long long* xb = p.x_acc + (size_t)b * H + 4 * i;
+        reinterpret_cast<ulonglong2*>(xb)[0] = make_ulonglong2(to_fix(v.x), to_fix(v.y));
+        reinterpret_cast<ulonglong2*>(xb)[1] = make_ulonglong2(to_fix(v.z), to_fix(v.w));
+      }
   }
   int o0, o1;
   cta_range(Hq * nrb, cta, ncta, o0, o1);
@@ -991,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     // ---------------------------------------------------------------- QKV
     r.ph = 0;
     int r0, r1;
-    cta_range(nqkv, cta, ncta, r0, r1);
+    qkv_range(nqkv, cta, ncta, r0, r1);
     // this CTA's q/k/v biases (at most NT rows): the load is issued before the barrier (the
     // biases do not depend on x), the store to shared memory after it (as.q is free until the
     // attention phase; stage_idp's barriers order the stores before the GEMV reads them)
@@ -1000,27 +1120,41 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
       const int row = r0 + tid;
       const int m = row < bounds[1] ? 0 : (row < bounds[2] ? 1 : 2);
-      const __half* b = w.bias[m];
-      if (b) bias_v = __half2float(__ldg(b + (row - bounds[m])));
+      const __half* bp = w.bias[m];
+      if (bp) bias_v = __half2float(__ldg(bp + (row - bounds[m])));
     }
     if (l > 0) grid_barrier(p, gen, sk);
     if (tid < r1 - r0) (&as.q[0][0])[tid] = bias_v;
-    if (l == 0) {
-      stage_idp(xo, load_emb, w.in_norm, p.eps, H, red, nullptr);
-    } else {
-      float* tr = (p.trace && cta == 0) ? p.trace + (size_t)(l - 1) * H : nullptr;
-      stage_idp(xo, load_x, w.in_norm, p.eps, H, red, tr);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (l == 0) {
+        stage_idp(xo[b], [&](int k) { return load_emb(b, k); }, w.in_norm, p.eps, H, red, nullptr);
+      } else {
+        float* tr = (p.trace && cta == 0 && b == 0) ? p.trace + (size_t)(l - 1) * H : nullptr;
+        stage_idp(xo[b], [&](int k) { return load_x(b, k); }, w.in_norm, p.eps, H, red, tr);
+      }
     }
     stamp(p, sk);
     {
       const float* bs = &as.q[0][0] - r0;
-      consume_rows<1>(r, xo, H, r0, r1,
-                          [&](int row, float y, float) { p.qkv[row] = y + bs[row]; });
+      consume_rows<1, NB>(r, xo, H, r0, r1, [&](int row, const float* y, const float*) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) p.qkv[(size_t)b * nqkv + row] = y[b] + bs[row];
+      });
     }
     // ---------------------------------------------------------------- ATTN
     r.ph = 1;
     grid_barrier(p, gen, sk);
-    for (int it = cta; it < Hkv * nt; it += ncta) attn_item(p, r, as, l, it / nt, it % nt, past, tt);
+    for (int it = cta; it < plan.total; it += ncta) {
+      int b, g, t;
+      attn_item_of(plan, Hkv, it, b, g, t);
+      if (p.kv_type == 0)
+        attn_item<KvF16>(p, r, as, l, b, g, t, past[b], plan.tt);
+      else if (p.kv_type == 1)
+        attn_item<KvBF16>(p, r, as, l, b, g, t, past[b], plan.tt);
+      else
+        attn_item<KvF32>(p, r, as, l, b, g, t, past[b], plan.tt);
+    }
     stamp(p, sk);
     // ---------------------------------------------------------------- O
     r.ph = 2;
@@ -1030,13 +1164,20 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       for (int i = o0; i < o1; ++i) {
         const int h = i / nrb, rb = i % nrb;
         if (h != cur_h) {
-          merge_head(p, h, nt, &as.pv[0][0][0], hbuf);
-          stage_idp(xo, [&](int k) { return *reinterpret_cast<const float4*>(hbuf + k); },
-                    nullptr, 0.f, D, red, nullptr);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            merge_head(p, b, h, plan.nt[b], &as.pv[0][0][0], hbuf[b]);
+            const float* hb = hbuf[b];
+            stage_idp(xo[b], [&](int k) { return *reinterpret_cast<const float4*>(hb + k); },
+                      nullptr, 0.f, D, red, nullptr);
+          }
           cur_h = h;
         }
         unsigned long long* xr = p.x_acc + (size_t)rb * kORows;
-        consume_cols(r, xo, kORows, 4, [&](int row, float y) { red_add_u64(xr + row, to_fix(y)); });
+        consume_cols<NB>(r, xo, kORows, 4, [&](int row, const float* y) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b) red_add_u64(xr + (size_t)b * H + row, to_fix(y[b]));
+        });
       }
     }
     stamp(p, sk);
@@ -1044,25 +1185,34 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     r.ph = 3;
     grid_barrier(p, gen, sk);
     if (nsl > 0) {
-      stage_idp(xo, load_x, w.post_norm, p.eps, H, red, nullptr);
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        stage_idp(xo[b], [&](int k) { return load_x(b, k); }, w.post_norm, p.eps, H, red, nullptr);
       stamp(p, sk);
       int j = 0;
       for (int s = cta; s < ns; s += ncta, ++j) {
-        float* hs = hbuf + j * kSlice - s * kSlice;
-        consume_rows<2>(r, xo, H, s * kSlice, (s + 1) * kSlice, [&](int row, float g, float u) {
-          hs[row] = g / (1.f + __expf(-g)) * u;
+        const int off = j * kSlice - s * kSlice;
+        consume_rows<2, NB>(r, xo, H, s * kSlice, (s + 1) * kSlice,
+                            [&](int row, const float* g, const float* u) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b) hbuf[b][off + row] = g[b] / (1.f + __expf(-g[b])) * u[b];
         });
       }
       cbar();
       stamp(p, sk);
       r.ph = 4;
-      stage_idp(xo, [&](int k) { return *reinterpret_cast<const float4*>(hbuf + k); }, nullptr,
-                0.f, nsl * kSlice, red, nullptr);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float* hb = hbuf[b];
+        stage_idp(xo[b], [&](int k) { return *reinterpret_cast<const float4*>(hb + k); }, nullptr,
+                  0.f, nsl * kSlice, red, nullptr);
+      }
       stamp(p, sk);
       const int rot = wd_rot(H, cta, ncta);
-      consume_cols(r, xo, H, 2 * nsl, [&](int i, float y) {
+      consume_cols<NB>(r, xo, H, 2 * nsl, [&](int i, const float* y) {
         const int row = i + rot < H ? i + rot : i + rot - H;
-        red_add_u64(p.x_acc + row, to_fix(y));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) red_add_u64(p.x_acc + (size_t)b * H + row, to_fix(y[b]));
       });
     } else {
       stamp(p, sk);
@@ -1074,14 +1224,15 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
   // ------------------------------------------------------------------------------ HEAD
   r.ph = 5;
   grid_barrier(p, gen, sk);
-  __half* xs = reinterpret_cast<__half*>(xo.xq);
-  {
+  const int nhb = H >> 4;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
     // final RMSNorm, x rounded once to fp16 in the pair layout of the fp16 head dot
-    const int nhb = H >> 4;
-    float* tr = (p.trace && cta == 0) ? p.trace + (size_t)(p.L - 1) * H : nullptr;
+    __half* xs = reinterpret_cast<__half*>(xo[b].xq);
+    float* tr = (p.trace && cta == 0 && b == 0) ? p.trace + (size_t)(p.L - 1) * H : nullptr;
     float ss = 0.f;
     for (int k = tid * 4; k < H; k += NT * 4) {
-      const float4 v = load_x(k);
+      const float4 v = load_x(b, k);
       if (tr) *reinterpret_cast<float4*>(tr + k) = v;
       ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     }
@@ -1093,7 +1244,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     for (int i = 0; i < NW; ++i) tot += red[i];
     const float inv = rsqrtf(tot / (float)H + p.eps);
     for (int k = tid * 4; k < H; k += NT * 4) {
-      const float4 v = load_x(k);
+      const float4 v = load_x(b, k);
       const float y[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -1102,8 +1253,13 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     cbar();
   }
   stamp(p, sk);
-  float best = -INFINITY;
-  int best_i = 0x7fffffff;
+  float best[NB];
+  int best_i[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    best[b] = -INFINITY;
+    best_i[b] = 0x7fffffff;
+  }
   {
     int r0, r1;
     cta_range(p.V, cta, ncta, r0, r1);
@@ -1111,16 +1267,17 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     const int rps = min(64, r.stage_bytes / rb);
     const int nch = H >> 3;  // 16-byte chunks per row
     // x of 16-byte weight chunk c (8 columns: half-block c/2, word c%2) = pair word (c%2, c/2);
-    // held in registers for c = lane + 32 j when the row fits (H <= 1536)
-    const int nhb = H >> 4;
-    const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
-    const bool regHead = nch <= 32 * 2 * kHeadRegHB;
+    // held in registers for c = lane + 32 j when the row fits (H <= 1536) and one sequence runs
+    const uint4* xs4[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) xs4[b] = reinterpret_cast<const uint4*>(xo[b].xq);
+    const bool regHead = NB == 1 && nch <= 32 * 2 * kHeadRegHB;
     uint4 xr[2 * kHeadRegHB];
     if (regHead) {
 #pragma unroll
       for (int j = 0; j < 2 * kHeadRegHB; ++j) {
         const int c = lane + 32 * j;
-        xr[j] = c < nch ? xs4[(c & 1) * nhb + (c >> 1)] : make_uint4(0u, 0u, 0u, 0u);
+        xr[j] = c < nch ? xs4[0][(c & 1) * nhb + (c >> 1)] : make_uint4(0u, 0u, 0u, 0u);
       }
     }
     for (int a = r0; a < r1; a += rps) {
@@ -1130,36 +1287,46 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
       const unsigned char* st = r.base + (size_t)slot * r.stage_bytes;
       for (int i = warp; i < n; i += NW) {
         const unsigned char* row = st + (size_t)i * rb;
-        float acc = 0.f;
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[b] = 0.f;
         // weights (w0,w1)(w2,w3)(w4,w5)(w6,w7) against x pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7)
-        auto chunk = [&](const uint4 wv, const uint4 xv) {
+        auto chunk = [&](const uint4 wv, auto xv_of) {
           uint32_t p04, p15, p26, p37;
           asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(p04) : "r"(wv.x), "r"(wv.z));
           asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(p15) : "r"(wv.x), "r"(wv.z));
           asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(p26) : "r"(wv.y), "r"(wv.w));
           asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(p37) : "r"(wv.y), "r"(wv.w));
-          acc = fma2_f16_f32(p04, xv.x, acc);
-          acc = fma2_f16_f32(p15, xv.y, acc);
-          acc = fma2_f16_f32(p26, xv.z, acc);
-          acc = fma2_f16_f32(p37, xv.w, acc);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const uint4 xv = xv_of(b);
+            acc[b] = fma2_f16_f32(p04, xv.x, acc[b]);
+            acc[b] = fma2_f16_f32(p15, xv.y, acc[b]);
+            acc[b] = fma2_f16_f32(p26, xv.z, acc[b]);
+            acc[b] = fma2_f16_f32(p37, xv.w, acc[b]);
+          }
         };
         if (regHead) {
 #pragma unroll
           for (int j = 0; j < 2 * kHeadRegHB; ++j) {
             const int c = lane + 32 * j;
-            if (c < nch) chunk(*reinterpret_cast<const uint4*>(row + c * 16), xr[j]);
+            if (c < nch) chunk(*reinterpret_cast<const uint4*>(row + c * 16), [&](int) { return xr[j]; });
           }
         } else {
           for (int c = lane; c < nch; c += 32)
-            chunk(*reinterpret_cast<const uint4*>(row + c * 16), xs4[(c & 1) * nhb + (c >> 1)]);
+            chunk(*reinterpret_cast<const uint4*>(row + c * 16),
+                  [&](int b) { return xs4[b][(c & 1) * nhb + (c >> 1)]; });
         }
-        const float v = warp_sum(acc);
-        if (lane == 0) {
-          const int vr = a + i;
-          if (p.logits) p.logits[vr] = v;
-          if (better(v, vr, best, best_i)) {
-            best = v;
-            best_i = vr;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float v = warp_sum(acc[b]);
+          if (lane == 0) {
+            const int vr = a + i;
+            if (p.logits) p.logits[(size_t)b * p.V + vr] = v;
+            if (better(v, vr, best[b], best_i[b])) {
+              best[b] = v;
+              best_i[b] = vr;
+            }
           }
         }
       }
@@ -1167,33 +1334,40 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     }
   }
   if (lane == 0) {
-    s_val[warp] = best;
-    s_idx[warp] = best_i;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      s_val[b][warp] = best[b];
+      s_idx[b][warp] = best_i[b];
+    }
   }
   cbar();
   stamp(p, sk);
   if (tid == 0) {
-    float bv = s_val[0];
-    int bi = s_idx[0];
-    for (int w2 = 1; w2 < NW; ++w2)
-      if (better(s_val[w2], s_idx[w2], bv, bi)) {
-        bv = s_val[w2];
-        bi = s_idx[w2];
-      }
-    p.head_val[cta] = bv;
-    p.head_idx[cta] = bi;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float bv = s_val[b][0];
+      int bi = s_idx[b][0];
+      for (int w2 = 1; w2 < NW; ++w2)
+        if (better(s_val[b][w2], s_idx[b][w2], bv, bi)) {
+          bv = s_val[b][w2];
+          bi = s_idx[b][w2];
+        }
+      p.head_val[(size_t)b * ncta + cta] = bv;
+      p.head_idx[(size_t)b * ncta + cta] = bi;
+    }
     __threadfence();
     s_last = atomicAdd(p.head_count, 1) == ncta - 1;
   }
   cbar();
   if (!s_last) return;
   __threadfence();
-  if (warp == 0) {
+  if (warp < NB) {  // warp b reduces sequence b
+    const int b = warp;
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     for (int i = lane; i < ncta; i += 32) {
-      const float v = __ldcg(p.head_val + i);
-      const int ix = __ldcg(p.head_idx + i);
+      const float v = __ldcg(p.head_val + (size_t)b * ncta + i);
+      const int ix = __ldcg(p.head_idx + (size_t)b * ncta + i);
       if (better(v, ix, bv, bi)) {
         bv = v;
         bi = ix;
@@ -1210,17 +1384,20 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     }
     if (lane == 0) {
       const int tok = bi == 0x7fffffff ? 0 : bi;
-      *p.argmax = tok;
-      *p.head_count = 0;
-      *p.bar_count = 0u;  // every CTA has passed every barrier of this launch
-      *p.length = past + 1;
-      if (p.gen_done) {  // every CTA read the position at its start, long before this point
+      p.argmax[b] = tok;
+      p.length[b] = past[b] + 1;
+      if (p.gen_done) {  // batch 1 only; every CTA read the position at its start
         *p.gen_count += 1;
         *p.gen_pos += 1;
         for (int j = 0; j < p.n_stop; ++j)
           if (tok == p.stop_ids[j]) *p.gen_done = 1;
       }
     }
+  }
+  cbar();  // warps 0..NB-1 have read the partials and the counter use is over
+  if (tid == 0) {
+    *p.head_count = 0;
+    *p.bar_count = 0u;  // every CTA has passed every barrier of this launch
   }
 }
 
@@ -1302,14 +1479,18 @@ size_t step_smem_bytes(const StepParams& p) {
   const int ns = p.I / kSlice;
   const int nsl_max = (ns + p.grid - 1) / p.grid;
   size_t b = (size_t)p.nstages * p.stage_bytes;
-  b += (size_t)nhb_max * 2 * 16 + (size_t)nhb_max * 4 + (size_t)nhb_max * 2;
-  b += (size_t)std::max(nsl_max * kSlice, D) * 4;
-  b = (b + 15) & ~size_t(15);
+  for (int s = 0; s < std::max(p.nb, 1); ++s) {
+    b += (size_t)nhb_max * 2 * 16 + (size_t)nhb_max * 4 + (size_t)nhb_max * 2;
+    b += (size_t)std::max(nsl_max * kSlice, D) * 4;
+    b = (b + 15) & ~size_t(15);
+  }
   b += sizeof(AttnScratch) + 64 * 4 + 16 + 2 * p.nstages * 8 + 64;
   return b;
 }
 
 int step_threads() { return kThreads; }
+
+int step_max_batch() { return kMaxB; }
 
 size_t step_attn_part_floats(int Hkv, int max_tiles) {
   return (size_t)Hkv * max_tiles * kMaxG * kPart;
@@ -1317,22 +1498,31 @@ size_t step_attn_part_floats(int Hkv, int max_tiles) {
 
 int step_max_tiles(int cap) { return (cap + 1 + TT / 2 - 1) / (TT / 2); }
 
+namespace {
+// The kernel instance of a batch size.
+const void* step_fn(int nb) {
+  return nb == 2 ? reinterpret_cast<const void*>(step_kernel<2>)
+                 : reinterpret_cast<const void*>(step_kernel<1>);
+}
+}  // namespace
+
 // Pick the largest stage size (>= one attention tile, 1 KB steps) for which one CTA per SM is
 // resident.
 cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
-  cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+  const void* fn = step_fn(p.nb);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                        (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   *blocks_per_sm = 0;
   for (; p.stage_bytes >= 2 * TT * D * 2; p.stage_bytes -= 1024) {
     const size_t smem = step_smem_bytes(p);
-    e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
       cudaGetLastError();
       continue;
     }
     int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, step_kernel, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (nb >= 1) {
       *blocks_per_sm = nb;
@@ -1342,9 +1532,9 @@ cudaError_t step_configure(StepParams& p, int* blocks_per_sm) {
   return cudaSuccess;
 }
 
-void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_bytes) {
+void step_func_info(int nb, int* regs, int* max_threads, int* static_smem, int* local_bytes) {
   cudaFuncAttributes fa = {};
-  cudaFuncGetAttributes(&fa, step_kernel);
+  cudaFuncGetAttributes(&fa, step_fn(nb));
   *regs = fa.numRegs;
   *max_threads = fa.maxThreadsPerBlock;
   *static_smem = (int)fa.sharedSizeBytes;
@@ -1352,9 +1542,9 @@ void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_by
 }
 
 cudaError_t launch_step(const StepParams& p, cudaStream_t s) {
+  const void* fn = step_fn(p.nb);
   const size_t smem = step_smem_bytes(p);
-  cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.grid);
@@ -1366,7 +1556,8 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t s) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, step_kernel, p);
+  void* args[] = {const_cast<StepParams*>(&p)};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 }  // namespace vv

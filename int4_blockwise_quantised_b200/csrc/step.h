@@ -25,15 +25,22 @@ struct StepLayer {
   const unsigned char* wd_img;  // per CTA: H rows x (2 x its slices) blocks
 };
 
+// Batch: nb sequences are stepped together (nb <= step_max_batch()); every weight byte is read
+// once for all of them.  Per-sequence buffers are laid out sequence-major: input_embeds [nb][H],
+// token / position / argmax / length [nb], logits [nb][V], x_acc [nb][H], qkv [nb][nqkv],
+// attn_part [nb][Hkv][max_tiles][8][132], head_val / head_idx [nb][grid], caches
+// [L][nb][Hkv][cap][D].
 struct StepParams {
   int H, L, Hq, Hkv, I, V;
+  int nb;
   float eps, scale;
   const StepLayer* layers;  // device array [L]
   const __half* embed;
   const __half* lm_head;
   const __half* final_norm;
-  __half* k_cache;
-  __half* v_cache;
+  void* k_cache;  // [L][nb][Hkv][cap][D] of the storage type kv_type
+  void* v_cache;
+  int kv_type;    // 0 fp16, 1 bf16, 2 fp32 (VV_KV_*)
   int cap;
   const float* rope_cos;
   const float* rope_sin;
@@ -77,7 +84,9 @@ int step_threads();
 size_t step_attn_part_floats(int Hkv, int max_tiles);
 int step_max_tiles(int cap);
 cudaError_t step_configure(StepParams& p, int* blocks_per_sm);
-void step_func_info(int* regs, int* max_threads, int* static_smem, int* local_bytes);
+void step_func_info(int nb, int* regs, int* max_threads, int* static_smem, int* local_bytes);
+// Largest batch (sequences per step) of the step kernel.
+int step_max_batch();
 cudaError_t launch_step(const StepParams& p, cudaStream_t s);
 // Column images: bytes per layer, and the kernels that build them from the caller's matrices.
 size_t step_wo_image_bytes(int H, int Hq);

@@ -77,20 +77,30 @@ class PackedModel:
         return mw, arr
 
 
-class Decoder:
-    """A vv_decoder with a caller-owned fp16 KV cache [L, 1, Hkv, cap, D] (K and V)."""
+KV_DTYPES = {torch.float16: _vv.VV_KV_F16, torch.bfloat16: _vv.VV_KV_BF16,
+             torch.float32: _vv.VV_KV_F32}
 
-    def __init__(self, model, kv_capacity, max_position=None, max_prefill=0):
+
+class Decoder:
+    """A vv_decoder with a caller-owned KV cache [L, batch, Hkv, cap, D] (K and V) of kv_dtype:
+    torch.float16 (the contract), or the bf16 / fp32 variants (decode only).  batch 2 steps two
+    sequences together (decode only); step() then takes [2]-shaped position / token / argmax,
+    [2, H] input_embeds and [2, V] logits."""
+
+    def __init__(self, model, kv_capacity, max_position=None, max_prefill=0,
+                 kv_dtype=torch.float16, batch=1):
         sh = model.shape
         self.model = model
         self.capacity = kv_capacity
+        self.batch = batch
         dev = model.device
-        kv_shape = (sh.layers, 1, sh.n_kv, kv_capacity, sh.head_dim)
-        self.k_cache = torch.zeros(kv_shape, dtype=torch.float16, device=dev)
-        self.v_cache = torch.zeros(kv_shape, dtype=torch.float16, device=dev)
+        kv_shape = (sh.layers, batch, sh.n_kv, kv_capacity, sh.head_dim)
+        self.k_cache = torch.zeros(kv_shape, dtype=kv_dtype, device=dev)
+        self.v_cache = torch.zeros(kv_shape, dtype=kv_dtype, device=dev)
         self.cfg = _vv.vv_config(sh.hidden, sh.layers, sh.n_q, sh.n_kv, sh.head_dim, sh.inter,
                                  sh.vocab, sh.eps, sh.theta, kv_capacity,
-                                 max_position or max(kv_capacity, 8192), max_prefill)
+                                 max_position or max(kv_capacity, 8192), max_prefill,
+                                 KV_DTYPES[kv_dtype], batch)
         self._mw, self._arr = model.c_weights()
         h = ctypes.c_void_p()
         check(_vv.lib.vv_decoder_create(ctypes.byref(self.cfg), ctypes.byref(self._mw),
@@ -120,6 +130,13 @@ class Decoder:
     def set_length(self, n, stream=None):
         check(_vv.lib.vv_decoder_set_length(self.handle, n, stream_handle(stream)))
 
+    def set_lengths(self, lens, stream=None):
+        arr = (ctypes.c_int32 * len(lens))(*[int(v) for v in lens])
+        check(_vv.lib.vv_decoder_set_lengths(self.handle, arr, stream_handle(stream)))
+
+    def sequence_length(self, b):
+        return _vv.lib.vv_decoder_sequence_length(self.handle, b)
+
     def set_trace(self, buf):
         self._trace = buf
         check(_vv.lib.vv_decoder_set_trace(self.handle, ptr(buf)))
@@ -135,7 +152,8 @@ class Decoder:
 
     def step(self, position, input_embeds=None, token=None, logits=None, argmax=None,
              stream=None):
-        """One decode step.  position/token: device int32 [1]; input_embeds fp16 [H]."""
+        """One decode step of every sequence.  position/token/argmax: device int32 [batch];
+        input_embeds fp16 [batch, H]; logits fp32 [batch, V]."""
         check(_vv.lib.vv_decoder_step(self.handle, ptr(input_embeds), ptr(token), ptr(position),
                                       ptr(logits), ptr(argmax), stream_handle(stream)))
 

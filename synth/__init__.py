@@ -49,6 +49,10 @@ class Shape:
 # Qwen2.5-1.5B backbone of VibeVoice-1.5B / ASR-BitNet and Qwen2.5-7B of VibeVoice-ASR(-HF).
 SHAPE_1P5B = Shape("qwen2-1.5b", 1536, 28, 12, 2, 128, 8960, 151936, tied=True)
 SHAPE_7B = Shape("qwen2-7b", 3584, 28, 28, 4, 128, 18944, 152064, tied=False)
+# Realtime-0.5B backbone: 20 layers, hidden 896 (the pages' figures).  The pages give no head
+# counts or MLP width: 7 query heads and 1 KV head of dimension 128 (7 x 128 = 896, the head
+# dimension of the other backbones) and the Qwen2.5-0.5B MLP width 4864 are this build's reading.
+SHAPE_0P5B = Shape("realtime-0.5b", 896, 20, 7, 1, 128, 4864, 151936, tied=True)
 # Small shapes for fast parity runs; several tiles and a ragged tail on every axis that has one.
 SHAPE_TINY = Shape("tiny", 256, 2, 4, 2, 128, 768, 1000, tied=True)
 SHAPE_SMALL = Shape("small", 1536, 2, 12, 2, 128, 8960, 4099, tied=True)

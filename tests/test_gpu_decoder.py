@@ -135,7 +135,9 @@ def test_capacity_and_range_errors():
 # ------------------------------------------------------------------------------------ prefill
 @pytest.mark.parametrize("shape,mode,S,N", [(synth.SHAPE_TINY, "int4", 37, 20),
                                             (synth.SHAPE_SMALL, "ternary", 70, 40),
-                                            (synth.SHAPE_SMALL, "int4", 300, 200)])
+                                            (synth.SHAPE_SMALL, "int4", 300, 200),
+                                            (synth.Shape("0.5b-2l", 896, 2, 7, 1, 128, 4864,
+                                                         2053, tied=True), "int4", 150, 100)])
 def test_prefill_then_steps_match_oracle(shape, mode, S, N):
     from int4_blockwise_quantised_b200.model import Decoder
 

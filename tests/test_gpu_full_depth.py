@@ -36,3 +36,9 @@ def test_decode_asr_ternary_across_p4736():
     """ASR-shaped long context, ternary weights: steps from P = 4731 to 4738 cross the point
     (past + 1 = 4737) where the 2 KV heads need 150 attention tiles, more than one per CTA."""
     run_steps(synth.SHAPE_SMALL, "ternary", 4731, 8)
+
+
+def test_decode_realtime_0p5b_20_layers():
+    """The Realtime-0.5B backbone at full depth (20 layers, hidden 896 = 7 column blocks of the
+    o-proj image, one KV head of 7 query heads, 76 gate/up slices on 148 CTAs), P = 512, 4 steps."""
+    run_steps(synth.SHAPE_0P5B, "int4", 512, 4)
