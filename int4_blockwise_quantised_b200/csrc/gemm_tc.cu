@@ -152,6 +152,122 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, const floa
   }
 }
 
+template <int EPI, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmEpilogue e, const int M, const int N, const int K) {
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::kStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + STAGES * kStageA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::kStageB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;   // [2] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;    // [2] epilogue -> MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = N / BN;
+  const int tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int kblocks = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+    }
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;  // running k-block counter across tiles
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (g >= STAGES) mbar_wait(&empty[s], ((g / STAGES) - 1) & 1);
+          mbar_arrive_expect_tx(&full[s], kStageA + C::kStageB);
+          tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m_blk * BM, &full[s]);
+          tma_load_2d(sB + s * C::kStageB, &tmB, kb * BK, n_blk * BN, &full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int g = 0, i = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2) mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1);  // epilogue done with it
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++g) {
+          const int s = g % STAGES;
+          mbar_wait(&full[s], (g / STAGES) & 1);
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * C::kStageB);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // 32 bytes per K=16 slice inside the swizzled row
+            umma_f16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), C::kIdesc,
+                     (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);  // stage free once these MMAs have read it
+        }
+        umma_commit(&acc_full[buf]);  // accumulator complete
+      }
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31
+    const int q = warp & 3;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int m_blk = t / n_tiles, n_blk = t % n_tiles;
+      const int buf = i & 1;
+      const int row = m_blk * BM + q * 32 + lane;
+      mbar_wait(&acc_full[buf], (i >> 1) & 1);
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(base + (uint32_t)c, v);
+        if (row < M) epilogue_chunk<EPI, BN>(e, v, row, n_blk * BN + c);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------- packed int4 B operand
 // The same GEMM with B given as MatMulNBits codes + fp16 scales (up to three row segments of one
 // matrix stack, or two segments interleaved row by row): the int4 weights are dequantised into
@@ -492,6 +608,87 @@ cudaError_t launch_q4_bn(const uint16_t* A, const PackedB& B, int M, int N, int 
 
 }  // namespace
 
+namespace {
+// The whole matrix stack dequantised to fp16 [total_rows, K] (the B operand of gemm_tc_kernel):
+// one thread per 32-weight block, (code - 8) * scale rounded once to fp16 (dequant8_f16), rows
+// of up to three segments, or two segments interleaved row by row.
+__global__ void __launch_bounds__(256) dequant_f16_kernel(const DequantSrc src, int total_rows,
+                                                          int K, __half* __restrict__ out) {
+  const int KB = K >> 5;
+  const int64_t nblk = (int64_t)total_rows * KB;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    const int orow = (int)(b / KB), kb = (int)(b % KB);
+    int m, r;
+    if (src.interleave) {
+      m = orow & 1;
+      r = orow >> 1;
+    } else {
+      m = 0;
+      r = orow;
+      while (m < src.nseg - 1 && r >= src.rows[m]) r -= src.rows[m++];
+    }
+    const uint4 codes = __ldg(reinterpret_cast<const uint4*>(src.q[m] + ((size_t)r * KB + kb) * 16));
+    const uint32_t sh = src.s[m][(size_t)r * KB + kb];
+    const uint32_t s2 = sh | (sh << 16);
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)orow * K + (size_t)kb * 32);
+    dst[0] = dequant8_f16(codes.x, s2);
+    dst[1] = dequant8_f16(codes.y, s2);
+    dst[2] = dequant8_f16(codes.z, s2);
+    dst[3] = dequant8_f16(codes.w, s2);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
+                               cudaStream_t s) {
+  const int64_t nblk = (int64_t)total_rows * (K >> 5);
+  int64_t grid = (nblk + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  dequant_f16_kernel<<<(int)grid, 256, 0, s>>>(src, total_rows, K, out);
+  return cudaGetLastError();
+}
+
+namespace {
+
+template <int BN>
+size_t smem_bytes() {
+  return Cfg<BN>::kStages * (kStageA + Cfg<BN>::kStageB) + 2 * Cfg<BN>::kStages * 8 + 4 * 8 + 16 +
+         1024;
+}
+
+template <int EPI, int BN>
+cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmEpilogue& e, int M,
+                     int N, int K, int grid, cudaStream_t s) {
+  const size_t smem = smem_bytes<BN>();
+  cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  gemm_tc_kernel<EPI, BN><<<grid, kThreads, smem, s>>>(ta, tb, e, M, N, K);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_bn(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                      const GemmEpilogue& e, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
+  const int tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  switch (epi) {
+    case kEpiBias: return run_gemm<kEpiBias, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiResid: return run_gemm<kEpiResid, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiSwiglu: return run_gemm<kEpiSwiglu, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiF16: return run_gemm<kEpiF16, BN>(ta, tb, e, M, N, K, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
 bool gemm_q4_supported(const PackedB& B, int N, int K) {
   if (K < BK || K % BK != 0 || B.nseg < 1 || B.nseg > 3) return false;
   const int sp = scale_pitch(B, K);
@@ -530,6 +727,29 @@ cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, in
     if (w == 256) return launch_q4_bn<256>(A, B, M, N, K, epi, e, s);
     if (w == 192) return launch_q4_bn<192>(A, B, M, N, K, epi, e, s);
     return launch_q4_bn<128>(A, B, M, N, K, epi, e, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t gemm_tc_smem() { return smem_bytes<256>(); }
+
+
+cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s) {
+  if (M < 1 || N % 64 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
+  if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
+  const int sms = sm_count();
+  const long mt = (M + BM - 1) / BM;
+  // the widest tile whose wave efficiency is within 0.1 of the best available width
+  const int widths[3] = {256, 192, 128};
+  double best = 0.0;
+  for (int w : widths)
+    if (N % w == 0) best = std::max(best, wave_eff(mt * (N / w), sms));
+  for (int w : widths) {
+    if (N % w != 0 || wave_eff(mt * (N / w), sms) < best - 0.1) continue;
+    if (w == 256) return launch_bn<256>(A, B, M, N, K, epi, e, s);
+    if (w == 192) return launch_bn<192>(A, B, M, N, K, epi, e, s);
+    return launch_bn<128>(A, B, M, N, K, epi, e, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -19,6 +19,25 @@ struct GemmEpilogue {
   int ldo;  // row stride of the output in elements
 };
 
+size_t gemm_tc_smem();
+// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 128 == 0 or N % 192 == 0, K % 64 == 0.
+cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
+                           const GemmEpilogue& e, cudaStream_t s);
+
+// Up to three packed MatMulNBits matrices (row segments, same K) dequantised into one fp16
+// [rows, K] matrix, element (code - 8) * scale rounded once to fp16.  interleave = 1 (two
+// segments of equal rows): output row 2n is row n of segment 0, row 2n + 1 row n of segment 1.
+// Scales with a row pitch of K/32.
+struct DequantSrc {
+  const uint8_t* q[3];
+  const uint16_t* s[3];
+  int rows[3];
+  int nseg;
+  int interleave;
+};
+cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
+                               cudaStream_t s);
+
 // B operand as packed MatMulNBits matrices, dequantised inside the GEMM (no fp16 copy in global
 // memory): up to three row segments (N = sum of rows, each a multiple of 128), or two segments
 // of equal rows interleaved row by row (interleave = 1, N = 2 * rows).  K % 64 == 0.  Codes

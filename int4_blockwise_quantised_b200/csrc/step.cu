@@ -365,12 +365,14 @@ __device__ void producer(const StepParams& p, Ring& r, const int* past) {
   const int ns = n_slices(p);
   int o0, o1;
   cta_range(Hq * nrb, cta, ncta, o0, o1);
+  int r0, r1;  // this CTA's lm_head rows
+  cta_range(p.V, cta, ncta, r0, r1);
   for (int l = 0; l < p.L; ++l) {
     const StepLayer& w = p.layers[l];
-    int r0, r1;
-    qkv_range(nqkv, cta, ncta, r0, r1);
+    int q0, q1;
+    qkv_range(nqkv, cta, ncta, q0, q1);
     const int bounds[4] = {0, Hq * D, (Hq + Hkv) * D, nqkv};
-    produce_qkv(r, w, H, r0, r1, bounds, pol);
+    produce_qkv(r, w, H, q0, q1, bounds, pol);
     for (int it = cta; it < plan.total; it += ncta) {
       int b, g, t;
       attn_item_of(plan, Hkv, it, b, g, t);
@@ -388,8 +390,6 @@ __device__ void producer(const StepParams& p, Ring& r, const int* past) {
     if (nsl > 0) produce_cols(r, w.wd_img + (size_t)cta * wd_cta_stride(p), H, 2 * nsl, pol);
   }
   // HEAD: fp16 rows of the lm_head
-  int r0, r1;
-  cta_range(p.V, cta, ncta, r0, r1);
   const int rb = H * 2;
   const int rps = min(64, r.stage_bytes / rb);
   for (int a = r0; a < r1; a += rps) {
@@ -1195,7 +1195,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
         consume_rows<2, NB>(r, xo, H, s * kSlice, (s + 1) * kSlice,
                             [&](int row, const float* g, const float* u) {
 #pragma unroll
-          for (int b = 0; b < NB; ++b) hbuf[b][off + row] = g[b] / (1.f + __expf(-g[b])) * u[b];
+          for (int b = 0; b < NB; ++b) hbuf[b][off + row] = __fdividef(g[b], 1.f + __expf(-g[b])) * u[b];
         });
       }
       cbar();
