@@ -288,8 +288,8 @@ vv_status vv_decoder_step(vv_decoder* dec, const uint16_t* input_embeds, const i
  *   input_ids, position_ids: device int32 [S]; audio_features: device fp16 [N, H] or NULL (N=0)
  * All S positions go through tensor-core GEMMs at once (each packed matrix is dequantised to an
  * fp16 operand, rounded once: exact for ternary weights, within 2^-12 relative for int4; for
- * S <= 256 inside the GEMM, for longer prompts one layer ahead on a second stream into a
- * two-layer fp16 buffer of the prefill workspace), with
+ * S <= 256 inside the GEMM, for longer prompts one launch per layer into a one-layer fp16 buffer
+ * of the prefill workspace), with
  * fp32 accumulation and an fp32 residual.  The first call allocates a prefill workspace sized
  * for max_prefill (kept until vv_decoder_destroy).  Asynchronous on `stream`.
  * Errors: VV_ERR_RANGE (audio_offset + N > S, negative offset), VV_ERR_CAPACITY (S > cap or
@@ -338,10 +338,10 @@ vv_status vv_decoder_generate(vv_decoder* dec, const int32_t* first_token, const
  * float [5] and launches: HOST int32 [5] receive the device time and the number of launches (or
  * copies) of each kind: [0] embedding splice, RMSNorm, RoPE/KV write, bias and trace copies;
  * [1] weight dequantisation to fp16; [2] tensor-core GEMMs; [3] causal attention; [4] final
- * norm + lm_head + argmax.  Kind [1] stays 0: prompts of S <= 256 positions run the GEMMs with
- * the int4 → fp16 expansion fused in; longer prompts run fp16 GEMMs on weights that a second
- * stream dequantises one layer ahead (overlapped with the GEMMs; a GEMM that waits for its
- * weights counts the wait in [2]).  Errors as vv_decoder_init. */
+ * norm + lm_head + argmax.  Prompts of S <= 256 positions run the GEMMs with the int4 → fp16
+ * expansion fused in (kind [1] stays 0); longer prompts dequantise each layer's four weight
+ * stacks in one launch into an fp16 buffer (kind [1]) and run fp16 GEMMs on it.  Errors as
+ * vv_decoder_init. */
 vv_status vv_decoder_profile_init(vv_decoder* dec, const int32_t* input_ids,
                                   const int32_t* position_ids, int64_t S,
                                   const uint16_t* audio_features, int64_t N, int64_t audio_offset,

@@ -273,9 +273,6 @@ vv_status vv_decoder_destroy(vv_decoder* d) {
   if (d->ws) cudaFree(d->ws);
   if (d->pws) cudaFree(d->pws);
   if (d->pf_pad) cudaFree(d->pf_pad);
-  for (cudaEvent_t ev : d->pf_ev)
-    if (ev) cudaEventDestroy(ev);
-  if (d->pf_side) cudaStreamDestroy(d->pf_side);
   cudaSetDevice(cur);
   delete d;
   return VV_OK;

@@ -39,9 +39,6 @@ struct vv_decoder {
   std::vector<const uint16_t*> pf_scales;
   int pf_pitch[7] = {0, 0, 0, 0, 0, 0, 0};
   uint16_t* pf_pad = nullptr;
-  // the long-prompt prefill's side stream (weight dequantisation one layer ahead) and its events
-  cudaStream_t pf_side = nullptr;
-  cudaEvent_t pf_ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 
   int nb = 1;                       // sequences stepped together (batch)
   int32_t len_host[2] = {0, 0};     // host copy of each sequence's length

@@ -641,6 +641,68 @@ __global__ void __launch_bounds__(256) dequant_f16_kernel(const DequantSrc src, 
 
 }  // namespace
 
+namespace {
+// Several matrix stacks in one launch: job j covers blocks [first[j], first[j + 1]) of the
+// launch's block range.
+struct DequantJobs {
+  DequantSrc src[4];
+  __half* out[4];
+  int K[4];
+  int64_t first[5];
+  int n;
+};
+
+__global__ void __launch_bounds__(256) dequant_jobs_kernel(const DequantJobs jb) {
+  const int64_t total = jb.first[jb.n];
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    int j = 0;
+    while (j + 1 < jb.n && g >= jb.first[j + 1]) ++j;
+    const DequantSrc& src = jb.src[j];
+    const int K = jb.K[j], KB = K >> 5;
+    const int64_t b = g - jb.first[j];
+    const int orow = (int)(b / KB), kb = (int)(b % KB);
+    int m, r;
+    if (src.interleave) {
+      m = orow & 1;
+      r = orow >> 1;
+    } else {
+      m = 0;
+      r = orow;
+      while (m < src.nseg - 1 && r >= src.rows[m]) r -= src.rows[m++];
+    }
+    const uint4 codes = __ldg(reinterpret_cast<const uint4*>(src.q[m] + ((size_t)r * KB + kb) * 16));
+    const uint32_t sh = src.s[m][(size_t)r * KB + kb];
+    const uint32_t s2 = sh | (sh << 16);
+    uint4* dst = reinterpret_cast<uint4*>(jb.out[j] + (size_t)orow * K + (size_t)kb * 32);
+    dst[0] = dequant8_f16(codes.x, s2);
+    dst[1] = dequant8_f16(codes.y, s2);
+    dst[2] = dequant8_f16(codes.z, s2);
+    dst[3] = dequant8_f16(codes.w, s2);
+  }
+}
+}  // namespace
+
+cudaError_t launch_dequant_many(const DequantSrc* src, const int* rows, const int* K,
+                                __half* const* out, int n, cudaStream_t s) {
+  if (n < 1 || n > 4) return cudaErrorInvalidValue;
+  DequantJobs jb = {};
+  jb.n = n;
+  jb.first[0] = 0;
+  for (int j = 0; j < n; ++j) {
+    jb.src[j] = src[j];
+    jb.out[j] = out[j];
+    jb.K[j] = K[j];
+    jb.first[j + 1] = jb.first[j] + (int64_t)rows[j] * (K[j] >> 5);
+  }
+  int64_t grid = (jb.first[n] + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  dequant_jobs_kernel<<<(int)grid, 256, 0, s>>>(jb);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
                                cudaStream_t s) {
   const int64_t nblk = (int64_t)total_rows * (K >> 5);

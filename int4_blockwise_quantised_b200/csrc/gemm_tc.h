@@ -37,6 +37,9 @@ struct DequantSrc {
 };
 cudaError_t launch_dequant_f16(const DequantSrc& src, int total_rows, int K, __half* out,
                                cudaStream_t s);
+// Up to four such matrix stacks (rows[j] x K[j] each, into out[j]) in one launch.
+cudaError_t launch_dequant_many(const DequantSrc* src, const int* rows, const int* K,
+                                __half* const* out, int n, cudaStream_t s);
 
 // B operand as packed MatMulNBits matrices, dequantised inside the GEMM (no fp16 copy in global
 // memory): up to three row segments (N = sum of rows, each a multiple of 128), or two segments

@@ -228,11 +228,11 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   const size_t o_q = take((size_t)SM * HQD * 2);
   const size_t o_h = take((size_t)SM * I * 2);
   const size_t o_bias = take((size_t)NQKV * 2);
-  // the two-pass path (S > kFusedMaxM): fp16 copies of two layers' weights, [q/k/v | o | gate/up
-  // interleaved | down] each; a side stream dequantises layer l + 1 while layer l computes
+  // the two-pass path (S > kFusedMaxM): the current layer's weights in fp16, [q/k/v | o |
+  // gate/up interleaved | down]
   const size_t w_qkv = (size_t)NQKV * H, w_o = (size_t)H * HQD, w_gu = (size_t)2 * I * H;
   const size_t w_layer = w_qkv + w_o + w_gu + (size_t)H * I;
-  const size_t o_w16 = take(SM > kFusedMaxM ? 2 * w_layer * 2 : 0);
+  const size_t o_w16 = take(SM > kFusedMaxM ? w_layer * 2 : 0);
   const size_t need = off_b;
   if (d->pws_bytes < need) {
     if (d->pws) cudaFree(d->pws);
@@ -252,10 +252,11 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   __half* W16 = reinterpret_cast<__half*>(b + o_w16);
   const bool two_pass = S > kFusedMaxM;
   // layer l's fp16 weights (two-pass path): matrix m = 0 q/k/v, 1 o, 2 gate/up, 3 down
-  auto w16_of = [&](int l, int m) {
+  auto w16_of = [&](int, int m) {
     const size_t offs[4] = {0, w_qkv, w_qkv + w_o, w_qkv + w_o + w_gu};
-    return W16 + (size_t)(l & 1) * w_layer + offs[m];
+    return W16 + offs[m];
   };
+  // one launch for the layer's four matrix stacks
   auto dequant_layer = [&](int l, cudaStream_t st) -> cudaError_t {
     const vv_layer_weights& w = d->layers[l];
     const DequantSrc ds[4] = {
@@ -264,15 +265,12 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
         {{w.wgate.q, w.wup.q, nullptr}, {w.wgate.scales, w.wup.scales, nullptr}, {I, I, 0}, 2, 1},
         {{w.wdown.q, nullptr, nullptr}, {w.wdown.scales, nullptr, nullptr}, {H, 0, 0}, 1, 0}};
     const int rows[4] = {NQKV, H, 2 * I, H}, ks[4] = {H, HQD, H, I};
-    for (int m = 0; m < 4; ++m) {
-      cudaError_t err = launch_dequant_f16(ds[m], rows[m], ks[m], w16_of(l, m), st);
-      if (err != cudaSuccess) return err;
-    }
-    return cudaSuccess;
+    __half* outs[4] = {w16_of(l, 0), w16_of(l, 1), w16_of(l, 2), w16_of(l, 3)};
+    return launch_dequant_many(ds, rows, ks, outs, 4, st);
   };
   // One projection of layer l (matrix m): fused dequantisation in the GEMM for short prompts
   // (each weight is expanded once per 128-row block of the prompt), else the fp16 GEMM on the
-  // weights the side stream dequantised (each weight expanded once).
+  // weights dequantised at the start of the layer (each weight expanded once).
   auto project = [&](int l, int m, const uint16_t* A, const PackedB& pb, int N, int K, int epi,
                      const GemmEpilogue& ep) -> cudaError_t {
     cudaError_t err;
@@ -283,26 +281,10 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     if (err != cudaSuccess) return err;
     return mark(kPfGemm);
   };
-  // side stream and events: [0] start (on s), [1..2] layer buffer ready (side), [3..4] layer
-  // buffer free again (s)
-  if (two_pass && !d->pf_side) {
-    cudaError_t err = cudaStreamCreateWithFlags(&d->pf_side, cudaStreamNonBlocking);
-    for (int i = 0; i < 5 && err == cudaSuccess; ++i)
-      err = cudaEventCreateWithFlags(&d->pf_ev[i], cudaEventDisableTiming);
-    if (err != cudaSuccess) return err;
-  }
   const size_t layer_kv = (size_t)Hkv * c.kv_capacity * D;
   cudaError_t e;
 
   VV_MARK(kPfMisc);
-  if (two_pass) {  // layers 0 and 1 into the two buffers, after all earlier work on s
-    if ((e = cudaEventRecord(d->pf_ev[0], s)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(d->pf_side, d->pf_ev[0], 0)) != cudaSuccess) return e;
-    for (int l = 0; l < 2 && l < c.layers; ++l) {
-      if ((e = dequant_layer(l, d->pf_side)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(d->pf_ev[1 + l], d->pf_side)) != cudaSuccess) return e;
-    }
-  }
   splice_x_kernel<<<S, 256, 0, s>>>(ids, S, reinterpret_cast<const __half*>(d->embed), c.vocab, H,
                                     reinterpret_cast<const __half*>(audio), N, off, X);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -337,7 +319,10 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     ep.out_f32 = QKV;
     ep.bias = Bqkv;
     ep.ldo = NQKV;
-    if (two_pass && (e = cudaStreamWaitEvent(s, d->pf_ev[1 + (l & 1)], 0)) != cudaSuccess) return e;
+    if (two_pass) {
+      if ((e = dequant_layer(l, s)) != cudaSuccess) return e;
+      VV_MARK(kPfDequant);
+    }
     if ((e = project(l, 0, reinterpret_cast<const uint16_t*>(Xn), pb, NQKV, H, kEpiBias, ep)) !=
         cudaSuccess)
       return e;
@@ -394,13 +379,7 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
     if ((e = project(l, 3, reinterpret_cast<const uint16_t*>(Hm), pb, H, I, kEpiResid, ep)) !=
         cudaSuccess)
       return e;
-    if (two_pass && l + 2 < c.layers) {
-      // layer l's buffer is free once its down GEMM has run: dequantise layer l + 2 into it
-      if ((e = cudaEventRecord(d->pf_ev[3 + (l & 1)], s)) != cudaSuccess) return e;
-      if ((e = cudaStreamWaitEvent(d->pf_side, d->pf_ev[3 + (l & 1)], 0)) != cudaSuccess) return e;
-      if ((e = dequant_layer(l + 2, d->pf_side)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(d->pf_ev[1 + (l & 1)], d->pf_side)) != cudaSuccess) return e;
-    }
+
     if (d->trace) {
       e = cudaMemcpyAsync(d->trace + (size_t)l * H, X + (size_t)(S - 1) * H, (size_t)H * 4,
                           cudaMemcpyDeviceToDevice, s);
