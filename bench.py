@@ -845,13 +845,14 @@ def phase_breakdown(st, L):
 
 
 def traffic_for(kernel, workload=None):
-    """DRAM bytes per launch from the committed ncu summary (entry "kernel/workload", else
-    "kernel"), or None when the kernel's source changed since the counters were taken."""
+    """DRAM bytes per launch from the committed ncu summary (entry "kernel/workload", or "kernel"
+    when no workload is named), or None when there is no capture of that workload or the
+    kernel's source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     tab = json.load(open(p))
-    d = tab.get(f"{kernel}/{workload}") or tab.get(kernel)
+    d = tab.get(f"{kernel}/{workload}") if workload else tab.get(kernel)
     if not d:
         return None
     src = os.path.join(ROOT, d["source"])
