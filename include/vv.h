@@ -206,8 +206,8 @@ typedef struct vv_config {
   int32_t kv_dtype;    /* VV_KV_F16 (0), VV_KV_BF16 (1) or VV_KV_F32 (2); the prefill needs F16 */
   int32_t batch;       /* sequences stepped together, 1 or 2 (0 means 1); batch 2 is the
                           CFG pair / two streams ("VibeVoice-1.5B — Current Status": the
-                          negative context stepped alongside the positive one); needs
-                          max_prefill == 0 */
+                          negative context stepped alongside the positive one); each sequence
+                          is prefilled by vv_decoder_init_seq */
 } vv_config;
 
 #define VV_KV_F16 0
@@ -298,6 +298,14 @@ vv_status vv_decoder_init(vv_decoder* dec, const int32_t* input_ids, const int32
                           int64_t S, const uint16_t* audio_features, int64_t N,
                           int64_t audio_offset, float* logits, int32_t* argmax_out,
                           vv_stream stream);
+
+/* vv_decoder_init for sequence `seq` of a batch decoder (vv_decoder_init is seq = 0): the
+ * prompt's K/V go to cache slice [L, seq, Hkv, ·, D] and only that sequence's length is set.
+ * Errors as vv_decoder_init, and VV_ERR_INVALID_ARG for seq outside [0, batch). */
+vv_status vv_decoder_init_seq(vv_decoder* dec, int32_t seq, const int32_t* input_ids,
+                              const int32_t* position_ids, int64_t S,
+                              const uint16_t* audio_features, int64_t N, int64_t audio_offset,
+                              float* logits, int32_t* argmax_out, vv_stream stream);
 
 /* Debug tap: when layer_out (device fp32 [L, H]) is non-NULL, each later step writes the
  * residual stream after every layer into it (init writes the last position's).  NULL turns it

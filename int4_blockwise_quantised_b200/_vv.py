@@ -92,6 +92,7 @@ def _load():
         "vv_decoder_batch": (c_int32, [P]),
         "vv_decoder_step": (S, [P, P, P, P, P, P, P]),
         "vv_decoder_init": (S, [P, P, P, c_int64, P, c_int64, c_int64, P, P, P]),
+        "vv_decoder_init_seq": (S, [P, c_int32, P, P, c_int64, P, c_int64, c_int64, P, P, P]),
         "vv_decoder_set_trace": (S, [P, P]),
         "vv_decoder_set_graph": (S, [P, c_int32]),
         "vv_decoder_set_wait_limit": (S, [P, c_int64]),

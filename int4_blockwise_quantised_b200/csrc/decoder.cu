@@ -66,8 +66,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
                  "kv_dtype %d", c.kv_dtype);
   VV_CHECK_SHAPE(c.batch >= 0 && c.batch <= vv::step_max_batch(), "batch %d (1 .. %d)", c.batch,
                  vv::step_max_batch());
-  VV_CHECK_SHAPE(c.batch <= 1 || c.max_prefill == 0,
-                 "batch %d: the prefill (max_prefill > 0) runs one sequence", c.batch);
+
   VV_CHECK_SHAPE(c.kv_dtype == VV_KV_F16 || c.max_prefill == 0,
                  "kv_dtype %d: the prefill (max_prefill > 0) writes an fp16 cache only", c.kv_dtype);
   VV_CHECK_SHAPE(c.n_kv >= 1 && c.n_kv <= 64 && c.n_q % c.n_kv == 0 && c.n_q / c.n_kv <= 8,
@@ -435,7 +434,16 @@ vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t
                           int64_t S, const uint16_t* audio_features, int64_t N,
                           int64_t audio_offset, float* logits, int32_t* argmax_out,
                           vv_stream stream) {
+  return vv_decoder_init_seq(d, 0, input_ids, position_ids, S, audio_features, N, audio_offset,
+                             logits, argmax_out, stream);
+}
+
+vv_status vv_decoder_init_seq(vv_decoder* d, int32_t seq, const int32_t* input_ids,
+                              const int32_t* position_ids, int64_t S,
+                              const uint16_t* audio_features, int64_t N, int64_t audio_offset,
+                              float* logits, int32_t* argmax_out, vv_stream stream) {
   VV_CHECK_ARG(d && input_ids && position_ids, "vv_decoder_init: null pointer");
+  VV_CHECK_ARG(seq >= 0 && seq < d->nb, "vv_decoder_init: sequence %d of a batch of %d", seq, d->nb);
   VV_CHECK_ARG(N == 0 || audio_features, "vv_decoder_init: audio_features null with N > 0");
   VV_CHECK_ARG(!audio_features || vv::aligned16(audio_features), "audio_features misaligned");
   if (S < 1) return set_error(VV_ERR_SHAPE, "S=%lld", (long long)S);
@@ -445,10 +453,10 @@ vv_status vv_decoder_init(vv_decoder* d, const int32_t* input_ids, const int32_t
   if (S > d->cfg.kv_capacity || S > d->cfg.max_prefill)
     return set_error(VV_ERR_CAPACITY, "S=%lld > capacity %d or max_prefill %d", (long long)S,
                      d->cfg.kv_capacity, d->cfg.max_prefill);
-  VV_CUDA(vv::prefill_run(d, input_ids, position_ids, (int)S, audio_features, (int)N,
+  VV_CUDA(vv::prefill_run(d, seq, input_ids, position_ids, (int)S, audio_features, (int)N,
                           (int)audio_offset, logits, argmax_out,
                           static_cast<cudaStream_t>(stream)));
-  d->len_host[0] = (int32_t)S;
+  d->len_host[seq] = (int32_t)S;
   return VV_OK;
 }
 
@@ -470,7 +478,7 @@ vv_status vv_decoder_profile_init(vv_decoder* d, const int32_t* input_ids,
                      d->cfg.kv_capacity, d->cfg.max_prefill);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   vv::PrefillTimer t;
-  vv_status st = vv::cuda_check(vv::prefill_run(d, input_ids, position_ids, (int)S, audio_features,
+  vv_status st = vv::cuda_check(vv::prefill_run(d, 0, input_ids, position_ids, (int)S, audio_features,
                                                 (int)N, (int)audio_offset, logits, argmax_out, s,
                                                 &t),
                                 "profile prefill");

@@ -71,7 +71,7 @@ cudaError_t enqueue_step(vv_decoder* d, const uint16_t* embeds, const int32_t* t
                          const int32_t* position, float* logits, int32_t* argmax, cudaStream_t s);
 // Prefill preparation at create: the pf_scales table (and padded scale copies where needed).
 cudaError_t prefill_prepare(vv_decoder* d);
-cudaError_t prefill_run(vv_decoder* dec, const int32_t* ids, const int32_t* pos, int S,
+cudaError_t prefill_run(vv_decoder* dec, int seq, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
                         cudaStream_t s, PrefillTimer* timer = nullptr);
 }  // namespace vv

@@ -194,7 +194,7 @@ cudaError_t prefill_prepare(vv_decoder* d) {
   return cudaDeviceSynchronize();
 }
 
-cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, int S,
+cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_t* pos, int S,
                         const uint16_t* audio, int N, int off, float* logits, int32_t* argmax,
                         cudaStream_t s, PrefillTimer* timer) {
   // mark(k): the work enqueued since the previous mark is of kind k
@@ -291,8 +291,9 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   VV_MARK(kPfMisc);
   for (int l = 0; l < c.layers; ++l) {
     const vv_layer_weights& w = d->layers[l];
-    __half* kc = reinterpret_cast<__half*>(d->k_cache) + (size_t)l * layer_kv;
-    __half* vc = reinterpret_cast<__half*>(d->v_cache) + (size_t)l * layer_kv;
+    // sequence seq's slice of layer l: caches are [L][batch][Hkv][cap][D]
+    __half* kc = reinterpret_cast<__half*>(d->k_cache) + ((size_t)l * d->nb + seq) * layer_kv;
+    __half* vc = reinterpret_cast<__half*>(d->v_cache) + ((size_t)l * d->nb + seq) * layer_kv;
     // ---- QKV
     rmsnorm_rows_kernel<<<S, 128, 0, s>>>(X, H, reinterpret_cast<const __half*>(w.input_norm), c.eps, Xn);
     VV_MARK(kPfMisc);
@@ -406,7 +407,7 @@ cudaError_t prefill_run(vv_decoder* d, const int32_t* ids, const int32_t* pos, i
   la.length = nullptr;
   if ((e = launch_lm_head(la, s, false)) != cudaSuccess) return e;
   VV_MARK(kPfHead);
-  set_int_kernel<<<1, 1, 0, s>>>(d->d_length, S);
+  set_int_kernel<<<1, 1, 0, s>>>(d->d_length + seq, S);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   VV_MARK(kPfMisc);
   return cudaSuccess;

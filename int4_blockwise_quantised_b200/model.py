@@ -172,12 +172,13 @@ class Decoder:
         return full[:, : n.value], full
 
     def init(self, input_ids, position_ids, audio_features=None, audio_offset=0, logits=None,
-             argmax=None, stream=None):
+             argmax=None, stream=None, seq=0):
+        """decoder_init of sequence `seq` (0 for a batch-1 decoder)."""
         S = input_ids.numel()
         N = 0 if audio_features is None else audio_features.shape[0]
-        check(_vv.lib.vv_decoder_init(self.handle, ptr(input_ids), ptr(position_ids), S,
-                                      ptr(audio_features), N, audio_offset, ptr(logits),
-                                      ptr(argmax), stream_handle(stream)))
+        check(_vv.lib.vv_decoder_init_seq(self.handle, seq, ptr(input_ids), ptr(position_ids), S,
+                                          ptr(audio_features), N, audio_offset, ptr(logits),
+                                          ptr(argmax), stream_handle(stream)))
 
     PREFILL_KINDS = ("misc", "dequant", "gemm", "attention", "lm_head")
 

@@ -115,14 +115,64 @@ def test_batch2_full_1p5b():
     run_pair(synth.SHAPE_1P5B, "int4", (1024, 700), 2)
 
 
-def test_batch2_rejects_prefill_and_generate():
+def test_batch2_rejects_bad_batch_and_generate():
     from int4_blockwise_quantised_b200 import _vv
     from int4_blockwise_quantised_b200.model import Decoder
 
     model = gpu_model(synth.SHAPE_TINY, "int4")
     with pytest.raises(_vv.VVError) as e:
-        Decoder(model, 64, max_prefill=16, batch=2)
-    assert e.value.code == _vv.VV_ERR_SHAPE
-    with pytest.raises(_vv.VVError) as e:
         Decoder(model, 64, batch=3)
     assert e.value.code == _vv.VV_ERR_SHAPE
+    dec = Decoder(model, 64, batch=2)
+    with pytest.raises(_vv.VVError) as e:
+        dec.generate(torch.zeros(1, dtype=torch.int32, device="cuda"),
+                     torch.zeros(1, dtype=torch.int32, device="cuda"), 4)
+    assert e.value.code == _vv.VV_ERR_SHAPE
+    ids = torch.zeros(8, dtype=torch.int32, device="cuda")
+    with pytest.raises(_vv.VVError) as e:
+        dec.init(ids, ids, seq=2)
+    assert e.value.code == _vv.VV_ERR_INVALID_ARG
+
+
+def test_batch2_prefill_each_sequence_then_step():
+    """The CFG pair from two prompts: each sequence prefilled into its own cache slice
+    (vv_decoder_init_seq), then batch-2 steps, every result against the oracle per sequence."""
+    from int4_blockwise_quantised_b200.model import Decoder
+
+    shape, mode = synth.SHAPE_SMALL, "int4"
+    cfg = ocfg(shape)
+    W = oracle_model(shape, mode)
+    model = gpu_model(shape, mode)
+    L, B = shape.layers, 2
+    prompts = [synth.asr_prompt(shape, 40, prefix=7, suffix=23), synth.asr_prompt(shape, 20, prefix=5,
+                                                                               suffix=12, base=3)]
+    Ss = [p[0].size for p in prompts]
+    dec = Decoder(model, max(Ss) + 8, max_prefill=max(Ss), batch=B)
+    lg1 = torch.zeros(shape.vocab, dtype=torch.float32, device="cuda")
+    kc, vc, toks = [], [], []
+    for b in range(B):
+        ids, pos, feats, off = prompts[b]
+        dec.init(dev(ids), dev(pos), dev(feats), off, logits=lg1, seq=b)
+        dec.sync_status()
+        ora = odec.decoder_init(cfg, W, ids, pos, feats, off)
+        assert normwise(lg1.cpu().numpy(), ora["logits"]) <= TOL
+        assert dec.sequence_length(b) == Ss[b]
+        assert normwise(dec.k_cache[:, b, :, :Ss[b]].cpu().numpy(), ora["k"]) <= TOL
+        kc.append([ora["k"][l] for l in range(L)])
+        vc.append([ora["v"][l] for l in range(L)])
+        toks.append(ora["argmax"])
+    # the other sequence's slice stays untouched by each prefill
+    assert torch.count_nonzero(dec.k_cache[:, 1, :, Ss[1]:]).item() == 0
+    logits = torch.zeros((B, shape.vocab), dtype=torch.float32, device="cuda")
+    for s in range(2):
+        pos_t = torch.tensor([Ss[b] + s for b in range(B)], dtype=torch.int32, device="cuda")
+        tok_t = torch.tensor(toks, dtype=torch.int32, device="cuda")
+        dec.step(pos_t, token=tok_t, logits=logits)
+        dec.sync_status()
+        lg = logits.cpu().numpy()
+        for b in range(B):
+            st = odec.decoder_step(cfg, W, W["embed"][toks[b]], Ss[b] + s, kc[b], vc[b])
+            assert normwise(lg[b], st["logits"]) <= TOL, (s, b)
+            kc[b] = [np.concatenate([kc[b][l], st["k_new"][l][:, None]], 1) for l in range(L)]
+            vc[b] = [np.concatenate([vc[b][l], st["v_new"][l][:, None]], 1) for l in range(L)]
+            toks[b] = st["argmax"]
