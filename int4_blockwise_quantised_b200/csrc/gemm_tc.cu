@@ -4,7 +4,7 @@
 //
 // Persistent: one CTA per SM walks the 128 x BN output tiles (BN = 256, 192 or 128: the widest
 // that fills the last wave of SMs about as well as any), K in blocks of 64.
-//   warp 0      : TMA producer (cp.async.bulk.tensor 2D, 128-byte swizzle, no multicast) into a
+//   warp 0      : TMA producer (cp.async.bulk.tensor 2D, 128-byte swizzle, this CTA only) into a
 //                 ring of (A 128x64, B BNx64) fp16 stages, mbarrier complete_tx; the ring runs on
 //                 across tile boundaries;
 //   warp 1      : allocates 2 x BN TMEM columns (two accumulators), one thread issues

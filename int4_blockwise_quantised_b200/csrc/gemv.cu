@@ -6,7 +6,7 @@
 //
 // Design (HBM-bound; every weight byte is read exactly once):
 //  * One producer warp streams whole weight rows (codes + scales, both contiguous per row) into
-//    a ring of shared-memory stages with cp.async.bulk (TMA, non-tensor, no multicast) and
+//    a ring of shared-memory stages with cp.async.bulk (TMA, non-tensor form, this CTA only) and
 //    mbarrier completion.  Weights do not depend on the previous kernel, so the producer fills
 //    the ring BEFORE griddepcontrol.wait: under programmatic dependent launch the next GEMV's
 //    weights are already in flight while the previous kernel finishes.

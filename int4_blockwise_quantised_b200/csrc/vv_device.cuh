@@ -51,7 +51,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 
 // ----------------------------------------------------------------------------------------------
-// mbarrier + bulk async copy (TMA, non-tensor form, no multicast).
+// mbarrier + bulk async copy (TMA, non-tensor form, into this CTA's shared memory).
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
