@@ -318,6 +318,13 @@ struct AttnPlan {
   int total;
 };
 __device__ __forceinline__ int kv_bytes(const StepParams& p) { return p.kv_type == 2 ? 4 : 2; }
+// lm_head rows per stage: as many as fit (at most 64), rounded down to a multiple of the compute
+// warps when there are more than NW (each warp takes whole rows: 16 rows on 15 warps would give
+// one warp two rows and make every stage take two rows' time).  Producer and consumers agree.
+__device__ __forceinline__ int head_rows_per_stage(int stage_bytes, int row_bytes) {
+  const int n = min(64, stage_bytes / row_bytes);
+  return n > NW ? n / NW * NW : n;
+}
 __device__ __forceinline__ int ntiles_for(int past, int tt) { return (past + 1 + tt - 1) / tt; }
 __device__ __forceinline__ AttnPlan attn_plan(const StepParams& p, const int* past) {
   AttnPlan a;
@@ -391,7 +398,7 @@ __device__ void producer(const StepParams& p, Ring& r, const int* past) {
   }
   // HEAD: fp16 rows of the lm_head
   const int rb = H * 2;
-  const int rps = min(64, r.stage_bytes / rb);
+  const int rps = head_rows_per_stage(r.stage_bytes, rb);
   for (int a = r0; a < r1; a += rps) {
     const int n = min(rps, r1 - a);
     Copy c[1] = {Copy{p.lm_head + (size_t)a * H, (uint32_t)(n * rb), 0u}};
@@ -1264,7 +1271,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p) {
     int r0, r1;
     cta_range(p.V, cta, ncta, r0, r1);
     const int rb = H * 2;
-    const int rps = min(64, r.stage_bytes / rb);
+    const int rps = head_rows_per_stage(r.stage_bytes, rb);
     const int nch = H >> 3;  // 16-byte chunks per row
     // x of 16-byte weight chunk c (8 columns: half-block c/2, word c%2) = pair word (c%2, c/2);
     // held in registers for c = lane + 32 j when the row fits (H <= 1536) and one sequence runs
