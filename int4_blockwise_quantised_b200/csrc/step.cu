@@ -813,35 +813,45 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     vt[(past - p0) * D + d] = vn;
   }
   cbar();
-  // scores: warp w -> head w/2, positions (w%2)*32 + lane.  K rows are 256 bytes apart, so each
-  // lane walks the 16 chunks of its row starting at chunk `lane % 16`: the 8 lanes of a 16-byte
-  // load phase then read 8 different K chunks (distinct banks; the q reads are 2-way).
-  for (int item = warp; item < 2 * G; item += NW) {
-    const int h = item >> 1, pp = (item & 1) * 32 + lane;
-    float sc = -INFINITY;
-    if (pp < n) {
-      const T* kr = kt + pp * D;
-      float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
+  // scores: item = (head, half of the tile); a warp takes one item, lpd lanes per position (1 for
+  // tiles of 64, 2 for tiles of 32, each lane then summing 64 of the 128 dims), so every lane has
+  // work.  K rows are 256 bytes apart: a lane walks its chunks starting at one that depends on the
+  // position, so the 8 lanes of a 16-byte load phase read 8 different chunks (distinct banks; the
+  // q reads are 2-way).
+  {
+    const int lpd = tt == TT ? 1 : 2;
+    const int nch = 16 / lpd;  // 16-byte chunks of the row per lane
+    const int half = lane % lpd;
+    for (int item = warp; item < 2 * G; item += NW) {
+      const int h = item >> 1, pp = (item & 1) * (32 / lpd) + lane / lpd;
+      float sc = -INFINITY;
+      if (pp < n) {
+        const T* kr = kt + pp * D;
+        float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
-      for (int c = 0; c < 16; ++c) {
-        const int cc = (c + lane) & 15;
-        float2 k8[4];
-        KV::load8(kr + cc * 8, k8);
-        const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
-        const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
-        acc = __ffma2_rn(k8[0], make_float2(qa4.x, qa4.y), acc);
-        acc2 = __ffma2_rn(k8[1], make_float2(qa4.z, qa4.w), acc2);
-        acc = __ffma2_rn(k8[2], make_float2(qb4.x, qb4.y), acc);
-        acc2 = __ffma2_rn(k8[3], make_float2(qb4.z, qb4.w), acc2);
+        for (int c = 0; c < nch; ++c) {
+          const int cc = ((c + pp) & (nch - 1)) + half * nch;
+          float2 k8[4];
+          KV::load8(kr + cc * 8, k8);
+          const float4 qa4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8]);
+          const float4 qb4 = *reinterpret_cast<const float4*>(&as.q[h][cc * 8 + 4]);
+          acc = __ffma2_rn(k8[0], make_float2(qa4.x, qa4.y), acc);
+          acc2 = __ffma2_rn(k8[1], make_float2(qa4.z, qa4.w), acc2);
+          acc = __ffma2_rn(k8[2], make_float2(qb4.x, qb4.y), acc);
+          acc2 = __ffma2_rn(k8[3], make_float2(qb4.z, qb4.w), acc2);
+        }
+        sc = (acc.x + acc.y) + (acc2.x + acc2.y);
       }
-      sc = (acc.x + acc.y) + (acc2.x + acc2.y);
+      if (lpd == 2) sc += __shfl_xor_sync(0xffffffffu, sc, 1);  // the pair's two halves
+      if (half == 0) as.s[h][pp] = sc;
     }
-    as.s[h][pp] = sc;
   }
   cbar();
   if (warp < G) {  // softmax statistics of this tile, per head
     const int h = warp;
-    const float s0 = as.s[h][lane], s1 = as.s[h][lane + 32];
+    // positions past the tile's n (all of 32..63 for tiles of 32) hold no score of this item
+    const float s0 = lane < n ? as.s[h][lane] : -INFINITY;
+    const float s1 = lane + 32 < n ? as.s[h][lane + 32] : -INFINITY;
     const float mt = warp_max(fmaxf(s0, s1));
     const float e0 = lane < n ? exp2f(s0 - mt) : 0.f;
     const float e1 = lane + 32 < n ? exp2f(s1 - mt) : 0.f;
@@ -854,17 +864,19 @@ __device__ void attn_item(const StepParams& p, Ring& r, AttnScratch& as, int l, 
     }
   }
   cbar();
-  // P.V: unit = (head h, 8-dim octet o, position quarter q); V rows read as 16-byte vectors (the
-  // 16 octets of a row on consecutive lanes: conflict-free), quarters combined through shared
-  // memory (as.pv), then written as the tile's partial.
+  // P.V: unit = (head h, 8-dim octet o, position quarter q of tt/4 positions); V rows read as
+  // 16-byte vectors (the 16 octets of a row on consecutive lanes: conflict-free), quarters
+  // combined through shared memory (as.pv), then written as the tile's partial.
   {
     const int units = G * 16 * 4;
+    const int ppu = tt / 4;
     for (int u = tid; u < units; u += NT) {
       const int o = u & 15, q = (u >> 4) & 3, h = u >> 6;
       float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
       const float* ph = as.s[h];
-      const int p_end = min(n, q * 16 + 16);
-      for (int pp = q * 16; pp < p_end; ++pp) {
+      const int p_end = min(n, q * ppu + ppu);
+#pragma unroll 4
+      for (int pp = q * ppu; pp < p_end; ++pp) {
         float2 v8[4];
         KV::load8(vt + pp * D + o * 8, v8);
         const float w = ph[pp];
