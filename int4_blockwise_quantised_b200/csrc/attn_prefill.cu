@@ -11,9 +11,10 @@
 //                 S_j = Q K_j^T  (kind::f16, A = Q and B = K_j from shared memory, K-major) into
 //                 S buffer j % 2, and O += P_j V_j (A = P_j from tensor memory, B = V_j from
 //                 shared memory read MN-major, i.e. straight from the row-major cache tile);
-//   warps 2..5  : softmax, one thread per query row (TMEM lane): reads S_j, applies the scale
-//                 (log2 domain) and the causal mask, exponentiates against the row's running
-//                 maximum and writes P_j (fp16) over S_j in tensor memory; O is rescaled only when
+//   warps 2..9  : softmax, two threads per query row (TMEM lane), 64 keys each: reads S_j,
+//                 applies the scale (log2 domain) and the causal mask, exponentiates against the
+//                 row's running maximum and writes P_j (fp16) over S_j in tensor memory (the two
+//                 halves of a row exchange the block maximum first); O is rescaled only when
 //                 a block's maximum exceeds the running one by more than 2^8 (the exponentials
 //                 stay below 2^8, and the final division uses the same maxima); at the end O / l
 //                 is rounded to fp16 and stored.
@@ -35,11 +36,12 @@ namespace {
 constexpr int D = 128;
 constexpr int BQ = 128;   // queries per CTA (TMEM lanes)
 constexpr int BKV = 128;  // keys per block
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, 8 softmax warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // log2 headroom before O is rescaled
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 tile: two 64-column atoms
 constexpr uint32_t kAtom = 128 * 128;      // 128 rows x 128 bytes
+constexpr uint32_t kBarBytes = 128;         // mbarriers + the TMEM address slot
 
 // instruction descriptors (kind::f16, D f32, M = 128, N = 128): S (both K-major); PV (B MN-major)
 constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -125,6 +127,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x by the special-function unit (flushes results below 2^-126 to zero; -inf -> 0).  P is
+// rounded to fp16 afterwards, far coarser than the instruction's error.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Named barrier of the two softmax warps that share TMEM lane quarter q (ids 1..4, 64 threads).
+__device__ __forceinline__ void pair_sync(int q) {
+  asm volatile("bar.sync %0, 64;" ::"r"(q + 1) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -152,6 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = bars + 9;    // [2]
   uint64_t* pv_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  // softmax exchange: block maxima [stage][half][row], final sums [half][row]
+  float (*xm)[2][BQ] = reinterpret_cast<float (*)[2][BQ]>(smem + 5 * kTile + kBarBytes);
+  float (*xl)[BQ] = reinterpret_cast<float (*)[BQ]>(smem + 5 * kTile + kBarBytes + 4 * BQ * 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -170,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 8);
     }
     mbar_init(pv_done, 1);
     fence_mbar_init();
@@ -247,84 +265,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // softmax / epilogue: TMEM lane quarter = warp % 4; row = query q0 + lane quarter * 32 + lane
+    // softmax / epilogue: two threads per query row.  TMEM lane quarter = warp % 4 (row = query
+    // q0 + quarter * 32 + lane); half = which 64 keys of a block (and which 64 columns of O) the
+    // thread takes.  The halves of a row exchange block maxima (and at the end their sums)
+    // through shared memory behind a named barrier of the quarter's two warps.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t col = (uint32_t)(half * 64);
     const float c = a.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < nkb; ++j) {
       const int st = j & 1;
       mbar_wait(&s_full[st], (j >> 1) & 1);
       tc_after();
-      uint32_t sr[4][32];
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS[st] + lane_off + (uint32_t)(cc * 32), sr[cc]);
+      for (int cc = 0; cc < 2; ++cc) tmem_ld32(tS[st] + lane_off + col + (uint32_t)(cc * 32), sr[cc]);
       tmem_wait_ld();
-      const int k0 = j * BKV;
-      const bool diag = j == nkb - 1;
-      float mb = -INFINITY;
+      const int k0 = j * BKV + half * 64;
+      float mb = -INFINITY;  // maximum of the raw scores (the scale c is positive)
+      if (j == nkb - 1) {    // diagonal block: keys after the query are masked
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          float v = __uint_as_float(sr[cc][t]) * c;
-          if (diag && k0 + cc * 32 + t > qi) v = -INFINITY;
-          sr[cc][t] = __float_as_uint(v);
-          mb = fmaxf(mb, v);
+          for (int t = 0; t < 32; ++t) {
+            if (k0 + cc * 32 + t > qi) sr[cc][t] = __float_as_uint(-INFINITY);
+            mb = fmaxf(mb, __uint_as_float(sr[cc][t]));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) mb = fmaxf(mb, __uint_as_float(sr[cc][t]));
         }
       }
+      mb *= c;  // into the log2 domain
+      // row maximum of the block: both halves' S loads are complete before either writes P
+      // over the S buffer (half 1's P columns hold half 0's S keys 32..63)
+      xm[st][half][r] = mb;
+      tc_before();
+      pair_sync(quarter);
+      tc_after();
+      mb = fmaxf(mb, xm[st][half ^ 1][r]);
       // lazy rescale: move the reference maximum only when this block's exceeds it by > 2^8
       const bool move = mb > m_used + kRescale;
       const float m_new = move ? mb : m_used;
       const float corr = move ? exp2f(m_used - m_new) : 1.f;  // 0 on the first block
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // O holds sum over blocks < j: wait until PV_{j-1} has written it, then rescale
+        // O holds sum over blocks < j: wait until PV_{j-1} has written it, then rescale this
+        // thread's 64 columns
         mbar_wait(pv_done, (j - 1) & 1);
         tc_after();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + (uint32_t)(cc * 32), o);
+          tmem_ld32(tO + lane_off + col + (uint32_t)(cc * 32), o);
           tmem_wait_ld();
 #pragma unroll
           for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * corr);
-          tmem_st32(tO + lane_off + (uint32_t)(cc * 32), o);
+          tmem_st32(tO + lane_off + col + (uint32_t)(cc * 32), o);
         }
       }
       l *= corr;
       m_used = m_new;
-      // P_j = 2^(s - m_used) as fp16 pairs into columns 0..63 of the S buffer
-      uint32_t pp[2][32];
-      float ls = 0.f;
+      // P_j = 2^(s - m_used) as fp16 pairs: keys 64 half .. 64 half + 63 into columns
+      // 32 half .. 32 half + 31 of the S buffer
+      uint32_t pp[32];
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
         for (int t = 0; t < 32; t += 2) {
-          const float e0 = exp2f(__uint_as_float(sr[cc][t]) - m_used);
-          const float e1 = exp2f(__uint_as_float(sr[cc][t + 1]) - m_used);
-          ls += e0 + e1;
-          pp[cc >> 1][(cc & 1) * 16 + (t >> 1)] = pack_h2(e0, e1);
+          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[cc][t]), c, -m_used));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[cc][t + 1]), c, -m_used));
+          ls0 += e0;
+          ls1 += e1;
+          pp[cc * 16 + (t >> 1)] = pack_h2(e0, e1);
         }
       }
+      const float ls = ls0 + ls1;
       l += ls;
-      tmem_st32(tS[st] + lane_off, pp[0]);
-      tmem_st32(tS[st] + lane_off + 32, pp[1]);
+      tmem_st32(tS[st] + lane_off + (uint32_t)(half * 32), pp);
       tmem_wait_st();
       tc_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[st]);
     }
-    // epilogue: O / l -> fp16
+    // epilogue: O / (l of both halves) -> fp16, this thread's 64 columns
+    xl[half][r] = l;
+    pair_sync(quarter);
+    l += xl[half ^ 1][r];
     mbar_wait(pv_done, (nkb - 1) & 1);
     tc_after();
     const float il = l > 0.f ? 1.f / l : 0.f;
-    __half* out = reinterpret_cast<__half*>(a.out) + (size_t)qi * a.Hq * D + (size_t)h * D;
+    __half* out = reinterpret_cast<__half*>(a.out) + (size_t)qi * a.Hq * D + (size_t)h * D + col;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
       uint32_t o[32];
-      tmem_ld32(tO + lane_off + (uint32_t)(cc * 32), o);
+      tmem_ld32(tO + lane_off + col + (uint32_t)(cc * 32), o);
       tmem_wait_ld();
       if (qi < S) {
 #pragma unroll
@@ -361,7 +403,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-constexpr size_t kSmem = 5 * kTile + 16 * 8 + 1024;
+constexpr size_t kSmem = 5 * kTile + kBarBytes + 6 * BQ * 4 + 1024;
 
 }  // namespace
 
