@@ -5,12 +5,16 @@
 //
 // Flash attention on the 5th-generation tensor cores.  One CTA = 128 queries x one query head;
 // key/value blocks of 128 positions up to the diagonal.
-//   warp 0      : TMA producer: the Q tile once, then K and V tiles (128 x 128 fp16, 128-byte
-//                 swizzle, two 64-column boxes each) into a two-stage ring;
-//   warp 1      : allocates TMEM (two S buffers + O), one thread issues the MMAs:
-//                 S_j = Q K_j^T  (kind::f16, A = Q and B = K_j from shared memory, K-major) into
-//                 S buffer j % 2, and O += P_j V_j (A = P_j from tensor memory, B = V_j from
-//                 shared memory read MN-major, i.e. straight from the row-major cache tile);
+//   warp 0      : TMA producer of the Q tile (once) and the K tiles (128 x 128 fp16, 128-byte
+//                 swizzle, two 64-column boxes each) into a three-stage ring; a K stage is free
+//                 again as soon as the S MMAs that read it are done;
+//   warp 10     : TMA producer of the V tiles into a two-stage ring (free after P.V);
+//   warp 1      : allocates TMEM (three S / P buffers + O: 512 columns), one thread issues the
+//                 MMAs: S_j = Q K_j^T (kind::f16, A = Q and B = K_j from shared memory,
+//                 K-major) into buffer j % 3, and O += P_j V_j (A = P_j from tensor memory, B =
+//                 V_j from shared memory read MN-major, i.e. straight from the row-major cache
+//                 tile); S_{j+2} is queued right behind P_j V_j, so the tensor pipe has the next
+//                 scores to compute while the softmax of block j + 1 runs;
 //   warps 2..9  : softmax, two threads per query row (TMEM lane), 64 keys each: reads S_j,
 //                 applies the scale (log2 domain) and the causal mask, exponentiates against the
 //                 row's running maximum and writes P_j (fp16) over S_j in tensor memory (the two
@@ -36,12 +40,17 @@ namespace {
 constexpr int D = 128;
 constexpr int BQ = 128;   // queries per CTA (TMEM lanes)
 constexpr int BKV = 128;  // keys per block
-constexpr int kThreads = 320;  // producer, MMA issuer, 8 softmax warps
+constexpr int kThreads = 352;  // K producer, MMA issuer, 8 softmax warps, V producer
+constexpr int kVWarp = 10;
+constexpr int kKStages = 3;   // K tiles in flight (a stage is free once its S MMAs are done)
+constexpr int kVStages = 2;   // V tiles in flight (free once the P.V MMAs are done)
+constexpr int kSBufs = 3;     // S / P buffers in tensor memory (+ O: 512 columns)
+constexpr int kTiles = 1 + kKStages + kVStages;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // log2 headroom before O is rescaled
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 tile: two 64-column atoms
 constexpr uint32_t kAtom = 128 * 128;      // 128 rows x 128 bytes
-constexpr uint32_t kBarBytes = 128;         // mbarriers + the TMEM address slot
+constexpr uint32_t kBarBytes = 256;         // mbarriers + the TMEM address slot
 
 // instruction descriptors (kind::f16, D f32, M = 128, N = 128): S (both K-major); PV (B MN-major)
 constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -156,20 +165,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = smem;
-  unsigned char* sK = smem + kTile;           // 2 stages
-  unsigned char* sV = smem + 3 * kTile;       // 2 stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTile);
+  unsigned char* sK = smem + kTile;      // kKStages stages
+  unsigned char* sV = smem + (1 + kKStages) * kTile;  // kVStages stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTiles * kTile);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;    // [2]
-  uint64_t* pv_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  // softmax exchange: block maxima [stage][half][row], final sums [half][row]
-  float (*xm)[2][BQ] = reinterpret_cast<float (*)[2][BQ]>(smem + 5 * kTile + kBarBytes);
-  float (*xl)[BQ] = reinterpret_cast<float (*)[BQ]>(smem + 5 * kTile + kBarBytes + 4 * BQ * 4);
+  uint64_t* k_full = bars + 1;                 // [kKStages]
+  uint64_t* k_empty = k_full + kKStages;       // [kKStages]
+  uint64_t* v_full = k_empty + kKStages;       // [kVStages]
+  uint64_t* v_empty = v_full + kVStages;       // [kVStages]
+  uint64_t* s_full = v_empty + kVStages;       // [kSBufs]
+  uint64_t* p_full = s_full + kSBufs;          // [kSBufs]
+  uint64_t* pv_done = p_full + kSBufs;         // [kSBufs]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + kSBufs);
+  // softmax exchange: block maxima [block parity][half][row], final sums [half][row]
+  float (*xm)[2][BQ] = reinterpret_cast<float (*)[2][BQ]>(smem + kTiles * kTile + kBarBytes);
+  float (*xl)[BQ] =
+      reinterpret_cast<float (*)[BQ]>(smem + kTiles * kTile + kBarBytes + 4 * BQ * 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -183,14 +194,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 8);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(pv_done, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -203,22 +219,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
+  auto tS = [tmem](int b) { return tmem + (uint32_t)(b * 128); };  // S_j / P_j: buffer j % 3
+  const uint32_t tO = tmem + 384;
 
   if (warp == 0) {
+    // Q once, then K_j into stage j % kKStages once S_{j - kKStages} has read that stage
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, kTile);
       tma_load_2d(sQ, &mp.q, h * D, q0, q_full);
       tma_load_2d(sQ + kAtom, &mp.q, h * D + 64, q0, q_full);
       for (int j = 0; j < nkb; ++j) {
-        const int st = j & 1;
-        if (j >= 2) mbar_wait(&kv_empty[st], ((j >> 1) - 1) & 1);
+        const int st = j % kKStages;
+        if (j >= kKStages) mbar_wait(&k_empty[st], (j / kKStages - 1) & 1);
         unsigned char* kt = sK + st * kTile;
-        unsigned char* vt = sV + st * kTile;
         mbar_arrive_expect_tx(&k_full[st], kTile);
         tma_load_3d(kt, &mp.kv[0], 0, j * BKV, g, &k_full[st]);
         tma_load_3d(kt + kAtom, &mp.kv[0], 64, j * BKV, g, &k_full[st]);
+      }
+    }
+  } else if (warp == kVWarp) {
+    // V_j into stage j % kVStages once PV_{j - kVStages} has read that stage
+    if (lane == 0) {
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j % kVStages;
+        if (j >= kVStages) mbar_wait(&v_empty[st], (j / kVStages - 1) & 1);
+        unsigned char* vt = sV + st * kTile;
         mbar_arrive_expect_tx(&v_full[st], kTile);
         tma_load_3d(vt, &mp.kv[1], 0, j * BKV, g, &v_full[st]);
         tma_load_3d(vt + kAtom, &mp.kv[1], 64, j * BKV, g, &v_full[st]);
@@ -228,37 +253,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       mbar_wait(q_full, 0);
       const uint32_t qa = smem_u32(sQ);
-      // S_j into buffer j % 2: 8 K-steps of 16 (32 bytes inside a 128-byte row, atom per 64)
+      // S_j into buffer j % 3: 8 K-steps of 16 (32 bytes inside a 128-byte row, atom per 64);
+      // the K stage is released when these MMAs complete
       auto issue_s = [&](int j) {
-        const int st = j & 1;
-        mbar_wait(&k_full[st], (j >> 1) & 1);
+        const int st = j % kKStages;
+        mbar_wait(&k_full[st], (j / kKStages) & 1);
         tc_after();
         const uint32_t kb = smem_u32(sK + st * kTile);
+        const uint32_t d = tS(j % kSBufs);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * kAtom + (uint32_t)(k & 3) * 32;
-          mma_ss(tS[st], desc_k_sw128(qa + off), desc_k_sw128(kb + off), kIdescS, k > 0 ? 1u : 0u);
+          mma_ss(d, desc_k_sw128(qa + off), desc_k_sw128(kb + off), kIdescS, k > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[st]);
+        mma_commit(&s_full[j % kSBufs]);
+        mma_commit(&k_empty[st]);
       };
       issue_s(0);
       if (nkb > 1) issue_s(1);
       for (int j = 0; j < nkb; ++j) {
-        const int st = j & 1;
-        mbar_wait(&p_full[st], (j >> 1) & 1);
-        mbar_wait(&v_full[st], (j >> 1) & 1);
+        const int bj = j % kSBufs, vs = j % kVStages;
+        mbar_wait(&p_full[bj], (j / kSBufs) & 1);
+        mbar_wait(&v_full[vs], (j / kVStages) & 1);
         tc_after();
-        const uint32_t vb = smem_u32(sV + st * kTile);
+        const uint32_t vb = smem_u32(sV + vs * kTile);
         // O += P_j V_j: K = keys, 16 per step (8 TMEM columns of fp16 pairs; 2 x 8 rows of V)
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
-          mma_ts(tO, tS[st] + (uint32_t)(k * 8), desc_mn_sw128(vb + (uint32_t)k * 2048), kIdescPV,
+          mma_ts(tO, tS(bj) + (uint32_t)(k * 8), desc_mn_sw128(vb + (uint32_t)k * 2048), kIdescPV,
                  (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[st]);
-        mma_commit(pv_done);
+        mma_commit(&v_empty[vs]);
+        mma_commit(&pv_done[bj]);
         if (j + 2 < nkb) {
-          // S_{j+2} overwrites P_j: after PV_j has read it
-          mbar_wait(pv_done, j & 1);
+          // S_{j+2} goes into the buffer of P_{j-1}: queued right behind PV_j once PV_{j-1}
+          // has read it
+          if (j >= 1) {
+            mbar_wait(&pv_done[(j - 1) % kSBufs], ((j - 1) / kSBufs) & 1);
+            tc_after();
+          }
           issue_s(j + 2);
         }
       }
@@ -278,12 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = a.scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < nkb; ++j) {
-      const int st = j & 1;
-      mbar_wait(&s_full[st], (j >> 1) & 1);
+      const int bj = j % kSBufs, xs = j & 1;
+      mbar_wait(&s_full[bj], (j / kSBufs) & 1);
       tc_after();
       uint32_t sr[2][32];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) tmem_ld32(tS[st] + lane_off + col + (uint32_t)(cc * 32), sr[cc]);
+      for (int cc = 0; cc < 2; ++cc) tmem_ld32(tS(bj) + lane_off + col + (uint32_t)(cc * 32), sr[cc]);
       tmem_wait_ld();
       const int k0 = j * BKV + half * 64;
       float mb = -INFINITY;  // maximum of the raw scores (the scale c is positive)
@@ -306,11 +338,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mb *= c;  // into the log2 domain
       // row maximum of the block: both halves' S loads are complete before either writes P
       // over the S buffer (half 1's P columns hold half 0's S keys 32..63)
-      xm[st][half][r] = mb;
+      xm[xs][half][r] = mb;
       tc_before();
       pair_sync(quarter);
       tc_after();
-      mb = fmaxf(mb, xm[st][half ^ 1][r]);
+      mb = fmaxf(mb, xm[xs][half ^ 1][r]);
       // lazy rescale: move the reference maximum only when this block's exceeds it by > 2^8
       const bool move = mb > m_used + kRescale;
       const float m_new = move ? mb : m_used;
@@ -318,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j > 0 && __any_sync(0xffffffffu, move)) {
         // O holds sum over blocks < j: wait until PV_{j-1} has written it, then rescale this
         // thread's 64 columns
-        mbar_wait(pv_done, (j - 1) & 1);
+        mbar_wait(&pv_done[(j - 1) % kSBufs], ((j - 1) / kSBufs) & 1);
         tc_after();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -349,17 +381,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float ls = ls0 + ls1;
       l += ls;
-      tmem_st32(tS[st] + lane_off + (uint32_t)(half * 32), pp);
+      tmem_st32(tS(bj) + lane_off + (uint32_t)(half * 32), pp);
       tmem_wait_st();
       tc_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[st]);
+      if (lane == 0) mbar_arrive(&p_full[bj]);
     }
     // epilogue: O / (l of both halves) -> fp16, this thread's 64 columns
     xl[half][r] = l;
     pair_sync(quarter);
     l += xl[half ^ 1][r];
-    mbar_wait(pv_done, (nkb - 1) & 1);
+    mbar_wait(&pv_done[(nkb - 1) % kSBufs], ((nkb - 1) / kSBufs) & 1);
     tc_after();
     const float il = l > 0.f ? 1.f / l : 0.f;
     __half* out = reinterpret_cast<__half*>(a.out) + (size_t)qi * a.Hq * D + (size_t)h * D + col;
@@ -403,7 +435,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-constexpr size_t kSmem = 5 * kTile + kBarBytes + 6 * BQ * 4 + 1024;
+constexpr size_t kSmem = kTiles * kTile + kBarBytes + 6 * BQ * 4 + 1024;
 
 }  // namespace
 
