@@ -14,7 +14,8 @@
 //                 the accumulator is released back to the MMA warp, so the epilogue of tile i
 //                 overlaps the main loop of tile i + 1.
 // Epilogues: BIAS (fp32 out + fp16 bias), RESID (fp32 x += acc), SWIGLU (columns interleaved
-// gate/up -> fp16 silu(g) * u), F16 (fp16 out + fp16 bias).  Rows >= M are masked (TMA
+// gate/up -> fp16 silu(g) * u), F16 (fp16 out + fp16 bias), ROPE (q/k/v + bias, rotary embedding
+// of the query and key heads, fp16 queries and K/V cache rows out).  Rows >= M are masked (TMA
 // zero-fills the A tail).  Every mbarrier wait is bounded; TMEM is released before the CTA exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -102,6 +103,57 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// kEpiRope: columns [c0 + p, +32) (v1) and [c0 + 64 + p, +32) (v2) of head c0 / 128 for one row.
+__device__ __forceinline__ void epilogue_rope(const GemmEpilogue& e, float (&v1)[32],
+                                              float (&v2)[32], int row, int c0, int p) {
+  constexpr int D = 128;
+  const int head = c0 / D;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    v1[j] += __half2float(e.bias[c0 + p + j]);
+    v2[j] += __half2float(e.bias[c0 + D / 2 + p + j]);
+  }
+  if (head < e.hq + e.hkv) {  // query or key head: rotate the pairs (d, d + 64), d = p + j
+    int pos = e.pos[row];
+    if (pos < 0 || pos >= e.max_pos) {
+      set_device_error(VV_ERR_RANGE);
+      pos = min(max(pos, 0), e.max_pos - 1);
+    }
+    const float* ct = e.rope_cos + (size_t)pos * (D / 2) + p;
+    const float* st = e.rope_sin + (size_t)pos * (D / 2) + p;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 cs = *reinterpret_cast<const float4*>(ct + j);
+      const float4 sn = *reinterpret_cast<const float4*>(st + j);
+      const float c4[4] = {cs.x, cs.y, cs.z, cs.w}, s4[4] = {sn.x, sn.y, sn.z, sn.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float x1 = v1[j + t], x2 = v2[j + t];
+        v1[j + t] = x1 * c4[t] - x2 * s4[t];
+        v2[j + t] = x2 * c4[t] + x1 * s4[t];
+      }
+    }
+  }
+  __half* dst;
+  if (head < e.hq)
+    dst = e.out_f16 + (size_t)row * e.ldo + (size_t)head * D;
+  else if (head < e.hq + e.hkv)
+    dst = e.kc + ((size_t)(head - e.hq) * e.cap + row) * D;
+  else
+    dst = e.vc + ((size_t)(head - e.hq - e.hkv) * e.cap + row) * D;
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    __align__(16) __half a[8], b[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      a[t] = __float2half_rn(v1[j + t]);
+      b[t] = __float2half_rn(v2[j + t]);
+    }
+    *reinterpret_cast<uint4*>(dst + p + j) = *reinterpret_cast<const uint4*>(a);
+    *reinterpret_cast<uint4*>(dst + D / 2 + p + j) = *reinterpret_cast<const uint4*>(b);
+  }
+}
+
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, const float (&v)[32], int row,
                                                int col) {
@@ -151,6 +203,32 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, const floa
     }
   }
 }
+
+// One accumulator row of a tile through the epilogue (kEpiRope: the two halves of each head
+// together).
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue_row(const GemmEpilogue& e, uint32_t base, int row, int M,
+                                             int col0) {
+  if constexpr (EPI == kEpiRope) {
+    static_assert(BN % 128 == 0, "rope tiles hold whole heads");
+#pragma unroll 1
+    for (int hb = 0; hb < BN; hb += 128)
+#pragma unroll 1
+      for (int p = 0; p < 64; p += 32) {
+        float v1[32], v2[32];
+        tmem_ld32(base + (uint32_t)(hb + p), v1);
+        tmem_ld32(base + (uint32_t)(hb + 64 + p), v2);
+        if (row < M) epilogue_rope(e, v1, v2, row, col0 + hb, p);
+      }
+  } else {
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(base + (uint32_t)c, v);
+      if (row < M) epilogue_chunk<EPI, BN>(e, v, row, col0 + c);
+    }
+  }
+}
+
 
 template <int EPI, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -248,11 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&acc_full[buf], (i >> 1) & 1);
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld32(base + (uint32_t)c, v);
-        if (row < M) epilogue_chunk<EPI, BN>(e, v, row, n_blk * BN + c);
-      }
+      epilogue_row<EPI, BN>(e, base, row, M, n_blk * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -443,11 +517,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       mbar_wait(&acc_full[buf], (i >> 1) & 1);
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld32(base + (uint32_t)c, v);
-        if (row < M) epilogue_chunk<EPI, BN>(e, v, row, n_blk * BN + c);
-      }
+      epilogue_row<EPI, BN>(e, base, row, M, n_blk * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -602,6 +672,9 @@ cudaError_t launch_q4_bn(const uint16_t* A, const PackedB& B, int M, int N, int 
     case kEpiResid: return run_q4<kEpiResid, BN>(ta, pm, e, M, N, K, grid, s);
     case kEpiSwiglu: return run_q4<kEpiSwiglu, BN>(ta, pm, e, M, N, K, grid, s);
     case kEpiF16: return run_q4<kEpiF16, BN>(ta, pm, e, M, N, K, grid, s);
+    case kEpiRope:
+      if constexpr (BN % 128 == 0) return run_q4<kEpiRope, BN>(ta, pm, e, M, N, K, grid, s);
+      return cudaErrorInvalidValue;  // tiles of 192 columns split heads
     default: return cudaErrorInvalidValue;
   }
 }
@@ -745,6 +818,9 @@ cudaError_t launch_bn(const uint16_t* A, const uint16_t* B, int M, int N, int K,
     case kEpiResid: return run_gemm<kEpiResid, BN>(ta, tb, e, M, N, K, grid, s);
     case kEpiSwiglu: return run_gemm<kEpiSwiglu, BN>(ta, tb, e, M, N, K, grid, s);
     case kEpiF16: return run_gemm<kEpiF16, BN>(ta, tb, e, M, N, K, grid, s);
+    case kEpiRope:
+      if constexpr (BN % 128 == 0) return run_gemm<kEpiRope, BN>(ta, tb, e, M, N, K, grid, s);
+      return cudaErrorInvalidValue;  // tiles of 192 columns split heads
     default: return cudaErrorInvalidValue;
   }
 }
@@ -767,6 +843,7 @@ bool gemm_q4_supported(const PackedB& B, int N, int K) {
 cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
   if (M < 1 || !gemm_q4_supported(B, N, K) || !aligned16(A)) return cudaErrorInvalidValue;
+  if (epi == kEpiRope && (N % 128 != 0 || !e.bias || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
   for (int g = 0; g < B.nseg; ++g)
     if (!aligned16(B.q[g]) || !aligned16(B.s[g])) return cudaErrorInvalidValue;
   const int sms = sm_count();
@@ -774,7 +851,7 @@ cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, in
   // tile width: segments (or interleaved pairs) must hold whole tiles; among the widths that
   // fit, the widest whose wave efficiency is within 0.1 of the best
   auto fits = [&](int w) {
-    if (N % w != 0) return false;
+    if (N % w != 0 || (epi == kEpiRope && w % 128 != 0)) return false;
     if (B.interleave) return (w / 2) % 8 == 0;
     for (int g = 0; g < B.nseg; ++g)
       if (B.rows[g] % w != 0) return false;
@@ -799,16 +876,18 @@ size_t gemm_tc_smem() { return smem_bytes<256>(); }
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
   if (M < 1 || N % 64 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
+  if (epi == kEpiRope && (N % 128 != 0 || !e.bias || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
   if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
   const int sms = sm_count();
   const long mt = (M + BM - 1) / BM;
   // the widest tile whose wave efficiency is within 0.1 of the best available width
   const int widths[3] = {256, 192, 128};
+  auto fits = [&](int w) { return N % w == 0 && (epi != kEpiRope || w % 128 == 0); };
   double best = 0.0;
   for (int w : widths)
-    if (N % w == 0) best = std::max(best, wave_eff(mt * (N / w), sms));
+    if (fits(w)) best = std::max(best, wave_eff(mt * (N / w), sms));
   for (int w : widths) {
-    if (N % w != 0 || wave_eff(mt * (N / w), sms) < best - 0.1) continue;
+    if (!fits(w) || wave_eff(mt * (N / w), sms) < best - 0.1) continue;
     if (w == 256) return launch_bn<256>(A, B, M, N, K, epi, e, s);
     if (w == 192) return launch_bn<192>(A, B, M, N, K, epi, e, s);
     return launch_bn<128>(A, B, M, N, K, epi, e, s);

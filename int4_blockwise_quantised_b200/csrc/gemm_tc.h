@@ -11,16 +11,28 @@ constexpr int kEpiBias = 0;    // out_f32[m, n] = acc + bias[n]
 constexpr int kEpiResid = 1;   // out_f32[m, n] += acc
 constexpr int kEpiSwiglu = 2;  // out_f16[m, n/2] = silu(acc[m, n]) * acc[m, n+1], n even
 constexpr int kEpiF16 = 3;     // out_f16[m, n] = fp16(acc + bias[n])
+// q/k/v with rotary embedding: y = acc + bias[n]; the columns of query and key heads are rotated
+// at position pos[m] (pairs d, d + D/2 of a head of D = 128); queries -> out_f16[m, n] (fp16,
+// row stride ldo = hq * D), keys / values -> kc / vc [head][cap][D] at slot m (fp16)
+constexpr int kEpiRope = 4;
 
 struct GemmEpilogue {
   float* out_f32;
   __half* out_f16;
   const __half* bias;
   int ldo;  // row stride of the output in elements
+  // kEpiRope only
+  const int32_t* pos;     // [M] position ids
+  const float* rope_cos;  // [max_pos][D/2]
+  const float* rope_sin;
+  int max_pos, hq, hkv, cap;
+  __half* kc;
+  __half* vc;
 };
 
 size_t gemm_tc_smem();
-// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 128 == 0 or N % 192 == 0, K % 64 == 0.
+// A: fp16 [M, K] row-major; B: fp16 [N, K] row-major; N % 128 == 0 or N % 192 == 0 (kEpiRope:
+// N % 128 == 0), K % 64 == 0.
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s);
 

@@ -4,15 +4,17 @@
 //
 // Tensor-core path, per layer (S prompt positions, fp32 residual X [S, H]):
 //   Xn  = RMSNorm(X)                                  (fp16, the GEMM operand)
-//   QKV = Xn . [Wq;Wk;Wv]^T + b                       tcgen05 GEMM, bias epilogue
-//   Q, K, V <- RoPE(QKV); K, V -> cache slots 0..S-1  (fp16)
-//   O   = causal GQA attention                       mma.sync flash attention
+//   Q, K, V = RoPE(Xn . [Wq;Wk;Wv]^T + b)             tcgen05 GEMM; its epilogue rotates q and k
+//                                                     and writes fp16 Q and cache slots 0..S-1
+//   O   = causal GQA attention                        tcgen05 flash attention (S, P, O in TMEM)
 //   X  += O . Wo^T                                    tcgen05 GEMM, residual epilogue
 //   Hm  = silu(Xn Wg^T) * (Xn Wu^T), Xn = RMSNorm(X)  tcgen05 GEMM over interleaved gate/up rows
 //   X  += Hm . Wd^T                                   tcgen05 GEMM, residual epilogue
-// The GEMMs read the packed int4 matrices as they are: converter warps inside the GEMM expand each
-// 64-column block of codes to fp16 ((code - 8) * scale, rounded once) in shared memory, right
-// before the tensor cores read it.  The last row then goes through the final RMSNorm + lm_head.
+// Weights: for prompts of at most kFusedMaxM positions the GEMMs read the packed int4 matrices
+// as they are (converter warps expand each 64-column block of codes to fp16, (code - 8) * scale
+// rounded once, in shared memory right before the tensor cores read it); longer prompts
+// dequantise the layer's four weight stacks to fp16 once at the start of the layer (one launch)
+// and run the fp16 GEMM on them.  The last row then goes through the final RMSNorm + lm_head.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -75,64 +77,6 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const float* __restri
     pk.x = *reinterpret_cast<uint32_t*>(&a);
     pk.y = *reinterpret_cast<uint32_t*>(&b);
     *reinterpret_cast<uint2*>(out + (size_t)row * H + i) = pk;
-  }
-}
-
-// RoPE of q and k at position_ids[s], then Q -> fp16 [S, Hq*D]; K, V -> cache slot s (fp16).
-// One CTA per position; each thread takes 8 consecutive dims of one head (vector loads of x and
-// of its rotate-half partner, one 16-byte store).
-__global__ void __launch_bounds__(256) rope_kv_kernel(const float* __restrict__ qkv, int S,
-                                                      int Hq, int Hkv, const int32_t* __restrict__ pos_ids,
-                                                      const float* __restrict__ cos_t,
-                                                      const float* __restrict__ sin_t, int max_pos,
-                                                      __half* __restrict__ q_out,
-                                                      __half* __restrict__ kc, __half* __restrict__ vc,
-                                                      int cap) {
-  const int s = blockIdx.x;
-  const int nh = Hq + 2 * Hkv;
-  int pos = pos_ids[s];
-  if (pos < 0 || pos >= max_pos) {
-    if (threadIdx.x == 0) set_device_error(VV_ERR_RANGE);
-    pos = min(max(pos, 0), max_pos - 1);
-  }
-  const float* row = qkv + (size_t)s * nh * D;
-  for (int c = threadIdx.x; c < nh * (D / 8); c += blockDim.x) {
-    const int hh = c / (D / 8), d0 = (c % (D / 8)) * 8;
-    const float* hr = row + hh * D;
-    float y[8];
-    if (hh >= Hq + Hkv) {  // value head: no rotation
-      const float4 a = *reinterpret_cast<const float4*>(hr + d0);
-      const float4 b = *reinterpret_cast<const float4*>(hr + d0 + 4);
-      y[0] = a.x; y[1] = a.y; y[2] = a.z; y[3] = a.w;
-      y[4] = b.x; y[5] = b.y; y[6] = b.z; y[7] = b.w;
-    } else {
-      const int f0 = d0 & (D / 2 - 1);
-      float x1[8], x2[8], cs[8], sn[8];
-      *reinterpret_cast<float4*>(x1) = *reinterpret_cast<const float4*>(hr + f0);
-      *reinterpret_cast<float4*>(x1 + 4) = *reinterpret_cast<const float4*>(hr + f0 + 4);
-      *reinterpret_cast<float4*>(x2) = *reinterpret_cast<const float4*>(hr + f0 + D / 2);
-      *reinterpret_cast<float4*>(x2 + 4) = *reinterpret_cast<const float4*>(hr + f0 + D / 2 + 4);
-      const float* ct = cos_t + (size_t)pos * (D / 2) + f0;
-      const float* st = sin_t + (size_t)pos * (D / 2) + f0;
-      *reinterpret_cast<float4*>(cs) = *reinterpret_cast<const float4*>(ct);
-      *reinterpret_cast<float4*>(cs + 4) = *reinterpret_cast<const float4*>(ct + 4);
-      *reinterpret_cast<float4*>(sn) = *reinterpret_cast<const float4*>(st);
-      *reinterpret_cast<float4*>(sn + 4) = *reinterpret_cast<const float4*>(st + 4);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        y[j] = d0 < D / 2 ? x1[j] * cs[j] - x2[j] * sn[j] : x2[j] * cs[j] + x1[j] * sn[j];
-    }
-    __align__(16) __half h[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) h[j] = __float2half_rn(y[j]);
-    __half* dst;
-    if (hh < Hq)
-      dst = q_out + (size_t)s * Hq * D + (size_t)hh * D + d0;
-    else if (hh < Hq + Hkv)
-      dst = kc + ((size_t)(hh - Hq) * cap + s) * D + d0;
-    else
-      dst = vc + ((size_t)(hh - Hq - Hkv) * cap + s) * D + d0;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
   }
 }
 
@@ -224,7 +168,6 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
   };
   const size_t o_x = take((size_t)SM * H * 4);
   const size_t o_xn = take((size_t)SM * (H > HQD ? H : HQD) * 2);
-  const size_t o_qkv = take((size_t)SM * NQKV * 4);
   const size_t o_q = take((size_t)SM * HQD * 2);
   const size_t o_h = take((size_t)SM * I * 2);
   const size_t o_bias = take((size_t)NQKV * 2);
@@ -245,7 +188,6 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
   unsigned char* b = d->pws;
   float* X = reinterpret_cast<float*>(b + o_x);
   __half* Xn = reinterpret_cast<__half*>(b + o_xn);  // also the attention output O
-  float* QKV = reinterpret_cast<float*>(b + o_qkv);
   __half* Q = reinterpret_cast<__half*>(b + o_q);
   __half* Hm = reinterpret_cast<__half*>(b + o_h);
   __half* Bqkv = reinterpret_cast<__half*>(b + o_bias);
@@ -316,20 +258,28 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
       boff += brows[m];
     }
     VV_MARK(kPfMisc);
+    // q/k/v + bias, rotary embedding at position_ids, fp16 Q and the K/V cache rows written by
+    // the GEMM's epilogue
     GemmEpilogue ep = {};
-    ep.out_f32 = QKV;
+    ep.out_f16 = Q;
     ep.bias = Bqkv;
-    ep.ldo = NQKV;
+    ep.ldo = HQD;
+    ep.pos = pos;
+    ep.rope_cos = d->rope_cos;
+    ep.rope_sin = d->rope_sin;
+    ep.max_pos = c.max_position;
+    ep.hq = Hq;
+    ep.hkv = Hkv;
+    ep.cap = c.kv_capacity;
+    ep.kc = kc;
+    ep.vc = vc;
     if (two_pass) {
       if ((e = dequant_layer(l, s)) != cudaSuccess) return e;
       VV_MARK(kPfDequant);
     }
-    if ((e = project(l, 0, reinterpret_cast<const uint16_t*>(Xn), pb, NQKV, H, kEpiBias, ep)) !=
+    if ((e = project(l, 0, reinterpret_cast<const uint16_t*>(Xn), pb, NQKV, H, kEpiRope, ep)) !=
         cudaSuccess)
       return e;
-    rope_kv_kernel<<<S, 256, 0, s>>>(QKV, S, Hq, Hkv, pos, d->rope_cos, d->rope_sin,
-                                                      c.max_position, Q, kc, vc, c.kv_capacity);
-    VV_MARK(kPfMisc);
     // ---- attention -> O (in the Xn buffer)
     AttnPrefillArgs aa = {};
     aa.q = reinterpret_cast<const uint16_t*>(Q);
