@@ -247,7 +247,8 @@ typedef struct vv_decoder vv_decoder;
  * lifetime; k_cache/v_cache likewise.  Allocates the decoder's workspace.  Length starts at 0.
  * Requirements: head_dim == 128, n_kv <= 64, n_q % n_kv == 0, n_q/n_kv <= 8, hidden a multiple
  * of 128 (<= 7680; 896 for the Realtime-0.5B backbone), inter a multiple of 256 (<= 65536),
- * n_q * head_dim <= 7680, 1 <= kv_capacity, 1 <= max_position.  With max_prefill > 0, the
+ * n_q * head_dim <= 7680, 1 <= kv_capacity, 1 <= max_position; every device pointer (caches,
+ * tables, packed matrices, norm gains, biases) 16-byte aligned.  With max_prefill > 0, the
  * scales of matrices whose K / 32 is not a multiple of 8 are copied once with a padded row
  * pitch for the prefill GEMMs (the decoder owns the copy).
  * Errors: VV_ERR_INVALID_ARG, VV_ERR_SHAPE, VV_ERR_CUDA (allocation). */

@@ -80,7 +80,7 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
                  "layers/vocab/capacity/max_position");
   VV_CHECK_ARG(w->embed && w->lm_head && w->final_norm, "embed/lm_head/final_norm null");
   VV_CHECK_ARG(vv::aligned16(k_cache) && vv::aligned16(v_cache) && vv::aligned16(w->lm_head) &&
-                   vv::aligned16(w->embed),
+                   vv::aligned16(w->embed) && vv::aligned16(w->final_norm),
                "cache / table pointers must be 16-byte aligned");
   for (int l = 0; l < c.layers; ++l) {
     const vv_layer_weights& L = w->layers[l];
@@ -89,6 +89,11 @@ vv_status vv_decoder_create(const vv_config* cfg, const vv_model_weights* w, uin
       VV_CHECK_ARG(p->q && p->scales && vv::aligned16(p->q) && vv::aligned16(p->scales),
                    "layer %d: packed weight null or not 16-byte aligned", l);
     VV_CHECK_ARG(L.input_norm && L.post_norm, "layer %d: norm gain null", l);
+    // the kernels read gains and biases as vectors
+    VV_CHECK_ARG(vv::aligned16(L.input_norm) && vv::aligned16(L.post_norm) &&
+                     (!L.bq || vv::aligned16(L.bq)) && (!L.bk || vv::aligned16(L.bk)) &&
+                     (!L.bv || vv::aligned16(L.bv)),
+                 "layer %d: norm gain or bias not 16-byte aligned", l);
   }
 
   vv_decoder* d = new (std::nothrow) vv_decoder();

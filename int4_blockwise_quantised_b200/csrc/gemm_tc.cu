@@ -108,10 +108,26 @@ __device__ __forceinline__ void epilogue_rope(const GemmEpilogue& e, float (&v1)
                                               float (&v2)[32], int row, int c0, int p) {
   constexpr int D = 128;
   const int head = c0 / D;
+  const __half* bh;  // this head's bias (uniform over the tile)
+  if (head < e.hq)
+    bh = e.bias ? e.bias + (size_t)head * D : nullptr;
+  else if (head < e.hq + e.hkv)
+    bh = e.bias_k ? e.bias_k + (size_t)(head - e.hq) * D : nullptr;
+  else
+    bh = e.bias_v ? e.bias_v + (size_t)(head - e.hq - e.hkv) * D : nullptr;
+  if (bh) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    v1[j] += __half2float(e.bias[c0 + p + j]);
-    v2[j] += __half2float(e.bias[c0 + D / 2 + p + j]);
+    for (int j = 0; j < 32; j += 8) {
+      const uint4 b1 = *reinterpret_cast<const uint4*>(bh + p + j);
+      const uint4 b2 = *reinterpret_cast<const uint4*>(bh + D / 2 + p + j);
+      const __half* h1 = reinterpret_cast<const __half*>(&b1);
+      const __half* h2 = reinterpret_cast<const __half*>(&b2);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        v1[j + t] += __half2float(h1[t]);
+        v2[j + t] += __half2float(h2[t]);
+      }
+    }
   }
   if (head < e.hq + e.hkv) {  // query or key head: rotate the pairs (d, d + 64), d = p + j
     int pos = e.pos[row];
@@ -715,26 +731,33 @@ __global__ void __launch_bounds__(256) dequant_f16_kernel(const DequantSrc src, 
 }  // namespace
 
 namespace {
-// Several matrix stacks in one launch: job j covers blocks [first[j], first[j + 1]) of the
-// launch's block range.
+// Several matrix stacks in one launch.  Work unit = (output row, piece of 1024 columns): one warp,
+// lane l expanding code words 128 * piece + l + 32 t (t < 4; 8 weights each), all loads issued
+// before the first store, so each store instruction of a warp writes 512 contiguous bytes.  Job j
+// covers units [first[j], first[j + 1]).
+constexpr int kDqWords = 4;                   // code words per lane per unit
+constexpr int kDqCols = 32 * kDqWords * 8;    // columns per unit
 struct DequantJobs {
   DequantSrc src[4];
   __half* out[4];
   int K[4];
-  int64_t first[5];
+  int first[5];
   int n;
 };
 
 __global__ void __launch_bounds__(256) dequant_jobs_kernel(const DequantJobs jb) {
-  const int64_t total = jb.first[jb.n];
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
-       g += (int64_t)gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int total = jb.first[jb.n];
+  const int nw = (int)gridDim.x * (int)(blockDim.x >> 5);
+  for (int u = (int)blockIdx.x * (int)(blockDim.x >> 5) + (int)(threadIdx.x >> 5); u < total;
+       u += nw) {
     int j = 0;
-    while (j + 1 < jb.n && g >= jb.first[j + 1]) ++j;
+    while (j + 1 < jb.n && u >= jb.first[j + 1]) ++j;
     const DequantSrc& src = jb.src[j];
-    const int K = jb.K[j], KB = K >> 5;
-    const int64_t b = g - jb.first[j];
-    const int orow = (int)(b / KB), kb = (int)(b % KB);
+    const int K = jb.K[j], KB = K >> 5, PK = (K + kDqCols - 1) / kDqCols, nwords = K >> 3;
+    const int v = u - jb.first[j];
+    const int orow = v / PK;
+    const int c0 = (v - orow * PK) * (32 * kDqWords) + lane;  // first code word of this lane
     int m, r;
     if (src.interleave) {
       m = orow & 1;
@@ -744,14 +767,22 @@ __global__ void __launch_bounds__(256) dequant_jobs_kernel(const DequantJobs jb)
       r = orow;
       while (m < src.nseg - 1 && r >= src.rows[m]) r -= src.rows[m++];
     }
-    const uint4 codes = __ldg(reinterpret_cast<const uint4*>(src.q[m] + ((size_t)r * KB + kb) * 16));
-    const uint32_t sh = src.s[m][(size_t)r * KB + kb];
-    const uint32_t s2 = sh | (sh << 16);
-    uint4* dst = reinterpret_cast<uint4*>(jb.out[j] + (size_t)orow * K + (size_t)kb * 32);
-    dst[0] = dequant8_f16(codes.x, s2);
-    dst[1] = dequant8_f16(codes.y, s2);
-    dst[2] = dequant8_f16(codes.z, s2);
-    dst[3] = dequant8_f16(codes.w, s2);
+    // word c of a row = word c % 4 of block c / 4: 8 consecutive weights
+    const uint32_t* qr = reinterpret_cast<const uint32_t*>(src.q[m]) + (size_t)r * KB * 4;
+    const uint16_t* sr = src.s[m] + (size_t)r * KB;
+    uint32_t w[kDqWords], sh[kDqWords];
+#pragma unroll
+    for (int t = 0; t < kDqWords; ++t) {
+      const int c = c0 + 32 * t;
+      w[t] = c < nwords ? __ldg(qr + c) : 0u;
+      sh[t] = c < nwords ? (uint32_t)__ldg(sr + (c >> 2)) : 0u;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(jb.out[j] + (size_t)orow * K);
+#pragma unroll
+    for (int t = 0; t < kDqWords; ++t) {
+      const int c = c0 + 32 * t;
+      if (c < nwords) dst[c] = dequant8_f16(w[t], sh[t] | (sh[t] << 16));
+    }
   }
 }
 }  // namespace
@@ -763,12 +794,15 @@ cudaError_t launch_dequant_many(const DequantSrc* src, const int* rows, const in
   jb.n = n;
   jb.first[0] = 0;
   for (int j = 0; j < n; ++j) {
+    if (K[j] % 32 != 0 || rows[j] < 0) return cudaErrorInvalidValue;
     jb.src[j] = src[j];
     jb.out[j] = out[j];
     jb.K[j] = K[j];
-    jb.first[j + 1] = jb.first[j] + (int64_t)rows[j] * (K[j] >> 5);
+    const int64_t next = (int64_t)jb.first[j] + (int64_t)rows[j] * ((K[j] + kDqCols - 1) / kDqCols);
+    if (next > 0x7fffffff) return cudaErrorInvalidValue;
+    jb.first[j + 1] = (int)next;
   }
-  int64_t grid = (jb.first[n] + 255) / 256;
+  int64_t grid = ((int64_t)jb.first[n] + 7) / 8;  // 8 warps per CTA
   const int64_t cap = (int64_t)sm_count() * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
@@ -843,7 +877,7 @@ bool gemm_q4_supported(const PackedB& B, int N, int K) {
 cudaError_t launch_gemm_q4(const uint16_t* A, const PackedB& B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
   if (M < 1 || !gemm_q4_supported(B, N, K) || !aligned16(A)) return cudaErrorInvalidValue;
-  if (epi == kEpiRope && (N % 128 != 0 || !e.bias || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
+  if (epi == kEpiRope && (N % 128 != 0 || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
   for (int g = 0; g < B.nseg; ++g)
     if (!aligned16(B.q[g]) || !aligned16(B.s[g])) return cudaErrorInvalidValue;
   const int sms = sm_count();
@@ -876,7 +910,7 @@ size_t gemm_tc_smem() { return smem_bytes<256>(); }
 cudaError_t launch_gemm_tc(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi,
                            const GemmEpilogue& e, cudaStream_t s) {
   if (M < 1 || N % 64 != 0 || K % BK != 0 || K < BK) return cudaErrorInvalidValue;
-  if (epi == kEpiRope && (N % 128 != 0 || !e.bias || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
+  if (epi == kEpiRope && (N % 128 != 0 || !e.pos || !e.kc || !e.vc)) return cudaErrorInvalidValue;
   if (!aligned16(A) || !aligned16(B)) return cudaErrorInvalidValue;
   const int sms = sm_count();
   const long mt = (M + BM - 1) / BM;

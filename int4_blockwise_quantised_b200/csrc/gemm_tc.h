@@ -11,7 +11,8 @@ constexpr int kEpiBias = 0;    // out_f32[m, n] = acc + bias[n]
 constexpr int kEpiResid = 1;   // out_f32[m, n] += acc
 constexpr int kEpiSwiglu = 2;  // out_f16[m, n/2] = silu(acc[m, n]) * acc[m, n+1], n even
 constexpr int kEpiF16 = 3;     // out_f16[m, n] = fp16(acc + bias[n])
-// q/k/v with rotary embedding: y = acc + bias[n]; the columns of query and key heads are rotated
+// q/k/v with rotary embedding: y = acc + the head's bias (bias / bias_k / bias_v); the columns of
+// query and key heads are rotated
 // at position pos[m] (pairs d, d + D/2 of a head of D = 128); queries -> out_f16[m, n] (fp16,
 // row stride ldo = hq * D), keys / values -> kc / vc [head][cap][D] at slot m (fp16)
 constexpr int kEpiRope = 4;
@@ -21,7 +22,9 @@ struct GemmEpilogue {
   __half* out_f16;
   const __half* bias;
   int ldo;  // row stride of the output in elements
-  // kEpiRope only
+  // kEpiRope only (bias = the query bias; any of the three may be null: no bias)
+  const __half* bias_k;   // [hkv * D]
+  const __half* bias_v;   // [hkv * D]
   const int32_t* pos;     // [M] position ids
   const float* rope_cos;  // [max_pos][D/2]
   const float* rope_sin;

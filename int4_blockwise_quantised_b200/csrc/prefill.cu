@@ -53,30 +53,41 @@ __global__ void __launch_bounds__(256) splice_x_kernel(const int32_t* __restrict
   for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)row * H + i] = __half2float(src[i]);
 }
 
-// Xn[s] = X[s] / sqrt(mean(X[s]^2) + eps) * gamma  -> fp16.  One CTA of 128 threads per row.
+// Xn[s] = X[s] / sqrt(mean(X[s]^2) + eps) * gamma  -> fp16.  One CTA of 128 threads per row; the
+// row is read once and held in registers (H <= 128 * 4 * kNormVec), gamma read as 8-byte vectors.
+constexpr int kNormVec = 15;  // hidden <= 7680
 __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const float* __restrict__ x, int H,
                                                            const __half* __restrict__ gamma,
                                                            float eps, __half* __restrict__ out) {
   const int row = blockIdx.x;
   const float* xr = x + (size_t)row * H;
+  float4 v[kNormVec];
   float ss = 0.f;
-  for (int i = threadIdx.x * 4; i < H; i += 512) {
-    const float4 v = *reinterpret_cast<const float4*>(xr + i);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int k = (threadIdx.x + i * 128) * 4;
+    v[i] = k < H ? *reinterpret_cast<const float4*>(xr + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
   __shared__ float red[4];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   const float inv = rsqrtf((red[0] + red[1] + red[2] + red[3]) / (float)H + eps);
-  for (int i = threadIdx.x * 4; i < H; i += 512) {
-    const float4 v = *reinterpret_cast<const float4*>(xr + i);
-    __half2 a = __floats2half2_rn(v.x * inv * __half2float(gamma[i]), v.y * inv * __half2float(gamma[i + 1]));
-    __half2 b = __floats2half2_rn(v.z * inv * __half2float(gamma[i + 2]), v.w * inv * __half2float(gamma[i + 3]));
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&a);
-    pk.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(out + (size_t)row * H + i) = pk;
+#pragma unroll
+  for (int i = 0; i < kNormVec; ++i) {
+    const int k = (threadIdx.x + i * 128) * 4;
+    if (k < H) {
+      const uint2 g = *reinterpret_cast<const uint2*>(gamma + k);
+      const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&g.x));
+      const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&g.y));
+      const __half2 a = __floats2half2_rn(v[i].x * inv * g01.x, v[i].y * inv * g01.y);
+      const __half2 b = __floats2half2_rn(v[i].z * inv * g23.x, v[i].w * inv * g23.y);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&a);
+      pk.y = *reinterpret_cast<const uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(out + (size_t)row * H + k) = pk;
+    }
   }
 }
 
@@ -170,7 +181,6 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
   const size_t o_xn = take((size_t)SM * (H > HQD ? H : HQD) * 2);
   const size_t o_q = take((size_t)SM * HQD * 2);
   const size_t o_h = take((size_t)SM * I * 2);
-  const size_t o_bias = take((size_t)NQKV * 2);
   // the two-pass path (S > kFusedMaxM): the current layer's weights in fp16, [q/k/v | o |
   // gate/up interleaved | down]
   const size_t w_qkv = (size_t)NQKV * H, w_o = (size_t)H * HQD, w_gu = (size_t)2 * I * H;
@@ -190,7 +200,6 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
   __half* Xn = reinterpret_cast<__half*>(b + o_xn);  // also the attention output O
   __half* Q = reinterpret_cast<__half*>(b + o_q);
   __half* Hm = reinterpret_cast<__half*>(b + o_h);
-  __half* Bqkv = reinterpret_cast<__half*>(b + o_bias);
   __half* W16 = reinterpret_cast<__half*>(b + o_w16);
   const bool two_pass = S > kFusedMaxM;
   // layer l's fp16 weights (two-pass path): matrix m = 0 q/k/v, 1 o, 2 gate/up, 3 down
@@ -246,23 +255,13 @@ cudaError_t prefill_run(vv_decoder* d, int seq, const int32_t* ids, const int32_
     pb.q[2] = w.wv.q; pb.s[2] = ps[2]; pb.rows[2] = Hkv * D;
     pb.nseg = 3;
     pb.s_pitch = d->pf_pitch[0];
-    const uint16_t* bsrc[3] = {w.bq, w.bk, w.bv};
-    const int brows[3] = {HQD, Hkv * D, Hkv * D};
-    int boff = 0;
-    for (int m = 0; m < 3; ++m) {
-      if (bsrc[m])
-        e = cudaMemcpyAsync(Bqkv + boff, bsrc[m], (size_t)brows[m] * 2, cudaMemcpyDeviceToDevice, s);
-      else
-        e = cudaMemsetAsync(Bqkv + boff, 0, (size_t)brows[m] * 2, s);
-      if (e != cudaSuccess) return e;
-      boff += brows[m];
-    }
-    VV_MARK(kPfMisc);
     // q/k/v + bias, rotary embedding at position_ids, fp16 Q and the K/V cache rows written by
     // the GEMM's epilogue
     GemmEpilogue ep = {};
     ep.out_f16 = Q;
-    ep.bias = Bqkv;
+    ep.bias = reinterpret_cast<const __half*>(w.bq);
+    ep.bias_k = reinterpret_cast<const __half*>(w.bk);
+    ep.bias_v = reinterpret_cast<const __half*>(w.bv);
     ep.ldo = HQD;
     ep.pos = pos;
     ep.rope_cos = d->rope_cos;

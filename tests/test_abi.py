@@ -65,3 +65,29 @@ def test_decoder_create_rejects_bad_config():
     st = vv.lib.vv_decoder_create(ctypes.byref(cfg), ctypes.byref(mw), 1 << 20, 1 << 20,
                                   ctypes.byref(h))
     assert st == vv.VV_ERR_INVALID_ARG
+
+
+def test_decoder_create_rejects_misaligned_gain_or_bias():
+    """Norm gains and q/k/v biases are read as vectors by the kernels: a pointer off a 16-byte
+    boundary is an argument error at create time (checked before any device work)."""
+    base = 1 << 20
+    cfg = vv.vv_config(1536, 1, 12, 2, 128, 8960, 1000, 1e-6, 1e6, 16, 16, 0)
+    layers = (vv.vv_layer_weights * 1)()
+    L = layers[0]
+    L.input_norm = L.post_norm = base
+    for name in ("wq", "wk", "wv", "wo", "wgate", "wup", "wdown"):
+        m = getattr(L, name)
+        m.q = m.scales = base
+    L.bq = L.bk = base
+    L.bv = base + 2  # fp16-aligned but not 16-byte aligned
+    mw = vv.vv_model_weights(base, base, base, layers)
+    h = ctypes.c_void_p()
+    st = vv.lib.vv_decoder_create(ctypes.byref(cfg), ctypes.byref(mw), base, base,
+                                  ctypes.byref(h))
+    code, text = vv.last_error()
+    assert st == vv.VV_ERR_INVALID_ARG and not h.value and "bias" in text
+    L.bv = base
+    L.post_norm = base + 8
+    st = vv.lib.vv_decoder_create(ctypes.byref(cfg), ctypes.byref(mw), base, base,
+                                  ctypes.byref(h))
+    assert st == vv.VV_ERR_INVALID_ARG and not h.value
